@@ -1,0 +1,257 @@
+// Sliding-window GQA attention of the block rows over the paged KV cache.
+//
+// Work split (flash-decoding): one CTA per (request, kv head, chunk of 64 cache
+// keys = 4 pages) plus one CTA for the block's own keys.  The query vectors of
+// a kv head's group (G query heads x Bk block rows, padded to 16-row mma
+// tiles) attend to the chunk; each warp owns 16 query vectors.  K and V rows of
+// the chunk are brought into shared memory by the TMA engine (1-D bulk copies,
+// 256 bytes per row into a padded 272-byte stride, completion on an mbarrier
+// with a bounded wait).  Scores and P.V use mma.sync m16n8k16; softmax
+// statistics are fp32.  A combine kernel merges the chunk partials.
+//
+// Visibility (FastFlowLM card, "Draft" row: sliding window 2048): block row t
+// sits at position p = Lb + t (Lb = cached tokens after this step's append);
+// cache key j is visible iff max(0, p - W + 1) <= j < Lb; all block keys are
+// visible to all block rows.
+#pragma once
+#include "common.cuh"
+
+namespace dfl {
+
+struct AttnParams {
+  const uint16_t *qb, *kb, *vb;  // [Mb][nq|nkv][128]
+  const uint16_t *kc, *vc;       // this layer's cache [pages][nkv][16][128]
+  const int32_t* page_table;
+  int max_pages, num_pages;
+  const int32_t *seq_len, *n_new;  // seq_len before the step (advanced later by the selector kernel)
+  int Bk, nq, nkv, W;
+  int NC;    // cache chunks per (request, kv head); chunk index NC = the block keys
+  int QVP;   // query vectors per (request, kv head), padded to 16
+  float *part_o, *part_ml;  // [B][nkv][NC+1][QVP][128], [B][nkv][NC+1][QVP][2]
+  float scale_log2;         // log2(e) / sqrt(128)
+  int* err;
+};
+
+DEVI void attn_geometry(const AttnParams& p, int b, long long& Lb, long long& cs, int& nact) {
+  Lb = (long long)p.seq_len[b] + p.n_new[b];
+  long long s0 = Lb - p.W + 1;
+  if (s0 < 0) s0 = 0;
+  cs = (s0 / kPage) * kPage;
+  nact = (int)((Lb - cs + kAttnKeys - 1) / kAttnKeys);
+}
+
+template <int MT>  // 16-row query tiles per CTA (= warps)
+__global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* Ks = Qs + MT * 16 * kAttnStride;
+  uint16_t* Vs = Ks + kAttnKeys * kAttnStride;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int row_ok[kAttnKeys];
+
+  const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.nq / p.nkv, nqv = G * p.Bk;
+  long long Lb, cs;
+  int nact;
+  attn_geometry(p, b, Lb, cs, nact);
+  const bool blk = c == p.NC;
+  if (!blk && c >= nact) return;
+  const long long key0 = cs + (long long)c * kAttnKeys;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  // queries of this (request, kv head): vector qv = t*G + gi -> head kvh*G + gi of block row t
+  for (int i = threadIdx.x; i < MT * 16 * 16; i += blockDim.x) {
+    const int qv = i >> 4, v = i & 15;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (qv < nqv) {
+      const int t = qv / G, gi = qv % G;
+      val = *reinterpret_cast<const uint4*>(p.qb + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + v * 8);
+    }
+    *reinterpret_cast<uint4*>(Qs + qv * kAttnStride + v * 8) = val;
+  }
+  if (blk) {
+    for (int i = threadIdx.x; i < kAttnKeys * 16; i += blockDim.x) {
+      const int u = i >> 4, v = i & 15;
+      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+      if (u < p.Bk) {
+        const size_t off = ((size_t)(b * p.Bk + u) * p.nkv + kvh) * kHeadDim + v * 8;
+        kv = *reinterpret_cast<const uint4*>(p.kb + off);
+        vv = *reinterpret_cast<const uint4*>(p.vb + off);
+      }
+      *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = kv;
+      *reinterpret_cast<uint4*>(Vs + u * kAttnStride + v * 8) = vv;
+    }
+    if (threadIdx.x < kAttnKeys) row_ok[threadIdx.x] = threadIdx.x < p.Bk;
+    __syncthreads();
+  } else {
+    __syncthreads();  // barrier initialised
+    if (warp == 0) {
+      int ok[2];
+      int32_t pg[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int kk = lane + 32 * h;
+        const long long j = key0 + kk;
+        ok[h] = 0;
+        pg[h] = -1;
+        if (j < Lb) {
+          const int lp = (int)(j / kPage);
+          pg[h] = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+          if (pg[h] >= 0 && pg[h] < p.num_pages) ok[h] = 1;
+          else set_err(p.err, DFLASH2_DEV_PAGE);
+        }
+        row_ok[kk] = ok[h];
+      }
+      const int nvalid = __popc(__ballot_sync(0xffffffffu, ok[0])) + __popc(__ballot_sync(0xffffffffu, ok[1]));
+      if (lane == 0) mbar_expect_tx(&bar, (uint32_t)nvalid * 2u * kHeadDim * 2u);
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int kk = lane + 32 * h;
+        if (ok[h]) {
+          const long long j = key0 + kk;
+          const size_t off = (((size_t)pg[h] * p.nkv + kvh) * kPage + j % kPage) * kHeadDim;
+          bulk_g2s(Ks + kk * kAttnStride, p.kc + off, kHeadDim * 2, &bar);
+          bulk_g2s(Vs + kk * kAttnStride, p.vc + off, kHeadDim * 2, &bar);
+        } else {
+          uint4* kr = reinterpret_cast<uint4*>(Ks + kk * kAttnStride);
+          uint4* vr = reinterpret_cast<uint4*>(Vs + kk * kAttnStride);
+          for (int v = 0; v < 16; ++v) kr[v] = vr[v] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(&bar, 0)) {
+      if (threadIdx.x == 0) set_err(p.err, DFLASH2_DEV_TIMEOUT);
+      return;
+    }
+  }
+
+  // ---- S = Q K^T for this warp's 16 query vectors x 64 keys ----
+  const int g = lane >> 2, t4 = lane & 3;
+  float s[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  const uint16_t* Qw = Qs + warp * 16 * kAttnStride;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t a[4];
+    ldmatrix_x4(a, Qw + (lane & 15) * kAttnStride + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      uint32_t b0, b1;
+      ldmatrix_x2(b0, b1, Ks + (n * 8 + (lane & 7)) * kAttnStride + ks * 16 + ((lane >> 3) & 1) * 8);
+      mma16816(s[n], a, b0, b1);
+    }
+  }
+  // ---- mask, chunk-local softmax (log2 domain) ----
+  float mrow[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int qv = warp * 16 + g + 8 * (e >> 1);
+      const int kk = n * 8 + 2 * t4 + (e & 1);
+      bool vis = qv < nqv && row_ok[kk];
+      if (vis && !blk) {
+        const long long j = key0 + kk;
+        const long long pos = Lb + qv / G;
+        vis = j >= pos - p.W + 1;
+      }
+      const float v = vis ? s[n][e] * p.scale_log2 : -INFINITY;
+      s[n][e] = v;
+      mrow[e >> 1] = fmaxf(mrow[e >> 1], v);
+    }
+  float lrow[2] = {0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 1));
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 2));
+  }
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = mrow[e >> 1];
+      const float pv = m == -INFINITY ? 0.f : exp2f(s[n][e] - m);
+      s[n][e] = pv;
+      lrow[e >> 1] += pv;
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+  }
+  // ---- O = P V ----
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t a[4];
+    a[0] = pack_bf2(s[2 * kk][0], s[2 * kk][1]);
+    a[1] = pack_bf2(s[2 * kk][2], s[2 * kk][3]);
+    a[2] = pack_bf2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+    a[3] = pack_bf2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      uint32_t b0, b1;
+      ldmatrix_x2_trans(b0, b1, Vs + (kk * 16 + (lane & 15)) * kAttnStride + n * 8);
+      mma16816(o[n], a, b0, b1);
+    }
+  }
+  // ---- write the chunk partial ----
+  const size_t base = (((size_t)b * p.nkv + kvh) * (p.NC + 1) + c) * p.QVP + warp * 16;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int row = g + 8 * h;
+    float* orow = p.part_o + (base + row) * kHeadDim;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(orow + n * 8 + 2 * t4) = make_float2(o[n][2 * h], o[n][2 * h + 1]);
+    if (t4 == 0) *reinterpret_cast<float2*>(p.part_ml + (base + row) * 2) = make_float2(mrow[h], lrow[h]);
+  }
+}
+
+// One warp per (request, kv head, query vector): merge the chunk partials -> o bf16 [Mb][nq][128].
+__global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
+  const int lane = threadIdx.x & 31;
+  const int qv = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int G = p.nq / p.nkv;
+  if (qv >= G * p.Bk) return;
+  long long Lb, cs;
+  int nact;
+  attn_geometry(p, b, Lb, cs, nact);
+  if (nact > p.NC) nact = p.NC;
+  const size_t base = ((size_t)b * p.nkv + kvh) * (p.NC + 1);
+  float M = -INFINITY;
+  for (int c = 0; c <= p.NC; ++c) {
+    if (c < p.NC && c >= nact) continue;
+    M = fmaxf(M, p.part_ml[((base + c) * p.QVP + qv) * 2]);
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
+  for (int c = 0; c <= p.NC; ++c) {
+    if (c < p.NC && c >= nact) continue;
+    const size_t idx = (base + c) * p.QVP + qv;
+    const float m = p.part_ml[idx * 2];
+    if (m == -INFINITY) continue;
+    const float w = exp2f(m - M);
+    L += w * p.part_ml[idx * 2 + 1];
+    const float4 v = *reinterpret_cast<const float4*>(p.part_o + idx * kHeadDim + lane * 4);
+    acc[0] += w * v.x;
+    acc[1] += w * v.y;
+    acc[2] += w * v.z;
+    acc[3] += w * v.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const int t = qv / G, gi = qv % G;
+  uint16_t* dst = ob + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + lane * 4;
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf2(acc[0] * inv, acc[1] * inv), pack_bf2(acc[2] * inv, acc[3] * inv));
+}
+
+}  // namespace dfl

@@ -1,0 +1,653 @@
+// C ABI of the DFlash 2 drafter block step (include/dflash2.h): argument
+// validation, workspace layout and the launch sequence of the sm_100a kernels.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "lmhead.cuh"
+#include "rowops.cuh"
+#include "selector.cuh"
+
+using namespace dfl;
+
+namespace {
+
+struct GemvPlan {
+  int NT = 1, ksplit = 1, units_per_split = 1, kc_units = 1, mgroups = 1, groups = 1;
+  size_t smem = 0;
+};
+
+struct Plan {
+  int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
+  bool q4;
+  GemvPlan fc, dc, qkv, o, gu, dn;
+  int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
+  size_t lm_smem;
+  size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
+      off_act, off_hn, off_cv, off_ci, off_z;
+  size_t off_s_taps, off_s_nnew, off_s_btok, off_s_tgt, off_s_path, off_s_scores, off_s_acc, off_s_emit;
+  size_t step_bytes, total;
+};
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
+  GemvPlan g;
+  const int R = rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
+  g.NT = R / 8;
+  g.mgroups = (rows + 63) / 64;
+  if (R < 64) g.mgroups = 1;
+  g.groups = (tiles + kWarps - 1) / kWarps;
+  const int units = K / kUnit;
+  const int target = 2 * nsm;
+  int ks = (int)lround((double)target / (double)(g.groups * g.mgroups));
+  ks = std::max(1, std::min(units, ks));
+  g.units_per_split = (units + ks - 1) / ks;
+  g.ksplit = (units + g.units_per_split - 1) / g.units_per_split;
+  const int per_unit = R * 512 + (q4 ? 8 * R * 4 : 0);
+  const int budget = 100 * 1024 - 64 * R - (q4 ? kWarps * 1024 : 0);
+  g.kc_units = std::max(1, std::min(g.units_per_split, budget / per_unit));
+  g.smem = (size_t)R * (g.kc_units * 512 + 64) + (q4 ? (size_t)g.kc_units * 8 * R * 4 + kWarps * 1024 : 0);
+  return g;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool cfg_ok(const dflash2_config* c) {
+  if (!c) return false;
+  const long long HQ = (long long)c->n_q * c->head_dim;
+  return c->layers >= 1 && c->layers <= DFLASH2_MAX_LAYERS && c->head_dim == kHeadDim && c->page_size == kPage &&
+         c->topk == kTopK && c->block >= 2 && c->block <= kMaxD + 1 && c->n_kv >= 1 && c->n_q % c->n_kv == 0 &&
+         (c->n_q / c->n_kv) * c->block <= 64 && c->hidden % kUnit == 0 && c->ffn % kUnit == 0 &&
+         HQ % kUnit == 0 && ((long long)c->n_taps * c->hidden) % kUnit == 0 && c->n_taps >= 1 &&
+         c->vocab % 16 == 0 && c->vocab > 0 && c->rank % 16 == 0 && c->rank >= 16 && c->rank <= kMaxR &&
+         c->window >= 1 && c->hidden <= 16384 && (c->wfmt == 0 || c->wfmt == 1) && c->rope_theta > 0.f &&
+         c->rms_eps >= 0.f;
+}
+
+Plan make_plan(const dflash2_config* c, int B) {
+  Plan p;
+  p.B = B;
+  p.Bk = c->block;
+  p.D = c->block - 1;
+  p.Mb = B * c->block;
+  p.H = c->hidden;
+  p.F = c->ffn;
+  p.HQ = c->n_q * kHeadDim;
+  p.HKV = c->n_kv * kHeadDim;
+  p.T = c->n_taps;
+  p.V = c->vocab;
+  p.R = c->rank;
+  p.nsm = device_sms();
+  p.q4 = c->wfmt == 0;
+  p.G = c->n_q / c->n_kv;
+  p.QV = p.G * p.Bk;
+  p.QVP = (p.QV + 15) / 16 * 16;
+  p.MT = p.QVP / 16;
+  p.NC = (c->window + kPage - 2 + kAttnKeys - 1) / kAttnKeys;
+  p.fc = plan_gemv(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
+  p.dc = plan_gemv((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
+  p.qkv = plan_gemv((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
+  p.o = plan_gemv(p.H / 16, p.Mb, p.HQ, p.q4, p.nsm);
+  p.gu = plan_gemv(2 * p.F / 16, p.Mb, p.H, p.q4, p.nsm);
+  p.dn = plan_gemv(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
+  p.lm_rows = B * p.D;
+  if (p.lm_rows <= 8) {
+    p.lm_NT = 1;
+    p.lm_rows_per_pass = 8;
+  } else {
+    p.lm_NT = 2;
+    p.lm_rows_per_pass = 16;
+  }
+  p.lm_passes = (p.lm_rows + p.lm_rows_per_pass - 1) / p.lm_rows_per_pass;
+  const int R8 = p.lm_NT * 8;
+  p.lm_smem = (size_t)R8 * (p.H * 2 + 64) + (size_t)kWarps * R8 * kTopK * 8;
+  const int lm_tiles = p.V / 16 + p.R / 16;
+  p.lm_nparts = std::min((p.lm_NT == 1 ? 2 : 1) * p.nsm, (lm_tiles + kWarps - 1) / kWarps);
+
+  auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.ksplit * rows * ldo * 4; };
+  size_t part = 0;
+  part = std::max(part, part_bytes(p.fc, p.Mb, p.H));
+  part = std::max(part, part_bytes(p.dc, p.Mb, p.H / 2));
+  part = std::max(part, part_bytes(p.qkv, 2 * p.Mb, p.HQ + 2 * p.HKV));
+  part = std::max(part, part_bytes(p.o, p.Mb, p.H));
+  part = std::max(part, part_bytes(p.gu, p.Mb, 2 * p.F));
+  part = std::max(part, part_bytes(p.dn, p.Mb, p.H));
+
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t r = o;
+    o = align256(o + bytes);
+    return r;
+  };
+  p.off_err = take(256);
+  p.off_h = take((size_t)p.Mb * p.H * 4);
+  p.off_xf = take((size_t)p.Mb * p.H * 4);
+  p.off_xb = take((size_t)p.Mb * p.H * 2);
+  p.off_yb = take((size_t)2 * p.Mb * p.H * 2);
+  p.off_part = take(part);
+  p.off_qb = take((size_t)p.Mb * p.HQ * 2);
+  p.off_kb = take((size_t)p.Mb * p.HKV * 2);
+  p.off_vb = take((size_t)p.Mb * p.HKV * 2);
+  const size_t nchunk = (size_t)B * c->n_kv * (p.NC + 1) * p.QVP;
+  p.off_ao = take(nchunk * kHeadDim * 4);
+  p.off_aml = take(nchunk * 2 * 4);
+  p.off_ob = take((size_t)p.Mb * p.HQ * 2);
+  p.off_act = take((size_t)p.Mb * p.F * 2);
+  p.off_hn = take((size_t)std::max(p.lm_rows, 1) * p.H * 2);
+  p.off_cv = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
+  p.off_ci = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
+  p.off_z = take((size_t)p.lm_rows * p.R * 4);
+  p.step_bytes = o;
+  p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
+  p.off_s_nnew = take((size_t)B * 4);
+  p.off_s_btok = take((size_t)p.Mb * 4);
+  p.off_s_tgt = take((size_t)p.Mb * 4);
+  p.off_s_path = take((size_t)B * p.D * 4);
+  p.off_s_scores = take((size_t)B * p.D * 4);
+  p.off_s_acc = take((size_t)B * 4);
+  p.off_s_emit = take((size_t)p.Mb * 4);
+  p.total = o;
+  return p;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+template <int NT, bool Q4>
+cudaError_t launch_gemv_t(const GemvPlan& g, const GemvParams& prm, int tiles, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemv<NT, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((tiles + kWarps - 1) / kWarps, g.ksplit, g.mgroups);
+  k_gemv<NT, Q4><<<grid, kWarps * 32, g.smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, const uint16_t* X, int ldx,
+                        int rows_stage, int K, float* out, int ldo, int out_rows, cudaStream_t s) {
+  GemvParams prm;
+  memset(&prm, 0, sizeof(prm));
+  int tiles = 0;
+  for (int i = 0; i < nseg; ++i) {
+    prm.seg[i] = segs[i];
+    tiles += segs[i].tiles;
+  }
+  prm.nseg = nseg;
+  prm.X = X;
+  prm.ldx = ldx;
+  prm.rows_stage = rows_stage;
+  prm.K = K;
+  prm.units_per_split = g.units_per_split;
+  prm.kc_units = g.kc_units;
+  prm.out = out;
+  prm.ldo = ldo;
+  prm.split_stride = (long long)out_rows * ldo;
+  prm.m_group_rows = 64;
+  switch (g.NT * 2 + (q4 ? 1 : 0)) {
+    case 2: return launch_gemv_t<1, false>(g, prm, tiles, s);
+    case 3: return launch_gemv_t<1, true>(g, prm, tiles, s);
+    case 4: return launch_gemv_t<2, false>(g, prm, tiles, s);
+    case 5: return launch_gemv_t<2, true>(g, prm, tiles, s);
+    case 8: return launch_gemv_t<4, false>(g, prm, tiles, s);
+    case 9: return launch_gemv_t<4, true>(g, prm, tiles, s);
+    case 16: return launch_gemv_t<8, false>(g, prm, tiles, s);
+    case 17: return launch_gemv_t<8, true>(g, prm, tiles, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_norm(const NormParams& np, int rows, cudaStream_t s) {
+  k_norm<<<rows, 256, np.H * sizeof(float), s>>>(np);
+  return cudaGetLastError();
+}
+
+template <int MT>
+cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
+  static bool attr = false;
+  const size_t smem = (size_t)(MT * 16 + 2 * kAttnKeys) * kAttnStride * 2;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_chunk<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_attn_chunk<MT><<<dim3(P.NC + 1, ap.nkv, P.B), MT * 32, smem, s>>>(ap);
+  return cudaGetLastError();
+}
+
+int fail(cudaError_t e) { return e == cudaSuccess ? DFLASH2_OK : DFLASH2_ERR_CUDA; }
+
+#define CK(expr)                          \
+  do {                                    \
+    cudaError_t e_ = (expr);              \
+    if (e_ != cudaSuccess) return fail(e_); \
+  } while (0)
+
+int check_weights(const dflash2_config* c, const dflash2_weights* w) {
+  if (!w) return DFLASH2_ERR_ARG;
+  if (c->wfmt == 0 && !w->prepared) return DFLASH2_ERR_LAYOUT;
+  const void* ptrs[] = {w->fc, w->fc_norm, w->final_norm, w->embed, w->lm_head, w->sel_proj, w->cb_a, w->cb_b};
+  for (const void* q : ptrs) {
+    if (!q) return DFLASH2_ERR_ARG;
+    if (!aligned16(q)) return DFLASH2_ERR_ALIGN;
+  }
+  for (int l = 0; l < c->layers; ++l) {
+    const dflash2_layer_weights& L = w->layer[l];
+    const void* lp[] = {L.wq, L.wk, L.wv, L.wo, L.wg, L.wu, L.wd, L.ln1, L.ln2, L.qn, L.kn, L.dc_w, L.dc_s0, L.dc_s1};
+    for (const void* q : lp) {
+      if (!q) return DFLASH2_ERR_ARG;
+      if (!aligned16(q)) return DFLASH2_ERR_ALIGN;
+    }
+  }
+  return DFLASH2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dflash2_workspace_size(const dflash2_config* cfg, int32_t batch) {
+  if (!cfg_ok(cfg) || batch < 1) return 0;
+  return make_plan(cfg, batch).total;
+}
+
+size_t dflash2_prepared_size(const dflash2_config* c) {
+  if (!cfg_ok(c) || c->wfmt != 0) return 0;
+  const size_t H = c->hidden, F = c->ffn, HQ = (size_t)c->n_q * kHeadDim, HKV = (size_t)c->n_kv * kHeadDim;
+  const size_t per_layer = HQ * H + 2 * HKV * H + H * HQ + 2 * F * H + H * F;
+  return (H * c->n_taps * H + c->layers * per_layer) / kUnit * 144;
+}
+
+int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src, void* dst, size_t dst_bytes,
+                            dflash2_weights* out, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (!src || !out) return DFLASH2_ERR_ARG;
+  dflash2_weights tmp = *src;
+  tmp.prepared = 0;
+  int rc = check_weights(c, &tmp);
+  if (rc != DFLASH2_OK && rc != DFLASH2_ERR_LAYOUT) return rc;
+  *out = *src;
+  out->prepared = 1;
+  if (c->wfmt != 0) return DFLASH2_OK;
+  if (!dst || !aligned16(dst)) return dst ? DFLASH2_ERR_ALIGN : DFLASH2_ERR_ARG;
+  if (dst_bytes < dflash2_prepared_size(c)) return DFLASH2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* d = (uint8_t*)dst;
+  const int H = c->hidden, F = c->ffn, HQ = c->n_q * kHeadDim, HKV = c->n_kv * kHeadDim;
+  auto prep = [&](const void* w, int N, int K) -> const void* {
+    k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K);
+    const void* r = d;
+    d += (size_t)N * K / kUnit * 144;
+    return r;
+  };
+  out->fc = prep(src->fc, H, c->n_taps * H);
+  for (int l = 0; l < c->layers; ++l) {
+    const dflash2_layer_weights& S = src->layer[l];
+    dflash2_layer_weights& O = out->layer[l];
+    O.wq = prep(S.wq, HQ, H);
+    O.wk = prep(S.wk, HKV, H);
+    O.wv = prep(S.wv, HKV, H);
+    O.wo = prep(S.wo, H, HQ);
+    O.wg = prep(S.wg, F, H);
+    O.wu = prep(S.wu, F, H);
+    O.wd = prep(S.wd, H, F);
+  }
+  return fail(cudaGetLastError());
+}
+
+int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const dflash2_inputs* in,
+                       const dflash2_kv* kv, int32_t batch, int32_t* out_path, float* out_scores, void* ws,
+                       size_t ws_bytes, const dflash2_debug* dbg, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (batch < 1 || !in || !kv || !out_path || !out_scores || !ws) return DFLASH2_ERR_ARG;
+  int rc = check_weights(c, w);
+  if (rc) return rc;
+  if (!in->taps || !in->n_new || !in->block_tokens || !kv->page_table || !kv->seq_len || kv->max_pages < 1 ||
+      kv->num_pages < 1)
+    return DFLASH2_ERR_ARG;
+  for (int l = 0; l < c->layers; ++l) {
+    if (!kv->k[l] || !kv->v[l]) return DFLASH2_ERR_ARG;
+    if (!aligned16(kv->k[l]) || !aligned16(kv->v[l])) return DFLASH2_ERR_ALIGN;
+  }
+  if (!aligned16(in->taps) || ((uintptr_t)ws & 255u)) return DFLASH2_ERR_ALIGN;
+  const Plan P = make_plan(c, batch);
+  if (ws_bytes < P.step_bytes) return DFLASH2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  int* err = at<int>(ws, P.off_err);
+  float* h = at<float>(ws, P.off_h);
+  float* xf = at<float>(ws, P.off_xf);
+  uint16_t* xb = at<uint16_t>(ws, P.off_xb);
+  uint16_t* yb = at<uint16_t>(ws, P.off_yb);
+  uint16_t* ctx = yb + (size_t)P.Mb * P.H;
+  float* part = at<float>(ws, P.off_part);
+  uint16_t* qb = at<uint16_t>(ws, P.off_qb);
+  uint16_t* kb = at<uint16_t>(ws, P.off_kb);
+  uint16_t* vb = at<uint16_t>(ws, P.off_vb);
+  uint16_t* ob = at<uint16_t>(ws, P.off_ob);
+  uint16_t* act = at<uint16_t>(ws, P.off_act);
+  uint16_t* hn = at<uint16_t>(ws, P.off_hn);
+  float* zbuf = at<float>(ws, P.off_z);
+  const int H = P.H, Mb = P.Mb;
+  const size_t hbytes = (size_t)Mb * H * 4;
+
+  CK(cudaMemsetAsync(err, 0, 4, s));
+  // A1: block rows from the shared embedding table
+  k_embed<<<Mb, 256, 0, s>>>(in->block_tokens, w->embed, h, H, P.V, err);
+  CK(cudaGetLastError());
+  if (dbg && dbg->hidden) CK(cudaMemcpyAsync(dbg->hidden, h, hbytes, cudaMemcpyDeviceToDevice, s));
+
+  // A2: context rows = RMSNorm_fc(W_fc . concat(taps))
+  {
+    GemvSeg seg{(const uint8_t*)w->fc, H / 16, Mb, 0};
+    CK(launch_gemv(P.fc, P.q4, &seg, 1, in->taps, P.T * H, Mb, P.T * H, part, H, Mb, s));
+    NormParams np{};
+    np.part = part;
+    np.nsplit = P.fc.ksplit;
+    np.split_stride = (long long)Mb * H;
+    np.ldp = H;
+    np.w = w->fc_norm;
+    np.eps = c->rms_eps;
+    np.H = H;
+    np.out_bf = ctx;
+    np.ldob = H;
+    np.mode = 1;
+    np.n_new = in->n_new;
+    np.Bk = P.Bk;
+    CK(launch_norm(np, Mb, s));
+    if (dbg && dbg->ctx) CK(cudaMemcpyAsync(dbg->ctx, ctx, (size_t)Mb * H * 2, cudaMemcpyDeviceToDevice, s));
+  }
+
+  AttnParams ap{};
+  ap.qb = qb;
+  ap.kb = kb;
+  ap.vb = vb;
+  ap.page_table = kv->page_table;
+  ap.max_pages = kv->max_pages;
+  ap.num_pages = kv->num_pages;
+  ap.seq_len = kv->seq_len;
+  ap.n_new = in->n_new;
+  ap.Bk = P.Bk;
+  ap.nq = c->n_q;
+  ap.nkv = c->n_kv;
+  ap.W = c->window;
+  ap.NC = P.NC;
+  ap.QVP = P.QVP;
+  ap.part_o = at<float>(ws, P.off_ao);
+  ap.part_ml = at<float>(ws, P.off_aml);
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
+  ap.err = err;
+
+  const GemvPlan* prev_down = nullptr;
+  for (int l = 0; l < c->layers; ++l) {
+    const dflash2_layer_weights& L = w->layer[l];
+    // A3a: x = RMSNorm(h; ln1) (adding the previous layer's MLP output), g = W_dc x, y = dynconv(x, g)
+    {
+      NormParams np{};
+      np.h = h;
+      if (prev_down) {
+        np.part = part;
+        np.nsplit = prev_down->ksplit;
+        np.split_stride = (long long)Mb * H;
+        np.ldp = H;
+      }
+      np.w = L.ln1;
+      np.eps = c->rms_eps;
+      np.H = H;
+      np.out_bf = xb;
+      np.ldob = H;
+      np.out_f = xf;
+      np.mode = 0;
+      np.Bk = P.Bk;
+      CK(launch_norm(np, Mb, s));
+      if (dbg && dbg->hidden && l > 0)
+        CK(cudaMemcpyAsync(dbg->hidden + (size_t)l * Mb * H, h, hbytes, cudaMemcpyDeviceToDevice, s));
+      GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
+      CK(launch_gemv(P.dc, false, &seg, 1, xb, H, Mb, H, part, H / 2, Mb, s));
+      k_dynconv<<<Mb, 256, 0, s>>>(xf, part, P.dc.ksplit, (long long)Mb * (H / 2), H / 2, L.dc_s0, L.dc_s1, H,
+                                   P.Bk, yb);
+      CK(cudaGetLastError());
+    }
+    // A3b: q from the block rows; k, v from block + context rows (stacked: read each matrix once)
+    {
+      const int ldo = P.HQ + 2 * P.HKV;
+      GemvSeg segs[3] = {{(const uint8_t*)L.wq, P.HQ / 16, Mb, 0},
+                         {(const uint8_t*)L.wk, P.HKV / 16, 2 * Mb, P.HQ},
+                         {(const uint8_t*)L.wv, P.HKV / 16, 2 * Mb, P.HQ + P.HKV}};
+      CK(launch_gemv(P.qkv, P.q4, segs, 3, yb, H, 2 * Mb, H, part, ldo, 2 * Mb, s));
+      // A3c: q/k norms, RoPE, context K/V appended to the paged cache
+      RopeParams rp{};
+      rp.part = part;
+      rp.nsplit = P.qkv.ksplit;
+      rp.split_stride = (long long)2 * Mb * ldo;
+      rp.ldp = ldo;
+      rp.qn = L.qn;
+      rp.kn = L.kn;
+      rp.eps = c->rms_eps;
+      rp.log2_theta = log2((double)c->rope_theta);
+      rp.Bk = P.Bk;
+      rp.nq = c->n_q;
+      rp.nkv = c->n_kv;
+      rp.Mb = Mb;
+      rp.seq_len = kv->seq_len;
+      rp.n_new = in->n_new;
+      rp.qb = qb;
+      rp.kb = kb;
+      rp.vb = vb;
+      rp.kc = kv->k[l];
+      rp.vc = kv->v[l];
+      rp.page_table = kv->page_table;
+      rp.max_pages = kv->max_pages;
+      rp.num_pages = kv->num_pages;
+      rp.err = err;
+      const int nslot = c->n_q + 2 * c->n_kv;
+      k_qk_rope_append<<<dim3((nslot + 3) / 4, 2 * Mb), 128, 0, s>>>(rp);
+      CK(cudaGetLastError());
+    }
+    // A3d: sliding-window GQA attention over cache + block keys
+    {
+      ap.kc = kv->k[l];
+      ap.vc = kv->v[l];
+      switch (P.MT) {
+        case 1: CK(launch_attn_t<1>(P, ap, s)); break;
+        case 2: CK(launch_attn_t<2>(P, ap, s)); break;
+        case 3: CK(launch_attn_t<3>(P, ap, s)); break;
+        default: CK(launch_attn_t<4>(P, ap, s)); break;
+      }
+      k_attn_combine<<<dim3((P.QV + 3) / 4, c->n_kv, batch), 128, 0, s>>>(ap, ob);
+      CK(cudaGetLastError());
+    }
+    // A3e: h += W_o o (added by the next norm)
+    {
+      GemvSeg seg{(const uint8_t*)L.wo, H / 16, Mb, 0};
+      CK(launch_gemv(P.o, P.q4, &seg, 1, ob, P.HQ, Mb, P.HQ, part, H, Mb, s));
+      NormParams np{};
+      np.h = h;
+      np.part = part;
+      np.nsplit = P.o.ksplit;
+      np.split_stride = (long long)Mb * H;
+      np.ldp = H;
+      np.w = L.ln2;
+      np.eps = c->rms_eps;
+      np.H = H;
+      np.out_bf = xb;
+      np.ldob = H;
+      np.mode = 0;
+      np.Bk = P.Bk;
+      CK(launch_norm(np, Mb, s));
+    }
+    // A3f: h += W_d (silu(W_g x2) * W_u x2)
+    {
+      GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wu, P.F / 16, Mb, P.F}};
+      CK(launch_gemv(P.gu, P.q4, segs, 2, xb, H, Mb, H, part, 2 * P.F, Mb, s));
+      const size_t n = (size_t)Mb * P.F;
+      const int blocks = (int)std::min<size_t>((n + 255) / 256, (size_t)P.nsm * 8);
+      k_silu_mul<<<blocks, 256, 0, s>>>(part, P.gu.ksplit, (long long)Mb * 2 * P.F, 2 * P.F, Mb, P.F, act);
+      CK(cudaGetLastError());
+      GemvSeg seg{(const uint8_t*)L.wd, H / 16, Mb, 0};
+      CK(launch_gemv(P.dn, P.q4, &seg, 1, act, P.F, Mb, P.F, part, H, Mb, s));
+      prev_down = &P.dn;
+    }
+  }
+  // A4: final norm of the drafted rows 1..block-1 (adding the last MLP output)
+  {
+    NormParams np{};
+    np.h = h;
+    np.part = part;
+    np.nsplit = P.dn.ksplit;
+    np.split_stride = (long long)Mb * H;
+    np.ldp = H;
+    np.w = w->final_norm;
+    np.eps = c->rms_eps;
+    np.H = H;
+    np.out_bf = hn;
+    np.ldob = H;
+    np.mode = 2;
+    np.Bk = P.Bk;
+    CK(launch_norm(np, Mb, s));
+    if (dbg && dbg->hidden)
+      CK(cudaMemcpyAsync(dbg->hidden + (size_t)c->layers * Mb * H, h, hbytes, cudaMemcpyDeviceToDevice, s));
+    if (dbg && dbg->final_h)
+      CK(cudaMemcpyAsync(dbg->final_h, hn, (size_t)P.lm_rows * H * 2, cudaMemcpyDeviceToDevice, s));
+  }
+  // A5: LM head + streaming top-16 (+ selector projection)
+  {
+    if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
+    for (int pass = 0; pass < P.lm_passes; ++pass) {
+      LmParams lp{};
+      lp.W = w->lm_head;
+      lp.Ws = w->sel_proj;
+      lp.V = P.V;
+      lp.R = P.R;
+      lp.H = H;
+      lp.row_base = pass * P.lm_rows_per_pass;
+      lp.X = hn + (size_t)lp.row_base * H;
+      lp.rows = std::min(P.lm_rows_per_pass, P.lm_rows - lp.row_base);
+      lp.rows_total = P.lm_rows;
+      lp.z = zbuf;
+      lp.cand_val = at<float>(ws, P.off_cv);
+      lp.cand_id = at<int32_t>(ws, P.off_ci);
+      if (P.lm_NT == 1) {
+        static bool attr = false;
+        if (!attr) {
+          CK(cudaFuncSetAttribute(k_lmhead_topk<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+          attr = true;
+        }
+        k_lmhead_topk<1><<<P.lm_nparts, kWarps * 32, P.lm_smem, s>>>(lp);
+      } else {
+        static bool attr = false;
+        if (!attr) {
+          CK(cudaFuncSetAttribute(k_lmhead_topk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+          attr = true;
+        }
+        k_lmhead_topk<2><<<P.lm_nparts, kWarps * 32, P.lm_smem, s>>>(lp);
+      }
+      CK(cudaGetLastError());
+    }
+    if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
+    if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  // A6: candidates, selector scores, Viterbi path; seq_len advanced
+  {
+    SelParams sp{};
+    sp.cand_val = at<float>(ws, P.off_cv);
+    sp.cand_id = at<int32_t>(ws, P.off_ci);
+    sp.nparts = P.lm_nparts;
+    sp.rows_total = P.lm_rows;
+    sp.z = zbuf;
+    sp.R = P.R;
+    sp.V = P.V;
+    sp.Bk = P.Bk;
+    sp.cb_a = w->cb_a;
+    sp.cb_b = w->cb_b;
+    sp.block_tokens = in->block_tokens;
+    sp.out_path = out_path;
+    sp.out_scores = out_scores;
+    sp.seq_len = kv->seq_len;
+    sp.n_new = in->n_new;
+    sp.dbg_cand = dbg ? dbg->cand : nullptr;
+    sp.dbg_logit = dbg ? dbg->cand_logit : nullptr;
+    sp.err = err;
+    if (sp.dbg_cand && !sp.dbg_logit) sp.dbg_cand = nullptr;
+    k_selector<<<batch, 256, 0, s>>>(sp);
+    CK(cudaGetLastError());
+  }
+  return DFLASH2_OK;
+}
+
+int dflash2_accept(const int32_t* draft, const int32_t* target, int32_t batch, int32_t block, int32_t* accepted,
+                   int32_t* emitted, void* stream) {
+  if (!draft || !target || !accepted || !emitted || batch < 1 || block < 2) return DFLASH2_ERR_ARG;
+  k_accept<<<(batch + 127) / 128, 128, 0, (cudaStream_t)stream>>>(draft, target, batch, block, accepted, emitted);
+  return fail(cudaGetLastError());
+}
+
+int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, const dflash2_kv* kv, int32_t batch,
+                           const uint16_t* taps_h, const int32_t* n_new_h, const int32_t* block_tokens_h,
+                           const int32_t* target_h, int32_t* path_h, float* scores_h, int32_t* accepted_h,
+                           int32_t* emitted_h, int32_t* dev_err, void* ws, size_t ws_bytes, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (batch < 1 || !taps_h || !n_new_h || !block_tokens_h || !target_h || !path_h || !scores_h || !accepted_h ||
+      !emitted_h || !ws)
+    return DFLASH2_ERR_ARG;
+  const Plan P = make_plan(c, batch);
+  if (ws_bytes < P.total) return DFLASH2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t Mb = P.Mb;
+  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_taps), taps_h, Mb * P.T * P.H * 2, cudaMemcpyHostToDevice, s));
+  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_nnew), n_new_h, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_btok), block_tokens_h, Mb * 4, cudaMemcpyHostToDevice, s));
+  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_tgt), target_h, Mb * 4, cudaMemcpyHostToDevice, s));
+  dflash2_inputs in{at<uint16_t>(ws, P.off_s_taps), at<int32_t>(ws, P.off_s_nnew), at<int32_t>(ws, P.off_s_btok)};
+  int rc = dflash2_draft_step(c, w, &in, kv, batch, at<int32_t>(ws, P.off_s_path), at<float>(ws, P.off_s_scores), ws,
+                              ws_bytes, nullptr, stream);
+  if (rc) return rc;
+  rc = dflash2_accept(at<int32_t>(ws, P.off_s_path), at<int32_t>(ws, P.off_s_tgt), batch, P.Bk,
+                      at<int32_t>(ws, P.off_s_acc), at<int32_t>(ws, P.off_s_emit), stream);
+  if (rc) return rc;
+  CK(cudaMemcpyAsync(path_h, at<void>(ws, P.off_s_path), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaMemcpyAsync(scores_h, at<void>(ws, P.off_s_scores), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaMemcpyAsync(accepted_h, at<void>(ws, P.off_s_acc), (size_t)batch * 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaMemcpyAsync(emitted_h, at<void>(ws, P.off_s_emit), Mb * 4, cudaMemcpyDeviceToHost, s));
+  if (dev_err) CK(cudaMemcpyAsync(dev_err, at<void>(ws, P.off_err), 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return DFLASH2_OK;
+}
+
+int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {
+  if (!ws || !out_bits) return DFLASH2_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  CK(cudaMemcpyAsync(out_bits, ws, 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return DFLASH2_OK;
+}
+
+const char* dflash2_strerror(int code) {
+  switch (code) {
+    case DFLASH2_OK: return "ok";
+    case DFLASH2_ERR_ARG: return "null pointer or bad argument";
+    case DFLASH2_ERR_SHAPE: return "configuration not supported by the kernels";
+    case DFLASH2_ERR_ALIGN: return "device pointer not 16-byte aligned (workspace: 256-byte)";
+    case DFLASH2_ERR_WORKSPACE: return "workspace or prepared-weight buffer too small";
+    case DFLASH2_ERR_CUDA: return "CUDA launch or copy failed";
+    case DFLASH2_ERR_LAYOUT: return "Q4_K weights must go through dflash2_prepare_weights";
+  }
+  return "unknown error";
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+// Candidate merge, selector transition scores and the Viterbi path, one CTA per
+// request (FastFlowLM card: "picks one coherent path through its top 16
+// candidates per position"; "Weights" row: selector projection and two
+// 248320 x 256 codebooks).
+//
+// Transition score (the reading fixed for the pages' unnamed formula):
+//   tau_t(a -> b) = sum_r A[a][r] * z_t[r] * Bc[b][r],  z_t = W_s h~_t,
+// sources at position 0 = the block's first token, at t > 0 the candidates of
+// t-1; unary = candidate logit;
+//   delta_0(j) = u_0(j) + tau_0(x0 -> c_0j)
+//   delta_t(j) = u_t(j) + max_i (delta_{t-1}(i) + tau_t(c_{t-1,i} -> c_tj)),
+// smaller candidate index on ties.  fp32 throughout.
+#pragma once
+#include "common.cuh"
+
+namespace dfl {
+
+constexpr int kMaxD = 15;
+constexpr int kMaxR = 256;
+
+struct SelParams {
+  const float* cand_val;  // [nparts][rows_total][16], each list sorted
+  const int32_t* cand_id;
+  int nparts, rows_total;
+  const float* z;  // [rows_total][R]
+  int R, V, Bk;
+  const uint16_t *cb_a, *cb_b;
+  const int32_t* block_tokens;
+  int32_t* out_path;
+  float* out_scores;
+  int32_t* seq_len;
+  const int32_t* n_new;
+  int32_t* dbg_cand;
+  float* dbg_logit;
+  int* err;
+};
+
+__global__ void __launch_bounds__(256) k_selector(SelParams p) {
+  const int b = blockIdx.x, D = p.Bk - 1, R = p.R;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int cand[kMaxD][kTopK];
+  __shared__ float cl[kMaxD][kTopK];
+  __shared__ float tau[kTopK][kTopK];
+  __shared__ float delta[kMaxD][kTopK];
+  __shared__ int bp[kMaxD][kTopK];
+  __shared__ int src_ids[kTopK];
+  // phase 1: per-lane merge lists [warps][32][16] (values, then ids); phase 2: codebook rows
+  __shared__ __align__(16) float big[2 * kTopK * kMaxR];
+  float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big);
+  float(*Wj)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big + kTopK * kMaxR);
+
+  // 1. merge the CTA lists of each drafted position into the final top-16
+  for (int t = warp; t < D; t += kWarps) {
+    const int row = b * D + t;
+    float* lv = big + (warp * 32 + lane) * kTopK;
+    int* li = reinterpret_cast<int*>(big + kWarps * 32 * kTopK) + (warp * 32 + lane) * kTopK;
+    for (int k = 0; k < kTopK; ++k) { lv[k] = -INFINITY; li[k] = 0x7fffffff; }
+    for (int part = lane; part < p.nparts; part += 32) {
+      const size_t o = ((size_t)part * p.rows_total + row) * kTopK;
+      for (int k = 0; k < kTopK; ++k) {
+        const float v = p.cand_val[o + k];
+        const int id = p.cand_id[o + k];
+        if (!better(v, id, lv[kTopK - 1], li[kTopK - 1])) break;  // list is sorted: the rest is worse
+        int pos = kTopK - 1;
+        while (pos > 0 && better(v, id, lv[pos - 1], li[pos - 1])) {
+          lv[pos] = lv[pos - 1];
+          li[pos] = li[pos - 1];
+          --pos;
+        }
+        lv[pos] = v;
+        li[pos] = id;
+      }
+    }
+    __syncwarp();
+    int head = 0;
+    for (int k = 0; k < kTopK; ++k) {
+      float bv = head < kTopK ? lv[head] : -INFINITY;
+      int bid = head < kTopK ? li[head] : 0x7fffffff;
+      int bl = lane;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+        const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+        if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) {
+          bv = ov;
+          bid = oid;
+          bl = ol;
+        }
+      }
+      if (lane == 0) {
+        cand[t][k] = bid;
+        cl[t][k] = bv;
+      }
+      if (lane == bl) ++head;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < D * kTopK) {
+    const int t = threadIdx.x / kTopK, k = threadIdx.x % kTopK;
+    const float v = cl[t][k];
+    int id = cand[t][k];
+    if (!isfinite(v)) set_err(p.err, DFLASH2_DEV_NONFINITE);
+    if (id < 0 || id >= p.V) {
+      set_err(p.err, DFLASH2_DEV_NONFINITE);
+      cand[t][k] = 0;
+    }
+  }
+  __syncthreads();
+
+  // 2. per position: transition scores tau_t, then one Viterbi step in warp 0
+  //    (lane j of warp 0 holds delta_t(j))
+  float d = 0.f;
+  for (int t = 0; t < D; ++t) {
+    const int nsrc = t == 0 ? 1 : kTopK;
+    if (threadIdx.x < kTopK) {
+      int a = t == 0 ? p.block_tokens[b * p.Bk] : cand[t - 1][threadIdx.x];
+      if (a < 0 || a >= p.V) a = 0;
+      src_ids[threadIdx.x] = a;
+    }
+    __syncthreads();
+    const float* zt = p.z + (size_t)(b * D + t) * R;
+    for (int i = threadIdx.x; i < kTopK * R; i += blockDim.x) {
+      const int j = i / R, r = i % R;
+      Wj[j][r] = zt[r] * bf2f(p.cb_b[(size_t)cand[t][j] * R + r]);
+      if (j < nsrc) As[j][r] = bf2f(p.cb_a[(size_t)src_ids[j] * R + r]);
+    }
+    __syncthreads();
+    {
+      const int i = threadIdx.x / kTopK, j = threadIdx.x % kTopK;
+      if (i < nsrc) {
+        float s = 0.f;
+        for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[j][r], s);
+        tau[i][j] = s;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int j = lane & 15;
+      int bi = 0;
+      if (t == 0) {
+        d = cl[0][j] + tau[0][j];
+      } else {
+        float best = 0.f;
+        bi = -1;
+        for (int i = 0; i < kTopK; ++i) {
+          const float s = __shfl_sync(0xffffffffu, d, i) + tau[i][j];
+          if (bi < 0 || s > best) { best = s; bi = i; }
+        }
+        d = cl[t][j] + best;
+      }
+      if (lane < kTopK) { delta[t][j] = d; bp[t][j] = bi; }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int jj = 0;
+    for (int i = 1; i < kTopK; ++i)
+      if (delta[D - 1][i] > delta[D - 1][jj]) jj = i;
+    for (int t = D - 1; t >= 0; --t) {
+      p.out_path[b * D + t] = cand[t][jj];
+      p.out_scores[b * D + t] = delta[t][jj];
+      jj = bp[t][jj];
+    }
+    p.seq_len[b] += p.n_new[b];
+  }
+  if (p.dbg_cand && threadIdx.x < D * kTopK) {
+    const int t = threadIdx.x / kTopK, k = threadIdx.x % kTopK;
+    p.dbg_cand[(b * D + t) * kTopK + k] = cand[t][k];
+    p.dbg_logit[(b * D + t) * kTopK + k] = cl[t][k];
+  }
+}
+
+}  // namespace dfl

@@ -73,6 +73,11 @@ class Workload:
     target_mode: str         # "uniform" or "first_mismatch"
     seed: int
     description: str = ""
+    weight_seed: int = 0     # seed of the weight set (0: use ``seed``)
+
+    @property
+    def wseed(self) -> int:
+        return self.weight_seed or self.seed
 
 
 TINY = Dims(layers=1, hidden=512, ffn=1536, n_q=4, n_kv=1, head_dim=128, window=64,
@@ -88,9 +93,9 @@ WORKLOADS: Dict[str, Workload] = {
                         "full DFlash2 shape, 1 request, 4096 cached tokens"),
     "full_b8_paged": Workload("full_b8_paged", FULL, 8, 2048, 32768, True, False, False,
                               "first_mismatch", 1003,
-                              "full shape, 8 requests, 2048..32768 cached, shuffled 16-token pages"),
+                              "full shape, 8 requests, 2048..32768 cached, shuffled 16-token pages", 1002),
     "full_b64": Workload("full_b64", FULL, 64, 512, 8192, False, False, False, "first_mismatch", 1004,
-                         "full shape, 64 requests (512 block rows), 512..8192 cached"),
+                         "full shape, 64 requests (512 block rows), 512..8192 cached", 1002),
     "full_bf16_b16": Workload("full_bf16_b16", FULL_BF16_B5, 16, 1, 262144, False, True, True,
                               "first_mismatch", 1005,
                               "bf16 layers, block 5, 16 requests, up to 262144 cached, 1% tap outliers"),

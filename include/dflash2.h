@@ -1,0 +1,201 @@
+/*
+ * dflash2.h — C ABI of the DFlash 2 drafter block step on one NVIDIA B200 (sm_100a).
+ *
+ * The step (FastFlowLM model card for Qwen3.8-27B-DFlash2, "Draft", "Weights",
+ * "Taps" and "How it is used" rows; MLX sidecar card, "Contents"): the target's
+ * residual features at five tapped layers are fused by an fc layer into
+ * context rows; a block of 8 positions (the last emitted token and 7 mask
+ * positions) runs through 5 Qwen3-style layers (RMSNorm, two-tap dynamic
+ * convolution, GQA attention with a 2048-token sliding window over the paged
+ * KV cache, SwiGLU MLP); the shared output head scores the 7 drafted positions,
+ * the 16 best tokens per position are kept, and a rank-256 selector picks one
+ * path through them; greedy acceptance then keeps the longest prefix that
+ * agrees with the target's tokens, plus one target token.
+ *
+ * Conventions for every call:
+ *  - Pointers named in the structs below are DEVICE pointers unless a comment
+ *    says host.  All memory is owned by the caller; the library allocates
+ *    nothing (no cudaMalloc, no host heap) and frees nothing.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls are asynchronous on it unless stated otherwise.
+ *  - bf16 tensors are uint16_t bit patterns; row-major; no padding.
+ *  - Return value: DFLASH2_OK (0) or a negative DFLASH2_ERR_* code.  Host-side
+ *    validation failures launch nothing.  Conditions only the GPU can see
+ *    (token id out of range, an unmapped KV page inside the window, non-finite
+ *    logits, an expired bounded wait) set bits in a device error word at the
+ *    start of the workspace; read it with dflash2_device_error().
+ */
+#ifndef DFLASH2_H
+#define DFLASH2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DFLASH2_MAX_LAYERS 8
+
+#define DFLASH2_OK 0
+#define DFLASH2_ERR_ARG (-1)       /* null pointer or bad scalar argument */
+#define DFLASH2_ERR_SHAPE (-2)     /* configuration outside what the kernels support */
+#define DFLASH2_ERR_ALIGN (-3)     /* a device pointer is not 16-byte aligned */
+#define DFLASH2_ERR_WORKSPACE (-4) /* workspace or prepared-weight buffer too small */
+#define DFLASH2_ERR_CUDA (-5)      /* a CUDA launch or copy failed */
+#define DFLASH2_ERR_LAYOUT (-6)    /* Q4_K weights passed without dflash2_prepare_weights */
+
+/* device error bits (dflash2_device_error) */
+#define DFLASH2_DEV_TOKEN 1     /* a block token id is outside [0, vocab) */
+#define DFLASH2_DEV_PAGE 2      /* a KV page needed by the window or an append is unmapped (-1) */
+#define DFLASH2_DEV_NONFINITE 4 /* a candidate logit is NaN or infinite */
+#define DFLASH2_DEV_TIMEOUT 8   /* a bounded wait on a bulk copy expired */
+
+/* Model dimensions.  The full drafter (FastFlowLM card, "Draft" row; aiqre.com
+ * model page, vocabulary): layers 5, hidden 5120, ffn 17408, n_q 32, n_kv 8,
+ * head_dim 128, window 2048, vocab 248320, n_taps 5, block 8, topk 16, rank 256.
+ * Supported: head_dim 128, page_size 16, topk 16, 2 <= block <= 16,
+ * n_q % n_kv == 0, (n_q / n_kv) * block <= 64, hidden, ffn, n_q*head_dim and
+ * n_taps*hidden multiples of 256, vocab and rank multiples of 16, rank <= 256.
+ * rope_theta: RoPE base (1e6); rms_eps: RMSNorm epsilon (1e-6).
+ * wfmt: storage of fc and the layer matrices, 0 = Q4_K, 1 = bf16. */
+typedef struct dflash2_config {
+  int32_t layers, hidden, ffn, n_q, n_kv, head_dim, window, vocab, n_taps, block, topk, rank,
+      page_size;
+  float rope_theta, rms_eps;
+  int32_t wfmt;
+} dflash2_config;
+
+/* One layer.  Matrices are [out, in] row-major: bf16, or Q4_K as 144-byte
+ * super-blocks of 256 consecutive inputs (d fp16, dmin fp16, eight 6-bit
+ * scales and eight 6-bit mins each packed little-endian into 6 bytes, 128
+ * bytes of 4-bit codes, low nibble first; weight = d*sc*q - dmin*m).  After
+ * dflash2_prepare_weights the Q4_K pointers refer to the prepared layout.
+ *   wq [n_q*hd, H], wk/wv [n_kv*hd, H], wo [H, n_q*hd], wg/wu [F, H], wd [H, F]
+ *   ln1, ln2 [H]: attention / MLP pre-norm weights; qn, kn [hd]: per-head q/k norms
+ *   dc_w [2*(H/4), H]: dynamic-convolution gate generator; dc_s0, dc_s1 [H]:
+ *   static taps.  y_t = (s0 + tanh g_t[c/4]) x_t + (s1 + tanh g_t[H/4 + c/4]) x_{t-1},
+ *   g_t = dc_w x_t, x = RMSNorm(h; ln1), causal along the block (x_{-1} = 0). */
+typedef struct dflash2_layer_weights {
+  const void *wq, *wk, *wv, *wo, *wg, *wu, *wd;
+  const uint16_t *ln1, *ln2, *qn, *kn, *dc_w, *dc_s0, *dc_s1;
+} dflash2_layer_weights;
+
+/* fc [H, n_taps*H] (wfmt), fc_norm [H]; final_norm [H]; embed and lm_head
+ * [vocab, H] bf16 (the target's shared embedding table and output head);
+ * sel_proj [rank, H]; cb_a, cb_b [vocab, rank] (the selector's projection and
+ * its two codebooks, FastFlowLM card, "Weights" row).  prepared: 0 for the
+ * canonical Q4_K layout, 1 once dflash2_prepare_weights has filled the struct. */
+typedef struct dflash2_weights {
+  const void *fc;
+  const uint16_t *fc_norm;
+  dflash2_layer_weights layer[DFLASH2_MAX_LAYERS];
+  const uint16_t *final_norm, *embed, *lm_head, *sel_proj, *cb_a, *cb_b;
+  int32_t prepared;
+} dflash2_weights;
+
+/* Paged KV cache of the context tokens (aiqre.com model page, "Memory": 20 KiB
+ * per token at 16-bit = 5 layers x 8 heads x 128 x {K,V} x 2 bytes).
+ * k[l], v[l]: bf16 [num_pages][n_kv][page_size][head_dim] per layer.
+ * page_table: int32 [batch][max_pages]; logical page i of a request holds its
+ * tokens page_size*i .. page_size*i + page_size-1; -1 = not backed (allowed for
+ * pages the window can no longer reach).  seq_len: int32 [batch], cached
+ * tokens before the step; the step appends n_new rows and advances it. */
+typedef struct dflash2_kv {
+  uint16_t *k[DFLASH2_MAX_LAYERS];
+  uint16_t *v[DFLASH2_MAX_LAYERS];
+  const int32_t *page_table;
+  int32_t max_pages, num_pages;
+  int32_t *seq_len;
+} dflash2_kv;
+
+/* Per-step inputs (device).
+ * taps: bf16 [batch][block][n_taps*hidden], row t of request b holds the target's
+ *   features at layers 5, 19, 33, 47, 61 (in that order) for its t-th new token;
+ *   rows t >= n_new[b] are ignored.
+ * n_new: int32 [batch], 0..block new context tokens per request.
+ * block_tokens: int32 [batch][block]: position 0 = last emitted token, 1..block-1 =
+ *   the caller's mask id. */
+typedef struct dflash2_inputs {
+  const uint16_t *taps;
+  const int32_t *n_new;
+  const int32_t *block_tokens;
+} dflash2_inputs;
+
+/* Optional device outputs for checking and profiling; any field may be NULL.
+ * hidden: fp32 [layers+1][batch*block][hidden] residual stream after the
+ *   embedding and after each layer; ctx: bf16 [batch*block][hidden] fused
+ *   context rows; final_h: bf16 [batch*(block-1)][hidden] final-normed rows (the
+ *   LM head's operand); cand: int32 and cand_logit: fp32 [batch*(block-1)][16];
+ *   z: fp32 [batch*(block-1)][rank] selector projection.
+ * ev_lm_begin / ev_lm_end: cudaEvent_t (as void*) recorded on `stream` around
+ *   the LM-head + top-16 kernel. */
+typedef struct dflash2_debug {
+  float *hidden;
+  uint16_t *ctx;
+  uint16_t *final_h;
+  int32_t *cand;
+  float *cand_logit;
+  float *z;
+  void *ev_lm_begin, *ev_lm_end;
+} dflash2_debug;
+
+/* Bytes of device workspace dflash2_draft_step needs for `batch` requests on
+ * the current device (depends on its SM count).  0 on an invalid config. */
+size_t dflash2_workspace_size(const dflash2_config *cfg, int32_t batch);
+
+/* Bytes of the prepared copy of the Q4_K matrices (0 for wfmt 1). */
+size_t dflash2_prepared_size(const dflash2_config *cfg);
+
+/* Repack the Q4_K matrices of `src` (canonical layout, device) into `dst`
+ * (device, dst_bytes >= dflash2_prepared_size) in the tile order the GEMV
+ * kernels stream, and fill `out` (host struct) with `src`'s pointers except the
+ * Q4_K matrices, which point into dst; out->prepared = 1.  Values are not
+ * changed: the prepared copy holds the same bits, reordered.  For wfmt 1 it
+ * copies the struct and sets prepared = 1.  Asynchronous on `stream`. */
+int dflash2_prepare_weights(const dflash2_config *cfg, const dflash2_weights *src, void *dst,
+                            size_t dst_bytes, dflash2_weights *out, void *stream);
+
+/* One block step for `batch` requests (the section comment at the top of this
+ * file).  out_path: int32 [batch][block-1] drafted token ids; out_scores: fp32
+ * [batch][block-1], the selector's cumulative path score at each position.
+ * Appends n_new context rows per request to every layer's cache and advances
+ * kv->seq_len.  workspace: device, >= dflash2_workspace_size bytes, 256-byte
+ * aligned; its first word is the device error word, cleared at the start of
+ * the step.  dbg may be NULL. */
+int dflash2_draft_step(const dflash2_config *cfg, const dflash2_weights *w, const dflash2_inputs *in,
+                       const dflash2_kv *kv, int32_t batch, int32_t *out_path, float *out_scores,
+                       void *workspace, size_t ws_bytes, const dflash2_debug *dbg, void *stream);
+
+/* Greedy acceptance (FastFlowLM card, "How it is used"): draft int32
+ * [batch][block-1], target int32 [batch][block] (the target's most likely token
+ * for block positions 1..block).  accepted[b] = longest n <= block-1 with
+ * draft[b][i] == target[b][i] for i < n; emitted[b] = draft[b][0..n-1], then
+ * target[b][n], then -1 padding to `block`.  Device pointers. */
+int dflash2_accept(const int32_t *draft, const int32_t *target, int32_t batch, int32_t block,
+                   int32_t *accepted, int32_t *emitted, void *stream);
+
+/* A whole speculative draft round with HOST buffers: copies taps, n_new,
+ * block_tokens and target (host, same layouts as above) into the workspace,
+ * runs dflash2_draft_step and dflash2_accept, copies path, scores, accepted and
+ * emitted back to host memory and synchronizes `stream`.  Page-locked host
+ * buffers make the copies asynchronous.  Weights and the KV cache stay on the
+ * device.  Returns the first error; device error bits are returned in
+ * *dev_err (host) when dev_err is not NULL. */
+int dflash2_spec_step_host(const dflash2_config *cfg, const dflash2_weights *w, const dflash2_kv *kv,
+                           int32_t batch, const uint16_t *taps_h, const int32_t *n_new_h,
+                           const int32_t *block_tokens_h, const int32_t *target_h, int32_t *path_h,
+                           float *scores_h, int32_t *accepted_h, int32_t *emitted_h,
+                           int32_t *dev_err, void *workspace, size_t ws_bytes, void *stream);
+
+/* Copy the device error word of `workspace` to *out_bits (host) and
+ * synchronize `stream`. */
+int dflash2_device_error(const void *workspace, int32_t *out_bits, void *stream);
+
+/* Static description of an error code. */
+const char *dflash2_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFLASH2_H */

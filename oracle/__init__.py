@@ -208,6 +208,17 @@ def selector(cand, cand_logit, z, x0: int, cb_a, cb_b):
     return path, sc
 
 
+def selector_trans(cand, z, x0: int, cb_a, cb_b) -> np.ndarray:
+    """Transition scores tau [D][K][K] of the selector (row = source index, column = destination)."""
+    cand = _np(cand, np.int32)
+    D, K = cand.shape
+    zz = np.ascontiguousarray(z, np.float64)
+    tr = np.empty((D, K, K), np.float64)
+    lib().orc_selector_trans(D, K, zz.shape[1], _p(cand), _p(zz), int(x0), _p(_np(cb_a, np.uint16)),
+                             _p(_np(cb_b, np.uint16)), _p(tr))
+    return tr
+
+
 def accept(draft, target):
     d = _np(draft, np.int32)
     t = _np(target, np.int32)

@@ -358,12 +358,10 @@ void orc_viterbi(int D, int K, const double *unary, const double *trans, int32_t
  * unary score = the candidate's raw logit (a per-position log-softmax shift
  * does not move the argmax path).  Sources at position 0 are the block's first
  * token x0, at position t > 0 the candidates of position t-1.
- * cand, cand_logit: [D][K]; z: [D][R].  path: token ids [D]; scores: [D]. */
-void orc_selector(int D, int K, int R, const int32_t *cand, const double *cand_logit,
-                  const double *z, int32_t x0, const uint16_t *cb_a, const uint16_t *cb_b,
-                  int32_t *path, double *scores) {
-  double *trans = (double *)calloc((size_t)D * K * K, sizeof(double));
-  int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)D);
+ * cand: [D][K]; z: [D][R]; trans: [D][K][K] (row = source index, column = destination). */
+void orc_selector_trans(int D, int K, int R, const int32_t *cand, const double *z, int32_t x0,
+                        const uint16_t *cb_a, const uint16_t *cb_b, double *trans) {
+  memset(trans, 0, sizeof(double) * (size_t)D * K * K);
   for (int t = 0; t < D; ++t) {
     int nsrc = t == 0 ? 1 : K;
     for (int i = 0; i < nsrc; ++i) {
@@ -378,6 +376,16 @@ void orc_selector(int D, int K, int R, const int32_t *cand, const double *cand_l
       }
     }
   }
+}
+
+/* The path itself: Viterbi over the candidates with tau as transitions and the
+ * raw logits as unary scores.  path: token ids [D]; scores: [D]. */
+void orc_selector(int D, int K, int R, const int32_t *cand, const double *cand_logit,
+                  const double *z, int32_t x0, const uint16_t *cb_a, const uint16_t *cb_b,
+                  int32_t *path, double *scores) {
+  double *trans = (double *)malloc(sizeof(double) * (size_t)D * K * K);
+  int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)D);
+  orc_selector_trans(D, K, R, cand, z, x0, cb_a, cb_b, trans);
   orc_viterbi(D, K, cand_logit, trans, idx, scores);
   for (int t = 0; t < D; ++t) path[t] = cand[t * K + idx[t]];
   free(trans);

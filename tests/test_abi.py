@@ -1,0 +1,78 @@
+"""The C ABI library loads on a host without a GPU and exports every declared entry point;
+host-side validation answers before any device work."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from block_diffusion_drafter_dflash2_b200 import build, inputs
+from block_diffusion_drafter_dflash2_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared():
+    txt = open(os.path.join(ROOT, "include", "dflash2.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(dflash2_\w+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared()
+    assert set(names) == set(binding.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror_and_sizes(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.dflash2_strerror(code)
+    cfg = binding.config(inputs.TINY)
+    assert lib.dflash2_workspace_size(C.byref(cfg), 1) > 0
+    d = inputs.TINY
+    H, F, HQ, HKV = d.hidden, d.ffn, d.n_q * 128, d.n_kv * 128
+    mats = H * d.n_taps * H + d.layers * (HQ * H + 2 * HKV * H + H * HQ + 3 * F * H)
+    assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144
+    full = binding.config(inputs.FULL)
+    # the prepared Q4_K copy has exactly the canonical size (973.2 MB of Q4_K matrices for the full drafter)
+    assert abs(lib.dflash2_prepared_size(C.byref(full)) / 1e6 - 973.2) < 0.5
+    assert lib.dflash2_prepared_size(C.byref(binding.config(inputs.FULL_BF16_B5))) == 0
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 64), ("page_size", 32), ("topk", 8), ("block", 1),
+                                         ("block", 17), ("hidden", 500), ("n_kv", 3), ("rank", 512),
+                                         ("vocab", 8200), ("layers", 9), ("wfmt", 2)])
+def test_unsupported_config_is_rejected(lib, field, value):
+    cfg = binding.config(inputs.TINY)
+    setattr(cfg, field, value)
+    assert lib.dflash2_workspace_size(C.byref(cfg), 1) == 0
+    rc = lib.dflash2_draft_step(C.byref(cfg), None, None, None, 1, None, None, None, 0, None, None)
+    assert rc == -2
+
+
+def test_null_arguments_are_rejected(lib):
+    cfg = binding.config(inputs.TINY)
+    assert lib.dflash2_draft_step(C.byref(cfg), None, None, None, 1, None, None, None, 0, None, None) == -1
+    w = binding.Weights()
+    assert lib.dflash2_draft_step(C.byref(cfg), C.byref(w), None, None, 0, None, None, None, 0, None, None) == -1
+    assert lib.dflash2_accept(None, None, 1, 8, None, None, None) == -1
+    out = C.c_int32()
+    assert lib.dflash2_device_error(None, C.byref(out), None) == -1
+
+
+def test_unprepared_q4k_weights_are_rejected(lib):
+    cfg = binding.config(inputs.TINY)
+    w = binding.Weights()
+    w.prepared = 0
+    ins, kv = binding.Inputs(), binding.KV()
+    buf = C.create_string_buffer(64)
+    rc = lib.dflash2_draft_step(C.byref(cfg), C.byref(w), C.byref(ins), C.byref(kv), 1, buf, buf, buf, 0, None,
+                                None)
+    assert rc == -6
