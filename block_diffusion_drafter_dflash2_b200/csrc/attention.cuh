@@ -49,6 +49,8 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int row_ok[kAttnKeys];
 
+  pdl_trigger();
+  pdl_wait();
   const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.nq / p.nkv, nqv = G * p.Bk;
@@ -218,9 +220,13 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
 }
 
 // One warp per (request, kv head, query vector): merge the chunk partials -> o bf16 [Mb][nq][128].
+// Lanes read the chunks' (m, l) in parallel; the weighted sum streams 16-byte rows.
 __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
-  const int lane = threadIdx.x & 31;
-  const int qv = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  __shared__ float wsh[4][64];
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int qv = blockIdx.x * (blockDim.x >> 5) + wi;
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int G = p.nq / p.nkv;
   if (qv >= G * p.Bk) return;
@@ -228,30 +234,50 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
   int nact;
   attn_geometry(p, b, Lb, cs, nact);
   if (nact > p.NC) nact = p.NC;
+  const int nc = nact + 1;  // cache chunks + the block-key chunk (index NC)
   const size_t base = ((size_t)b * p.nkv + kvh) * (p.NC + 1);
+  float m[2], l[2];
   float M = -INFINITY;
-  for (int c = 0; c <= p.NC; ++c) {
-    if (c < p.NC && c >= nact) continue;
-    M = fmaxf(M, p.part_ml[((base + c) * p.QVP + qv) * 2]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = lane + 32 * h;
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+    if (i < nc) {
+      const int c = i < nact ? i : p.NC;
+      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + ((base + c) * p.QVP + qv) * 2);
+      m[h] = ml.x;
+      l[h] = ml.y;
+    }
+    M = fmaxf(M, m[h]);
   }
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
-  for (int c = 0; c <= p.NC; ++c) {
-    if (c < p.NC && c >= nact) continue;
-    const size_t idx = (base + c) * p.QVP + qv;
-    const float m = p.part_ml[idx * 2];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    L += w * p.part_ml[idx * 2 + 1];
-    const float4 v = *reinterpret_cast<const float4*>(p.part_o + idx * kHeadDim + lane * 4);
-    acc[0] += w * v.x;
-    acc[1] += w * v.y;
-    acc[2] += w * v.z;
-    acc[3] += w * v.w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = lane + 32 * h;
+    const float w = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - M);
+    if (i < 64) wsh[wi][i] = w;
+    L += w * l[h];
+  }
+  L = warp_sum(L);
+  __syncwarp();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int i = 0; i < nc; ++i) {
+    const int c = i < nact ? i : p.NC;
+    const float w = wsh[wi][i];
+    const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((base + c) * p.QVP + qv) * kHeadDim + lane * 4);
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const int t = qv / G, gi = qv % G;
   uint16_t* dst = ob + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + lane * 4;
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf2(acc[0] * inv, acc[1] * inv), pack_bf2(acc[2] * inv, acc[3] * inv));
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf2(acc.x * inv, acc.y * inv), pack_bf2(acc.z * inv, acc.w * inv));
 }
 
 }  // namespace dfl

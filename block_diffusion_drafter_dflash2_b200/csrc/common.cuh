@@ -108,6 +108,11 @@ DEVI float warp_sum(float v) {
 // Ordering of candidates: larger logit first, smaller token id on equal logits.
 DEVI bool better(float a, int ia, float b, int ib) { return a > b || (a == b && ia < ib); }
 
+// Programmatic dependent launch: let the next kernel on the stream start its prologue, and
+// wait until every earlier kernel has finished and its writes are visible.
+DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 DEVI void set_err(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }

@@ -11,13 +11,15 @@
 #include "lmhead.cuh"
 #include "rowops.cuh"
 #include "selector.cuh"
+#include "stream.cuh"
 
 using namespace dfl;
 
 namespace {
 
 struct GemvPlan {
-  int NT = 1, ksplit = 1, units_per_split = 1, kc_units = 1, mgroups = 1, groups = 1;
+  int NT = 1, R = 8, groups = 1, mgroups = 1, U = 1, P = 1, kc_units = 1, max_pieces = 1;
+  long long W = 1;
   size_t smem = 0;
 };
 
@@ -26,9 +28,11 @@ struct Plan {
   bool q4;
   GemvPlan fc, dc, qkv, o, gu, dn;
   int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
+  bool lm_stream;
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
-      off_act, off_hn, off_cv, off_ci, off_z;
+      off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
+  size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_total;
   size_t off_s_taps, off_s_nnew, off_s_btok, off_s_tgt, off_s_path, off_s_scores, off_s_acc, off_s_emit;
   size_t step_bytes, total;
 };
@@ -40,23 +44,28 @@ int device_sms() {
   return n;
 }
 
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kStaticSmem = 2048;  // mbarriers and flags of the streaming kernels
+
+// tiles: 16-row tiles over all segments; paired: gate/up (groups = tiles / 8 still, 4 + 4 tiles each)
 GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   GemvPlan g;
-  const int R = rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
-  g.NT = R / 8;
-  g.mgroups = (rows + 63) / 64;
-  if (R < 64) g.mgroups = 1;
-  g.groups = (tiles + kWarps - 1) / kWarps;
-  const int units = K / kUnit;
-  const int target = 2 * nsm;
-  int ks = (int)lround((double)target / (double)(g.groups * g.mgroups));
-  ks = std::max(1, std::min(units, ks));
-  g.units_per_split = (units + ks - 1) / ks;
-  g.ksplit = (units + g.units_per_split - 1) / g.units_per_split;
-  const int per_unit = R * 512 + (q4 ? 8 * R * 4 : 0);
-  const int budget = 100 * 1024 - 64 * R - (q4 ? kWarps * 1024 : 0);
-  g.kc_units = std::max(1, std::min(g.units_per_split, budget / per_unit));
-  g.smem = (size_t)R * (g.kc_units * 512 + 64) + (q4 ? (size_t)g.kc_units * 8 * R * 4 + kWarps * 1024 : 0);
+  g.R = rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
+  g.NT = g.R / 8;
+  g.mgroups = g.R == 64 ? (rows + 63) / 64 : 1;
+  g.groups = (tiles + kConsumers - 1) / kConsumers;
+  const int unitK = q4 ? 256 : 128, slot = q4 ? Ring<true>::kSlot : Ring<false>::kSlot;
+  const int ns = q4 ? Ring<true>::kNS : Ring<false>::kNS;
+  g.U = K / unitK;
+  g.W = (long long)g.groups * g.mgroups * g.U;
+  g.P = (int)std::min<long long>(nsm, g.W);
+  g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
+  const int ring = kConsumers * ns * slot;
+  const int per_unit = g.R * unitK * 2 + (q4 ? 8 * g.R * 4 : 0);
+  const int budget = kSmemLimit - kStaticSmem - ring - (q4 ? kConsumers * 1024 : 0) - 64 * g.R;
+  g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) +
+           (q4 ? (size_t)g.kc_units * 8 * g.R * 4 + kConsumers * 1024 : 0);
   return g;
 }
 
@@ -70,7 +79,7 @@ bool cfg_ok(const dflash2_config* c) {
          (c->n_q / c->n_kv) * c->block <= 64 && c->hidden % kUnit == 0 && c->ffn % kUnit == 0 &&
          HQ % kUnit == 0 && ((long long)c->n_taps * c->hidden) % kUnit == 0 && c->n_taps >= 1 &&
          c->vocab % 16 == 0 && c->vocab > 0 && c->rank % 16 == 0 && c->rank >= 16 && c->rank <= kMaxR &&
-         c->window >= 1 && c->hidden <= 16384 && (c->wfmt == 0 || c->wfmt == 1) && c->rope_theta > 0.f &&
+         c->window >= 1 && c->window <= 4032 && c->hidden <= 16384 && (c->wfmt == 0 || c->wfmt == 1) && c->rope_theta > 0.f &&
          c->rms_eps >= 0.f;
 }
 
@@ -101,20 +110,23 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.gu = plan_gemv(2 * p.F / 16, p.Mb, p.H, p.q4, p.nsm);
   p.dn = plan_gemv(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
   p.lm_rows = B * p.D;
-  if (p.lm_rows <= 8) {
+  const int lm_tiles = p.V / 16 + p.R / 16;
+  p.lm_stream = p.lm_rows <= 8;
+  if (p.lm_stream) {
     p.lm_NT = 1;
     p.lm_rows_per_pass = 8;
+    p.lm_smem = (size_t)kConsumers * Ring<false>::kNS * Ring<false>::kSlot + (size_t)8 * (p.H * 2 + 64) +
+                (size_t)kConsumers * 8 * kTopK * 8;
+    p.lm_nparts = std::min(p.nsm, (lm_tiles + kConsumers - 1) / kConsumers);
   } else {
     p.lm_NT = 2;
     p.lm_rows_per_pass = 16;
+    p.lm_smem = (size_t)16 * (p.H * 2 + 64) + (size_t)kWarps * 16 * kTopK * 8;
+    p.lm_nparts = std::min(p.nsm, (lm_tiles + kWarps - 1) / kWarps);
   }
   p.lm_passes = (p.lm_rows + p.lm_rows_per_pass - 1) / p.lm_rows_per_pass;
-  const int R8 = p.lm_NT * 8;
-  p.lm_smem = (size_t)R8 * (p.H * 2 + 64) + (size_t)kWarps * R8 * kTopK * 8;
-  const int lm_tiles = p.V / 16 + p.R / 16;
-  p.lm_nparts = std::min((p.lm_NT == 1 ? 2 : 1) * p.nsm, (lm_tiles + kWarps - 1) / kWarps);
 
-  auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.ksplit * rows * ldo * 4; };
+  auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.max_pieces * rows * ldo * 4; };
   size_t part = 0;
   part = std::max(part, part_bytes(p.fc, p.Mb, p.H));
   part = std::max(part, part_bytes(p.dc, p.Mb, p.H / 2));
@@ -147,6 +159,19 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_cv = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
   p.off_ci = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
+  p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
+  // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
+  auto nctr = [](const GemvPlan& g) { return (size_t)g.groups * g.mgroups; };
+  const GemvPlan* lp[5] = {&p.dc, &p.qkv, &p.o, &p.gu, &p.dn};
+  p.ctr_fc = nctr(p.fc);
+  size_t acc = 0;
+  for (int i = 0; i < 5; ++i) {
+    p.ctr_layer[i] = acc;
+    acc += nctr(*lp[i]);
+  }
+  p.ctr_per_layer = acc;
+  p.ctr_total = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;
+  p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
   p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
   p.off_s_nnew = take((size_t)B * 4);
@@ -167,55 +192,87 @@ T* at(void* ws, size_t off) {
 
 bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
+// Launch with programmatic dependent launch: the kernel may start while the previous kernel on
+// the stream drains; every kernel launched this way calls griddepcontrol.wait before it touches
+// data written by earlier kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 template <int NT, bool Q4>
-cudaError_t launch_gemv_t(const GemvPlan& g, const GemvParams& prm, int tiles, cudaStream_t s) {
+cudaError_t launch_sgemv_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemv<NT, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(k_sgemv<NT, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemLimit - kStaticSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid((tiles + kWarps - 1) / kWarps, g.ksplit, g.mgroups);
-  k_gemv<NT, Q4><<<grid, kWarps * 32, g.smem, s>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kStreamThreads), g.smem, s, prm);
 }
 
-cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, const uint16_t* X, int ldx,
-                        int rows_stage, int K, float* out, int ldo, int out_rows, cudaStream_t s) {
-  GemvParams prm;
+struct Epi {
+  int mode = EPI_STORE;
+  float* y = nullptr;
+  int ldy = 0;
+  uint16_t* act = nullptr;
+  int F = 0;
+  QkvEpi qkv{};
+};
+
+cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X,
+                        int ldx, int rows, float* part, int ldo, int out_rows, int* counters, const Epi& e, int* err,
+                        cudaStream_t s) {
+  SGemvParams prm;
   memset(&prm, 0, sizeof(prm));
-  int tiles = 0;
-  for (int i = 0; i < nseg; ++i) {
-    prm.seg[i] = segs[i];
-    tiles += segs[i].tiles;
-  }
+  for (int i = 0; i < nseg; ++i) prm.seg[i] = segs[i];
   prm.nseg = nseg;
+  prm.paired = paired ? 1 : 0;
   prm.X = X;
   prm.ldx = ldx;
-  prm.rows_stage = rows_stage;
-  prm.K = K;
-  prm.units_per_split = g.units_per_split;
+  prm.rows = rows;
+  prm.U = g.U;
+  prm.groups = g.groups;
+  prm.mgroups = g.mgroups;
+  prm.W = g.W;
   prm.kc_units = g.kc_units;
-  prm.out = out;
+  prm.part = part;
   prm.ldo = ldo;
-  prm.split_stride = (long long)out_rows * ldo;
-  prm.m_group_rows = 64;
+  prm.piece_stride = (long long)out_rows * ldo;
+  prm.counters = counters;
+  prm.epi = e.mode;
+  prm.y = e.y;
+  prm.ldy = e.ldy;
+  prm.act = e.act;
+  prm.F = e.F;
+  prm.qkv = e.qkv;
+  prm.err = err;
   switch (g.NT * 2 + (q4 ? 1 : 0)) {
-    case 2: return launch_gemv_t<1, false>(g, prm, tiles, s);
-    case 3: return launch_gemv_t<1, true>(g, prm, tiles, s);
-    case 4: return launch_gemv_t<2, false>(g, prm, tiles, s);
-    case 5: return launch_gemv_t<2, true>(g, prm, tiles, s);
-    case 8: return launch_gemv_t<4, false>(g, prm, tiles, s);
-    case 9: return launch_gemv_t<4, true>(g, prm, tiles, s);
-    case 16: return launch_gemv_t<8, false>(g, prm, tiles, s);
-    case 17: return launch_gemv_t<8, true>(g, prm, tiles, s);
+    case 2: return launch_sgemv_t<1, false>(g, prm, s);
+    case 3: return launch_sgemv_t<1, true>(g, prm, s);
+    case 4: return launch_sgemv_t<2, false>(g, prm, s);
+    case 5: return launch_sgemv_t<2, true>(g, prm, s);
+    case 8: return launch_sgemv_t<4, false>(g, prm, s);
+    case 9: return launch_sgemv_t<4, true>(g, prm, s);
+    case 16: return launch_sgemv_t<8, false>(g, prm, s);
+    case 17: return launch_sgemv_t<8, true>(g, prm, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_norm(const NormParams& np, int rows, cudaStream_t s) {
-  k_norm<<<rows, 256, np.H * sizeof(float), s>>>(np);
-  return cudaGetLastError();
+  return launch_pdl(k_norm, dim3(rows), dim3(256), np.H * sizeof(float), s, np);
 }
 
 template <int MT>
@@ -227,8 +284,7 @@ cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_attn_chunk<MT><<<dim3(P.NC + 1, ap.nkv, P.B), MT * 32, smem, s>>>(ap);
-  return cudaGetLastError();
+  return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(MT * 32), smem, s, ap);
 }
 
 int fail(cudaError_t e) { return e == cudaSuccess ? DFLASH2_OK : DFLASH2_ERR_CUDA; }
@@ -241,7 +297,7 @@ int fail(cudaError_t e) { return e == cudaSuccess ? DFLASH2_OK : DFLASH2_ERR_CUD
 
 int check_weights(const dflash2_config* c, const dflash2_weights* w) {
   if (!w) return DFLASH2_ERR_ARG;
-  if (c->wfmt == 0 && !w->prepared) return DFLASH2_ERR_LAYOUT;
+  if (!w->prepared) return DFLASH2_ERR_LAYOUT;
   const void* ptrs[] = {w->fc, w->fc_norm, w->final_norm, w->embed, w->lm_head, w->sel_proj, w->cb_a, w->cb_b};
   for (const void* q : ptrs) {
     if (!q) return DFLASH2_ERR_ARG;
@@ -268,10 +324,14 @@ size_t dflash2_workspace_size(const dflash2_config* cfg, int32_t batch) {
 }
 
 size_t dflash2_prepared_size(const dflash2_config* c) {
-  if (!cfg_ok(c) || c->wfmt != 0) return 0;
+  if (!cfg_ok(c)) return 0;
   const size_t H = c->hidden, F = c->ffn, HQ = (size_t)c->n_q * kHeadDim, HKV = (size_t)c->n_kv * kHeadDim;
   const size_t per_layer = HQ * H + 2 * HKV * H + H * HQ + 2 * F * H + H * F;
-  return (H * c->n_taps * H + c->layers * per_layer) / kUnit * 144;
+  const size_t mats = H * c->n_taps * H + c->layers * per_layer;
+  const size_t mat_bytes = c->wfmt == 0 ? mats / kUnit * 144 : mats * 2;
+  const size_t dyn = (size_t)c->layers * 2 * (H / 4) * H * 2;
+  const size_t head = ((size_t)c->vocab + c->rank) * H * 2;
+  return mat_bytes + dyn + head;
 }
 
 int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src, void* dst, size_t dst_bytes,
@@ -279,35 +339,45 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
   if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
   if (!src || !out) return DFLASH2_ERR_ARG;
   dflash2_weights tmp = *src;
-  tmp.prepared = 0;
+  tmp.prepared = 1;
   int rc = check_weights(c, &tmp);
-  if (rc != DFLASH2_OK && rc != DFLASH2_ERR_LAYOUT) return rc;
+  if (rc != DFLASH2_OK) return rc;
+  if (!dst) return DFLASH2_ERR_ARG;
+  if (!aligned16(dst)) return DFLASH2_ERR_ALIGN;
+  if (dst_bytes < dflash2_prepared_size(c)) return DFLASH2_ERR_WORKSPACE;
   *out = *src;
   out->prepared = 1;
-  if (c->wfmt != 0) return DFLASH2_OK;
-  if (!dst || !aligned16(dst)) return dst ? DFLASH2_ERR_ALIGN : DFLASH2_ERR_ARG;
-  if (dst_bytes < dflash2_prepared_size(c)) return DFLASH2_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* d = (uint8_t*)dst;
   const int H = c->hidden, F = c->ffn, HQ = c->n_q * kHeadDim, HKV = c->n_kv * kHeadDim;
-  auto prep = [&](const void* w, int N, int K) -> const void* {
-    k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K);
+  auto prep = [&](const void* w, int N, int K, bool q4) -> const void* {
     const void* r = d;
-    d += (size_t)N * K / kUnit * 144;
+    if (q4) {
+      k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K);
+      d += (size_t)N * K / kUnit * 144;
+    } else {
+      k_bf16_prepare<<<dim3(K / 128, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K);
+      d += (size_t)N * K * 2;
+    }
     return r;
   };
-  out->fc = prep(src->fc, H, c->n_taps * H);
+  const bool q4 = c->wfmt == 0;
+  out->fc = prep(src->fc, H, c->n_taps * H, q4);
   for (int l = 0; l < c->layers; ++l) {
     const dflash2_layer_weights& S = src->layer[l];
     dflash2_layer_weights& O = out->layer[l];
-    O.wq = prep(S.wq, HQ, H);
-    O.wk = prep(S.wk, HKV, H);
-    O.wv = prep(S.wv, HKV, H);
-    O.wo = prep(S.wo, H, HQ);
-    O.wg = prep(S.wg, F, H);
-    O.wu = prep(S.wu, F, H);
-    O.wd = prep(S.wd, H, F);
+    O.wq = prep(S.wq, HQ, H, q4);
+    O.wk = prep(S.wk, HKV, H, q4);
+    O.wv = prep(S.wv, HKV, H, q4);
+    O.wo = prep(S.wo, H, HQ, q4);
+    O.wg = prep(S.wg, F, H, q4);
+    O.wu = prep(S.wu, F, H, q4);
+    O.wd = prep(S.wd, H, F, q4);
+    O.dc_w = (const uint16_t*)prep(S.dc_w, 2 * (H / 4), H, false);
   }
+  // the output head and the selector projection as one tile-contiguous [V + R, H] matrix
+  out->lm_head = (const uint16_t*)prep(src->lm_head, c->vocab, H, false);
+  out->sel_proj = (const uint16_t*)prep(src->sel_proj, c->rank, H, false);
   return fail(cudaGetLastError());
 }
 
@@ -346,21 +416,24 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   const int H = P.H, Mb = P.Mb;
   const size_t hbytes = (size_t)Mb * H * 4;
 
+  float* gbuf = at<float>(ws, P.off_g);
+  int* ctr = at<int>(ws, P.off_ctr);
   CK(cudaMemsetAsync(err, 0, 4, s));
+  CK(cudaMemsetAsync(ctr, 0, P.ctr_total * 4, s));
   // A1: block rows from the shared embedding table
-  k_embed<<<Mb, 256, 0, s>>>(in->block_tokens, w->embed, h, H, P.V, err);
-  CK(cudaGetLastError());
+  CK(launch_pdl(k_embed, dim3(Mb), dim3(256), 0, s, in->block_tokens, w->embed, h, H, P.V, err));
   if (dbg && dbg->hidden) CK(cudaMemcpyAsync(dbg->hidden, h, hbytes, cudaMemcpyDeviceToDevice, s));
 
-  // A2: context rows = RMSNorm_fc(W_fc . concat(taps))
+  // A2: context rows = RMSNorm_fc(W_fc . concat(taps)); fc output staged in xf
   {
     GemvSeg seg{(const uint8_t*)w->fc, H / 16, Mb, 0};
-    CK(launch_gemv(P.fc, P.q4, &seg, 1, in->taps, P.T * H, Mb, P.T * H, part, H, Mb, s));
+    Epi e;
+    e.mode = EPI_STORE;
+    e.y = xf;
+    e.ldy = H;
+    CK(launch_gemv(P.fc, P.q4, &seg, 1, false, in->taps, P.T * H, Mb, part, H, Mb, ctr, e, err, s));
     NormParams np{};
-    np.part = part;
-    np.nsplit = P.fc.ksplit;
-    np.split_stride = (long long)Mb * H;
-    np.ldp = H;
+    np.in = xf;
     np.w = w->fc_norm;
     np.eps = c->rms_eps;
     np.H = H;
@@ -393,19 +466,13 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
   ap.err = err;
 
-  const GemvPlan* prev_down = nullptr;
   for (int l = 0; l < c->layers; ++l) {
     const dflash2_layer_weights& L = w->layer[l];
-    // A3a: x = RMSNorm(h; ln1) (adding the previous layer's MLP output), g = W_dc x, y = dynconv(x, g)
+    int* lctr = ctr + P.ctr_fc + (size_t)l * P.ctr_per_layer;
+    // A3a: x = RMSNorm(h; ln1), g = W_dc x, y = dynconv(x, g)
     {
       NormParams np{};
-      np.h = h;
-      if (prev_down) {
-        np.part = part;
-        np.nsplit = prev_down->ksplit;
-        np.split_stride = (long long)Mb * H;
-        np.ldp = H;
-      }
+      np.in = h;
       np.w = L.ln1;
       np.eps = c->rms_eps;
       np.H = H;
@@ -418,46 +485,44 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       if (dbg && dbg->hidden && l > 0)
         CK(cudaMemcpyAsync(dbg->hidden + (size_t)l * Mb * H, h, hbytes, cudaMemcpyDeviceToDevice, s));
       GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
-      CK(launch_gemv(P.dc, false, &seg, 1, xb, H, Mb, H, part, H / 2, Mb, s));
-      k_dynconv<<<Mb, 256, 0, s>>>(xf, part, P.dc.ksplit, (long long)Mb * (H / 2), H / 2, L.dc_s0, L.dc_s1, H,
-                                   P.Bk, yb);
-      CK(cudaGetLastError());
+      Epi e;
+      e.mode = EPI_STORE;
+      e.y = gbuf;
+      e.ldy = H / 2;
+      CK(launch_gemv(P.dc, false, &seg, 1, false, xb, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err, s));
+      CK(launch_pdl(k_dynconv, dim3(Mb, (H / 4 + 255) / 256), dim3(256), 0, s, (const float*)xf, (const float*)gbuf,
+                    L.dc_s0, L.dc_s1, H, P.Bk, yb));
     }
-    // A3b: q from the block rows; k, v from block + context rows (stacked: read each matrix once)
+    // A3b+c: q from the block rows; k, v from block + context rows (stacked: each matrix read once);
+    // the last CTA of each head applies q/k RMSNorm + RoPE and appends context K/V to the cache
     {
       const int ldo = P.HQ + 2 * P.HKV;
       GemvSeg segs[3] = {{(const uint8_t*)L.wq, P.HQ / 16, Mb, 0},
                          {(const uint8_t*)L.wk, P.HKV / 16, 2 * Mb, P.HQ},
                          {(const uint8_t*)L.wv, P.HKV / 16, 2 * Mb, P.HQ + P.HKV}};
-      CK(launch_gemv(P.qkv, P.q4, segs, 3, yb, H, 2 * Mb, H, part, ldo, 2 * Mb, s));
-      // A3c: q/k norms, RoPE, context K/V appended to the paged cache
-      RopeParams rp{};
-      rp.part = part;
-      rp.nsplit = P.qkv.ksplit;
-      rp.split_stride = (long long)2 * Mb * ldo;
-      rp.ldp = ldo;
-      rp.qn = L.qn;
-      rp.kn = L.kn;
-      rp.eps = c->rms_eps;
-      rp.log2_theta = log2((double)c->rope_theta);
-      rp.Bk = P.Bk;
-      rp.nq = c->n_q;
-      rp.nkv = c->n_kv;
-      rp.Mb = Mb;
-      rp.seq_len = kv->seq_len;
-      rp.n_new = in->n_new;
-      rp.qb = qb;
-      rp.kb = kb;
-      rp.vb = vb;
-      rp.kc = kv->k[l];
-      rp.vc = kv->v[l];
-      rp.page_table = kv->page_table;
-      rp.max_pages = kv->max_pages;
-      rp.num_pages = kv->num_pages;
-      rp.err = err;
-      const int nslot = c->n_q + 2 * c->n_kv;
-      k_qk_rope_append<<<dim3((nslot + 3) / 4, 2 * Mb), 128, 0, s>>>(rp);
-      CK(cudaGetLastError());
+      Epi e;
+      e.mode = EPI_QKV;
+      QkvEpi& q = e.qkv;
+      q.qn = L.qn;
+      q.kn = L.kn;
+      q.eps = c->rms_eps;
+      q.log2_theta = log2((double)c->rope_theta);
+      q.Bk = P.Bk;
+      q.nq = c->n_q;
+      q.nkv = c->n_kv;
+      q.Mb = Mb;
+      q.seq_len = kv->seq_len;
+      q.n_new = in->n_new;
+      q.qb = qb;
+      q.kb = kb;
+      q.vb = vb;
+      q.kc = kv->k[l];
+      q.vc = kv->v[l];
+      q.page_table = kv->page_table;
+      q.max_pages = kv->max_pages;
+      q.num_pages = kv->num_pages;
+      q.err = err;
+      CK(launch_gemv(P.qkv, P.q4, segs, 3, false, yb, H, 2 * Mb, part, ldo, 2 * Mb, lctr + P.ctr_layer[1], e, err, s));
     }
     // A3d: sliding-window GQA attention over cache + block keys
     {
@@ -469,19 +534,18 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
         case 3: CK(launch_attn_t<3>(P, ap, s)); break;
         default: CK(launch_attn_t<4>(P, ap, s)); break;
       }
-      k_attn_combine<<<dim3((P.QV + 3) / 4, c->n_kv, batch), 128, 0, s>>>(ap, ob);
-      CK(cudaGetLastError());
+      CK(launch_pdl(k_attn_combine, dim3((P.QV + 3) / 4, c->n_kv, batch), dim3(128), 0, s, ap, ob));
     }
-    // A3e: h += W_o o (added by the next norm)
+    // A3e: h += W_o o (residual added by the last CTA of each column group)
     {
       GemvSeg seg{(const uint8_t*)L.wo, H / 16, Mb, 0};
-      CK(launch_gemv(P.o, P.q4, &seg, 1, ob, P.HQ, Mb, P.HQ, part, H, Mb, s));
+      Epi e;
+      e.mode = EPI_RESID;
+      e.y = h;
+      e.ldy = H;
+      CK(launch_gemv(P.o, P.q4, &seg, 1, false, ob, P.HQ, Mb, part, H, Mb, lctr + P.ctr_layer[2], e, err, s));
       NormParams np{};
-      np.h = h;
-      np.part = part;
-      np.nsplit = P.o.ksplit;
-      np.split_stride = (long long)Mb * H;
-      np.ldp = H;
+      np.in = h;
       np.w = L.ln2;
       np.eps = c->rms_eps;
       np.H = H;
@@ -491,27 +555,26 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       np.Bk = P.Bk;
       CK(launch_norm(np, Mb, s));
     }
-    // A3f: h += W_d (silu(W_g x2) * W_u x2)
+    // A3f: h += W_d (silu(W_g x2) * W_u x2); gate and up tiles paired per CTA so the SwiGLU is fused
     {
       GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wu, P.F / 16, Mb, P.F}};
-      CK(launch_gemv(P.gu, P.q4, segs, 2, xb, H, Mb, H, part, 2 * P.F, Mb, s));
-      const size_t n = (size_t)Mb * P.F;
-      const int blocks = (int)std::min<size_t>((n + 255) / 256, (size_t)P.nsm * 8);
-      k_silu_mul<<<blocks, 256, 0, s>>>(part, P.gu.ksplit, (long long)Mb * 2 * P.F, 2 * P.F, Mb, P.F, act);
-      CK(cudaGetLastError());
+      Epi e;
+      e.mode = EPI_SWIGLU;
+      e.act = act;
+      e.F = P.F;
+      CK(launch_gemv(P.gu, P.q4, segs, 2, true, xb, H, Mb, part, 2 * P.F, Mb, lctr + P.ctr_layer[3], e, err, s));
       GemvSeg seg{(const uint8_t*)L.wd, H / 16, Mb, 0};
-      CK(launch_gemv(P.dn, P.q4, &seg, 1, act, P.F, Mb, P.F, part, H, Mb, s));
-      prev_down = &P.dn;
+      Epi e2;
+      e2.mode = EPI_RESID;
+      e2.y = h;
+      e2.ldy = H;
+      CK(launch_gemv(P.dn, P.q4, &seg, 1, false, act, P.F, Mb, part, H, Mb, lctr + P.ctr_layer[4], e2, err, s));
     }
   }
-  // A4: final norm of the drafted rows 1..block-1 (adding the last MLP output)
+  // A4: final norm of the drafted rows 1..block-1
   {
     NormParams np{};
-    np.h = h;
-    np.part = part;
-    np.nsplit = P.dn.ksplit;
-    np.split_stride = (long long)Mb * H;
-    np.ldp = H;
+    np.in = h;
     np.w = w->final_norm;
     np.eps = c->rms_eps;
     np.H = H;
@@ -528,36 +591,46 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   // A5: LM head + streaming top-16 (+ selector projection)
   {
     if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
-    for (int pass = 0; pass < P.lm_passes; ++pass) {
-      LmParams lp{};
-      lp.W = w->lm_head;
-      lp.Ws = w->sel_proj;
+    if (P.lm_stream) {
+      static bool attr = false;
+      if (!attr) {
+        CK(cudaFuncSetAttribute(k_slmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit - kStaticSmem));
+        attr = true;
+      }
+      SLmParams lp{};
+      lp.W = (const uint8_t*)w->lm_head;
       lp.V = P.V;
       lp.R = P.R;
       lp.H = H;
-      lp.row_base = pass * P.lm_rows_per_pass;
-      lp.X = hn + (size_t)lp.row_base * H;
-      lp.rows = std::min(P.lm_rows_per_pass, P.lm_rows - lp.row_base);
-      lp.rows_total = P.lm_rows;
+      lp.X = hn;
+      lp.rows = P.lm_rows;
       lp.z = zbuf;
       lp.cand_val = at<float>(ws, P.off_cv);
       lp.cand_id = at<int32_t>(ws, P.off_ci);
-      if (P.lm_NT == 1) {
+      lp.err = err;
+      CK(launch_pdl(k_slmhead, dim3(P.lm_nparts), dim3(kStreamThreads), P.lm_smem, s, lp));
+    } else {
+      for (int pass = 0; pass < P.lm_passes; ++pass) {
+        LmParams lp{};
+        lp.W = (const uint8_t*)w->lm_head;
+        lp.V = P.V;
+        lp.R = P.R;
+        lp.H = H;
+        lp.row_base = pass * P.lm_rows_per_pass;
+        lp.X = hn + (size_t)lp.row_base * H;
+        lp.rows = std::min(P.lm_rows_per_pass, P.lm_rows - lp.row_base);
+        lp.rows_total = P.lm_rows;
+        lp.z = zbuf;
+        lp.cand_val = at<float>(ws, P.off_cv);
+        lp.cand_id = at<int32_t>(ws, P.off_ci);
         static bool attr = false;
         if (!attr) {
-          CK(cudaFuncSetAttribute(k_lmhead_topk<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-          attr = true;
-        }
-        k_lmhead_topk<1><<<P.lm_nparts, kWarps * 32, P.lm_smem, s>>>(lp);
-      } else {
-        static bool attr = false;
-        if (!attr) {
-          CK(cudaFuncSetAttribute(k_lmhead_topk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+          CK(cudaFuncSetAttribute(k_lmhead_topk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit - kStaticSmem));
           attr = true;
         }
         k_lmhead_topk<2><<<P.lm_nparts, kWarps * 32, P.lm_smem, s>>>(lp);
+        CK(cudaGetLastError());
       }
-      CK(cudaGetLastError());
     }
     if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
     if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
@@ -584,8 +657,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     sp.dbg_logit = dbg ? dbg->cand_logit : nullptr;
     sp.err = err;
     if (sp.dbg_cand && !sp.dbg_logit) sp.dbg_cand = nullptr;
-    k_selector<<<batch, 256, 0, s>>>(sp);
-    CK(cudaGetLastError());
+    CK(launch_pdl(k_selector, dim3(batch), dim3(256), 0, s, sp));
   }
   return DFLASH2_OK;
 }

@@ -1,8 +1,8 @@
-// Skinny GEMM Y[m][n] = sum_k W[n][k] X[m][k] for the block step's few rows
-// (8 block rows per request, 16 with the context rows), weights streamed once
-// from HBM.  Weights are the M side of a warp mma.sync m16n8k16 ("swap AB"): a
-// warp owns 16 output features and streams them along K; the activations,
-// staged once per CTA in shared memory, are the n = 8 side.
+// Per-warp compute pieces of the skinny GEMM Y[m][n] = sum_k W[n][k] X[m][k]
+// (the block step's few rows: 8 block rows per request, 16 with the context
+// rows).  Weights are the M side of a warp mma.sync m16n8k16 ("swap AB"): a
+// warp owns 16 output features; the activations, staged in shared memory, are
+// the n = 8 side.
 //
 // Q4_K (prepared layout, one 2304-byte record per 16-feature tile and
 // 256-wide super-block): 2048 bytes of codes arranged so that lane (g, t)
@@ -28,54 +28,22 @@ struct GemvSeg {
   int out_col;       // first output column
 };
 
-struct GemvParams {
-  GemvSeg seg[3];
-  int nseg;
-  const uint16_t* X;  // bf16 activations [rows][ldx]
-  int ldx;
-  int rows_stage;     // rows staged in shared memory (max over segments)
-  int K;              // reduction length (multiple of 256)
-  int units_per_split;
-  int kc_units;       // units staged per shared-memory chunk
-  float* out;         // fp32 partial sums [split][rows][ldo]
-  int ldo;
-  long long split_stride;
-  int m_group_rows;   // rows per grid.z group (64)
+enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3 };
+
+// Fused epilogue of the q|k|v projection: per-head q/k RMSNorm, RoPE at the absolute
+// position, block rows -> qb/kb/vb, context rows (t < n_new) -> the layer's paged cache.
+struct QkvEpi {
+  const uint16_t *qn, *kn;
+  float eps;
+  double log2_theta;
+  int Bk, nq, nkv, Mb;
+  const int32_t *seq_len, *n_new;
+  uint16_t *qb, *kb, *vb;  // [Mb][heads][128]
+  uint16_t *kc, *vc;       // [pages][nkv][16][128]
+  const int32_t* page_table;
+  int max_pages, num_pages;
+  int* err;
 };
-
-template <int NT>
-struct GemvSmem {
-  static constexpr int kRows = NT * 8;
-};
-
-DEVI int gemv_stride_bytes(int kc_units) { return kc_units * kUnit * 2 + 64; }
-
-// Stage X[:, k0 : k0+cu*256] into shared memory (rows >= rows_valid zero-filled)
-// and, for Q4_K, the 32-wide sums X_j.
-template <int NT, bool Q4>
-DEVI void gemv_stage(const GemvParams& p, const uint16_t* X, int rows_valid, int u0, int cu, uint8_t* Xs,
-                     float* Xsum, int stride) {
-  constexpr int R = NT * 8;
-  const int vec_per_row = cu * kUnit / 8;  // 16-byte vectors
-  for (int i = threadIdx.x; i < R * vec_per_row; i += blockDim.x) {
-    int r = i / vec_per_row, v = i % vec_per_row;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < rows_valid) val = *reinterpret_cast<const uint4*>(X + (size_t)r * p.ldx + (size_t)u0 * kUnit + v * 8);
-    *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = val;
-  }
-  if (Q4) {
-    __syncthreads();
-    const int nsub = cu * 8;
-    for (int i = threadIdx.x; i < R * nsub; i += blockDim.x) {
-      int r = i % R, j = i / R;
-      const uint16_t* row = reinterpret_cast<const uint16_t*>(Xs + r * stride) + j * 32;
-      float s = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < 32; ++k) s += bf2f(row[k]);
-      Xsum[j * R + r] = s;
-    }
-  }
-}
 
 template <int NT>
 DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8_t* Xs, int stride,
@@ -150,121 +118,52 @@ DEVI void bf16_step(const uint4 (&w)[8], const uint8_t* Xs, int stride, int kbyt
   }
 }
 
-template <int NT, bool Q4>
-__global__ void __launch_bounds__(kWarps * 32) k_gemv(GemvParams p) {
-  constexpr int R = NT * 8;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int stride = gemv_stride_bytes(p.kc_units);
-  uint8_t* Xs = smem;
-  float* Xsum = reinterpret_cast<float*>(smem + R * stride);
-  float2* coef = reinterpret_cast<float2*>(Xsum + (Q4 ? p.kc_units * 8 * R : 0)) + warp * 128;
-
-  // the warp's tile
-  int gt = blockIdx.x * kWarps + warp, si = -1, tile = 0;
-  {
-    int acc_t = 0;
-    for (int s = 0; s < p.nseg; ++s) {
-      if (gt < acc_t + p.seg[s].tiles) {
-        si = s;
-        tile = gt - acc_t;
-        break;
-      }
-      acc_t += p.seg[s].tiles;
+// q/k RMSNorm + RoPE of one head of one row (lane holds dims 2L, 2L+1, 64+2L, 65+2L), then store.
+DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float (&xin)[4], int lane) {
+  const bool ctx = row >= e.Mb;
+  const int rr = ctx ? row - e.Mb : row;
+  const int b = rr / e.Bk, t = rr % e.Bk;
+  const int L0 = e.seq_len[b], nn = e.n_new[b];
+  if (ctx && t >= nn) return;
+  float x[4] = {xin[0], xin[1], xin[2], xin[3]};
+  const int dims[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
+  if (kind < 2) {
+    const uint16_t* w = kind == 0 ? e.qn : e.kn;
+    const float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+    const float rs = rsqrtf(ss / kHeadDim + e.eps);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = x[i] * rs * bf2f(w[dims[i]]);
+    const long long pos = ctx ? (long long)L0 + t : (long long)L0 + nn + t;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      // angle pos * theta^(-2i/128) reduced modulo 2 pi in double, rotated in fp32
+      const double inv = exp2(-(2.0 * dims[i] / kHeadDim) * e.log2_theta);
+      double a = (double)pos * inv;
+      a -= 6.283185307179586 * rint(a / 6.283185307179586);
+      float sn, cs;
+      sincosf((float)a, &sn, &cs);
+      const float x0 = x[i], x1 = x[i + 2];
+      x[i] = x0 * cs - x1 * sn;
+      x[i + 2] = x1 * cs + x0 * sn;
     }
   }
-  const int mz = blockIdx.z * p.m_group_rows;
-  const uint16_t* X = p.X + (size_t)mz * p.ldx;
-  int stage_rows = p.rows_stage - mz;
-  stage_rows = stage_rows > R ? R : stage_rows;
-  int my_rows = 0;
-  const uint8_t* W = nullptr;
-  int out_col = 0;
-  if (si >= 0) {
-    my_rows = p.seg[si].rows - mz;
-    my_rows = my_rows > R ? R : (my_rows < 0 ? 0 : my_rows);
-    W = p.seg[si].W;
-    out_col = p.seg[si].out_col + tile * 16;
-  }
-  const int ntact = (my_rows + 7) >> 3;
-  const bool active = si >= 0 && ntact > 0;
-
-  const int nunits = p.K / kUnit;
-  const int u_lo = blockIdx.y * p.units_per_split;
-  int u_hi = u_lo + p.units_per_split;
-  u_hi = u_hi > nunits ? nunits : u_hi;
-
-  float acc[NT][4];
-#pragma unroll
-  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-
-  for (int c0 = u_lo; c0 < u_hi; c0 += p.kc_units) {
-    const int cu = (u_hi - c0) < p.kc_units ? (u_hi - c0) : p.kc_units;
-    __syncthreads();
-    gemv_stage<NT, Q4>(p, X, stage_rows, c0, cu, Xs, Xsum, stride);
-    __syncthreads();
-    if (!active) continue;
-    if (Q4) {
-      // stream this warp's tile: 2304 bytes per super-block, two super-blocks in flight
-      const uint8_t* base = W + ((size_t)tile * nunits) * kQ4Bytes;
-      uint4 qa[4], qb[4], sa, sb;
-      auto load = [&](uint4 (&q)[4], uint4& s, int u) {
-        const uint8_t* b = base + (size_t)u * kQ4Bytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = ldg_stream(b + (i * 32 + lane) * 16);
-        s = ldg_stream(b + 2048 + (lane >> 1) * 16);
-      };
-      load(qa, sa, c0);
-      if (c0 + 1 < c0 + cu) load(qb, sb, c0 + 1);
-      for (int u = c0; u < c0 + cu; u += 2) {
-        q4_unit<NT>(qa, sa, coef, Xs, stride, Xsum + (u - c0) * 8 * R, (u - c0) * 512, ntact, acc, lane);
-        if (u + 2 < c0 + cu) load(qa, sa, u + 2);
-        if (u + 1 < c0 + cu) {
-          q4_unit<NT>(qb, sb, coef, Xs, stride, Xsum + (u + 1 - c0) * 8 * R, (u + 1 - c0) * 512, ntact, acc, lane);
-          if (u + 3 < c0 + cu) load(qb, sb, u + 3);
-        }
-      }
-    } else {
-      const uint16_t* Wr = reinterpret_cast<const uint16_t*>(W) + (size_t)(tile * 16 + g) * p.K;
-      const size_t row8 = (size_t)8 * p.K;
-      const int s_lo = c0 * 2, s_hi = (c0 + cu) * 2;  // 128-wide steps
-      uint4 wa[8], wb[8];
-      auto load = [&](uint4 (&w)[8], int s) {
-        const uint16_t* b = Wr + (size_t)s * 128 + t * 8;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          w[2 * j] = ldg_stream(b + j * 32);
-          w[2 * j + 1] = ldg_stream(b + row8 + j * 32);
-        }
-      };
-      load(wa, s_lo);
-      if (s_lo + 1 < s_hi) load(wb, s_lo + 1);
-      for (int s = s_lo; s < s_hi; s += 2) {
-        bf16_step<NT>(wa, Xs, stride, (s - s_lo) * 256, ntact, acc, lane);
-        if (s + 2 < s_hi) load(wa, s + 2);
-        if (s + 1 < s_hi) {
-          bf16_step<NT>(wb, Xs, stride, (s + 1 - s_lo) * 256, ntact, acc, lane);
-          if (s + 3 < s_hi) load(wb, s + 3);
-        }
-      }
+  uint16_t* dst;
+  if (!ctx) {
+    uint16_t* base = kind == 0 ? e.qb : (kind == 1 ? e.kb : e.vb);
+    const int nh = kind == 0 ? e.nq : e.nkv;
+    dst = base + ((size_t)row * nh + head) * kHeadDim;
+  } else {
+    const long long pos = (long long)L0 + t;
+    const int lp = (int)(pos / kPage);
+    const int pg = lp < e.max_pages ? e.page_table[(size_t)b * e.max_pages + lp] : -1;
+    if (pg < 0 || pg >= e.num_pages) {
+      if (lane == 0) set_err(e.err, DFLASH2_DEV_PAGE);
+      return;
     }
+    dst = (kind == 1 ? e.kc : e.vc) + (((size_t)pg * e.nkv + head) * kPage + pos % kPage) * kHeadDim;
   }
-  if (!active) return;
-  float* out = p.out + (size_t)blockIdx.y * p.split_stride + (size_t)mz * p.ldo;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    if (nt < ntact) {
-      const int r0 = nt * 8 + 2 * t;
-      if (r0 < my_rows) {
-        out[(size_t)r0 * p.ldo + out_col + g] = acc[nt][0];
-        out[(size_t)r0 * p.ldo + out_col + g + 8] = acc[nt][2];
-      }
-      if (r0 + 1 < my_rows) {
-        out[(size_t)(r0 + 1) * p.ldo + out_col + g] = acc[nt][1];
-        out[(size_t)(r0 + 1) * p.ldo + out_col + g + 8] = acc[nt][3];
-      }
-    }
-  }
+  *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf2(x[0], x[1]);
+  *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf2(x[2], x[3]);
 }
 
 // Canonical Q4_K [N][K/256][144 B] -> prepared tiles [N/16][K/256][2304 B].

@@ -2,9 +2,10 @@
 // over the 248320-token vocabulary, 16 candidates kept per drafted position),
 // with the selector projection z = W_s h~ riding along as extra tiles.
 //
-// Persistent CTAs of 8 warps.  The final-normed rows (bf16, <= 16 per pass)
-// sit in shared memory; each warp streams 16-row vocabulary tiles of W_lm
-// (bf16, 16-byte streaming loads, two 128-wide K steps in flight) through
+// This kernel serves more than 8 drafted rows (16 per pass); up to 8 rows use
+// the TMA-ring engine k_slmhead.  Persistent CTAs of 8 warps.  The final-normed
+// rows (bf16) sit in shared memory; each warp streams prepared 16-row vocabulary
+// tiles (16-byte streaming loads, two 128-wide K steps in flight) through
 // mma.sync m16n8k16 with the vocabulary as the M side.  Logits never leave the
 // SM: after each tile every lane offers its values to a per-warp, per-row
 // sorted top-16 list in shared memory (threshold test first; insertions
@@ -17,7 +18,7 @@
 namespace dfl {
 
 struct LmParams {
-  const uint16_t *W, *Ws;  // lm_head [V][H], sel_proj [R][H]
+  const uint8_t* W;        // prepared bf16 tiles of [lm_head; sel_proj]
   int V, R, H;
   const uint16_t* X;       // final-normed rows of this pass [rows][H]
   int rows;                // rows in this pass (<= 8*NT)
@@ -71,17 +72,14 @@ __global__ void __launch_bounds__(kWarps * 32) k_lmhead_topk(LmParams p) {
   const int nit = ntiles * spt;
   const int ntact = (p.rows + 7) >> 3;
 
-  auto wrow = [&](int it) -> const uint16_t* {
-    const int tile = wg + (it / spt) * nw;
-    const uint16_t* base = tile < vt ? p.W + (size_t)tile * 16 * H : p.Ws + (size_t)(tile - vt) * 16 * H;
-    return base + (size_t)g * H + (size_t)(it % spt) * 128 + t * 8;
-  };
+  // prepared bf16 tiles of [lm_head; sel_proj]: 4096 bytes per (tile, 128-wide step)
   auto load = [&](uint4 (&w)[8], int it) {
-    const uint16_t* b = wrow(it);
+    const int tile = wg + (it / spt) * nw;
+    const uint8_t* b = p.W + ((size_t)tile * spt + it % spt) * 4096 + lane * 16;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      w[2 * j] = ldg_stream(b + j * 32);
-      w[2 * j + 1] = ldg_stream(b + (size_t)8 * H + j * 32);
+      w[2 * j] = ldg_stream(b + j * 1024);
+      w[2 * j + 1] = ldg_stream(b + j * 1024 + 512);
     }
   };
   float acc[NT][4];

@@ -1,6 +1,5 @@
-// Row-wise kernels of the block step: embedding gather, residual + RMSNorm,
-// two-tap dynamic convolution, SwiGLU combine, q/k norm + RoPE + cache append,
-// greedy acceptance.
+// Row-wise kernels of the block step: embedding gather, RMSNorm, two-tap
+// dynamic convolution, greedy acceptance.
 #pragma once
 #include "common.cuh"
 
@@ -9,6 +8,8 @@ namespace dfl {
 // h[r] = E[block_tokens[r]] (fp32); ids outside [0, V) flag DFLASH2_DEV_TOKEN and read row 0.
 __global__ void k_embed(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E, float* __restrict__ h,
                         int H, int V, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x;
   int id = tok[r];
   if (id < 0 || id >= V) {
@@ -20,11 +21,7 @@ __global__ void k_embed(const int32_t* __restrict__ tok, const uint16_t* __restr
 }
 
 struct NormParams {
-  float* h;            // residual stream [rows][H]; read (+ partials) and written back, or null
-  const float* part;   // partial sums [nsplit][rows][ldp] added to the row (from column pcol), or null
-  int nsplit;
-  long long split_stride;
-  int ldp, pcol;
+  const float* in;     // fp32 rows [rows][H]: the residual stream or the fc output
   const uint16_t* w;   // RMSNorm weight [H]
   float eps;
   int H;
@@ -36,24 +33,27 @@ struct NormParams {
   int Bk;
 };
 
-// One CTA per row: v = h + sum_s part_s; h = v; y = v / sqrt(mean v^2 + eps) * w.
+// One CTA per row: y = x / sqrt(mean x^2 + eps) * w, 16-byte loads.
 __global__ void __launch_bounds__(256) k_norm(NormParams p) {
-  extern __shared__ float vrow[];
+  extern __shared__ float4 vrow4[];
   __shared__ float red[8];
-  const int r = blockIdx.x, H = p.H;
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x, H4 = p.H / 4;
   const int b = r / p.Bk, t = r % p.Bk;
   if (p.mode == 1 && t >= p.n_new[b]) {
-    for (int c = threadIdx.x; c < H; c += blockDim.x) p.out_bf[(size_t)r * p.ldob + c] = 0;
+    for (int c = threadIdx.x; c < H4; c += blockDim.x)
+      *reinterpret_cast<uint2*>(p.out_bf + (size_t)r * p.ldob + 4 * c) = make_uint2(0, 0);
     return;
   }
+  if (p.mode == 2 && t == 0) return;
+  const float4* in = reinterpret_cast<const float4*>(p.in + (size_t)r * p.H);
   float ss = 0.f;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    float v = p.h ? p.h[(size_t)r * H + c] : 0.f;
-    if (p.part)
-      for (int s = 0; s < p.nsplit; ++s) v += p.part[s * p.split_stride + (size_t)r * p.ldp + p.pcol + c];
-    if (p.h) p.h[(size_t)r * H + c] = v;
-    vrow[c] = v;
-    ss += v * v;
+#pragma unroll 4
+  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+    const float4 v = in[c];
+    vrow4[c] = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -64,132 +64,37 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
     if (threadIdx.x == 0) red[0] = v;
   }
   __syncthreads();
-  const float rs = rsqrtf(red[0] / H + p.eps);
-  int orow = r;
-  if (p.mode == 2) {
-    if (t == 0) return;
-    orow = b * (p.Bk - 1) + t - 1;
-  }
-  for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    const float y = vrow[c] * rs * bf2f(p.w[c]);
-    if (p.out_bf) p.out_bf[(size_t)orow * p.ldob + c] = f2bf(y);
-    if (p.out_f) p.out_f[(size_t)r * H + c] = y;
+  const float rs = rsqrtf(red[0] / p.H + p.eps);
+  const int orow = p.mode == 2 ? b * (p.Bk - 1) + t - 1 : r;
+  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+    const float4 v = vrow4[c];
+    const uint2 wv = *reinterpret_cast<const uint2*>(p.w + 4 * c);
+    const float y0 = v.x * rs * bf2f(wv.x & 0xffff), y1 = v.y * rs * bf2f(wv.x >> 16);
+    const float y2 = v.z * rs * bf2f(wv.y & 0xffff), y3 = v.w * rs * bf2f(wv.y >> 16);
+    if (p.out_bf)
+      *reinterpret_cast<uint2*>(p.out_bf + (size_t)orow * p.ldob + 4 * c) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
+    if (p.out_f) reinterpret_cast<float4*>(p.out_f + (size_t)r * p.H)[c] = make_float4(y0, y1, y2, y3);
   }
 }
 
 // y_t[c] = (s0[c] + tanh g_t[c/4]) x_t[c] + (s1[c] + tanh g_t[H/4 + c/4]) x_{t-1}[c], x_{-1} = 0.
-__global__ void k_dynconv(const float* __restrict__ xf, const float* __restrict__ gpart, int nsplit,
-                          long long split_stride, int ldg, const uint16_t* __restrict__ s0,
+// Thread = 4 channels sharing one gate pair; grid (rows, H/1024).
+__global__ void k_dynconv(const float* __restrict__ xf, const float* __restrict__ g, const uint16_t* __restrict__ s0,
                           const uint16_t* __restrict__ s1, int H, int Bk, uint16_t* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x, t = r % Bk, G = H / 4;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    float g0 = 0.f, g1 = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-      g0 += gpart[s * split_stride + (size_t)r * ldg + c / 4];
-      g1 += gpart[s * split_stride + (size_t)r * ldg + G + c / 4];
-    }
-    const float xc = xf[(size_t)r * H + c];
-    const float xp = t > 0 ? xf[(size_t)(r - 1) * H + c] : 0.f;
-    y[(size_t)r * H + c] = f2bf((bf2f(s0[c]) + tanhf(g0)) * xc + (bf2f(s1[c]) + tanhf(g1)) * xp);
-  }
-}
-
-// act[r][f] = silu(sum_s gate) * sum_s up; gate in columns [0, F), up in [F, 2F) of the partials.
-__global__ void k_silu_mul(const float* __restrict__ part, int nsplit, long long split_stride, int ldp, int rows,
-                           int F, uint16_t* __restrict__ act) {
-  const size_t n = (size_t)rows * F;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const size_t r = i / F, f = i % F;
-    float g = 0.f, u = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-      g += part[s * split_stride + r * ldp + f];
-      u += part[s * split_stride + r * ldp + F + f];
-    }
-    act[i] = f2bf(g / (1.f + __expf(-g)) * u);
-  }
-}
-
-struct RopeParams {
-  const float* part;  // q|k|v partial sums [nsplit][2*Mb][ldp]: rows [0,Mb) block, [Mb,2Mb) context
-  int nsplit;
-  long long split_stride;
-  int ldp;
-  const uint16_t *qn, *kn;
-  float eps;
-  double log2_theta;
-  int Bk, nq, nkv, Mb;
-  const int32_t *seq_len, *n_new;
-  uint16_t *qb, *kb, *vb;   // [Mb][heads][128] bf16
-  uint16_t *kc, *vc;        // this layer's cache [pages][nkv][16][128]
-  const int32_t* page_table;
-  int max_pages, num_pages;
-  int* err;
-};
-
-// One warp per (row, head slot); slots: n_q query heads, n_kv key heads, n_kv value heads.
-// Lane L holds dims {2L, 2L+1, 64+2L, 65+2L}: the RoPE pairs (i, i+64) stay inside the lane.
-__global__ void k_qk_rope_append(RopeParams p) {
-  const int lane = threadIdx.x & 31;
-  const int slot = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int r = blockIdx.y;
-  const int nslot = p.nq + 2 * p.nkv;
-  if (slot >= nslot) return;
-  const bool ctx = r >= p.Mb;
-  const int rr = ctx ? r - p.Mb : r;
-  const int b = rr / p.Bk, t = rr % p.Bk;
-  const int L0 = p.seq_len[b], nn = p.n_new[b];
-  if (ctx && (slot < p.nq || t >= nn)) return;
-  int kind, head, col;
-  if (slot < p.nq) { kind = 0; head = slot; col = slot * kHeadDim; }
-  else if (slot < p.nq + p.nkv) { kind = 1; head = slot - p.nq; col = p.nq * kHeadDim + head * kHeadDim; }
-  else { kind = 2; head = slot - p.nq - p.nkv; col = (p.nq + p.nkv) * kHeadDim + head * kHeadDim; }
-  const int dims[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
-  float x[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float v = 0.f;
-    for (int s = 0; s < p.nsplit; ++s) v += p.part[s * p.split_stride + (size_t)r * p.ldp + col + dims[i]];
-    x[i] = v;
-  }
-  if (kind < 2) {
-    const uint16_t* w = kind == 0 ? p.qn : p.kn;
-    float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-    const float rs = rsqrtf(ss / kHeadDim + p.eps);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = x[i] * rs * bf2f(w[dims[i]]);
-    // RoPE (rotate-half) at the absolute position; angle reduced in double, rotated in fp32
-    const long long pos = ctx ? (long long)L0 + t : (long long)L0 + nn + t;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int fi = dims[i];  // 0..63
-      const double inv = exp2(-(2.0 * fi / kHeadDim) * p.log2_theta);
-      double a = (double)pos * inv;
-      a -= 6.283185307179586 * rint(a / 6.283185307179586);
-      float sn, cs;
-      sincosf((float)a, &sn, &cs);
-      const float x0 = x[i], x1 = x[i + 2];
-      x[i] = x0 * cs - x1 * sn;
-      x[i + 2] = x1 * cs + x0 * sn;
-    }
-  }
-  uint16_t* dst;
-  if (!ctx) {
-    uint16_t* base = kind == 0 ? p.qb : (kind == 1 ? p.kb : p.vb);
-    const int nh = kind == 0 ? p.nq : p.nkv;
-    dst = base + ((size_t)r * nh + head) * kHeadDim;
-  } else {
-    const long long pos = (long long)L0 + t;
-    const int lp = (int)(pos / kPage);
-    const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
-    if (pg < 0 || pg >= p.num_pages) {
-      if (lane == 0) set_err(p.err, DFLASH2_DEV_PAGE);
-      return;
-    }
-    uint16_t* base = kind == 1 ? p.kc : p.vc;
-    dst = base + (((size_t)pg * p.nkv + head) * kPage + pos % kPage) * kHeadDim;
-  }
-  *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf2(x[0], x[1]);
-  *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf2(x[2], x[3]);
+  const int q = blockIdx.y * blockDim.x + threadIdx.x;
+  if (q >= G) return;
+  const float a0 = tanhf(g[(size_t)r * (H / 2) + q]), a1 = tanhf(g[(size_t)r * (H / 2) + G + q]);
+  const float4 xc = reinterpret_cast<const float4*>(xf + (size_t)r * H)[q];
+  const float4 xp = t > 0 ? reinterpret_cast<const float4*>(xf + (size_t)(r - 1) * H)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint2 w0 = *reinterpret_cast<const uint2*>(s0 + 4 * q), w1 = *reinterpret_cast<const uint2*>(s1 + 4 * q);
+  const float y0 = (bf2f(w0.x & 0xffff) + a0) * xc.x + (bf2f(w1.x & 0xffff) + a1) * xp.x;
+  const float y1 = (bf2f(w0.x >> 16) + a0) * xc.y + (bf2f(w1.x >> 16) + a1) * xp.y;
+  const float y2 = (bf2f(w0.y & 0xffff) + a0) * xc.z + (bf2f(w1.y & 0xffff) + a1) * xp.z;
+  const float y3 = (bf2f(w0.y >> 16) + a0) * xc.w + (bf2f(w1.y >> 16) + a1) * xp.w;
+  *reinterpret_cast<uint2*>(y + (size_t)r * H + 4 * q) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
 }
 
 __global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,

@@ -36,6 +36,8 @@ struct SelParams {
 };
 
 __global__ void __launch_bounds__(256) k_selector(SelParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x, D = p.Bk - 1, R = p.R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int cand[kMaxD][kTopK];
@@ -49,50 +51,97 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
   float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big);
   float(*Wj)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big + kTopK * kMaxR);
 
-  // 1. merge the CTA lists of each drafted position into the final top-16
+  // 1. merge the CTA lists of each drafted position into the final top-16.
+  //    T0 = the best 16th entry over the lists bounds the final 16th from below, so only
+  //    list prefixes >= T0 survive (a few dozen entries); an exact selection runs on those.
+  constexpr int kCap = 512;
+  __shared__ int surv_n[kWarps];
   for (int t = warp; t < D; t += kWarps) {
     const int row = b * D + t;
-    float* lv = big + (warp * 32 + lane) * kTopK;
-    int* li = reinterpret_cast<int*>(big + kWarps * 32 * kTopK) + (warp * 32 + lane) * kTopK;
-    for (int k = 0; k < kTopK; ++k) { lv[k] = -INFINITY; li[k] = 0x7fffffff; }
+    float T0 = -INFINITY;
+    for (int part = lane; part < p.nparts; part += 32)
+      T0 = fmaxf(T0, p.cand_val[((size_t)part * p.rows_total + row) * kTopK + kTopK - 1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) T0 = fmaxf(T0, __shfl_xor_sync(0xffffffffu, T0, o));
+    float* sv = big + warp * kCap;
+    int* si = reinterpret_cast<int*>(big + kWarps * kCap) + warp * kCap;
+    if (lane == 0) surv_n[warp] = 0;
+    __syncwarp();
     for (int part = lane; part < p.nparts; part += 32) {
       const size_t o = ((size_t)part * p.rows_total + row) * kTopK;
       for (int k = 0; k < kTopK; ++k) {
         const float v = p.cand_val[o + k];
-        const int id = p.cand_id[o + k];
-        if (!better(v, id, lv[kTopK - 1], li[kTopK - 1])) break;  // list is sorted: the rest is worse
-        int pos = kTopK - 1;
-        while (pos > 0 && better(v, id, lv[pos - 1], li[pos - 1])) {
-          lv[pos] = lv[pos - 1];
-          li[pos] = li[pos - 1];
-          --pos;
+        if (!(v >= T0)) break;  // lists are sorted
+        const int slot = atomicAdd(&surv_n[warp], 1);
+        if (slot < kCap) {
+          sv[slot] = v;
+          si[slot] = p.cand_id[o + k];
         }
-        lv[pos] = v;
-        li[pos] = id;
       }
     }
     __syncwarp();
-    int head = 0;
-    for (int k = 0; k < kTopK; ++k) {
-      float bv = head < kTopK ? lv[head] : -INFINITY;
-      int bid = head < kTopK ? li[head] : 0x7fffffff;
-      int bl = lane;
+    const int n = surv_n[warp];
+    if (n <= kCap) {
+      for (int k = 0; k < kTopK; ++k) {
+        float bv = -INFINITY;
+        int bid = 0x7fffffff, bslot = -1;
+        for (int i = lane; i < n; i += 32)
+          if (better(sv[i], si[i], bv, bid)) { bv = sv[i]; bid = si[i]; bslot = i; }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-        const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
-        if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) {
-          bv = ov;
-          bid = oid;
-          bl = ol;
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+          const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
+          if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && os > bslot)) { bv = ov; bid = oid; bslot = os; }
+        }
+        if (lane == 0) {
+          cand[t][k] = bid;
+          cl[t][k] = bv;
+          if (bslot >= 0) { sv[bslot] = -INFINITY; si[bslot] = 0x7fffffff; }
+        }
+        __syncwarp();
+      }
+    } else {
+      // pathological ties: exact per-lane insertion merge of every list, then 16 rounds over lane heads
+      float* lv = big + (warp * 32 + lane) * kTopK;
+      int* li = reinterpret_cast<int*>(big + kWarps * 32 * kTopK) + (warp * 32 + lane) * kTopK;
+      __syncwarp();
+      for (int k = 0; k < kTopK; ++k) { lv[k] = -INFINITY; li[k] = 0x7fffffff; }
+      for (int part = lane; part < p.nparts; part += 32) {
+        const size_t o = ((size_t)part * p.rows_total + row) * kTopK;
+        for (int k = 0; k < kTopK; ++k) {
+          const float v = p.cand_val[o + k];
+          const int id = p.cand_id[o + k];
+          if (!better(v, id, lv[kTopK - 1], li[kTopK - 1])) break;
+          int pos = kTopK - 1;
+          while (pos > 0 && better(v, id, lv[pos - 1], li[pos - 1])) {
+            lv[pos] = lv[pos - 1];
+            li[pos] = li[pos - 1];
+            --pos;
+          }
+          lv[pos] = v;
+          li[pos] = id;
         }
       }
-      if (lane == 0) {
-        cand[t][k] = bid;
-        cl[t][k] = bv;
+      __syncwarp();
+      int head = 0;
+      for (int k = 0; k < kTopK; ++k) {
+        float bv = head < kTopK ? lv[head] : -INFINITY;
+        int bid = head < kTopK ? li[head] : 0x7fffffff;
+        int bl = lane;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+          const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+          if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) { bv = ov; bid = oid; bl = ol; }
+        }
+        if (lane == 0) {
+          cand[t][k] = bid;
+          cl[t][k] = bv;
+        }
+        if (lane == bl) ++head;
       }
-      if (lane == bl) ++head;
     }
   }
   __syncthreads();
@@ -120,10 +169,25 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
     }
     __syncthreads();
     const float* zt = p.z + (size_t)(b * D + t) * R;
-    for (int i = threadIdx.x; i < kTopK * R; i += blockDim.x) {
-      const int j = i / R, r = i % R;
-      Wj[j][r] = zt[r] * bf2f(p.cb_b[(size_t)cand[t][j] * R + r]);
-      if (j < nsrc) As[j][r] = bf2f(p.cb_a[(size_t)src_ids[j] * R + r]);
+    const int R8 = R / 8;
+    for (int i = threadIdx.x; i < kTopK * R8; i += blockDim.x) {
+      const int j = i / R8, r = (i % R8) * 8;
+      const uint4 bv = *reinterpret_cast<const uint4*>(p.cb_b + (size_t)cand[t][j] * R + r);
+      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        Wj[j][r + 2 * e] = zt[r + 2 * e] * bf2f(bw[e] & 0xffff);
+        Wj[j][r + 2 * e + 1] = zt[r + 2 * e + 1] * bf2f(bw[e] >> 16);
+      }
+      if (j < nsrc) {
+        const uint4 av = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
+        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          As[j][r + 2 * e] = bf2f(aw[e] & 0xffff);
+          As[j][r + 2 * e + 1] = bf2f(aw[e] >> 16);
+        }
+      }
     }
     __syncthreads();
     {

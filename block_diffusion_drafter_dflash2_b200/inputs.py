@@ -99,6 +99,9 @@ WORKLOADS: Dict[str, Workload] = {
     "full_bf16_b16": Workload("full_bf16_b16", FULL_BF16_B5, 16, 1, 262144, False, True, True,
                               "first_mismatch", 1005,
                               "bf16 layers, block 5, 16 requests, up to 262144 cached, 1% tap outliers"),
+    # profiling case: full layer shapes, one layer, a 65536-token vocabulary (about 1.7 GB on the device)
+    "prof_small": Workload("prof_small", dataclasses.replace(FULL, layers=1, vocab=65536), 1, 4096, 4096, False, False,
+                           False, "first_mismatch", 1006, "profiling case: 1 full-shape layer, vocab 65536"),
 }
 
 

@@ -39,11 +39,15 @@ def test_strerror_and_sizes(lib):
     d = inputs.TINY
     H, F, HQ, HKV = d.hidden, d.ffn, d.n_q * 128, d.n_kv * 128
     mats = H * d.n_taps * H + d.layers * (HQ * H + 2 * HKV * H + H * HQ + 3 * F * H)
-    assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144
+    dyn = d.layers * 2 * (H // 4) * H * 2
+    head = (d.vocab + d.rank) * H * 2
+    # prepared copy: the Q4_K matrices keep their size, bf16 matrices and the output head theirs
+    assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144 + dyn + head
     full = binding.config(inputs.FULL)
-    # the prepared Q4_K copy has exactly the canonical size (973.2 MB of Q4_K matrices for the full drafter)
-    assert abs(lib.dflash2_prepared_size(C.byref(full)) / 1e6 - 973.2) < 0.5
-    assert lib.dflash2_prepared_size(C.byref(binding.config(inputs.FULL_BF16_B5))) == 0
+    # full drafter: 973.2 MB of Q4_K matrices + 131.1 MB dynamic-convolution generators + 2545.5 MB head
+    assert abs(lib.dflash2_prepared_size(C.byref(full)) / 1e6 - (973.2 + 131.1 + 2545.5)) < 1.0
+    bf = binding.config(inputs.FULL_BF16_B5)
+    assert lib.dflash2_prepared_size(C.byref(bf)) > lib.dflash2_prepared_size(C.byref(full))
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 64), ("page_size", 32), ("topk", 8), ("block", 1),
