@@ -55,7 +55,7 @@ def launches_per_step(dims: Dims, batch: int) -> int:
     """Kernels the library launches for one draft step plus one acceptance."""
     rows = batch * (dims.block - 1)
     lm_passes = 1 if rows <= 8 else (rows + 15) // 16
-    # embed, fc GEMV, fc norm | per layer: norm, W_dc GEMV, dynconv, QKV GEMV, rope/append,
-    # attention, combine, W_o GEMV, norm, gate/up GEMV, SwiGLU, W_d GEMV | final norm,
-    # LM head passes, selector | acceptance
-    return 3 + 12 * dims.layers + 1 + lm_passes + 1 + 1
+    # embed, fc GEMV, fc norm | per layer: norm, W_dc GEMV, dynconv, QKV GEMV (+ norm/RoPE/append),
+    # attention, combine, W_o GEMV (+ residual), norm, gate/up GEMV (+ SwiGLU), W_d GEMV (+ residual) |
+    # final norm, LM head, selector | acceptance
+    return 3 + 10 * dims.layers + 1 + lm_passes + 1 + 1

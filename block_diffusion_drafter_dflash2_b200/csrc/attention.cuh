@@ -65,27 +65,53 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
-  // queries of this (request, kv head): vector qv = t*G + gi -> head kvh*G + gi of block row t
-  for (int i = threadIdx.x; i < MT * 16 * 16; i += blockDim.x) {
-    const int qv = i >> 4, v = i & 15;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (qv < nqv) {
-      const int t = qv / G, gi = qv % G;
-      val = *reinterpret_cast<const uint4*>(p.qb + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + v * 8);
+  // queries of this (request, kv head): vector qv = t*G + gi -> head kvh*G + gi of block row t.
+  // Every thread issues its 8 loads before any store (no load->store chains).
+  {
+    uint4 qv8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = threadIdx.x + k * blockDim.x, qv = i >> 4, v = i & 15;
+      qv8[k] = make_uint4(0, 0, 0, 0);
+      if (qv < nqv) {
+        const int t = qv / G, gi = qv % G;
+        qv8[k] = *reinterpret_cast<const uint4*>(p.qb + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + v * 8);
+      }
     }
-    *reinterpret_cast<uint4*>(Qs + qv * kAttnStride + v * 8) = val;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = threadIdx.x + k * blockDim.x, qv = i >> 4, v = i & 15;
+      *reinterpret_cast<uint4*>(Qs + qv * kAttnStride + v * 8) = qv8[k];
+    }
   }
   if (blk) {
+    // the block's own keys: Bk rows loaded (4 vectors per thread at most), the rest zero
     for (int i = threadIdx.x; i < kAttnKeys * 16; i += blockDim.x) {
       const int u = i >> 4, v = i & 15;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-      if (u < p.Bk) {
-        const size_t off = ((size_t)(b * p.Bk + u) * p.nkv + kvh) * kHeadDim + v * 8;
-        kv = *reinterpret_cast<const uint4*>(p.kb + off);
-        vv = *reinterpret_cast<const uint4*>(p.vb + off);
+      if (u >= p.Bk) {
+        *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(Vs + u * kAttnStride + v * 8) = make_uint4(0, 0, 0, 0);
       }
-      *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = kv;
-      *reinterpret_cast<uint4*>(Vs + u * kAttnStride + v * 8) = vv;
+    }
+    {
+      uint4 kv4[8], vv4[8];  // Bk <= 16 rows x 16 vectors over >= 32 threads
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = threadIdx.x + k * blockDim.x, u = i >> 4, v = i & 15;
+        if (u < p.Bk) {
+          const size_t off = ((size_t)(b * p.Bk + u) * p.nkv + kvh) * kHeadDim + v * 8;
+          kv4[k] = *reinterpret_cast<const uint4*>(p.kb + off);
+          vv4[k] = *reinterpret_cast<const uint4*>(p.vb + off);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = threadIdx.x + k * blockDim.x, u = i >> 4, v = i & 15;
+        if (u < p.Bk) {
+          *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = kv4[k];
+          *reinterpret_cast<uint4*>(Vs + u * kAttnStride + v * 8) = vv4[k];
+        }
+      }
     }
     if (threadIdx.x < kAttnKeys) row_ok[threadIdx.x] = threadIdx.x < p.Bk;
     __syncthreads();
@@ -264,7 +290,7 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
   L = warp_sum(L);
   __syncwarp();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+#pragma unroll 8
   for (int i = 0; i < nc; ++i) {
     const int c = i < nact ? i : p.NC;
     const float w = wsh[wi][i];

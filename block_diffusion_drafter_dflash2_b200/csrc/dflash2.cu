@@ -60,12 +60,11 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   g.W = (long long)g.groups * g.mgroups * g.U;
   g.P = (int)std::min<long long>(nsm, g.W);
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
-  const int ring = kConsumers * ns * slot;
-  const int per_unit = g.R * unitK * 2 + (q4 ? 8 * g.R * 4 : 0);
+  const int ring = ns * slot;
+  const int per_unit = g.R * unitK * 2;
   const int budget = kSmemLimit - kStaticSmem - ring - (q4 ? kConsumers * 1024 : 0) - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) +
-           (q4 ? (size_t)g.kc_units * 8 * g.R * 4 + kConsumers * 1024 : 0);
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + (q4 ? kConsumers * 1024 : 0);
   return g;
 }
 
@@ -115,7 +114,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   if (p.lm_stream) {
     p.lm_NT = 1;
     p.lm_rows_per_pass = 8;
-    p.lm_smem = (size_t)kConsumers * Ring<false>::kNS * Ring<false>::kSlot + (size_t)8 * (p.H * 2 + 64) +
+    p.lm_smem = (size_t)Ring<false>::kNS * Ring<false>::kSlot + (size_t)8 * (p.H * 2 + 64) +
                 (size_t)kConsumers * 8 * kTopK * 8;
     p.lm_nparts = std::min(p.nsm, (lm_tiles + kConsumers - 1) / kConsumers);
   } else {
@@ -330,8 +329,8 @@ size_t dflash2_prepared_size(const dflash2_config* c) {
   const size_t mats = H * c->n_taps * H + c->layers * per_layer;
   const size_t mat_bytes = c->wfmt == 0 ? mats / kUnit * 144 : mats * 2;
   const size_t dyn = (size_t)c->layers * 2 * (H / 4) * H * 2;
-  const size_t head = ((size_t)c->vocab + c->rank) * H * 2;
-  return mat_bytes + dyn + head;
+  const size_t head_groups = ((size_t)(c->vocab + c->rank) / 16 + 7) / 8;
+  return mat_bytes + dyn + head_groups * 8 * 16 * H * 2;
 }
 
 int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src, void* dst, size_t dst_bytes,
@@ -350,15 +349,18 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* d = (uint8_t*)dst;
   const int H = c->hidden, F = c->ffn, HQ = c->n_q * kHeadDim, HKV = c->n_kv * kHeadDim;
+  // one matrix (or a set sharing one buffer) into group-interleaved records at d
+  auto place = [&](const void* w, int N, int K, bool q4, PrepPlace pl) {
+    if (q4)
+      k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K, pl);
+    else
+      k_bf16_prepare<<<dim3(K / 128, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K, pl);
+  };
+  auto bytes = [&](int N, int K, bool q4) { return q4 ? (size_t)N * K / kUnit * 144 : (size_t)N * K * 2; };
   auto prep = [&](const void* w, int N, int K, bool q4) -> const void* {
     const void* r = d;
-    if (q4) {
-      k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K);
-      d += (size_t)N * K / kUnit * 144;
-    } else {
-      k_bf16_prepare<<<dim3(K / 128, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K);
-      d += (size_t)N * K * 2;
-    }
+    place(w, N, K, q4, PrepPlace{0, 8, 0});
+    d += bytes(N, K, q4);
     return r;
   };
   const bool q4 = c->wfmt == 0;
@@ -370,14 +372,21 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
     O.wk = prep(S.wk, HKV, H, q4);
     O.wv = prep(S.wv, HKV, H, q4);
     O.wo = prep(S.wo, H, HQ, q4);
-    O.wg = prep(S.wg, F, H, q4);
-    O.wu = prep(S.wu, F, H, q4);
+    // gate and up interleaved 4 + 4 tiles per group; wu aliases the same buffer
+    place(S.wg, F, H, q4, PrepPlace{0, 4, 0});
+    place(S.wu, F, H, q4, PrepPlace{0, 4, 4});
+    O.wg = O.wu = d;
+    d += 2 * bytes(F, H, q4);
     O.wd = prep(S.wd, H, F, q4);
     O.dc_w = (const uint16_t*)prep(S.dc_w, 2 * (H / 4), H, false);
   }
-  // the output head and the selector projection as one tile-contiguous [V + R, H] matrix
-  out->lm_head = (const uint16_t*)prep(src->lm_head, c->vocab, H, false);
-  out->sel_proj = (const uint16_t*)prep(src->sel_proj, c->rank, H, false);
+  // the output head and the selector projection as one [V + R, H] matrix, padded to whole groups
+  const size_t groups = ((size_t)(c->vocab + c->rank) / 16 + 7) / 8, gbytes = (size_t)8 * 16 * H * 2;
+  CK(cudaMemsetAsync(d + (groups - 1) * gbytes, 0, gbytes, s));
+  place(src->lm_head, c->vocab, H, false, PrepPlace{0, 8, 0});
+  place(src->sel_proj, c->rank, H, false, PrepPlace{c->vocab / 16, 8, 0});
+  out->lm_head = (const uint16_t*)d;
+  out->sel_proj = (const uint16_t*)(d + (size_t)c->vocab / 16 * 16 * H * 2);
   return fail(cudaGetLastError());
 }
 
@@ -557,7 +566,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     }
     // A3f: h += W_d (silu(W_g x2) * W_u x2); gate and up tiles paired per CTA so the SwiGLU is fused
     {
-      GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wu, P.F / 16, Mb, P.F}};
+      GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wg, P.F / 16, Mb, P.F}};
       Epi e;
       e.mode = EPI_SWIGLU;
       e.act = act;

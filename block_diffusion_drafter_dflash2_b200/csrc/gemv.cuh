@@ -13,7 +13,8 @@
 // offset and the sub-block scale/min are applied per 32-wide sub-block on the
 // fp32 accumulators:
 //   y += (d*sc_j) * S_j - (dmin*m_j + 128*d*sc_j) * X_j,
-//   S_j = sum_k (128+q_k) x_k,  X_j = sum_k x_k  (bf16 x as fed to the mma).
+//   S_j = sum_k (128+q_k) x_k,  X_j = sum_k x_k  (bf16 x as fed to the mma; X_j comes
+//   from a second mma with an all-ones A operand).
 // The logical k order inside an mma is permuted identically on A and B, which
 // leaves the dot product unchanged.
 #pragma once
@@ -46,10 +47,11 @@ struct QkvEpi {
 };
 
 template <int NT>
-DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8_t* Xs, int stride,
-                  const float* Xsum_u, int kbyte, int ntact, float (&acc)[NT][4], int lane) {
-  constexpr int R = NT * 8;
+DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8_t* Xs, int stride, int kbyte,
+                  int ntact, float (&acc)[NT][4], int lane) {
   const int g = lane >> 2, t = lane & 3;
+  // A = 1.0 in every slot: the mma then yields X_j = sum_k x_k (bf16 x, fp32 accumulate) per row
+  const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
   {
     // lane decodes (d*sc_j, dmin*m_j + 128*d*sc_j) of feature lane/2, sub-blocks 4*(lane&1) .. +3
     const int f = lane >> 1, jb = (lane & 1) * 4;
@@ -84,14 +86,15 @@ DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8
     for (int nt = 0; nt < NT; ++nt) {
       if (nt < ntact) {
         const uint4 bx = *reinterpret_cast<const uint4*>(Xs + (nt * 8 + g) * stride + kbyte + j * 64 + t * 16);
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, xs[4] = {0.f, 0.f, 0.f, 0.f};
         mma16816(s, a0, bx.x, bx.y);
         mma16816(s, a1, bx.z, bx.w);
-        const float2 xs = *reinterpret_cast<const float2*>(Xsum_u + j * R + nt * 8 + 2 * t);
-        acc[nt][0] = fmaf(cg.x, s[0], fmaf(-cg.y, xs.x, acc[nt][0]));
-        acc[nt][1] = fmaf(cg.x, s[1], fmaf(-cg.y, xs.y, acc[nt][1]));
-        acc[nt][2] = fmaf(ch.x, s[2], fmaf(-ch.y, xs.x, acc[nt][2]));
-        acc[nt][3] = fmaf(ch.x, s[3], fmaf(-ch.y, xs.y, acc[nt][3]));
+        mma16816(xs, ones, bx.x, bx.y);
+        mma16816(xs, ones, bx.z, bx.w);
+        acc[nt][0] = fmaf(cg.x, s[0], fmaf(-cg.y, xs[0], acc[nt][0]));
+        acc[nt][1] = fmaf(cg.x, s[1], fmaf(-cg.y, xs[1], acc[nt][1]));
+        acc[nt][2] = fmaf(ch.x, s[2], fmaf(-ch.y, xs[2], acc[nt][2]));
+        acc[nt][3] = fmaf(ch.x, s[3], fmaf(-ch.y, xs[3], acc[nt][3]));
       }
     }
   }
@@ -166,8 +169,19 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
   *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf2(x[2], x[3]);
 }
 
-// Canonical Q4_K [N][K/256][144 B] -> prepared tiles [N/16][K/256][2304 B].
-__global__ void k_q4k_prepare(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K) {
+// Placement of 16-row tile T of a matrix in a group-interleaved prepared buffer: tile T' = T + tile0
+// sits in group T' / per_grp at slot slot0 + T' % per_grp; a group record of one K unit holds its 8
+// slots back to back, so one bulk copy brings a whole group's unit.
+struct PrepPlace {
+  int tile0, per_grp, slot0;
+};
+DEVI size_t prep_offset(const PrepPlace& pl, int T, int s, int U, int unit_bytes) {
+  const int tt = T + pl.tile0, grp = tt / pl.per_grp, slot = pl.slot0 + tt % pl.per_grp;
+  return (((size_t)grp * U + s) * 8 + slot) * unit_bytes;
+}
+
+// Canonical Q4_K [N][K/256][144 B] -> prepared tiles (group records of 8 x 2304 B per super-block).
+__global__ void k_q4k_prepare(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K, PrepPlace pl) {
   const int nsb = K / kUnit, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
   const uint8_t* bg = src + ((size_t)(T * 16 + g) * nsb + s) * 144;
@@ -186,13 +200,29 @@ __global__ void k_q4k_prepare(const uint8_t* __restrict__ src, uint8_t* __restri
       w[j][h] = q(bg, e) | (q(bh, e) << 4) | (q(bg, e + 2) << 8) | (q(bh, e + 2) << 12) | (q(bg, e + 1) << 16) |
                 (q(bh, e + 1) << 20) | (q(bg, e + 3) << 24) | (q(bh, e + 3) << 28);
     }
-  uint8_t* out = dst + ((size_t)T * nsb + s) * kQ4Bytes;
+  uint8_t* out = dst + prep_offset(pl, T, s, nsb, kQ4Bytes);
 #pragma unroll
   for (int p = 0; p < 4; ++p)
     reinterpret_cast<uint4*>(out)[p * 32 + lane] = make_uint4(w[2 * p][0], w[2 * p][1], w[2 * p + 1][0], w[2 * p + 1][1]);
   if (lane < 16) {
     const uint8_t* b = src + ((size_t)(T * 16 + lane) * nsb + s) * 144;
     for (int i = 0; i < 16; ++i) out[2048 + lane * 16 + i] = b[i];
+  }
+}
+
+// Canonical bf16 [N][K] -> prepared tiles (group records of 8 x 4096 B per 128-wide K step): for each
+// 32-wide sub-block j, 512 bytes of lane (g, t)'s W[row g][32j + 8t ..], then 512 bytes for row g + 8.
+__global__ void k_bf16_prepare(const uint16_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K,
+                               PrepPlace pl) {
+  const int S = K / 128, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x, g = lane >> 2, t = lane & 3;
+  uint8_t* out = dst + prep_offset(pl, T, s, S, 4096);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const size_t k = (size_t)s * 128 + j * 32 + t * 8;
+    *reinterpret_cast<uint4*>(out + j * 1024 + lane * 16) =
+        *reinterpret_cast<const uint4*>(src + (size_t)(T * 16 + g) * K + k);
+    *reinterpret_cast<uint4*>(out + j * 1024 + 512 + lane * 16) =
+        *reinterpret_cast<const uint4*>(src + (size_t)(T * 16 + g + 8) * K + k);
   }
 }
 

@@ -16,8 +16,13 @@ __global__ void k_embed(const int32_t* __restrict__ tok, const uint16_t* __restr
     if (threadIdx.x == 0) set_err(err, DFLASH2_DEV_TOKEN);
     id = 0;
   }
-  const uint16_t* e = E + (size_t)id * H;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) h[(size_t)r * H + c] = bf2f(e[c]);
+  const uint4* e = reinterpret_cast<const uint4*>(E + (size_t)id * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = e[c];
+    float4* o = reinterpret_cast<float4*>(h + (size_t)r * H + c * 8);
+    o[0] = make_float4(bf2f(v.x & 0xffff), bf2f(v.x >> 16), bf2f(v.y & 0xffff), bf2f(v.y >> 16));
+    o[1] = make_float4(bf2f(v.z & 0xffff), bf2f(v.z >> 16), bf2f(v.w & 0xffff), bf2f(v.w >> 16));
+  }
 }
 
 struct NormParams {
@@ -49,7 +54,7 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
   if (p.mode == 2 && t == 0) return;
   const float4* in = reinterpret_cast<const float4*>(p.in + (size_t)r * p.H);
   float ss = 0.f;
-#pragma unroll 4
+#pragma unroll 8
   for (int c = threadIdx.x; c < H4; c += blockDim.x) {
     const float4 v = in[c];
     vrow4[c] = v;
@@ -66,6 +71,7 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
   __syncthreads();
   const float rs = rsqrtf(red[0] / p.H + p.eps);
   const int orow = p.mode == 2 ? b * (p.Bk - 1) + t - 1 : r;
+#pragma unroll 8
   for (int c = threadIdx.x; c < H4; c += blockDim.x) {
     const float4 v = vrow4[c];
     const uint2 wv = *reinterpret_cast<const uint2*>(p.w + 4 * c);

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
   // phase 1: per-lane merge lists [warps][32][16] (values, then ids); phase 2: codebook rows
   __shared__ __align__(16) float big[2 * kTopK * kMaxR];
   float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big);
-  float(*Wj)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big + kTopK * kMaxR);
+  float(*Wj)[kTopK] = reinterpret_cast<float(*)[kTopK]>(big + kTopK * kMaxR);  // [r][j]: conflict-free reads
 
   // 1. merge the CTA lists of each drafted position into the final top-16.
   //    T0 = the best 16th entry over the lists bounds the final 16th from below, so only
@@ -58,11 +58,35 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
   __shared__ int surv_n[kWarps];
   for (int t = warp; t < D; t += kWarps) {
     const int row = b * D + t;
+    // T0 = max(best 16th entry of a list, 16th best list head): either way at least 16
+    // entries are >= T0, so the final 16 are all >= T0
     float T0 = -INFINITY;
-    for (int part = lane; part < p.nparts; part += 32)
-      T0 = fmaxf(T0, p.cand_val[((size_t)part * p.rows_total + row) * kTopK + kTopK - 1]);
+    float heads[8];
+    int nh = 0;
+    for (int part = lane; part < p.nparts; part += 32) {
+      const size_t o = ((size_t)part * p.rows_total + row) * kTopK;
+      T0 = fmaxf(T0, p.cand_val[o + kTopK - 1]);
+      if (nh < 8) heads[nh++] = p.cand_val[o];
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) T0 = fmaxf(T0, __shfl_xor_sync(0xffffffffu, T0, o));
+    if (p.nparts <= 8 * 32) {
+      // 16th largest head: 16 rounds of a warp max, removing one occurrence each time
+      float hb = -INFINITY;
+      for (int k = 0; k < kTopK; ++k) {
+        float lb = -INFINITY;
+        int li_ = -1;
+        for (int i = 0; i < nh; ++i)
+          if (heads[i] > lb) { lb = heads[i]; li_ = i; }
+        float m = lb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const unsigned who = __ballot_sync(0xffffffffu, li_ >= 0 && lb == m);
+        if (who && lane == __ffs(who) - 1) heads[li_] = -INFINITY;
+        hb = m;
+      }
+      T0 = fmaxf(T0, hb);
+    }
     float* sv = big + warp * kCap;
     int* si = reinterpret_cast<int*>(big + kWarps * kCap) + warp * kCap;
     if (lane == 0) surv_n[warp] = 0;
@@ -176,8 +200,8 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
       const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        Wj[j][r + 2 * e] = zt[r + 2 * e] * bf2f(bw[e] & 0xffff);
-        Wj[j][r + 2 * e + 1] = zt[r + 2 * e + 1] * bf2f(bw[e] >> 16);
+        Wj[r + 2 * e][j] = zt[r + 2 * e] * bf2f(bw[e] & 0xffff);
+        Wj[r + 2 * e + 1][j] = zt[r + 2 * e + 1] * bf2f(bw[e] >> 16);
       }
       if (j < nsrc) {
         const uint4 av = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
@@ -194,7 +218,7 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
       const int i = threadIdx.x / kTopK, j = threadIdx.x % kTopK;
       if (i < nsrc) {
         float s = 0.f;
-        for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[j][r], s);
+        for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[r][j], s);
         tau[i][j] = s;
       }
     }

@@ -1,23 +1,27 @@
 // Weight-streaming engine of the block step (all of its matrices are read once
 // per step, so the step is bound by HBM bandwidth).
 //
-// One CTA per SM, warp-specialised: a producer warp streams tile-contiguous
-// weight chunks (prepared layouts, below) into a per-warp ring of shared-memory
-// slots with 1-D bulk copies on the TMA engine, completion counted on mbarriers;
-// 8 consumer warps each own one 16-feature tile at a time and run warp
-// mma.sync m16n8k16 with the weights as the M side and the step's few
-// activation rows (staged once in shared memory) as the N side.  The producer
-// starts before the activations exist (the weights do not depend on the
-// previous kernel), so with programmatic dependent launch the weight stream
-// overlaps the previous kernel's tail and this kernel's own prologue.
+// One CTA per SM, warp-specialised: one producer thread streams weight
+// records into a ring of shared-memory slots with 1-D bulk copies on the TMA
+// engine (completion counted on mbarriers); 8 consumer warps each own one
+// 16-feature tile of the current 8-tile column group and run warp mma.sync
+// m16n8k16 with the weights as the M side and the step's few activation rows
+// (brought into shared memory by bulk copies as well) as the N side.  The
+// producer starts before the activations exist (the weights do not depend on
+// the previous kernel), so with programmatic dependent launch the weight
+// stream overlaps the previous kernel's tail and this kernel's prologue.
 //
-// Prepared layouts (made by dflash2_prepare_weights, values unchanged):
-//  * Q4_K: per 16-row tile and 256-wide super-block a 2304-byte record: 2048
-//    bytes of 4-bit codes in mma A-fragment order, then the 16 canonical 16-byte
-//    scale records of the tile's rows (see q4_unit).
-//  * bf16: per 16-row tile and 128-wide K step a 4096-byte record: for each
-//    32-wide sub-block j, 512 bytes holding lane L = (g, t)'s 8 values
-//    W[row g][32j + 8t ..] then 512 bytes for row g + 8.
+// Prepared layouts (made by dflash2_prepare_weights, values unchanged): the
+// 8 tiles of a column group are interleaved per K unit, so one bulk copy moves
+// a whole group's unit (18 KB of Q4_K, 32 KB of bf16):
+//  * Q4_K: per tile and 256-wide super-block a 2304-byte record: 2048 bytes of
+//    4-bit codes in mma A-fragment order, then the 16 canonical 16-byte scale
+//    records of the tile's rows (see q4_unit).
+//  * bf16: per tile and 128-wide K step a 4096-byte record: for each 32-wide
+//    sub-block j, 512 bytes holding lane L = (g, t)'s 8 values W[row g][32j + 8t ..]
+//    then 512 bytes for row g + 8.
+//  * gate/up of the MLP are interleaved 4 + 4 tiles per group, so one CTA holds
+//    both halves of the SwiGLU for 64 features.
 //
 // Work split of the GEMV (stream-K): the (column group, K unit) plane is cut
 // into gridDim.x equal contiguous ranges, so every SM streams the same number
@@ -27,6 +31,7 @@
 // order — deterministic — and runs the epilogue.
 #pragma once
 #include "gemv.cuh"
+#include "lmhead.cuh"
 
 namespace dfl {
 
@@ -37,11 +42,11 @@ template <bool Q4>
 struct Ring;
 template <>
 struct Ring<true> {
-  static constexpr int kSlot = kQ4Bytes, kNS = 6, kUnitK = 256;
+  static constexpr int kUnitBytes = kQ4Bytes, kSlot = 8 * kQ4Bytes, kNS = 6, kUnitK = 256;
 };
 template <>
 struct Ring<false> {
-  static constexpr int kSlot = 4096, kNS = 4, kUnitK = 128;
+  static constexpr int kUnitBytes = 4096, kSlot = 8 * 4096, kNS = 4, kUnitK = 128;
 };
 
 DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory"); }
@@ -50,7 +55,7 @@ DEVI void mbar_arrive(uint64_t* bar) {
 }
 
 struct SGemvParams {
-  GemvSeg seg[3];
+  GemvSeg seg[3];     // output column ranges; weights of a paired launch live in seg[0].W
   int nseg;
   int paired;
   const uint16_t* X;  // bf16 activations [rows][ldx]
@@ -76,12 +81,11 @@ struct SGemvParams {
 // Owner CTA of global position x when [0, W) is cut into P ranges [c*W/P, (c+1)*W/P).
 DEVI long long sk_owner(long long x, long long W, long long P) { return ((x + 1) * P + W - 1) / W - 1; }
 
-// Tile of consumer warp w in column group grp; -1 when idle.
+// Tile (output columns) of consumer warp w in column group grp.
 DEVI int sk_tile(const SGemvParams& p, int grp, int w, int& si) {
   if (p.paired) {
     si = w >> 2;
-    const int tile = grp * 4 + (w & 3);
-    return tile < p.seg[si].tiles ? tile : -1;
+    return grp * 4 + (w & 3);
   }
   int gt = grp * kConsumers + w, acc = 0;
   for (int s = 0; s < p.nseg; ++s) {
@@ -91,12 +95,24 @@ DEVI int sk_tile(const SGemvParams& p, int grp, int w, int& si) {
     }
     acc += p.seg[s].tiles;
   }
-  si = -1;
+  si = 0;
   return -1;
 }
 
+// Weight records of column group grp (one group record per K unit).
+template <bool Q4>
+DEVI const uint8_t* sk_group_src(const SGemvParams& p, int grp) {
+  if (p.paired) return p.seg[0].W + (size_t)grp * p.U * Ring<Q4>::kSlot;
+  int acc = 0;
+  for (int s = 0; s < p.nseg; ++s) {
+    const int ng = p.seg[s].tiles / 8;
+    if (grp < acc + ng) return p.seg[s].W + (size_t)(grp - acc) * p.U * Ring<Q4>::kSlot;
+    acc += ng;
+  }
+  return nullptr;
+}
+
 DEVI int sk_rows(const SGemvParams& p, int si, int mz, int R) {
-  if (si < 0) return 0;
   int r = p.seg[si].rows - mz;
   return r > R ? R : (r < 0 ? 0 : r);
 }
@@ -116,18 +132,15 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
     const int rows = sk_rows(p, 0, mz, R);
     for (int i = tid; i < rows * 64; i += nthr) {
       const int r = i >> 6, f = f0 + (i & 63);
-      if (f >= p.F) continue;
       const float gv = sum_pieces(p, npieces, mz + r, p.seg[0].out_col + f);
       const float uv = sum_pieces(p, npieces, mz + r, p.seg[1].out_col + f);
       p.act[(size_t)(mz + r) * p.F + f] = f2bf(gv / (1.f + __expf(-gv)) * uv);
     }
     return;
   }
-  int si = -1;
+  int si = 0;
   const int tile0 = sk_tile(p, grp, 0, si);
   if (tile0 < 0) return;
-  int ncol = (p.seg[si].tiles - tile0) * 16;
-  ncol = ncol > 128 ? 128 : ncol;
   const int col0 = p.seg[si].out_col + tile0 * 16;
   const int rows = sk_rows(p, si, mz, R);
   if (p.epi == EPI_QKV) {
@@ -141,8 +154,8 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
     }
     return;
   }
-  for (int i = tid; i < rows * ncol; i += nthr) {
-    const int r = i / ncol, c = col0 + i % ncol;
+  for (int i = tid; i < rows * 128; i += nthr) {
+    const int r = i >> 7, c = col0 + (i & 127);
     const float v = sum_pieces(p, npieces, mz + r, c);
     float* y = p.y + (size_t)(mz + r) * p.ldy + c;
     if (p.epi == EPI_RESID) *y += v;
@@ -150,27 +163,45 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   }
 }
 
+// Bring rows [0, nrows) of an X chunk (row stride ldx elements, `bytes` per row) into Xs (row
+// stride `stride` bytes) with bulk copies on xbar; rows [nrows, R) are zeroed.  Consumer threads.
+DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes, uint8_t* Xs, int stride,
+                        uint64_t* xbar, uint32_t& xph, int* err) {
+  consumers_sync();  // every consumer is done with the previous chunk
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(xbar, (uint32_t)(nrows * bytes));
+    for (int r = 0; r < nrows; ++r) bulk_g2s(Xs + r * stride, X + (size_t)r * ldx, bytes, xbar);
+  }
+  for (int i = threadIdx.x; i < (R - nrows) * (bytes / 16); i += kConsumers * 32) {
+    const int r = nrows + i / (bytes / 16), v = i % (bytes / 16);
+    *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = make_uint4(0, 0, 0, 0);
+  }
+  consumers_sync();
+  if (!mbar_wait_bounded(xbar, xph) && threadIdx.x == 0) set_err(err, DFLASH2_DEV_TIMEOUT);
+  xph ^= 1u;
+}
+
 template <int NT, bool Q4>
 __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
   using RC = Ring<Q4>;
   constexpr int R = NT * 8;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full[kConsumers][RC::kNS];
-  __shared__ __align__(8) uint64_t empty[kConsumers][RC::kNS];
+  __shared__ __align__(8) uint64_t full[RC::kNS];
+  __shared__ __align__(8) uint64_t empty[RC::kNS];
+  __shared__ __align__(8) uint64_t xbar;
   __shared__ int s_last;
   uint8_t* ring = smem;
-  uint8_t* Xs = smem + kConsumers * RC::kNS * RC::kSlot;
+  uint8_t* Xs = smem + RC::kNS * RC::kSlot;
   const int stride = p.kc_units * RC::kUnitK * 2 + 64;
-  float* Xsum = reinterpret_cast<float*>(Xs + R * stride);
-  float2* coef_all = reinterpret_cast<float2*>(Xsum + (Q4 ? p.kc_units * 8 * R : 0));
+  float2* coef_all = reinterpret_cast<float2*>(Xs + R * stride);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 
   if (threadIdx.x == 0) {
-    for (int w = 0; w < kConsumers; ++w)
-      for (int s = 0; s < RC::kNS; ++s) {
-        mbar_init(&full[w][s], 1);
-        mbar_init(&empty[w][s], 1);
-      }
+    for (int s = 0; s < RC::kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -181,32 +212,26 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
   if (warp == kConsumers) {
     // ---- producer: weights only, so it may run ahead of the previous kernel ----
     if (lane != 0) return;
-    int cnt[kConsumers];
-    for (int w = 0; w < kConsumers; ++w) cnt[w] = 0;
+    int cnt = 0;
     for (long long x = x0; x < x1;) {
       const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
       const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
       const int grp = gidx % p.groups, mz = (gidx / p.groups) * 64;
-      const uint8_t* src[kConsumers];
-      for (int w = 0; w < kConsumers; ++w) {
-        int si;
-        const int tile = sk_tile(p, grp, w, si);
-        src[w] = (tile >= 0 && sk_rows(p, si, mz, R) > 0)
-                     ? p.seg[si].W + ((size_t)tile * p.U) * RC::kSlot
-                     : nullptr;
-      }
-      for (int u = ua; u < ub; ++u)
-        for (int w = 0; w < kConsumers; ++w) {
-          if (!src[w]) continue;
-          const int slot = cnt[w] % RC::kNS, round = cnt[w] / RC::kNS;
-          if (round > 0 && !mbar_wait_bounded(&empty[w][slot], (round - 1) & 1)) {
+      int si;
+      sk_tile(p, grp, 0, si);
+      if (sk_rows(p, si, mz, R) > 0) {
+        const uint8_t* src = sk_group_src<Q4>(p, grp);
+        for (int u = ua; u < ub; ++u) {
+          const int slot = cnt % RC::kNS, round = cnt / RC::kNS;
+          if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
             set_err(p.err, DFLASH2_DEV_TIMEOUT);
             return;
           }
-          mbar_expect_tx(&full[w][slot], RC::kSlot);
-          bulk_g2s(ring + (w * RC::kNS + slot) * RC::kSlot, src[w] + (size_t)u * RC::kSlot, RC::kSlot, &full[w][slot]);
-          ++cnt[w];
+          mbar_expect_tx(&full[slot], RC::kSlot);
+          bulk_g2s(ring + slot * RC::kSlot, src + (size_t)u * RC::kSlot, RC::kSlot, &full[slot]);
+          ++cnt;
         }
+      }
       x += ub - ua;
     }
     return;
@@ -216,6 +241,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
   pdl_wait();  // activations and the partial/ticket buffers come from earlier kernels
   float2* coef = coef_all + warp * 128;
   int cnt = 0;
+  uint32_t xph = 0;
   bool dead = false;
   for (long long x = x0; x < x1;) {
     const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
@@ -223,66 +249,47 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
     const int grp = gidx % p.groups, mz = (gidx / p.groups) * 64;
     int si;
     const int tile = sk_tile(p, grp, warp, si);
-    const int my_rows = tile >= 0 ? sk_rows(p, si, mz, R) : 0;
+    const int my_rows = sk_rows(p, si, mz, R);
     const int ntact = (my_rows + 7) >> 3;
     int stage_rows = p.rows - mz;
     stage_rows = stage_rows > R ? R : stage_rows;
     float acc[NT][4];
 #pragma unroll
     for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    for (int c0 = ua; c0 < ub; c0 += p.kc_units) {
-      const int cu = (ub - c0) < p.kc_units ? (ub - c0) : p.kc_units;
-      // stage X[mz.., c0*unitK ..] and, for Q4_K, the 32-wide sums
-      consumers_sync();
-      const int vec_per_row = cu * RC::kUnitK / 8;
-      const uint16_t* X = p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK;
-      for (int i = threadIdx.x; i < R * vec_per_row; i += kConsumers * 32) {
-        const int r = i / vec_per_row, v = i % vec_per_row;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (r < stage_rows) val = *reinterpret_cast<const uint4*>(X + (size_t)r * p.ldx + v * 8);
-        *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = val;
-      }
-      consumers_sync();
-      if (Q4) {
-        for (int i = threadIdx.x; i < R * cu * 8; i += kConsumers * 32) {
-          const int r = i % R, j = i / R;
-          const uint16_t* row = reinterpret_cast<const uint16_t*>(Xs + r * stride) + j * 32;
-          float s = 0.f;
-#pragma unroll 8
-          for (int k = 0; k < 32; ++k) s += bf2f(row[k]);
-          Xsum[j * R + r] = s;
-        }
-        consumers_sync();
-      }
-      if (ntact == 0) continue;
-      for (int u = c0; u < c0 + cu; ++u) {
-        const int slot = cnt % RC::kNS;
-        // a consumer never leaves early (the named barriers count on it): after an expired
-        // wait it flags the error and skips its remaining work
-        if (!dead && !mbar_wait_bounded(&full[warp][slot], (cnt / RC::kNS) & 1)) {
-          set_err(p.err, DFLASH2_DEV_TIMEOUT);
-          dead = true;
-        }
-        ++cnt;
-        if (dead) continue;
-        const uint8_t* sb = ring + (warp * RC::kNS + slot) * RC::kSlot;
-        if (Q4) {
-          uint4 q[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
-          const uint4 sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
-          q4_unit<NT>(q, sc, coef, Xs, stride, Xsum + (u - c0) * 8 * R, (u - c0) * 512, ntact, acc, lane);
-        } else {
-          uint4 wv[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
-            wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+    if (ntact > 0) {
+      for (int c0 = ua; c0 < ub; c0 += p.kc_units) {
+        const int cu = (ub - c0) < p.kc_units ? (ub - c0) : p.kc_units;
+        stage_x_chunk(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R, cu * RC::kUnitK * 2,
+                      Xs, stride, &xbar, xph, p.err);
+        for (int u = c0; u < c0 + cu; ++u) {
+          const int slot = cnt % RC::kNS;
+          // a consumer never leaves early (the named barriers count on it): after an expired
+          // wait it flags the error and skips its remaining work
+          if (!dead && !mbar_wait_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
+            set_err(p.err, DFLASH2_DEV_TIMEOUT);
+            dead = true;
           }
-          bf16_step<NT>(wv, Xs, stride, (u - c0) * 256, ntact, acc, lane);
+          ++cnt;
+          if (dead) continue;
+          const uint8_t* sb = ring + slot * RC::kSlot + warp * RC::kUnitBytes;
+          if (Q4) {
+            uint4 q[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
+            const uint4 sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
+            q4_unit<NT>(q, sc, coef, Xs, stride, (u - c0) * 512, ntact, acc, lane);
+          } else {
+            uint4 wv[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
+              wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+            }
+            bf16_step<NT>(wv, Xs, stride, (u - c0) * 256, ntact, acc, lane);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[warp][slot]);
       }
     }
     // partial of this piece
@@ -308,6 +315,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
         }
       }
     }
+    // split-K: the last CTA of this column group to arrive sums the partials in range order
+    // (deterministic) and runs the epilogue; nobody waits
     __threadfence();
     consumers_sync();
     if (threadIdx.x == 0) {
@@ -316,7 +325,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
       if (s_last) p.counters[gidx] = 0;
     }
     consumers_sync();
-    if (s_last) {
+    if (s_last && ntact > 0) {
       __threadfence();
       sk_fixup(p, grp, mz, R, npieces);
     }
@@ -326,10 +335,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
 
 // ---------------------------------------------------------------------------
 // Shared output head + streaming top-16 (<= 8 drafted rows), same engine: the
-// prepared [V + R rows] bf16 matrix (output head, then the selector projection)
-// is cut into 8-tile sets handed round-robin to the persistent CTAs.
+// prepared [V + R rows] bf16 matrix (output head, then the selector projection,
+// padded to whole 8-tile groups) is handed out group by group to the
+// persistent CTAs.  Logits never leave the SM: after each tile every lane
+// offers its values to a per-warp, per-row sorted top-16 list in shared memory
+// (threshold test first; insertions serialised over the warp by ballot); at the
+// end the CTA merges its 8 warp lists, and the selector kernel merges the CTAs'.
 struct SLmParams {
-  const uint8_t* W;  // prepared bf16 tiles of [lm_head; sel_proj]
+  const uint8_t* W;  // prepared bf16 groups of [lm_head; sel_proj]
   int V, R, H;
   const uint16_t* X;  // final-normed rows [rows][H]
   int rows;
@@ -342,23 +355,24 @@ struct SLmParams {
 __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
   using RC = Ring<false>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full[kConsumers][RC::kNS];
-  __shared__ __align__(8) uint64_t empty[kConsumers][RC::kNS];
+  __shared__ __align__(8) uint64_t full[RC::kNS];
+  __shared__ __align__(8) uint64_t empty[RC::kNS];
+  __shared__ __align__(8) uint64_t xbar;
   const int H = p.H, stride = H * 2 + 64;
   uint8_t* ring = smem;
-  uint8_t* Xs = smem + kConsumers * RC::kNS * RC::kSlot;
+  uint8_t* Xs = smem + RC::kNS * RC::kSlot;
   float* lv_all = reinterpret_cast<float*>(Xs + 8 * stride);          // [warps][8][16]
   int* li_all = reinterpret_cast<int*>(lv_all + kConsumers * 8 * kTopK);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int vt = p.V / 16, total = vt + p.R / 16, S = H / 128;
-  const int nsets = (total + kConsumers - 1) / kConsumers;
+  const int ngroups = (total + kConsumers - 1) / kConsumers;
 
   if (threadIdx.x == 0) {
-    for (int w = 0; w < kConsumers; ++w)
-      for (int s = 0; s < RC::kNS; ++s) {
-        mbar_init(&full[w][s], 1);
-        mbar_init(&empty[w][s], 1);
-      }
+    for (int s = 0; s < RC::kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -366,23 +380,18 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
 
   if (warp == kConsumers) {
     if (lane != 0) return;
-    int cnt[kConsumers];
-    for (int w = 0; w < kConsumers; ++w) cnt[w] = 0;
-    for (int set = blockIdx.x; set < nsets; set += gridDim.x)
-      for (int s = 0; s < S; ++s)
-        for (int w = 0; w < kConsumers; ++w) {
-          const int tile = set * kConsumers + w;
-          if (tile >= total) continue;
-          const int slot = cnt[w] % RC::kNS, round = cnt[w] / RC::kNS;
-          if (round > 0 && !mbar_wait_bounded(&empty[w][slot], (round - 1) & 1)) {
-            set_err(p.err, DFLASH2_DEV_TIMEOUT);
-            return;
-          }
-          mbar_expect_tx(&full[w][slot], RC::kSlot);
-          bulk_g2s(ring + (w * RC::kNS + slot) * RC::kSlot, p.W + ((size_t)tile * S + s) * RC::kSlot, RC::kSlot,
-                   &full[w][slot]);
-          ++cnt[w];
+    int cnt = 0;
+    for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x)
+      for (int s = 0; s < S; ++s) {
+        const int slot = cnt % RC::kNS, round = cnt / RC::kNS;
+        if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
+          set_err(p.err, DFLASH2_DEV_TIMEOUT);
+          return;
         }
+        mbar_expect_tx(&full[slot], RC::kSlot);
+        bulk_g2s(ring + slot * RC::kSlot, p.W + ((size_t)grp * S + s) * RC::kSlot, RC::kSlot, &full[slot]);
+        ++cnt;
+      }
     return;
   }
 
@@ -391,29 +400,24 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
     li_all[i] = 0x7fffffff;
   }
   pdl_wait();
-  for (int i = threadIdx.x; i < 8 * (H / 8); i += kConsumers * 32) {
-    const int r = i / (H / 8), v = i % (H / 8);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < p.rows) val = *reinterpret_cast<const uint4*>(p.X + (size_t)r * H + v * 8);
-    *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = val;
-  }
-  consumers_sync();
+  uint32_t xph = 0;
+  stage_x_chunk(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
   float* lv = lv_all + warp * 8 * kTopK;
   int* li = li_all + warp * 8 * kTopK;
   int cnt = 0;
-  bool ok = true;
-  for (int set = blockIdx.x; set < nsets && ok; set += gridDim.x) {
-    const int tile = set * kConsumers + warp;
-    if (tile >= total) continue;
+  bool dead = false;
+  for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x) {
+    const int tile = grp * kConsumers + warp;
     float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
     for (int s = 0; s < S; ++s) {
       const int slot = cnt % RC::kNS;
-      if (!mbar_wait_bounded(&full[warp][slot], (cnt / RC::kNS) & 1)) {
+      if (!dead && !mbar_wait_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
         set_err(p.err, DFLASH2_DEV_TIMEOUT);
-        ok = false;
-        break;
+        dead = true;
       }
-      const uint8_t* sb = ring + (warp * RC::kNS + slot) * RC::kSlot;
+      ++cnt;
+      if (dead) continue;
+      const uint8_t* sb = ring + slot * RC::kSlot + warp * RC::kUnitBytes;
       uint4 wv[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -422,10 +426,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
       }
       bf16_step<1>(wv, Xs, stride, s * 256, 1, acc, lane);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[warp][slot]);
-      ++cnt;
+      if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    if (!ok) break;
+    if (dead || tile >= total) continue;
     if (tile >= vt) {
       const int c0 = (tile - vt) * 16;
 #pragma unroll
@@ -497,20 +500,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
           if (i == bi) { v[i] = -INFINITY; id[i] = 0x7fffffff; }
       }
     }
-  }
-}
-
-// Canonical bf16 [N][K] -> prepared tiles [N/16][K/128][4096 B].
-__global__ void k_bf16_prepare(const uint16_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K) {
-  const int S = K / 128, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x, g = lane >> 2, t = lane & 3;
-  uint8_t* out = dst + ((size_t)T * S + s) * 4096;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const size_t k = (size_t)s * 128 + j * 32 + t * 8;
-    *reinterpret_cast<uint4*>(out + j * 1024 + lane * 16) =
-        *reinterpret_cast<const uint4*>(src + (size_t)(T * 16 + g) * K + k);
-    *reinterpret_cast<uint4*>(out + j * 1024 + 512 + lane * 16) =
-        *reinterpret_cast<const uint4*>(src + (size_t)(T * 16 + g + 8) * K + k);
   }
 }
 
