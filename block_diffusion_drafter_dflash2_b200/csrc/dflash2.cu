@@ -62,9 +62,10 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
   const int ring = ns * slot;
   const int per_unit = g.R * unitK * 2;
-  const int budget = kSmemLimit - kStaticSmem - ring - (q4 ? kConsumers * 1024 : 0) - 64 * g.R;
+  const int extra = kGemvConsumers * 1024 + kConsumers * 32 * g.NT * 4 * 4;  // per-warp scale tables, set reduction
+  const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + (q4 ? kConsumers * 1024 : 0);
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
   return g;
 }
 
@@ -218,7 +219,7 @@ cudaError_t launch_sgemv_t(const GemvPlan& g, const SGemvParams& prm, cudaStream
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kStreamThreads), g.smem, s, prm);
+  return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kGemvThreads), g.smem, s, prm);
 }
 
 struct Epi {

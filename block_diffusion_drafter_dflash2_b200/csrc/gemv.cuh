@@ -91,10 +91,16 @@ DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8
         mma16816(s, a1, bx.z, bx.w);
         mma16816(xs, ones, bx.x, bx.y);
         mma16816(xs, ones, bx.z, bx.w);
-        acc[nt][0] = fmaf(cg.x, s[0], fmaf(-cg.y, xs[0], acc[nt][0]));
-        acc[nt][1] = fmaf(cg.x, s[1], fmaf(-cg.y, xs[1], acc[nt][1]));
-        acc[nt][2] = fmaf(ch.x, s[2], fmaf(-ch.y, xs[2], acc[nt][2]));
-        acc[nt][3] = fmaf(ch.x, s[3], fmaf(-ch.y, xs[3], acc[nt][3]));
+        // acc += D * S - M * X, two accumulators per packed FMA
+        float2 a01 = make_float2(acc[nt][0], acc[nt][1]), a23 = make_float2(acc[nt][2], acc[nt][3]);
+        a01 = ffma2(make_float2(-cg.y, -cg.y), make_float2(xs[0], xs[1]), a01);
+        a01 = ffma2(make_float2(cg.x, cg.x), make_float2(s[0], s[1]), a01);
+        a23 = ffma2(make_float2(-ch.y, -ch.y), make_float2(xs[2], xs[3]), a23);
+        a23 = ffma2(make_float2(ch.x, ch.x), make_float2(s[2], s[3]), a23);
+        acc[nt][0] = a01.x;
+        acc[nt][1] = a01.y;
+        acc[nt][2] = a23.x;
+        acc[nt][3] = a23.y;
       }
     }
   }

@@ -52,13 +52,22 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
     return;
   }
   if (p.mode == 2 && t == 0) return;
-  const float4* in = reinterpret_cast<const float4*>(p.in + (size_t)r * p.H);
+  const float4* __restrict__ in = reinterpret_cast<const float4*>(p.in + (size_t)r * p.H);
   float ss = 0.f;
-#pragma unroll 8
-  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
-    const float4 v = in[c];
-    vrow4[c] = v;
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  {
+    float4 v4[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int c = threadIdx.x + k * blockDim.x;
+      if (c < H4) v4[k] = in[c];
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int c = threadIdx.x + k * blockDim.x;
+      if (c >= H4) break;
+      vrow4[c] = v4[k];
+      ss += v4[k].x * v4[k].x + v4[k].y * v4[k].y + v4[k].z * v4[k].z + v4[k].w * v4[k].w;
+    }
   }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -71,15 +80,27 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
   __syncthreads();
   const float rs = rsqrtf(red[0] / p.H + p.eps);
   const int orow = p.mode == 2 ? b * (p.Bk - 1) + t - 1 : r;
-#pragma unroll 8
-  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+  // the weight loads go first: with the stores in the same loop the compiler cannot prove the
+  // global pointers apart and would serialise a load->store round trip per iteration
+  const uint2* __restrict__ w2 = reinterpret_cast<const uint2*>(p.w);
+  uint16_t* __restrict__ ob = p.out_bf ? p.out_bf + (size_t)orow * p.ldob : nullptr;
+  float4* __restrict__ of = p.out_f ? reinterpret_cast<float4*>(p.out_f + (size_t)r * p.H) : nullptr;
+  constexpr int kMaxIt = 16;  // H <= 16384 over 256 threads
+  uint2 wv[kMaxIt];
+#pragma unroll
+  for (int k = 0; k < kMaxIt; ++k) {
+    const int c = threadIdx.x + k * blockDim.x;
+    if (c < H4) wv[k] = w2[c];
+  }
+#pragma unroll
+  for (int k = 0; k < kMaxIt; ++k) {
+    const int c = threadIdx.x + k * blockDim.x;
+    if (c >= H4) break;
     const float4 v = vrow4[c];
-    const uint2 wv = *reinterpret_cast<const uint2*>(p.w + 4 * c);
-    const float y0 = v.x * rs * bf2f(wv.x & 0xffff), y1 = v.y * rs * bf2f(wv.x >> 16);
-    const float y2 = v.z * rs * bf2f(wv.y & 0xffff), y3 = v.w * rs * bf2f(wv.y >> 16);
-    if (p.out_bf)
-      *reinterpret_cast<uint2*>(p.out_bf + (size_t)orow * p.ldob + 4 * c) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
-    if (p.out_f) reinterpret_cast<float4*>(p.out_f + (size_t)r * p.H)[c] = make_float4(y0, y1, y2, y3);
+    const float y0 = v.x * rs * bf2f(wv[k].x & 0xffff), y1 = v.y * rs * bf2f(wv[k].x >> 16);
+    const float y2 = v.z * rs * bf2f(wv[k].y & 0xffff), y3 = v.w * rs * bf2f(wv[k].y >> 16);
+    if (ob) *reinterpret_cast<uint2*>(ob + 4 * c) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
+    if (of) of[c] = make_float4(y0, y1, y2, y3);
   }
 }
 

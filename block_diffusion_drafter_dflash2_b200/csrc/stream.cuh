@@ -35,8 +35,11 @@
 
 namespace dfl {
 
-constexpr int kConsumers = 8;
+constexpr int kConsumers = 8;                          // consumer warps of the LM-head kernel = tiles per group
 constexpr int kStreamThreads = (kConsumers + 1) * 32;
+constexpr int kGemvSets = 2;                           // GEMV: two warp sets alternate ring slots
+constexpr int kGemvConsumers = kGemvSets * kConsumers;
+constexpr int kGemvThreads = (kGemvConsumers + 1) * 32;
 
 template <bool Q4>
 struct Ring;
@@ -49,7 +52,8 @@ struct Ring<false> {
   static constexpr int kUnitBytes = 4096, kSlot = 8 * 4096, kNS = 4, kUnitK = 128;
 };
 
-DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory"); }
+template <int NTHR>
+DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NTHR) : "memory"); }
 DEVI void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -126,7 +130,7 @@ DEVI float sum_pieces(const SGemvParams& p, int npieces, int row, int col) {
 
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
-  const int tid = threadIdx.x, nthr = kConsumers * 32, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, nthr = kGemvConsumers * 32, warp = tid >> 5, lane = tid & 31;
   if (p.paired) {
     const int f0 = grp * 64;
     const int rows = sk_rows(p, 0, mz, R);
@@ -145,7 +149,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   const int rows = sk_rows(p, si, mz, R);
   if (p.epi == EPI_QKV) {
     const int head = tile0 / 8;
-    for (int r = warp; r < rows; r += kConsumers) {
+    for (int r = warp; r < rows; r += kGemvConsumers) {
       float x[4];
       const int dims[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
 #pragma unroll
@@ -165,26 +169,28 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
 
 // Bring rows [0, nrows) of an X chunk (row stride ldx elements, `bytes` per row) into Xs (row
 // stride `stride` bytes) with bulk copies on xbar; rows [nrows, R) are zeroed.  Consumer threads.
+template <int NTHR>
 DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes, uint8_t* Xs, int stride,
                         uint64_t* xbar, uint32_t& xph, int* err) {
-  consumers_sync();  // every consumer is done with the previous chunk
+  consumers_sync<NTHR>();  // every consumer is done with the previous chunk
   if (threadIdx.x == 0) {
     mbar_expect_tx(xbar, (uint32_t)(nrows * bytes));
     for (int r = 0; r < nrows; ++r) bulk_g2s(Xs + r * stride, X + (size_t)r * ldx, bytes, xbar);
   }
-  for (int i = threadIdx.x; i < (R - nrows) * (bytes / 16); i += kConsumers * 32) {
+  for (int i = threadIdx.x; i < (R - nrows) * (bytes / 16); i += NTHR) {
     const int r = nrows + i / (bytes / 16), v = i % (bytes / 16);
     *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = make_uint4(0, 0, 0, 0);
   }
-  consumers_sync();
+  consumers_sync<NTHR>();
   if (!mbar_wait_bounded(xbar, xph) && threadIdx.x == 0) set_err(err, DFLASH2_DEV_TIMEOUT);
   xph ^= 1u;
 }
 
 template <int NT, bool Q4>
-__global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
   using RC = Ring<Q4>;
   constexpr int R = NT * 8;
+  constexpr int NC = kGemvConsumers * 32;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[RC::kNS];
   __shared__ __align__(8) uint64_t empty[RC::kNS];
@@ -193,13 +199,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
   uint8_t* ring = smem;
   uint8_t* Xs = smem + RC::kNS * RC::kSlot;
   const int stride = p.kc_units * RC::kUnitK * 2 + 64;
-  float2* coef_all = reinterpret_cast<float2*>(Xs + R * stride);
+  float2* coef_all = reinterpret_cast<float2*>(Xs + R * stride);                // [16 warps][128]
+  float* red = reinterpret_cast<float*>(coef_all + kGemvConsumers * 128);       // [8][32][NT*4]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int set = warp / kConsumers, wt = warp % kConsumers;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < RC::kNS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers);
+      mbar_init(&empty[s], kConsumers);  // the 8 warps of the set that owns the slot
     }
     mbar_init(&xbar, 1);
     fence_mbar_init();
@@ -209,7 +217,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
   const long long P = gridDim.x, c = blockIdx.x;
   const long long x0 = c * p.W / P, x1 = (c + 1) * p.W / P;
 
-  if (warp == kConsumers) {
+  if (warp == kGemvConsumers) {
     // ---- producer: weights only, so it may run ahead of the previous kernel ----
     if (lane != 0) return;
     int cnt = 0;
@@ -237,7 +245,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
     return;
   }
 
-  // ---- consumers ----
+  // ---- consumers: ring slot k is consumed by warp set (k & 1) ----
   pdl_wait();  // activations and the partial/ticket buffers come from earlier kernels
   float2* coef = coef_all + warp * 128;
   int cnt = 0;
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
     const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
     const int grp = gidx % p.groups, mz = (gidx / p.groups) * 64;
     int si;
-    const int tile = sk_tile(p, grp, warp, si);
+    const int tile = sk_tile(p, grp, wt, si);
     const int my_rows = sk_rows(p, si, mz, R);
     const int ntact = (my_rows + 7) >> 3;
     int stage_rows = p.rows - mz;
@@ -259,19 +267,22 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
     if (ntact > 0) {
       for (int c0 = ua; c0 < ub; c0 += p.kc_units) {
         const int cu = (ub - c0) < p.kc_units ? (ub - c0) : p.kc_units;
-        stage_x_chunk(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R, cu * RC::kUnitK * 2,
-                      Xs, stride, &xbar, xph, p.err);
+        stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R,
+                          cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err);
         for (int u = c0; u < c0 + cu; ++u) {
           const int slot = cnt % RC::kNS;
+          const bool mine = (cnt & 1) == set;
+          const uint32_t par = (cnt / RC::kNS) & 1;
+          ++cnt;
+          if (!mine) continue;
           // a consumer never leaves early (the named barriers count on it): after an expired
           // wait it flags the error and skips its remaining work
-          if (!dead && !mbar_wait_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
+          if (!dead && !mbar_wait_bounded(&full[slot], par)) {
             set_err(p.err, DFLASH2_DEV_TIMEOUT);
             dead = true;
           }
-          ++cnt;
           if (dead) continue;
-          const uint8_t* sb = ring + slot * RC::kSlot + warp * RC::kUnitBytes;
+          const uint8_t* sb = ring + slot * RC::kSlot + wt * RC::kUnitBytes;
           if (Q4) {
             uint4 q[4];
 #pragma unroll
@@ -292,12 +303,25 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
         }
       }
     }
-    // partial of this piece
+    // the two sets' accumulators meet in shared memory; set 0 writes the piece's partial
+    if (ntact > 0 && set == 1) {
+      float* rd = red + (wt * 32 + lane) * (NT * 4);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rd[nt * 4 + e] = acc[nt][e];
+    }
+    consumers_sync<NC>();
     const long long gstart = (long long)gidx * p.U;
     const long long first = sk_owner(gstart, p.W, P);
     const int piece = (int)(c - first);
     const int npieces = (int)(sk_owner(gstart + p.U - 1, p.W, P) - first + 1);
-    if (ntact > 0) {
+    if (ntact > 0 && set == 0) {
+      const float* rd = red + (wt * 32 + lane) * (NT * 4);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] += rd[nt * 4 + e];
       float* out = p.part + (size_t)piece * p.piece_stride + (size_t)mz * p.ldo;
       const int out_col = p.seg[si].out_col + tile * 16;
 #pragma unroll
@@ -318,13 +342,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_sgemv(SGemvParams p) {
     // split-K: the last CTA of this column group to arrive sums the partials in range order
     // (deterministic) and runs the epilogue; nobody waits
     __threadfence();
-    consumers_sync();
+    consumers_sync<NC>();
     if (threadIdx.x == 0) {
       const int prev = atomicAdd(p.counters + gidx, 1);
       s_last = prev == npieces - 1;
       if (s_last) p.counters[gidx] = 0;
     }
-    consumers_sync();
+    consumers_sync<NC>();
     if (s_last && ntact > 0) {
       __threadfence();
       sk_fixup(p, grp, mz, R, npieces);
@@ -401,7 +425,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
   }
   pdl_wait();
   uint32_t xph = 0;
-  stage_x_chunk(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
+  stage_x_chunk<kConsumers * 32>(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
   float* lv = lv_all + warp * 8 * kTopK;
   int* li = li_all + warp * 8 * kTopK;
   int cnt = 0;
@@ -460,7 +484,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
       }
     }
   }
-  consumers_sync();
+  consumers_sync<kConsumers * 32>();
   // merge the 8 warp lists of each row
   for (int r = warp; r < p.rows; r += kConsumers) {
     float v[4];
