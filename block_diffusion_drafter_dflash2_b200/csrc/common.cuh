@@ -102,6 +102,22 @@ DEVI bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
+// Same, but the waiting thread is suspended (up to a few microseconds per try) instead of
+// spinning, leaving issue slots to the warps that do work (the producer in particular).
+DEVI bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(4000u)
+      : "memory");
+  return ok != 0;
+}
+DEVI bool mbar_wait_sleep_bounded(uint64_t* bar, uint32_t parity) {
+  for (long long i = 0; i < (kWaitLimit >> 6); ++i)
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+  return false;
+}
 // global -> shared bulk copy; dst/src 16-byte aligned, bytes a multiple of 16.
 DEVI void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -182,7 +182,7 @@ DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes,
     *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = make_uint4(0, 0, 0, 0);
   }
   consumers_sync<NTHR>();
-  if (!mbar_wait_bounded(xbar, xph) && threadIdx.x == 0) set_err(err, DFLASH2_DEV_TIMEOUT);
+  if (!mbar_wait_sleep_bounded(xbar, xph) && threadIdx.x == 0) set_err(err, DFLASH2_DEV_TIMEOUT);
   xph ^= 1u;
 }
 
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
   // ---- consumers: ring slot k is consumed by warp set (k & 1) ----
   pdl_wait();  // activations and the partial/ticket buffers come from earlier kernels
   float2* coef = coef_all + warp * 128;
-  int cnt = 0;
+  int cnt = 0, staged_mz = -1;
   uint32_t xph = 0;
   bool dead = false;
   for (long long x = x0; x < x1;) {
@@ -265,10 +265,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 #pragma unroll
     for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     if (ntact > 0) {
+      const bool whole = p.kc_units >= p.U;  // all of K fits: stage X once per row group and keep it
       for (int c0 = ua; c0 < ub; c0 += p.kc_units) {
         const int cu = (ub - c0) < p.kc_units ? (ub - c0) : p.kc_units;
-        stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R,
-                          cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err);
+        int base = c0;
+        if (whole) {
+          base = 0;
+          if (staged_mz != mz) {
+            stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx, p.ldx, stage_rows, R, p.U * RC::kUnitK * 2, Xs, stride, &xbar,
+                              xph, p.err);
+            staged_mz = mz;
+          }
+        } else {
+          stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R,
+                            cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err);
+        }
         for (int u = c0; u < c0 + cu; ++u) {
           const int slot = cnt % RC::kNS;
           const bool mine = (cnt & 1) == set;
@@ -277,7 +288,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
           if (!mine) continue;
           // a consumer never leaves early (the named barriers count on it): after an expired
           // wait it flags the error and skips its remaining work
-          if (!dead && !mbar_wait_bounded(&full[slot], par)) {
+          if (!dead && !mbar_wait_sleep_bounded(&full[slot], par)) {
             set_err(p.err, DFLASH2_DEV_TIMEOUT);
             dead = true;
           }
@@ -288,7 +299,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
             const uint4 sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
-            q4_unit<NT>(q, sc, coef, Xs, stride, (u - c0) * 512, ntact, acc, lane);
+            q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane);
           } else {
             uint4 wv[8];
 #pragma unroll
@@ -296,7 +307,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
               wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
               wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
             }
-            bf16_step<NT>(wv, Xs, stride, (u - c0) * 256, ntact, acc, lane);
+            bf16_step<NT>(wv, Xs, stride, (u - base) * 256, ntact, acc, lane);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);
@@ -435,7 +446,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
     float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
     for (int s = 0; s < S; ++s) {
       const int slot = cnt % RC::kNS;
-      if (!dead && !mbar_wait_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
+      if (!dead && !mbar_wait_sleep_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
         set_err(p.err, DFLASH2_DEV_TIMEOUT);
         dead = true;
       }
