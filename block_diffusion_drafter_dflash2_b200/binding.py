@@ -16,7 +16,9 @@ MAX_LAYERS = 8
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdflash2.so")
 
-ERR_NAMES = {0: "OK", -1: "ARG", -2: "SHAPE", -3: "ALIGN", -4: "WORKSPACE", -5: "CUDA", -6: "LAYOUT"}
+ERR_NAMES = {0: "OK", -1: "ARG", -2: "SHAPE", -3: "ALIGN", -4: "WORKSPACE", -5: "CUDA", -6: "LAYOUT",
+             -7: "STATIC_LIMIT"}
+STATIC_SCRATCH_BYTES = 16 << 20
 DEV_TOKEN, DEV_PAGE, DEV_NONFINITE, DEV_TIMEOUT = 1, 2, 4, 8
 
 
@@ -54,7 +56,8 @@ class Debug(C.Structure):
 
 
 EXPORTS = ("dflash2_workspace_size", "dflash2_prepared_size", "dflash2_prepare_weights", "dflash2_draft_step",
-           "dflash2_accept", "dflash2_spec_step_host", "dflash2_device_error", "dflash2_strerror")
+           "dflash2_draft_step_static", "dflash2_accept", "dflash2_spec_step_host", "dflash2_device_error",
+           "dflash2_strerror")
 
 _lib = None
 
@@ -76,6 +79,9 @@ def load(path: str = LIB_PATH):
     lib.dflash2_draft_step.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(Inputs), C.POINTER(KV),
                                        C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.POINTER(Debug),
                                        C.c_void_p]
+    lib.dflash2_draft_step_static.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(Inputs),
+                                              C.POINTER(KV), C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                                              C.POINTER(Debug), C.c_void_p]
     lib.dflash2_accept.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
     lib.dflash2_spec_step_host.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(KV), C.c_int32] + \
         [C.c_void_p] * 9 + [C.c_void_p, C.c_size_t, C.c_void_p]
@@ -170,6 +176,16 @@ class Drafter:
                                          _ptr(out_path), _ptr(out_scores), _ptr(self.workspace), self.ws_bytes,
                                          C.byref(dbg) if dbg is not None else None, _stream(stream))
         check(rc, "draft_step")
+
+    def draft_step_static(self, inputs: dict, state: dict, out_path: torch.Tensor, out_scores: torch.Tensor,
+                          dev_err: Optional[torch.Tensor] = None, stream=None, kv: Optional[KV] = None):
+        """The allocation-free entry point: same step, scratch compiled into the library (no workspace)."""
+        ins = Inputs(inputs["taps"].data_ptr(), inputs["n_new"].data_ptr(), inputs["block_tokens"].data_ptr())
+        kvs = kv if kv is not None else kv_struct(state)
+        rc = self.lib.dflash2_draft_step_static(C.byref(self.cfg), C.byref(self.w), C.byref(ins), C.byref(kvs),
+                                                self.batch, _ptr(out_path), _ptr(out_scores), _ptr(dev_err), None,
+                                                _stream(stream))
+        check(rc, "draft_step_static")
 
     def accept(self, draft: torch.Tensor, target: torch.Tensor, accepted: torch.Tensor, emitted: torch.Tensor,
                stream=None):

@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "attention.cuh"
 #include "common.cuh"
@@ -312,6 +313,30 @@ int check_weights(const dflash2_config* c, const dflash2_weights* w) {
     }
   }
   return DFLASH2_OK;
+}
+
+// Scratch of the allocation-free entry point: file-scope device memory, present on every GPU
+// that loads this library for the life of the process.
+static __device__ __align__(256) uint8_t g_static_scratch[DFLASH2_STATIC_SCRATCH_BYTES];
+
+// Device address of g_static_scratch on the current device, looked up once per device.  (The
+// symbol's name in host code is only a host-side stand-in, not a device address.)
+void* static_scratch(cudaError_t* err) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<void*> cache[kMaxDevices];
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  *err = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (*err != cudaSuccess) return nullptr;
+  cache[dev].store(p, std::memory_order_release);
+  return p;
 }
 
 }  // namespace
@@ -672,6 +697,23 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   return DFLASH2_OK;
 }
 
+int dflash2_draft_step_static(const dflash2_config* c, const dflash2_weights* w, const dflash2_inputs* in,
+                              const dflash2_kv* kv, int32_t batch, int32_t* out_path, float* out_scores,
+                              int32_t* dev_err, const dflash2_debug* dbg, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (batch < 1) return DFLASH2_ERR_ARG;
+  if (make_plan(c, batch).step_bytes > DFLASH2_STATIC_SCRATCH_BYTES) return DFLASH2_ERR_STATIC_LIMIT;
+  cudaError_t e = cudaSuccess;
+  void* ws = static_scratch(&e);
+  if (!ws) return fail(e == cudaSuccess ? cudaErrorUnknown : e);
+  const int rc = dflash2_draft_step(c, w, in, kv, batch, out_path, out_scores, ws, DFLASH2_STATIC_SCRATCH_BYTES, dbg,
+                                    stream);
+  if (rc != DFLASH2_OK) return rc;
+  if (dev_err)  // the error word sits at the start of the scratch
+    CK(cudaMemcpyAsync(dev_err, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return DFLASH2_OK;
+}
+
 int dflash2_accept(const int32_t* draft, const int32_t* target, int32_t batch, int32_t block, int32_t* accepted,
                    int32_t* emitted, void* stream) {
   if (!draft || !target || !accepted || !emitted || batch < 1 || block < 2) return DFLASH2_ERR_ARG;
@@ -728,6 +770,7 @@ const char* dflash2_strerror(int code) {
     case DFLASH2_ERR_WORKSPACE: return "workspace or prepared-weight buffer too small";
     case DFLASH2_ERR_CUDA: return "CUDA launch or copy failed";
     case DFLASH2_ERR_LAYOUT: return "Q4_K weights must go through dflash2_prepare_weights";
+    case DFLASH2_ERR_STATIC_LIMIT: return "request needs more scratch than the allocation-free entry point holds";
   }
   return "unknown error";
 }

@@ -44,6 +44,7 @@ extern "C" {
 #define DFLASH2_ERR_WORKSPACE (-4) /* workspace or prepared-weight buffer too small */
 #define DFLASH2_ERR_CUDA (-5)      /* a CUDA launch or copy failed */
 #define DFLASH2_ERR_LAYOUT (-6)    /* Q4_K weights passed without dflash2_prepare_weights */
+#define DFLASH2_ERR_STATIC_LIMIT (-7) /* request larger than the built-in scratch of dflash2_draft_step_static */
 
 /* device error bits (dflash2_device_error) */
 #define DFLASH2_DEV_TOKEN 1     /* a block token id is outside [0, vocab) */
@@ -166,6 +167,32 @@ int dflash2_prepare_weights(const dflash2_config *cfg, const dflash2_weights *sr
 int dflash2_draft_step(const dflash2_config *cfg, const dflash2_weights *w, const dflash2_inputs *in,
                        const dflash2_kv *kv, int32_t batch, int32_t *out_path, float *out_scores,
                        void *workspace, size_t ws_bytes, const dflash2_debug *dbg, void *stream);
+
+/* Allocation-free variant of dflash2_draft_step.  (This entry point has no
+ * counterpart in the drafter's description; it exists for callers, not for the
+ * method.)  Some callers cannot hand the library a workspace: code embedded in a
+ * host framework whose device memory is owned by its own pool and that forbids
+ * direct cudaMalloc, or a latency-critical path where an allocation (which may
+ * synchronise the device) is not acceptable.  This call needs no workspace: its
+ * scratch is a 16 MiB array compiled into the library (DFLASH2_STATIC_SCRATCH_BYTES),
+ * which every GPU that loads the library keeps until the process exits.  It
+ * allocates nothing itself.
+ *  - Enough for the full drafter at batch 1 (about 8 MiB); requests whose step
+ *    workspace (dflash2_workspace_size minus its host-copy staging) exceeds the
+ *    array are rejected with DFLASH2_ERR_STATIC_LIMIT before any launch.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents; the step clears what must start at zero.  Calls that overlap on
+ *    the GPU (different streams, or threads without ordering) race on it: order
+ *    them on one stream.
+ *  - dev_err: optional DEVICE pointer to one int32 that receives the step's device
+ *    error bits (DFLASH2_DEV_*), copied on `stream` after the step; NULL to skip.
+ * Other arguments, outputs and errors as dflash2_draft_step. */
+#define DFLASH2_STATIC_SCRATCH_BYTES (16u << 20)
+int dflash2_draft_step_static(const dflash2_config *cfg, const dflash2_weights *w, const dflash2_inputs *in,
+                              const dflash2_kv *kv, int32_t batch, int32_t *out_path, float *out_scores,
+                              int32_t *dev_err, const dflash2_debug *dbg, void *stream);
 
 /* Greedy acceptance (FastFlowLM card, "How it is used"): draft int32
  * [batch][block-1], target int32 [batch][block] (the target's most likely token
