@@ -145,15 +145,19 @@ typedef struct dflash2_debug {
  * the current device (depends on its SM count).  0 on an invalid config. */
 size_t dflash2_workspace_size(const dflash2_config *cfg, int32_t batch);
 
-/* Bytes of the prepared copy of the Q4_K matrices (0 for wfmt 1). */
+/* Bytes of the prepared weight copy: every streamed matrix (fc, the layer matrices, the
+ * dynamic-convolution generators, the output head with the selector projection). */
 size_t dflash2_prepared_size(const dflash2_config *cfg);
 
-/* Repack the Q4_K matrices of `src` (canonical layout, device) into `dst`
- * (device, dst_bytes >= dflash2_prepared_size) in the tile order the GEMV
- * kernels stream, and fill `out` (host struct) with `src`'s pointers except the
- * Q4_K matrices, which point into dst; out->prepared = 1.  Values are not
- * changed: the prepared copy holds the same bits, reordered.  For wfmt 1 it
- * copies the struct and sets prepared = 1.  Asynchronous on `stream`. */
+/* Repack the streamed matrices of `src` (canonical layouts, device) into `dst`
+ * (device, 16-byte aligned, dst_bytes >= dflash2_prepared_size): the 8 tiles of 16 rows
+ * of each column group interleaved per K unit (Q4_K: 256-wide super-blocks, codes in
+ * mma fragment order; bf16: 128-wide steps), gate and up interleaved 4 + 4 tiles per
+ * group, and the output head followed by the selector projection as one matrix padded
+ * to whole groups.  Values are not changed: the prepared copy holds the same bits,
+ * reordered.  Fills `out` (host struct) with `src`'s pointers except the streamed
+ * matrices, which point into dst (wu aliases wg); out->prepared = 1.  The embedding
+ * table, norms, static taps and codebooks stay where they are.  Asynchronous on `stream`. */
 int dflash2_prepare_weights(const dflash2_config *cfg, const dflash2_weights *src, void *dst,
                             size_t dst_bytes, dflash2_weights *out, void *stream);
 
