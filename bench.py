@@ -274,8 +274,13 @@ def main():
     L_after = [int(v) + Bk for v in inputs.context_lengths(wl)]
     byt = accounting.step_bytes(dims, L_after, [Bk] * B)
     hbm, peak_kind = peaks()
-    lm_b = accounting.lmhead_bytes(dims, B * D)
-    lm_gbs = lm_b / (lm_ms * 1e-3) / 1e9
+    nk = dr.step_kernels()
+    if nk == 1:  # the whole step is one persistent kernel: its bytes are the step's
+        rk_name, rk_bytes = "k_step_persistent (whole block step, one cooperative launch)", byt["total"]
+    else:
+        rk_name = "k_slmhead / k_lmhead_topk (LM head + streaming top-16 + selector projection)"
+        rk_bytes = accounting.lmhead_bytes(dims, B * D)
+    rk_gbs = rk_bytes / (lm_ms * 1e-3) / 1e9
     value = ws / (ms_max * 1e-3)  # draft steps/s over all ranks (one step = a rank's whole batch)
     line = {
         "metric": "DFlash2 draft steps/s (8-token block)",
@@ -297,12 +302,12 @@ def main():
         "step_hbm": {"algorithmic_bytes": byt["total"], "achieved_gbs": byt["total"] / (ms_max * 1e-3) / 1e9,
                      "frac_of_8tbs": byt["total"] / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                      "frac_of_measured": byt["total"] / (ms_max * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind},
-        "roofline": {"kernel": "k_lmhead_topk (LM head + streaming top-16 + selector projection)", "bound": "hbm",
-                     "achieved": lm_gbs, "peak": hbm, "unit": "GB/s", "frac": lm_gbs / hbm, "traffic": None,
-                     "algorithmic_bytes": lm_b, "avg_launch_ms": lm_ms, "peak_kind": peak_kind},
+        "roofline": {"kernel": rk_name, "bound": "hbm",
+                     "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm, "traffic": None,
+                     "algorithmic_bytes": rk_bytes, "avg_launch_ms": lm_ms, "peak_kind": peak_kind},
         "e2e": {"value": ws / (e2e_ms * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": accounting.launches_per_step(dims, B) * K,
+        "gpu_launches": accounting.launches_per_step(dims, B, nk) * K,
         "clocks": clk.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -57,7 +57,7 @@ class Debug(C.Structure):
 
 EXPORTS = ("dflash2_workspace_size", "dflash2_prepared_size", "dflash2_prepare_weights", "dflash2_draft_step",
            "dflash2_draft_step_static", "dflash2_accept", "dflash2_spec_step_host", "dflash2_device_error",
-           "dflash2_strerror")
+           "dflash2_step_kernels", "dflash2_strerror")
 
 _lib = None
 
@@ -86,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.dflash2_spec_step_host.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(KV), C.c_int32] + \
         [C.c_void_p] * 9 + [C.c_void_p, C.c_size_t, C.c_void_p]
     lib.dflash2_device_error.argtypes = [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]
+    lib.dflash2_step_kernels.restype = C.c_int32
+    lib.dflash2_step_kernels.argtypes = [C.POINTER(Config), C.c_int32]
     lib.dflash2_strerror.restype = C.c_char_p
     lib.dflash2_strerror.argtypes = [C.c_int]
     _lib = lib
@@ -203,6 +205,10 @@ class Drafter:
             C.addressof(dev_err), _ptr(self.workspace), self.ws_bytes, _stream(stream))
         check(rc, "spec_step_host")
         return dev_err.value
+
+    def step_kernels(self) -> int:
+        """Kernels one draft_step launches (1: the whole step is one persistent kernel)."""
+        return int(self.lib.dflash2_step_kernels(C.byref(self.cfg), self.batch))
 
     def device_error(self, stream=None) -> int:
         out = C.c_int32(0)

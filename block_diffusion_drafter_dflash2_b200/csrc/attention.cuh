@@ -40,18 +40,16 @@ DEVI void attn_geometry(const AttnParams& p, int b, long long& Lb, long long& cs
   nact = (int)((Lb - cs + kAttnKeys - 1) / kAttnKeys);
 }
 
-template <int MT>  // 16-row query tiles per CTA (= warps)
-__global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
+// One chunk item (request b, kv head kvh, chunk c) processed by the first NTHR threads of the CTA
+// (named barrier 1); warps 0..MT-1 do the math.  buf: (MT*16 + 2*64) * 272 bytes of shared memory;
+// bar: an initialised mbarrier whose phase `phase` tracks across items; row_ok: 64 ints.
+// Returns without touching anything when the chunk lies outside the request's window.
+template <int MT, int NTHR>
+DEVI void attn_item(const AttnParams& p, int c, int kvh, int b, uint8_t* buf, uint64_t* bar, uint32_t& phase,
+                    int* row_ok) {
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(buf);
   uint16_t* Ks = Qs + MT * 16 * kAttnStride;
   uint16_t* Vs = Ks + kAttnKeys * kAttnStride;
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ int row_ok[kAttnKeys];
-
-  pdl_trigger();
-  pdl_wait();
-  const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.nq / p.nkv, nqv = G * p.Bk;
   long long Lb, cs;
@@ -60,33 +58,31 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
   const bool blk = c == p.NC;
   if (!blk && c >= nact) return;
   const long long key0 = cs + (long long)c * kAttnKeys;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
+  consumers_sync<NTHR>();  // the buffer is free (previous item done)
   // queries of this (request, kv head): vector qv = t*G + gi -> head kvh*G + gi of block row t.
   // Every thread issues its 8 loads before any store (no load->store chains).
   {
-    uint4 qv8[8];
+    constexpr int kQv = MT * 16 * 16;  // 16-byte vectors of the query tile
+    constexpr int kPer = (kQv + NTHR - 1) / NTHR;
+    uint4 qv8[kPer];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = threadIdx.x + k * blockDim.x, qv = i >> 4, v = i & 15;
+    for (int k = 0; k < kPer; ++k) {
+      const int i = threadIdx.x + k * NTHR, qv = i >> 4, v = i & 15;
       qv8[k] = make_uint4(0, 0, 0, 0);
-      if (qv < nqv) {
+      if (i < kQv && qv < nqv) {
         const int t = qv / G, gi = qv % G;
-        qv8[k] = *reinterpret_cast<const uint4*>(p.qb + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + v * 8);
+        qv8[k] = __ldcg(reinterpret_cast<const uint4*>(p.qb + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + v * 8));
       }
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = threadIdx.x + k * blockDim.x, qv = i >> 4, v = i & 15;
-      *reinterpret_cast<uint4*>(Qs + qv * kAttnStride + v * 8) = qv8[k];
+    for (int k = 0; k < kPer; ++k) {
+      const int i = threadIdx.x + k * NTHR, qv = i >> 4, v = i & 15;
+      if (i < kQv) *reinterpret_cast<uint4*>(Qs + qv * kAttnStride + v * 8) = qv8[k];
     }
   }
   if (blk) {
     // the block's own keys: Bk rows loaded (4 vectors per thread at most), the rest zero
-    for (int i = threadIdx.x; i < kAttnKeys * 16; i += blockDim.x) {
+    for (int i = threadIdx.x; i < kAttnKeys * 16; i += NTHR) {
       const int u = i >> 4, v = i & 15;
       if (u >= p.Bk) {
         *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = make_uint4(0, 0, 0, 0);
@@ -94,19 +90,20 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
       }
     }
     {
-      uint4 kv4[8], vv4[8];  // Bk <= 16 rows x 16 vectors over >= 32 threads
+      constexpr int kPerK = (16 * 16 + NTHR - 1) / NTHR;  // Bk <= 16 rows x 16 vectors
+      uint4 kv4[kPerK], vv4[kPerK];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int i = threadIdx.x + k * blockDim.x, u = i >> 4, v = i & 15;
+      for (int k = 0; k < kPerK; ++k) {
+        const int i = threadIdx.x + k * NTHR, u = i >> 4, v = i & 15;
         if (u < p.Bk) {
           const size_t off = ((size_t)(b * p.Bk + u) * p.nkv + kvh) * kHeadDim + v * 8;
-          kv4[k] = *reinterpret_cast<const uint4*>(p.kb + off);
-          vv4[k] = *reinterpret_cast<const uint4*>(p.vb + off);
+          kv4[k] = __ldcg(reinterpret_cast<const uint4*>(p.kb + off));
+          vv4[k] = __ldcg(reinterpret_cast<const uint4*>(p.vb + off));
         }
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int i = threadIdx.x + k * blockDim.x, u = i >> 4, v = i & 15;
+      for (int k = 0; k < kPerK; ++k) {
+        const int i = threadIdx.x + k * NTHR, u = i >> 4, v = i & 15;
         if (u < p.Bk) {
           *reinterpret_cast<uint4*>(Ks + u * kAttnStride + v * 8) = kv4[k];
           *reinterpret_cast<uint4*>(Vs + u * kAttnStride + v * 8) = vv4[k];
@@ -114,10 +111,10 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
       }
     }
     if (threadIdx.x < kAttnKeys) row_ok[threadIdx.x] = threadIdx.x < p.Bk;
-    __syncthreads();
+    consumers_sync<NTHR>();
   } else {
-    __syncthreads();  // barrier initialised
     if (warp == 0) {
+      fence_proxy_async();  // cache rows written by earlier kernels/CTAs are read by the bulk copies
       int ok[2];
       int32_t pg[2];
 #pragma unroll
@@ -135,7 +132,7 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
         row_ok[kk] = ok[h];
       }
       const int nvalid = __popc(__ballot_sync(0xffffffffu, ok[0])) + __popc(__ballot_sync(0xffffffffu, ok[1]));
-      if (lane == 0) mbar_expect_tx(&bar, (uint32_t)nvalid * 2u * kHeadDim * 2u);
+      if (lane == 0) mbar_expect_tx(bar, (uint32_t)nvalid * 2u * kHeadDim * 2u);
       __syncwarp();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -143,8 +140,8 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
         if (ok[h]) {
           const long long j = key0 + kk;
           const size_t off = (((size_t)pg[h] * p.nkv + kvh) * kPage + j % kPage) * kHeadDim;
-          bulk_g2s(Ks + kk * kAttnStride, p.kc + off, kHeadDim * 2, &bar);
-          bulk_g2s(Vs + kk * kAttnStride, p.vc + off, kHeadDim * 2, &bar);
+          bulk_g2s(Ks + kk * kAttnStride, p.kc + off, kHeadDim * 2, bar);
+          bulk_g2s(Vs + kk * kAttnStride, p.vc + off, kHeadDim * 2, bar);
         } else {
           uint4* kr = reinterpret_cast<uint4*>(Ks + kk * kAttnStride);
           uint4* vr = reinterpret_cast<uint4*>(Vs + kk * kAttnStride);
@@ -152,12 +149,15 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
         }
       }
     }
-    __syncthreads();
-    if (!mbar_wait_bounded(&bar, 0)) {
+    consumers_sync<NTHR>();
+    const bool ok = mbar_wait_sleep_bounded(bar, phase);
+    phase ^= 1u;
+    if (!ok) {
       if (threadIdx.x == 0) set_err(p.err, DFLASH2_DEV_TIMEOUT);
       return;
     }
   }
+  if (warp >= MT) return;
 
   // ---- S = Q K^T for this warp's 16 query vectors x 64 keys ----
   const int g = lane >> 2, t4 = lane & 3;
@@ -245,15 +245,27 @@ __global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
   }
 }
 
+
+template <int MT>  // 16-row query tiles per CTA (= warps)
+__global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int row_ok[kAttnKeys];
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  uint32_t phase = 0;
+  attn_item<MT, MT * 32>(p, blockIdx.x, blockIdx.y, blockIdx.z, smem, &bar, phase, row_ok);
+}
+
 // One warp per (request, kv head, query vector): merge the chunk partials -> o bf16 [Mb][nq][128].
 // Lanes read the chunks' (m, l) in parallel; the weighted sum streams 16-byte rows.
-__global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
-  __shared__ float wsh[4][64];
-  pdl_trigger();
-  pdl_wait();
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
-  const int qv = blockIdx.x * (blockDim.x >> 5) + wi;
-  const int kvh = blockIdx.y, b = blockIdx.z;
+DEVI void attn_combine_warp(const AttnParams& p, uint16_t* __restrict__ ob, int qv, int kvh, int b, float* wsh) {
+  const int lane = threadIdx.x & 31;
   const int G = p.nq / p.nkv;
   if (qv >= G * p.Bk) return;
   long long Lb, cs;
@@ -271,7 +283,7 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
     l[h] = 0.f;
     if (i < nc) {
       const int c = i < nact ? i : p.NC;
-      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + ((base + c) * p.QVP + qv) * 2);
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((base + c) * p.QVP + qv) * 2));
       m[h] = ml.x;
       l[h] = ml.y;
     }
@@ -284,7 +296,7 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
   for (int h = 0; h < 2; ++h) {
     const int i = lane + 32 * h;
     const float w = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - M);
-    if (i < 64) wsh[wi][i] = w;
+    if (i < 64) wsh[i] = w;
     L += w * l[h];
   }
   L = warp_sum(L);
@@ -293,8 +305,8 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
 #pragma unroll 8
   for (int i = 0; i < nc; ++i) {
     const int c = i < nact ? i : p.NC;
-    const float w = wsh[wi][i];
-    const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((base + c) * p.QVP + qv) * kHeadDim + lane * 4);
+    const float w = wsh[i];
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((base + c) * p.QVP + qv) * kHeadDim + lane * 4));
     acc.x += w * v.x;
     acc.y += w * v.y;
     acc.z += w * v.z;
@@ -304,6 +316,14 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
   const int t = qv / G, gi = qv % G;
   uint16_t* dst = ob + ((size_t)(b * p.Bk + t) * p.nq + kvh * G + gi) * kHeadDim + lane * 4;
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf2(acc.x * inv, acc.y * inv), pack_bf2(acc.z * inv, acc.w * inv));
+}
+
+__global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
+  __shared__ float wsh[4][64];
+  pdl_trigger();
+  pdl_wait();
+  const int wi = threadIdx.x >> 5;
+  attn_combine_warp(p, ob, blockIdx.x * (blockDim.x >> 5) + wi, blockIdx.y, blockIdx.z, wsh[wi]);
 }
 
 }  // namespace dfl

@@ -141,6 +141,12 @@ DEVI bool better(float a, int ia, float b, int ib) { return a > b || (a == b && 
 DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Named barrier 1 over the first NTHR threads of the CTA.
+template <int NTHR>
+DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NTHR) : "memory"); }
+// Order this thread's view of global memory before its later bulk (async-proxy) copies.
+DEVI void fence_proxy_async() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 DEVI void set_err(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }

@@ -1,6 +1,7 @@
 // C ABI of the DFlash 2 drafter block step (include/dflash2.h): argument
 // validation, workspace layout and the launch sequence of the sm_100a kernels.
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -11,6 +12,7 @@
 #include "gemv.cuh"
 #include "lmhead.cuh"
 #include "rowops.cuh"
+#include "persist.cuh"
 #include "selector.cuh"
 #include "stream.cuh"
 
@@ -28,6 +30,9 @@ struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
   bool q4;
   GemvPlan fc, dc, qkv, o, gu, dn;
+  GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
+  bool persistent;
+  size_t psmem, off_cfv, off_cfi, off_ssp;
   int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
   bool lm_stream;
   size_t lm_smem;
@@ -55,7 +60,7 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   g.NT = g.R / 8;
   g.mgroups = g.R == 64 ? (rows + 63) / 64 : 1;
   g.groups = (tiles + kConsumers - 1) / kConsumers;
-  const int unitK = q4 ? 256 : 128, slot = q4 ? Ring<true>::kSlot : Ring<false>::kSlot;
+  const int unitK = q4 ? Ring<true>::kUnitK : Ring<false>::kUnitK, slot = q4 ? Ring<true>::kSlot : Ring<false>::kSlot;
   const int ns = q4 ? Ring<true>::kNS : Ring<false>::kNS;
   g.U = K / unitK;
   g.W = (long long)g.groups * g.mgroups * g.U;
@@ -67,6 +72,25 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
   g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
+  return g;
+}
+
+// Plan of one streamed product inside the persistent step: every SM takes part (P = #SMs) and the
+// activations live in the fixed staging region of that kernel.
+GemvPlan plan_gemv_persistent(int tiles, int rows, int K, bool q4, int nsm) {
+  GemvPlan g;
+  g.R = rows <= 8 ? 8 : 16;
+  g.NT = g.R / 8;
+  g.mgroups = 1;
+  g.groups = (tiles + kConsumers - 1) / kConsumers;
+  const int unitK = q4 ? 256 : 64;
+  g.U = K / unitK;
+  g.W = (long long)g.groups * g.U;
+  g.P = (int)std::min<long long>(nsm, g.W);  // every CTA in [0, P) owns at least one unit
+  g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
+  g.kc_units = std::max(1, std::min(g.U, (kPXBytes - 64 * g.R) / (g.R * unitK * 2)));
+  if (g.kc_units < g.U && g.kc_units > 1) g.kc_units &= ~1;  // whole slots (two units each) per chunk
+  g.smem = 0;
   return g;
 }
 
@@ -126,6 +150,19 @@ Plan make_plan(const dflash2_config* c, int B) {
     p.lm_nparts = std::min(p.nsm, (lm_tiles + kWarps - 1) / kWarps);
   }
   p.lm_passes = (p.lm_rows + p.lm_rows_per_pass - 1) / p.lm_rows_per_pass;
+  // one request with a block of <= 8: the whole step runs as one persistent launch
+  p.persistent = B == 1 && p.Bk <= 8 && p.QVP == 32 && 8 * (p.H * 2 + 64) <= kPXBytes &&
+                 (size_t)(p.MT * 16 + 2 * kAttnKeys) * kAttnStride * 2 <= (size_t)kPXBytes;
+  p.psmem = (size_t)kPNS * kPSlot + kPXBytes + (size_t)kGemvConsumers * 128 * 8 + (size_t)kConsumers * 32 * 8 * 4 +
+            (size_t)kGemvConsumers * 64 * 4;
+  if (p.persistent) {
+    p.pfc = plan_gemv_persistent(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
+    p.pdc = plan_gemv_persistent((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
+    p.pqkv = plan_gemv_persistent((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
+    p.po = plan_gemv_persistent(p.H / 16, p.Mb, p.HQ, p.q4, p.nsm);
+    p.pgu = plan_gemv_persistent(2 * p.F / 16, p.Mb, p.H, p.q4, p.nsm);
+    p.pdn = plan_gemv_persistent(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
+  }
 
   auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.max_pieces * rows * ldo * 4; };
   size_t part = 0;
@@ -135,6 +172,14 @@ Plan make_plan(const dflash2_config* c, int B) {
   part = std::max(part, part_bytes(p.o, p.Mb, p.H));
   part = std::max(part, part_bytes(p.gu, p.Mb, 2 * p.F));
   part = std::max(part, part_bytes(p.dn, p.Mb, p.H));
+  if (p.persistent) {
+    part = std::max(part, part_bytes(p.pfc, p.Mb, p.H));
+    part = std::max(part, part_bytes(p.pdc, p.Mb, p.H / 2));
+    part = std::max(part, part_bytes(p.pqkv, 2 * p.Mb, p.HQ + 2 * p.HKV));
+    part = std::max(part, part_bytes(p.po, p.Mb, p.H));
+    part = std::max(part, part_bytes(p.pgu, p.Mb, 2 * p.F));
+    part = std::max(part, part_bytes(p.pdn, p.Mb, p.H));
+  }
 
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -157,8 +202,12 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_ob = take((size_t)p.Mb * p.HQ * 2);
   p.off_act = take((size_t)p.Mb * p.F * 2);
   p.off_hn = take((size_t)std::max(p.lm_rows, 1) * p.H * 2);
-  p.off_cv = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
-  p.off_ci = take((size_t)p.lm_nparts * p.lm_rows * kTopK * 4);
+  const size_t nlists = (size_t)std::max(p.lm_nparts, p.persistent ? p.nsm : 0);
+  p.off_cv = take(nlists * p.lm_rows * kTopK * 4);
+  p.off_ci = take(nlists * p.lm_rows * kTopK * 4);
+  p.off_cfv = take((size_t)p.lm_rows * kTopK * 4);
+  p.off_cfi = take((size_t)p.lm_rows * kTopK * 4);
+  p.off_ssp = take((size_t)(p.H / 128) * 4 * p.Mb * 4);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
@@ -171,7 +220,7 @@ Plan make_plan(const dflash2_config* c, int B) {
     acc += nctr(*lp[i]);
   }
   p.ctr_per_layer = acc;
-  p.ctr_total = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;
+  p.ctr_total = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer + 1;  // + the persistent step's grid barrier
   p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
   p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
@@ -232,9 +281,8 @@ struct Epi {
   QkvEpi qkv{};
 };
 
-cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X,
-                        int ldx, int rows, float* part, int ldo, int out_rows, int* counters, const Epi& e, int* err,
-                        cudaStream_t s) {
+SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X, int ldx,
+                         int rows, float* part, int ldo, int out_rows, int* counters, const Epi& e, int* err) {
   SGemvParams prm;
   memset(&prm, 0, sizeof(prm));
   for (int i = 0; i < nseg; ++i) prm.seg[i] = segs[i];
@@ -259,6 +307,13 @@ cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nse
   prm.F = e.F;
   prm.qkv = e.qkv;
   prm.err = err;
+  return prm;
+}
+
+cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X,
+                        int ldx, int rows, float* part, int ldo, int out_rows, int* counters, const Epi& e, int* err,
+                        cudaStream_t s) {
+  const SGemvParams prm = sgemv_params(g, segs, nseg, paired, X, ldx, rows, part, ldo, out_rows, counters, e, err);
   switch (g.NT * 2 + (q4 ? 1 : 0)) {
     case 2: return launch_sgemv_t<1, false>(g, prm, s);
     case 3: return launch_sgemv_t<1, true>(g, prm, s);
@@ -339,6 +394,31 @@ void* static_scratch(cudaError_t* err) {
   return p;
 }
 
+// The persistent step needs its shared memory opted in and one CTA of it resident on every SM
+// (cooperative launch); checked once per device.
+bool persistent_ready(const Plan& P) {
+  const char* env = getenv("DFLASH2_PERSISTENT");  // opt in with "1" (the kernel sequence is the default)
+  if (!env || env[0] != '1') return false;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> state[kMaxDevices];  // 0 unknown, 1 ready, 2 not available
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  int st = state[dev].load(std::memory_order_acquire);
+  if (st == 0) {
+    int coop = 0, nb = 0;
+    st = 2;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
+        cudaFuncSetAttribute(k_step_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.psmem) ==
+            cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_step_persistent, kPThreads, P.psmem) == cudaSuccess &&
+        nb >= 1)
+      st = 1;
+    cudaGetLastError();
+    state[dev].store(st, std::memory_order_release);
+  }
+  return st == 1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -380,7 +460,7 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
     if (q4)
       k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K, pl);
     else
-      k_bf16_prepare<<<dim3(K / 128, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K, pl);
+      k_bf16_prepare<<<dim3(K / 64, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K, pl);
   };
   auto bytes = [&](int N, int K, bool q4) { return q4 ? (size_t)N * K / kUnit * 144 : (size_t)N * K * 2; };
   auto prep = [&](const void* w, int N, int K, bool q4) -> const void* {
@@ -450,11 +530,196 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   float* zbuf = at<float>(ws, P.off_z);
   const int H = P.H, Mb = P.Mb;
   const size_t hbytes = (size_t)Mb * H * 4;
+  AttnParams ap{};
+  ap.qb = qb;
+  ap.kb = kb;
+  ap.vb = vb;
+  ap.page_table = kv->page_table;
+  ap.max_pages = kv->max_pages;
+  ap.num_pages = kv->num_pages;
+  ap.seq_len = kv->seq_len;
+  ap.n_new = in->n_new;
+  ap.Bk = P.Bk;
+  ap.nq = c->n_q;
+  ap.nkv = c->n_kv;
+  ap.W = c->window;
+  ap.NC = P.NC;
+  ap.QVP = P.QVP;
+  ap.part_o = at<float>(ws, P.off_ao);
+  ap.part_ml = at<float>(ws, P.off_aml);
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
+  ap.err = err;
 
   float* gbuf = at<float>(ws, P.off_g);
   int* ctr = at<int>(ws, P.off_ctr);
   CK(cudaMemsetAsync(err, 0, 4, s));
   CK(cudaMemsetAsync(ctr, 0, P.ctr_total * 4, s));
+  if (P.persistent && persistent_ready(P)) {
+    if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
+    StepParams S;
+    memset(&S, 0, sizeof(S));
+    S.layers = c->layers;
+    S.Bk = P.Bk;
+    S.Mb = Mb;
+    S.H = H;
+    S.D = P.D;
+    S.V = P.V;
+    S.R = P.R;
+    S.eps = c->rms_eps;
+    S.block_tokens = in->block_tokens;
+    S.embed = w->embed;
+    S.fc_norm = w->fc_norm;
+    S.fcout = xf;
+    S.ctx = ctx;
+    S.n_new = in->n_new;
+    S.ap = ap;
+    S.ob = ob;
+    S.head = (const uint8_t*)w->lm_head;
+    S.final_norm = w->final_norm;
+    S.z = zbuf;
+    S.cand_val = at<float>(ws, P.off_cv);
+    S.cand_id = at<int32_t>(ws, P.off_ci);
+    S.cand_fval = at<float>(ws, P.off_cfv);
+    S.cand_fid = at<int32_t>(ws, P.off_cfi);
+    S.h = h;
+    S.ssp = at<float>(ws, P.off_ssp);
+    S.gbar = reinterpret_cast<unsigned*>(ctr + P.ctr_total - 1);
+    S.err = err;
+    S.dbg_hidden = dbg ? dbg->hidden : nullptr;
+    S.dbg_ctx = dbg ? dbg->ctx : nullptr;
+    S.dbg_final_h = dbg ? dbg->final_h : nullptr;
+    {
+      SelParams& sp = S.sel;
+      sp.cand_val = S.cand_fval;
+      sp.cand_id = S.cand_fid;
+      sp.nparts = 1;
+      sp.rows_total = P.D;
+      sp.z = zbuf;
+      sp.R = P.R;
+      sp.V = P.V;
+      sp.Bk = P.Bk;
+      sp.cb_a = w->cb_a;
+      sp.cb_b = w->cb_b;
+      sp.block_tokens = in->block_tokens;
+      sp.out_path = out_path;
+      sp.out_scores = out_scores;
+      sp.seq_len = kv->seq_len;
+      sp.n_new = in->n_new;
+      sp.dbg_cand = dbg ? dbg->cand : nullptr;
+      sp.dbg_logit = dbg ? dbg->cand_logit : nullptr;
+      sp.err = err;
+      if (sp.dbg_cand && !sp.dbg_logit) sp.dbg_cand = nullptr;
+    }
+    // A2: fc over the taps (operand copied), output to xf
+    {
+      GemvSeg seg{(const uint8_t*)w->fc, H / 16, Mb, 0};
+      Epi e;
+      e.mode = EPI_STORE;
+      e.y = xf;
+      e.ldy = H;
+      S.fc.g = sgemv_params(P.pfc, &seg, 1, false, in->taps, P.T * H, Mb, part, H, Mb, ctr, e, err);
+      S.fc.P = P.pfc.P;
+      S.fc.q4 = P.q4;
+      S.fc.stage = STG_COPY;
+    }
+    for (int l = 0; l < c->layers; ++l) {
+      const dflash2_layer_weights& L = w->layer[l];
+      int* lctr = ctr + P.ctr_fc + (size_t)l * P.ctr_per_layer;
+      PLayer& Q = S.L[l];
+      Q.kc = kv->k[l];
+      Q.vc = kv->v[l];
+      {  // A3a: g = W_dc RMSNorm(h; ln1), operand computed in the staging
+        GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
+        Epi e;
+        e.mode = EPI_STORE;
+        e.y = gbuf;
+        e.ldy = H / 2;
+        Q.dc.g = sgemv_params(P.pdc, &seg, 1, false, nullptr, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err);
+        Q.dc.P = P.pdc.P;
+        Q.dc.q4 = 0;
+        Q.dc.stage = STG_NORM;
+        Q.dc.nw = L.ln1;
+      }
+      {  // A3b+c: q|k|v of [dynconv rows; context rows], the dynconv computed in the staging
+        const int ldo = P.HQ + 2 * P.HKV;
+        GemvSeg segs[3] = {{(const uint8_t*)L.wq, P.HQ / 16, Mb, 0},
+                           {(const uint8_t*)L.wk, P.HKV / 16, 2 * Mb, P.HQ},
+                           {(const uint8_t*)L.wv, P.HKV / 16, 2 * Mb, P.HQ + P.HKV}};
+        Epi e;
+        e.mode = EPI_QKV;
+        QkvEpi& q = e.qkv;
+        q.qn = L.qn;
+        q.kn = L.kn;
+        q.eps = c->rms_eps;
+        q.log2_theta = log2((double)c->rope_theta);
+        q.Bk = P.Bk;
+        q.nq = c->n_q;
+        q.nkv = c->n_kv;
+        q.Mb = Mb;
+        q.seq_len = kv->seq_len;
+        q.n_new = in->n_new;
+        q.qb = qb;
+        q.kb = kb;
+        q.vb = vb;
+        q.kc = kv->k[l];
+        q.vc = kv->v[l];
+        q.page_table = kv->page_table;
+        q.max_pages = kv->max_pages;
+        q.num_pages = kv->num_pages;
+        q.err = err;
+        Q.qkv.g = sgemv_params(P.pqkv, segs, 3, false, nullptr, H, 2 * Mb, part, ldo, 2 * Mb, lctr + P.ctr_layer[1], e, err);
+        Q.qkv.P = P.pqkv.P;
+        Q.qkv.q4 = P.q4;
+        Q.qkv.stage = STG_DYNCONV;
+        Q.qkv.nw = L.ln1;
+        Q.qkv.gdc = gbuf;
+        Q.qkv.s0 = L.dc_s0;
+        Q.qkv.s1 = L.dc_s1;
+        Q.qkv.ctx = ctx;
+      }
+      {  // A3e: h += W_o o
+        GemvSeg seg{(const uint8_t*)L.wo, H / 16, Mb, 0};
+        Epi e;
+        e.mode = EPI_RESID;
+        e.y = h;
+        e.ldy = H;
+        Q.o.g = sgemv_params(P.po, &seg, 1, false, ob, P.HQ, Mb, part, H, Mb, lctr + P.ctr_layer[2], e, err);
+        Q.o.g.ssp = S.ssp;  // sums of squares of the new h for the gate/up RMSNorm
+        Q.o.g.ssp_rows = Mb;
+        Q.o.P = P.po.P;
+        Q.o.q4 = P.q4;
+        Q.o.stage = STG_COPY;
+      }
+      {  // A3f: act = SwiGLU of gate|up over RMSNorm(h; ln2) (computed in the staging); h += W_d act
+        GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wg, P.F / 16, Mb, P.F}};
+        Epi e;
+        e.mode = EPI_SWIGLU;
+        e.act = act;
+        e.F = P.F;
+        Q.gu.g = sgemv_params(P.pgu, segs, 2, true, nullptr, H, Mb, part, 2 * P.F, Mb, lctr + P.ctr_layer[3], e, err);
+        Q.gu.P = P.pgu.P;
+        Q.gu.q4 = P.q4;
+        Q.gu.stage = STG_NORM;
+        Q.gu.nw = L.ln2;
+        GemvSeg seg{(const uint8_t*)L.wd, H / 16, Mb, 0};
+        Epi e2;
+        e2.mode = EPI_RESID;
+        e2.y = h;
+        e2.ldy = H;
+        Q.dn.g = sgemv_params(P.pdn, &seg, 1, false, act, P.F, Mb, part, H, Mb, lctr + P.ctr_layer[4], e2, err);
+        Q.dn.g.ssp = S.ssp;  // ... for the next layer's RMSNorm or the final norm
+        Q.dn.g.ssp_rows = Mb;
+        Q.dn.P = P.pdn.P;
+        Q.dn.q4 = P.q4;
+        Q.dn.stage = STG_COPY;
+      }
+    }
+    void* args[] = {&S};
+    CK(cudaLaunchCooperativeKernel((const void*)k_step_persistent, dim3(P.nsm), dim3(kPThreads), args, P.psmem, s));
+    if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
+    if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
+    return DFLASH2_OK;
+  }
   // A1: block rows from the shared embedding table
   CK(launch_pdl(k_embed, dim3(Mb), dim3(256), 0, s, in->block_tokens, w->embed, h, H, P.V, err));
   if (dbg && dbg->hidden) CK(cudaMemcpyAsync(dbg->hidden, h, hbytes, cudaMemcpyDeviceToDevice, s));
@@ -481,25 +746,6 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     if (dbg && dbg->ctx) CK(cudaMemcpyAsync(dbg->ctx, ctx, (size_t)Mb * H * 2, cudaMemcpyDeviceToDevice, s));
   }
 
-  AttnParams ap{};
-  ap.qb = qb;
-  ap.kb = kb;
-  ap.vb = vb;
-  ap.page_table = kv->page_table;
-  ap.max_pages = kv->max_pages;
-  ap.num_pages = kv->num_pages;
-  ap.seq_len = kv->seq_len;
-  ap.n_new = in->n_new;
-  ap.Bk = P.Bk;
-  ap.nq = c->n_q;
-  ap.nkv = c->n_kv;
-  ap.W = c->window;
-  ap.NC = P.NC;
-  ap.QVP = P.QVP;
-  ap.part_o = at<float>(ws, P.off_ao);
-  ap.part_ml = at<float>(ws, P.off_aml);
-  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
-  ap.err = err;
 
   for (int l = 0; l < c->layers; ++l) {
     const dflash2_layer_weights& L = w->layer[l];
@@ -751,6 +997,15 @@ int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, co
   if (dev_err) CK(cudaMemcpyAsync(dev_err, at<void>(ws, P.off_err), 4, cudaMemcpyDeviceToHost, s));
   CK(cudaStreamSynchronize(s));
   return DFLASH2_OK;
+}
+
+int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
+  if (!cfg_ok(c) || batch < 1) return 0;
+  const Plan P = make_plan(c, batch);
+  if (P.persistent && persistent_ready(P)) return 1;
+  // embed, fc GEMV, fc norm | per layer: norm, W_dc GEMV, dynconv, QKV GEMV, attention, combine,
+  // W_o GEMV, norm, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector
+  return 3 + 10 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 1;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

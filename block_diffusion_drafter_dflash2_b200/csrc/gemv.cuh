@@ -106,13 +106,13 @@ DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8
   }
 }
 
-// bf16 weights: one 128-wide K step = 8 16-byte vectors per lane (rows g, g+8; 4 sub-blocks of 32).
-template <int NT>
-DEVI void bf16_step(const uint4 (&w)[8], const uint8_t* Xs, int stride, int kbyte, int ntact, float (&acc)[NT][4],
+// bf16 weights: one K step of NJ 32-wide sub-blocks = 2*NJ 16-byte vectors per lane (rows g, g+8).
+template <int NT, int NJ>
+DEVI void bf16_step(const uint4 (&w)[2 * NJ], const uint8_t* Xs, int stride, int kbyte, int ntact, float (&acc)[NT][4],
                     int lane) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < NJ; ++j) {
     const uint4 u = w[2 * j], v = w[2 * j + 1];
     const uint32_t a0[4] = {u.x, v.x, u.y, v.y};
     const uint32_t a1[4] = {u.z, v.z, u.w, v.w};
@@ -216,15 +216,15 @@ __global__ void k_q4k_prepare(const uint8_t* __restrict__ src, uint8_t* __restri
   }
 }
 
-// Canonical bf16 [N][K] -> prepared tiles (group records of 8 x 4096 B per 128-wide K step): for each
+// Canonical bf16 [N][K] -> prepared tiles (group records of 8 x 2048 B per 64-wide K step): for each
 // 32-wide sub-block j, 512 bytes of lane (g, t)'s W[row g][32j + 8t ..], then 512 bytes for row g + 8.
 __global__ void k_bf16_prepare(const uint16_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K,
                                PrepPlace pl) {
-  const int S = K / 128, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x, g = lane >> 2, t = lane & 3;
-  uint8_t* out = dst + prep_offset(pl, T, s, S, 4096);
+  const int S = K / 64, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x, g = lane >> 2, t = lane & 3;
+  uint8_t* out = dst + prep_offset(pl, T, s, S, 2048);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const size_t k = (size_t)s * 128 + j * 32 + t * 8;
+  for (int j = 0; j < 2; ++j) {
+    const size_t k = (size_t)s * 64 + j * 32 + t * 8;
     *reinterpret_cast<uint4*>(out + j * 1024 + lane * 16) =
         *reinterpret_cast<const uint4*>(src + (size_t)(T * 16 + g) * K + k);
     *reinterpret_cast<uint4*>(out + j * 1024 + 512 + lane * 16) =

@@ -68,16 +68,16 @@ __global__ void __launch_bounds__(kWarps * 32) k_lmhead_topk(LmParams p) {
   const int vt = p.V / 16, total = vt + p.R / 16;
   const int wg = blockIdx.x * kWarps + warp, nw = gridDim.x * kWarps;
   const int ntiles = wg < total ? (total - wg + nw - 1) / nw : 0;
-  const int spt = H / 128;  // 128-wide K steps per tile
+  const int spt = H / 64;  // 64-wide K steps per tile
   const int nit = ntiles * spt;
   const int ntact = (p.rows + 7) >> 3;
 
-  // prepared bf16 [lm_head; sel_proj]: 4096 bytes per (tile, 128-wide step), 8 tiles interleaved per group
-  auto load = [&](uint4 (&w)[8], int it) {
+  // prepared bf16 [lm_head; sel_proj]: 2048 bytes per (tile, 64-wide step), 8 tiles interleaved per group
+  auto load = [&](uint4 (&w)[4], int it) {
     const int tile = wg + (it / spt) * nw;
-    const uint8_t* b = p.W + (((size_t)(tile >> 3) * spt + it % spt) * 8 + (tile & 7)) * 4096 + lane * 16;
+    const uint8_t* b = p.W + (((size_t)(tile >> 3) * spt + it % spt) * 8 + (tile & 7)) * 2048 + lane * 16;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 2; ++j) {
       w[2 * j] = ldg_stream(b + j * 1024);
       w[2 * j + 1] = ldg_stream(b + j * 1024 + 512);
     }
@@ -129,14 +129,14 @@ __global__ void __launch_bounds__(kWarps * 32) k_lmhead_topk(LmParams p) {
   };
 
   if (nit > 0) {
-    uint4 wa[8], wb[8];
+    uint4 wa[4], wb[4];
     load(wa, 0);
     if (1 < nit) load(wb, 1);
     for (int it = 0; it < nit; it += 2) {
       {
-        const int kbyte = (it % spt) * 256;
+        const int kbyte = (it % spt) * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
           const uint4 u = wa[2 * j], v = wa[2 * j + 1];
           const uint32_t a0[4] = {u.x, v.x, u.y, v.y}, a1[4] = {u.z, v.z, u.w, v.w};
 #pragma unroll
@@ -152,9 +152,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_lmhead_topk(LmParams p) {
         if ((it % spt) == spt - 1) finish_tile(it);
       }
       if (it + 1 < nit) {
-        const int kbyte = ((it + 1) % spt) * 256;
+        const int kbyte = ((it + 1) % spt) * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
           const uint4 u = wb[2 * j], v = wb[2 * j + 1];
           const uint32_t a0[4] = {u.x, v.x, u.y, v.y}, a1[4] = {u.z, v.z, u.w, v.w};
 #pragma unroll

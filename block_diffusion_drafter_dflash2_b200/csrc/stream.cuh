@@ -13,11 +13,11 @@
 //
 // Prepared layouts (made by dflash2_prepare_weights, values unchanged): the
 // 8 tiles of a column group are interleaved per K unit, so one bulk copy moves
-// a whole group's unit (18 KB of Q4_K, 32 KB of bf16):
+// a whole group's unit (18 KB of Q4_K, 16 KB of bf16):
 //  * Q4_K: per tile and 256-wide super-block a 2304-byte record: 2048 bytes of
 //    4-bit codes in mma A-fragment order, then the 16 canonical 16-byte scale
 //    records of the tile's rows (see q4_unit).
-//  * bf16: per tile and 128-wide K step a 4096-byte record: for each 32-wide
+//  * bf16: per tile and 64-wide K step a 2048-byte record: for each 32-wide
 //    sub-block j, 512 bytes holding lane L = (g, t)'s 8 values W[row g][32j + 8t ..]
 //    then 512 bytes for row g + 8.
 //  * gate/up of the MLP are interleaved 4 + 4 tiles per group, so one CTA holds
@@ -49,11 +49,9 @@ struct Ring<true> {
 };
 template <>
 struct Ring<false> {
-  static constexpr int kUnitBytes = 4096, kSlot = 8 * 4096, kNS = 4, kUnitK = 128;
+  static constexpr int kUnitBytes = 2048, kSlot = 8 * 2048, kNS = 8, kUnitK = 64;
 };
 
-template <int NTHR>
-DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NTHR) : "memory"); }
 DEVI void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -79,6 +77,8 @@ struct SGemvParams {
   uint16_t* act;
   int F;
   QkvEpi qkv;
+  float* ssp;         // EPI_RESID: per-row sums of squares of the new rows, or null
+  int ssp_rows;       // row stride of ssp: [column group][quarter][ssp_rows]
   int* err;
 };
 
@@ -162,8 +162,16 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
     const int r = i >> 7, c = col0 + (i & 127);
     const float v = sum_pieces(p, npieces, mz + r, c);
     float* y = p.y + (size_t)(mz + r) * p.ldy + c;
-    if (p.epi == EPI_RESID) *y += v;
-    else *y = v;
+    if (p.epi == EPI_RESID) {
+      const float nv = __ldcg(y) + v;  // L2 read: another CTA may have written it
+      *y = nv;
+      if (p.ssp) {  // sum of squares of this warp's 32 columns of the new row, for the next RMSNorm
+        const float q = warp_sum(nv * nv);
+        if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
+      }
+    } else {
+      *y = v;
+    }
   }
 }
 
@@ -299,18 +307,22 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
             const uint4 sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
+            // the slot is free as soon as its bytes are in registers: release it before the math
+            // so the producer's next copy overlaps the decode
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
             q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane);
           } else {
-            uint4 wv[8];
+            uint4 wv[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
               wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
               wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
             }
-            bf16_step<NT>(wv, Xs, stride, (u - base) * 256, ntact, acc, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            bf16_step<NT, 2>(wv, Xs, stride, (u - base) * 128, ntact, acc, lane);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[slot]);
         }
       }
     }
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
   float* lv_all = reinterpret_cast<float*>(Xs + 8 * stride);          // [warps][8][16]
   int* li_all = reinterpret_cast<int*>(lv_all + kConsumers * 8 * kTopK);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int vt = p.V / 16, total = vt + p.R / 16, S = H / 128;
+  const int vt = p.V / 16, total = vt + p.R / 16, S = H / 64;
   const int ngroups = (total + kConsumers - 1) / kConsumers;
 
   if (threadIdx.x == 0) {
@@ -453,15 +465,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
       ++cnt;
       if (dead) continue;
       const uint8_t* sb = ring + slot * RC::kSlot + warp * RC::kUnitBytes;
-      uint4 wv[8];
+      uint4 wv[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
         wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
       }
-      bf16_step<1>(wv, Xs, stride, s * 256, 1, acc, lane);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (lane == 0) mbar_arrive(&empty[slot]);  // bytes in registers: release before the math
+      bf16_step<1, 2>(wv, Xs, stride, s * 128, 1, acc, lane);
     }
     if (dead || tile >= total) continue;
     if (tile >= vt) {

@@ -130,7 +130,8 @@ typedef struct dflash2_inputs {
  *   LM head's operand); cand: int32 and cand_logit: fp32 [batch*(block-1)][16];
  *   z: fp32 [batch*(block-1)][rank] selector projection.
  * ev_lm_begin / ev_lm_end: cudaEvent_t (as void*) recorded on `stream` around
- *   the LM-head + top-16 kernel. */
+ *   the LM-head + top-16 kernel, or, when the step runs as one persistent kernel
+ *   (dflash2_step_kernels() == 1), around that kernel. */
 typedef struct dflash2_debug {
   float *hidden;
   uint16_t *ctx;
@@ -152,7 +153,7 @@ size_t dflash2_prepared_size(const dflash2_config *cfg);
 /* Repack the streamed matrices of `src` (canonical layouts, device) into `dst`
  * (device, 16-byte aligned, dst_bytes >= dflash2_prepared_size): the 8 tiles of 16 rows
  * of each column group interleaved per K unit (Q4_K: 256-wide super-blocks, codes in
- * mma fragment order; bf16: 128-wide steps), gate and up interleaved 4 + 4 tiles per
+ * mma fragment order; bf16: 64-wide steps), gate and up interleaved 4 + 4 tiles per
  * group, and the output head followed by the selector projection as one matrix padded
  * to whole groups.  Values are not changed: the prepared copy holds the same bits,
  * reordered.  Fills `out` (host struct) with `src`'s pointers except the streamed
@@ -222,6 +223,15 @@ int dflash2_spec_step_host(const dflash2_config *cfg, const dflash2_weights *w, 
 /* Copy the device error word of `workspace` to *out_bits (host) and
  * synchronize `stream`. */
 int dflash2_device_error(const void *workspace, int32_t *out_bits, void *stream);
+
+/* Kernels one dflash2_draft_step call launches for `batch` requests on the
+ * current device (memsets not counted).  A single request with a block of at
+ * most 8 runs as ONE persistent cooperative kernel (one CTA per SM, grid
+ * barriers between dependent operations) when the device supports cooperative
+ * launch and the environment variable DFLASH2_PERSISTENT is "1"; otherwise
+ * the step is a sequence of kernels (about ten per layer).
+ * 0 on an invalid config or batch. */
+int32_t dflash2_step_kernels(const dflash2_config *cfg, int32_t batch);
 
 /* Static description of an error code. */
 const char *dflash2_strerror(int code);

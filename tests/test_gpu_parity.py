@@ -31,6 +31,37 @@ def test_tiny_step_matches_oracle():
     parity.check_accept(run)
 
 
+def test_tiny_single_request_runs_as_one_persistent_kernel(monkeypatch):
+    monkeypatch.setenv("DFLASH2_PERSISTENT", "1")
+    wl = inputs.WORKLOADS["tiny"]
+    w, hw_t, hw = weights_for(wl)
+    run = parity.run_gpu(wl, w, [0])
+    assert run["drafter"].step_kernels() == 1
+    parity.check_request(run, hw_t, hw, 0)
+
+
+def test_tiny_kernel_sequence_matches_oracle(monkeypatch):
+    """The same single request through the multi-kernel sequence (persistent kernel switched off)."""
+    monkeypatch.setenv("DFLASH2_PERSISTENT", "0")
+    wl = inputs.WORKLOADS["tiny"]
+    w, hw_t, hw = weights_for(wl)
+    run = parity.run_gpu(wl, w, [0])
+    assert run["drafter"].step_kernels() > 1
+    parity.check_request(run, hw_t, hw, 0)
+    parity.check_accept(run)
+
+
+def test_tiny_bf16_layers_single_request_block5(monkeypatch):
+    """bf16 layer matrices in the persistent kernel (block 5: 4 drafted rows, ragged query tile)."""
+    import dataclasses
+    monkeypatch.setenv("DFLASH2_PERSISTENT", "1")
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=1, block=5),
+                             batch=1, ctx_lo=77, ctx_hi=77)
+    w, hw_t, hw = weights_for(wl)
+    run = parity.run_gpu(wl, w, [0])
+    parity.check_request(run, hw_t, hw, 0)
+
+
 @pytest.mark.parametrize("n_new", [[0], [1], [3], [8]])
 def test_tiny_ragged_new_rows(n_new):
     """0, 1, some or all block rows carry new context tokens (ragged appends)."""
@@ -84,6 +115,17 @@ def test_steps_chain_and_device_state_advances():
     st["n_new"][0] = 3
     run2 = parity.run_gpu(wl, w, [0], state=st)
     parity.check_request(run2, hw_t, hw, 0)
+
+
+@pytest.mark.slow
+def test_full_b1_persistent(monkeypatch):
+    """The full single-request step as one persistent kernel."""
+    monkeypatch.setenv("DFLASH2_PERSISTENT", "1")
+    wl = inputs.WORKLOADS["full_b1"]
+    w, hw_t, hw = weights_for(wl)
+    run = parity.run_gpu(wl, w, [0])
+    assert run["drafter"].step_kernels() == 1
+    print("full_b1 persistent", parity.check_request(run, hw_t, hw, 0))
 
 
 @pytest.mark.slow
