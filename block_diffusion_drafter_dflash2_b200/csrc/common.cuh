@@ -19,6 +19,7 @@ constexpr int kHeadDim = 128;
 constexpr int kPage = 16;
 constexpr int kAttnKeys = 64;         // cache keys per attention chunk (4 pages)
 constexpr int kAttnStride = 136;      // bf16 elements per staged K/V/Q row (272 B, conflict-free ldmatrix)
+constexpr int kHeadTiles = 16;  // tiles (of 16 rows) per prepared output-head record
 constexpr long long kWaitLimit = 1ll << 26;  // bounded spin on an mbarrier
 
 DEVI float bf2f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -34,6 +35,18 @@ DEVI uint4 ldg_stream(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
+  return r;
+}
+
+// 16-byte load of a ring slot that the slot's release hands back to the copy engine: a volatile
+// shared load, so the compiler neither repeats it after the release (rematerialising the value
+// from memory that may by then hold the next copy) nor moves it past the release.
+DEVI uint4 lds_slot(const void* p) {
+  uint4 r;
+  asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"((uint32_t)__cvta_generic_to_shared(p))
+               : "memory");
   return r;
 }
 

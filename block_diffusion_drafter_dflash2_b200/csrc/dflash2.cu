@@ -140,9 +140,8 @@ Plan make_plan(const dflash2_config* c, int B) {
   if (p.lm_stream) {
     p.lm_NT = 1;
     p.lm_rows_per_pass = 8;
-    p.lm_smem = (size_t)Ring<false>::kNS * Ring<false>::kSlot + (size_t)8 * (p.H * 2 + 64) +
-                (size_t)kConsumers * 8 * kTopK * 8;
-    p.lm_nparts = std::min(p.nsm, (lm_tiles + kConsumers - 1) / kConsumers);
+    p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
+    p.lm_nparts = std::min(p.nsm, (lm_tiles + kHeadTiles - 1) / kHeadTiles);
   } else {
     p.lm_NT = 2;
     p.lm_rows_per_pass = 16;
@@ -435,8 +434,8 @@ size_t dflash2_prepared_size(const dflash2_config* c) {
   const size_t mats = H * c->n_taps * H + c->layers * per_layer;
   const size_t mat_bytes = c->wfmt == 0 ? mats / kUnit * 144 : mats * 2;
   const size_t dyn = (size_t)c->layers * 2 * (H / 4) * H * 2;
-  const size_t head_groups = ((size_t)(c->vocab + c->rank) / 16 + 7) / 8;
-  return mat_bytes + dyn + head_groups * 8 * 16 * H * 2;
+  const size_t head_groups = ((size_t)(c->vocab + c->rank) / 16 + kHeadTiles - 1) / kHeadTiles;
+  return mat_bytes + dyn + head_groups * kHeadTiles * 16 * H * 2;
 }
 
 int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src, void* dst, size_t dst_bytes,
@@ -465,7 +464,7 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
   auto bytes = [&](int N, int K, bool q4) { return q4 ? (size_t)N * K / kUnit * 144 : (size_t)N * K * 2; };
   auto prep = [&](const void* w, int N, int K, bool q4) -> const void* {
     const void* r = d;
-    place(w, N, K, q4, PrepPlace{0, 8, 0});
+    place(w, N, K, q4, PrepPlace{0, 8, 0, 8});
     d += bytes(N, K, q4);
     return r;
   };
@@ -479,20 +478,22 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
     O.wv = prep(S.wv, HKV, H, q4);
     O.wo = prep(S.wo, H, HQ, q4);
     // gate and up interleaved 4 + 4 tiles per group; wu aliases the same buffer
-    place(S.wg, F, H, q4, PrepPlace{0, 4, 0});
-    place(S.wu, F, H, q4, PrepPlace{0, 4, 4});
+    place(S.wg, F, H, q4, PrepPlace{0, 4, 0, 8});
+    place(S.wu, F, H, q4, PrepPlace{0, 4, 4, 8});
     O.wg = O.wu = d;
     d += 2 * bytes(F, H, q4);
     O.wd = prep(S.wd, H, F, q4);
     O.dc_w = (const uint16_t*)prep(S.dc_w, 2 * (H / 4), H, false);
   }
-  // the output head and the selector projection as one [V + R, H] matrix, padded to whole groups
-  const size_t groups = ((size_t)(c->vocab + c->rank) / 16 + 7) / 8, gbytes = (size_t)8 * 16 * H * 2;
+  // the output head and the selector projection as one [V + R, H] matrix in records of 16 tiles
+  // (32 KB per 64-wide step: one bulk copy feeds two 8-tile column groups), padded to whole records
+  const size_t groups = ((size_t)(c->vocab + c->rank) / 16 + kHeadTiles - 1) / kHeadTiles;
+  const size_t gbytes = (size_t)kHeadTiles * 16 * H * 2;
   CK(cudaMemsetAsync(d + (groups - 1) * gbytes, 0, gbytes, s));
-  place(src->lm_head, c->vocab, H, false, PrepPlace{0, 8, 0});
-  place(src->sel_proj, c->rank, H, false, PrepPlace{c->vocab / 16, 8, 0});
+  place(src->lm_head, c->vocab, H, false, PrepPlace{0, kHeadTiles, 0, kHeadTiles});
+  place(src->sel_proj, c->rank, H, false, PrepPlace{c->vocab / 16, kHeadTiles, 0, kHeadTiles});
   out->lm_head = (const uint16_t*)d;
-  out->sel_proj = (const uint16_t*)(d + (size_t)c->vocab / 16 * 16 * H * 2);
+  out->sel_proj = (const uint16_t*)d;  // interleaved into the head's records
   return fail(cudaGetLastError());
 }
 
@@ -889,7 +890,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       lp.cand_val = at<float>(ws, P.off_cv);
       lp.cand_id = at<int32_t>(ws, P.off_ci);
       lp.err = err;
-      CK(launch_pdl(k_slmhead, dim3(P.lm_nparts), dim3(kStreamThreads), P.lm_smem, s, lp));
+      CK(launch_pdl(k_slmhead, dim3(P.lm_nparts), dim3(kGemvThreads), P.lm_smem, s, lp));
     } else {
       for (int pass = 0; pass < P.lm_passes; ++pass) {
         LmParams lp{};

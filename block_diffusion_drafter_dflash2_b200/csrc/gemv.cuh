@@ -178,12 +178,14 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
 // Placement of 16-row tile T of a matrix in a group-interleaved prepared buffer: tile T' = T + tile0
 // sits in group T' / per_grp at slot slot0 + T' % per_grp; a group record of one K unit holds its 8
 // slots back to back, so one bulk copy brings a whole group's unit.
+// Tile T of a matrix goes to record grp = (T + tile0) / per_grp, position slot0 + (T + tile0) % per_grp
+// of the `rec` tiles a record holds (per K unit s).
 struct PrepPlace {
-  int tile0, per_grp, slot0;
+  int tile0, per_grp, slot0, rec;
 };
 DEVI size_t prep_offset(const PrepPlace& pl, int T, int s, int U, int unit_bytes) {
   const int tt = T + pl.tile0, grp = tt / pl.per_grp, slot = pl.slot0 + tt % pl.per_grp;
-  return (((size_t)grp * U + s) * 8 + slot) * unit_bytes;
+  return (((size_t)grp * U + s) * pl.rec + slot) * unit_bytes;
 }
 
 // Canonical Q4_K [N][K/256][144 B] -> prepared tiles (group records of 8 x 2304 B per super-block).

@@ -72,10 +72,11 @@ __global__ void __launch_bounds__(kWarps * 32) k_lmhead_topk(LmParams p) {
   const int nit = ntiles * spt;
   const int ntact = (p.rows + 7) >> 3;
 
-  // prepared bf16 [lm_head; sel_proj]: 2048 bytes per (tile, 64-wide step), 8 tiles interleaved per group
+  // prepared bf16 [lm_head; sel_proj]: 2048 bytes per (tile, 64-wide step), 16 tiles per record
   auto load = [&](uint4 (&w)[4], int it) {
     const int tile = wg + (it / spt) * nw;
-    const uint8_t* b = p.W + (((size_t)(tile >> 3) * spt + it % spt) * 8 + (tile & 7)) * 2048 + lane * 16;
+    const uint8_t* b =
+        p.W + (((size_t)(tile / kHeadTiles) * spt + it % spt) * kHeadTiles + tile % kHeadTiles) * 2048 + lane * 16;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       w[2 * j] = ldg_stream(b + j * 1024);

@@ -24,7 +24,7 @@
 namespace dfl {
 
 constexpr int kPUnits = 2;                      // K units per ring slot
-constexpr int kPSlot = kQ4Bytes * 8 * kPUnits;  // two Q4_K group units (36864 B) or two bf16 64-wide steps (32768 B)
+constexpr int kPSlot = kQ4Bytes * 8 * kPUnits;  // two Q4_K group units (36864 B), two bf16 64-wide steps or one head record step (32768 B)
 constexpr int kPNS = 3;
 constexpr int kPThreads = kGemvThreads;     // 16 consumer warps + 1 producer warp
 constexpr int kPNC = kGemvConsumers * 32;   // consumer threads
@@ -175,12 +175,13 @@ DEVI bool produce_gemv(const PGemv& pg, const PRing& r, int& cnt, int* err) {
   return true;
 }
 
+// Output head records (16 tiles x one 64-wide step = 32 KB) of this CTA: rec = c, c + P, ...
 DEVI bool produce_head(const StepParams& S, const PRing& r, int& cnt) {
-  const int total = S.V / 16 + S.R / 16, ngroups = (total + 7) / 8, St = S.H / 64;
+  const int total = S.V / 16 + S.R / 16, nrec = (total + kHeadTiles - 1) / kHeadTiles, St = S.H / 64;
   const int P = gridDim.x, c = blockIdx.x;
-  for (int grp = c; grp < ngroups; grp += P)
-    for (int s = 0; s < St; s += kPUnits)
-      if (!produce_slot(r, cnt, S.head + ((size_t)grp * St + s) * 16384, kPUnits * 16384, S.err)) return false;
+  for (int rec = c; rec < nrec; rec += P)
+    for (int s = 0; s < St; ++s)
+      if (!produce_slot(r, cnt, S.head + ((size_t)rec * St + s) * kHeadSlot, kHeadSlot, S.err)) return false;
   return true;
 }
 
@@ -344,28 +345,26 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
         const bool have = k + half < cu;
         const uint8_t* sb = st.ring + slot * kPSlot + half * rec + wt * unitB;
         if (Q4) {
-          uint4 q[4], sc = make_uint4(0, 0, 0, 0);
+          const uint4 z4 = make_uint4(0, 0, 0, 0);
+          uint4 q[4] = {z4, z4, z4, z4}, sc = z4;
           if (have) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
-            sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
+            for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
+            sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
           }
-          // the slot is free as soon as its bytes are in registers: release it before the math
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&st.empty[slot]);
           if (have && ntact > 0) q4_unit<NT>(q, sc, coef, st.Xs, stride, (u - base) * 512, ntact, acc, lane);
+          slot_release(&st.empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
         } else {
-          uint4 wv[4];
+          uint4 wv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
           if (have) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
-              wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+              wv[2 * j] = lds_slot(sb + j * 1024 + lane * 16);
+              wv[2 * j + 1] = lds_slot(sb + j * 1024 + 512 + lane * 16);
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&st.empty[slot]);
           if (have && ntact > 0) bf16_step<NT, 2>(wv, st.Xs, stride, (u - base) * 128, ntact, acc, lane);
+          slot_release(&st.empty[slot], wv[0].x ^ wv[1].x ^ wv[2].x ^ wv[3].x, lane);
         }
       }
     }
@@ -461,134 +460,50 @@ DEVI void stage_final_rows(const StepParams& S, int stride, PState& st) {
 }
 
 // Output head + top-16 of the drafted rows; this CTA's lists -> cand_val/cand_id[blockIdx.x].
-// Group k of this CTA: both halves stream it (steps 2j + half), then the half (k & 1) adds the
-// other's accumulators and offers the tile's logits to its warps' per-row lists.
+// Every consumer warp takes every slot (one 32 KB record step): warp (half, wt) owns tile
+// 8 * half + wt of the record, then offers its logits to its own per-row lists.
 __device__ __noinline__ void consume_head(const StepParams& S, PState& st) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int half = warp >> 3, wt = warp & 7;
-  const int H = S.H, stride = H * 2 + 64, vt = S.V / 16, total = vt + S.R / 16, ngroups = (total + 7) / 8;
-  const int St = H / 64, P = gridDim.x, c = blockIdx.x, D = S.D;
-  // per-warp sorted lists of (logit bits, id), in the scale-table region (unused by bf16 work)
-  uint2* lists = reinterpret_cast<uint2*>(st.coef);  // [16 warps][8 rows][16]
+  const int H = S.H, stride = H * 2 + 64, vt = S.V / 16, total = vt + S.R / 16;
+  const int nrec = (total + kHeadTiles - 1) / kHeadTiles, St = H / 64, P = gridDim.x, c = blockIdx.x, D = S.D;
+  uint2* lists = reinterpret_cast<uint2*>(st.coef);  // [16 warps][8 rows][16], in the scale-table region
   rs_from_ssp(S, S.Bk, st);
   stage_final_rows(S, stride, st);
   for (int i = threadIdx.x; i < kGemvConsumers * 8 * kTopK; i += kPNC)
     lists[i] = make_uint2(__float_as_uint(-INFINITY), 0x7fffffffu);
   consumers_sync<kPNC>();
   uint2* my = lists + warp * 8 * kTopK;
-  int k = 0;
-  for (int grp = c; grp < ngroups; grp += P, ++k) {
-    const int tile = grp * 8 + wt;
+  for (int rec = c; rec < nrec; rec += P) {
+    const int tile = rec * kHeadTiles + half * 8 + wt;
     float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-    for (int s = 0; s < St; s += kPUnits) {
+    for (int s = 0; s < St; ++s) {
       int slot;
       if (!slot_wait(st, slot, S.err)) continue;
-      const uint8_t* sb = st.ring + slot * kPSlot + half * 16384 + wt * 2048;
+      const uint8_t* sb = st.ring + slot * kPSlot + (half * 8 + wt) * 2048;
       uint4 wv[4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
-        wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+        wv[2 * j] = lds_slot(sb + j * 1024 + lane * 16);
+        wv[2 * j + 1] = lds_slot(sb + j * 1024 + 512 + lane * 16);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&st.empty[slot]);  // bytes in registers: release before the math
-      bf16_step<1, 2>(wv, st.Xs, stride, (s + half) * 128, 1, acc, lane);
+      bf16_step<1, 2>(wv, st.Xs, stride, s * 128, 1, acc, lane);
+      slot_release(&st.empty[slot], wv[0].x ^ wv[1].x ^ wv[2].x ^ wv[3].x, lane);
     }
-    const int owner = k & 1;
-    float* rd = st.red + (wt * 32 + lane) * 4;
-    if (half != owner) {
+    if (st.dead || tile >= total) continue;
+    if (tile >= vt) {
+      const int c0 = (tile - vt) * 16;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) rd[e] = acc[0][e];
-    }
-    consumers_sync<kPNC>();
-    if (half == owner && tile < total && !st.dead) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[0][e] += rd[e];
-      if (tile >= vt) {
-        const int c0 = (tile - vt) * 16;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = 2 * t + (e & 1);
-          if (r < D) S.z[(size_t)r * S.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
-        }
-      } else {
-        const int id0 = tile * 16;
-        bool want = false;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = 2 * t + (e & 1);
-          if (r < D) {
-            const uint2 last = my[r * kTopK + kTopK - 1];
-            if (better(acc[0][e], id0 + g + 8 * (e >> 1), __uint_as_float(last.x), (int)last.y)) want = true;
-          }
-        }
-        unsigned m = __ballot_sync(0xffffffffu, want);
-        while (m) {
-          const int l = __ffs(m) - 1;
-          if (lane == l) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = 2 * t + (e & 1);
-              if (r >= D) continue;
-              uint2* lst = my + r * kTopK;
-              const float v = acc[0][e];
-              const int id = id0 + g + 8 * (e >> 1);
-              if (!better(v, id, __uint_as_float(lst[kTopK - 1].x), (int)lst[kTopK - 1].y)) continue;
-              int pos = kTopK - 1;
-              while (pos > 0 && better(v, id, __uint_as_float(lst[pos - 1].x), (int)lst[pos - 1].y)) {
-                lst[pos] = lst[pos - 1];
-                --pos;
-              }
-              lst[pos] = make_uint2(__float_as_uint(v), (unsigned)id);
-            }
-          }
-          __syncwarp();
-          m &= m - 1;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const int r = 2 * t + (e & 1);
+        if (r < D) S.z[(size_t)r * S.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
       }
-    }
-    consumers_sync<kPNC>();  // red is reused by the next group
-  }
-  // merge the 16 warp lists of each row (lane holds 8 entries: warp lane/2, entries 8*(lane&1)..+7)
-  for (int r = warp; r < D; r += kGemvConsumers) {
-    float v[8];
-    int id[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint2 e = lists[((lane >> 1) * 8 + r) * kTopK + (lane & 1) * 8 + i];
-      v[i] = __uint_as_float(e.x);
-      id[i] = (int)e.y;
-    }
-    for (int kk = 0; kk < kTopK; ++kk) {
-      int bi = 0;
-#pragma unroll
-      for (int i = 1; i < 8; ++i)
-        if (better(v[i], id[i], v[bi], id[bi])) bi = i;
-      float bv = v[0];
-      int bid = id[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i)
-        if (i == bi) { bv = v[i]; bid = id[i]; }
-      int bl = lane;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-        const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
-        if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) { bv = ov; bid = oid; bl = ol; }
-      }
-      if (lane == 0) {
-        const size_t o = ((size_t)c * D + r) * kTopK + kk;
-        S.cand_val[o] = bv;
-        S.cand_id[o] = bid;
-      }
-      if (lane == bl) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i == bi) { v[i] = -INFINITY; id[i] = 0x7fffffff; }
-      }
+    } else {
+      offer_tile(my, acc[0], tile * 16, D, lane);
     }
   }
+  consumers_sync<kPNC>();
+  merge_warp_lists(lists, D, S.cand_val, S.cand_id, c, warp, kGemvConsumers, lane);
 }
 
 // Row r's final top-16 from the CTAs' lists (warp 0 of CTA r), into cand_fval/cand_fid.

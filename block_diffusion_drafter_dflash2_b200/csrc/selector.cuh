@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(256) k_selector(SelParams p) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x, D = p.Bk - 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   __shared__ int cand[kMaxD][kTopK];
   __shared__ float cl[kMaxD][kTopK];
   // phase 1: per-lane merge lists [warps][32][16] (values, then ids); phase 2: codebook rows

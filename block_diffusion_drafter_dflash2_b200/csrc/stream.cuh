@@ -36,7 +36,6 @@
 namespace dfl {
 
 constexpr int kConsumers = 8;                          // consumer warps of the LM-head kernel = tiles per group
-constexpr int kStreamThreads = (kConsumers + 1) * 32;
 constexpr int kGemvSets = 2;                           // GEMV: two warp sets alternate ring slots
 constexpr int kGemvConsumers = kGemvSets * kConsumers;
 constexpr int kGemvThreads = (kGemvConsumers + 1) * 32;
@@ -54,6 +53,16 @@ struct Ring<false> {
 
 DEVI void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Hand a ring slot back to the producer: dep folds one word of every load this lane made from
+// the slot, and the warp vote on it cannot complete until all lanes' loads have landed in
+// registers; the arrive consumes the vote, so it is issued only then.  The consumers call it
+// after the math on the slot's bytes: releasing between the loads and the math measured no
+// faster and, at 64 activation rows, let results go wrong.
+DEVI void slot_release(uint64_t* bar, uint32_t dep, int lane) {
+  const unsigned v = __ballot_sync(0xffffffffu, dep == 0x9e3779b9u);
+  if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)), "r"(v) : "memory");
 }
 
 struct SGemvParams {
@@ -305,23 +314,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
           if (Q4) {
             uint4 q[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(sb + (i * 32 + lane) * 16);
-            const uint4 sc = *reinterpret_cast<const uint4*>(sb + 2048 + (lane >> 1) * 16);
-            // the slot is free as soon as its bytes are in registers: release it before the math
-            // so the producer's next copy overlaps the decode
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+            for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
+            const uint4 sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
             q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane);
+            slot_release(&empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
           } else {
             uint4 wv[4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
-              wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+              wv[2 * j] = lds_slot(sb + j * 1024 + lane * 16);
+              wv[2 * j + 1] = lds_slot(sb + j * 1024 + 512 + lane * 16);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
             bf16_step<NT, 2>(wv, Xs, stride, (u - base) * 128, ntact, acc, lane);
+            slot_release(&empty[slot], wv[0].x ^ wv[1].x ^ wv[2].x ^ wv[3].x, lane);
           }
         }
       }
@@ -381,152 +386,74 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Shared output head + streaming top-16 (<= 8 drafted rows), same engine: the
-// prepared [V + R rows] bf16 matrix (output head, then the selector projection,
-// padded to whole 8-tile groups) is handed out group by group to the
-// persistent CTAs.  Logits never leave the SM: after each tile every lane
-// offers its values to a per-warp, per-row sorted top-16 list in shared memory
-// (threshold test first; insertions serialised over the warp by ballot); at the
-// end the CTA merges its 8 warp lists, and the selector kernel merges the CTAs'.
-struct SLmParams {
-  const uint8_t* W;  // prepared bf16 groups of [lm_head; sel_proj]
-  int V, R, H;
-  const uint16_t* X;  // final-normed rows [rows][H]
-  int rows;
-  float* z;           // [rows][R]
-  float* cand_val;    // [gridDim.x][rows][16]
-  int32_t* cand_id;
-  int* err;
-};
+// Shared output head + streaming top-16 (<= 8 drafted rows), same engine: the prepared
+// [V + R rows] bf16 matrix (output head, then the selector projection) is stored in records of
+// 16 tiles per 64-wide K step (32 KB, one bulk copy), handed out record by record to the
+// persistent CTAs.  All 16 consumer warps take every slot: warp (half, wt) owns tile
+// 8 * half + wt of the record and accumulates it over all K steps.  Logits never leave the SM:
+// after its tile each warp offers the values to its own per-row sorted top-16 lists in shared
+// memory; at the end the CTA merges its 16 warp lists, and the selector merges the CTAs'.
 
-__global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
-  using RC = Ring<false>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full[RC::kNS];
-  __shared__ __align__(8) uint64_t empty[RC::kNS];
-  __shared__ __align__(8) uint64_t xbar;
-  const int H = p.H, stride = H * 2 + 64;
-  uint8_t* ring = smem;
-  uint8_t* Xs = smem + RC::kNS * RC::kSlot;
-  float* lv_all = reinterpret_cast<float*>(Xs + 8 * stride);          // [warps][8][16]
-  int* li_all = reinterpret_cast<int*>(lv_all + kConsumers * 8 * kTopK);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int vt = p.V / 16, total = vt + p.R / 16, S = H / 64;
-  const int ngroups = (total + kConsumers - 1) / kConsumers;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < RC::kNS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers);
-    }
-    mbar_init(&xbar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  pdl_trigger();
-
-  if (warp == kConsumers) {
-    if (lane != 0) return;
-    int cnt = 0;
-    for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x)
-      for (int s = 0; s < S; ++s) {
-        const int slot = cnt % RC::kNS, round = cnt / RC::kNS;
-        if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
-          set_err(p.err, DFLASH2_DEV_TIMEOUT);
-          return;
-        }
-        mbar_expect_tx(&full[slot], RC::kSlot);
-        bulk_g2s(ring + slot * RC::kSlot, p.W + ((size_t)grp * S + s) * RC::kSlot, RC::kSlot, &full[slot]);
-        ++cnt;
-      }
-    return;
-  }
-
-  for (int i = threadIdx.x; i < kConsumers * 8 * kTopK; i += kConsumers * 32) {
-    lv_all[i] = -INFINITY;
-    li_all[i] = 0x7fffffff;
-  }
-  pdl_wait();
-  uint32_t xph = 0;
-  stage_x_chunk<kConsumers * 32>(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
-  float* lv = lv_all + warp * 8 * kTopK;
-  int* li = li_all + warp * 8 * kTopK;
-  int cnt = 0;
-  bool dead = false;
-  for (int grp = blockIdx.x; grp < ngroups; grp += gridDim.x) {
-    const int tile = grp * kConsumers + warp;
-    float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-    for (int s = 0; s < S; ++s) {
-      const int slot = cnt % RC::kNS;
-      if (!dead && !mbar_wait_sleep_bounded(&full[slot], (cnt / RC::kNS) & 1)) {
-        set_err(p.err, DFLASH2_DEV_TIMEOUT);
-        dead = true;
-      }
-      ++cnt;
-      if (dead) continue;
-      const uint8_t* sb = ring + slot * RC::kSlot + warp * RC::kUnitBytes;
-      uint4 wv[4];
+// Offer one tile's logits (this lane: rows 2t, 2t+1 at vocabulary ids id0 + g and id0 + g + 8,
+// i.e. acc[e] at row 2t + (e & 1), id id0 + g + 8 * (e >> 1)) to the warp's sorted per-row lists
+// lists[r * 16 + k] = (value bits, id), best first.  Entries beating a row's current 16th are
+// inserted one at a time, the 16 list positions shifting in parallel across lanes 0-15.
+DEVI void offer_tile(uint2* lists, const float (&acc)[4], int id0, int rows, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  unsigned m[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        wv[2 * j] = *reinterpret_cast<const uint4*>(sb + j * 1024 + lane * 16);
-        wv[2 * j + 1] = *reinterpret_cast<const uint4*>(sb + j * 1024 + 512 + lane * 16);
+  for (int e = 0; e < 4; ++e) {
+    const int r = 2 * t + (e & 1);
+    bool want = false;
+    if (r < rows) {
+      const uint2 last = lists[r * kTopK + kTopK - 1];
+      want = better(acc[e], id0 + g + 8 * (e >> 1), __uint_as_float(last.x), (int)last.y);
+    }
+    m[e] = __ballot_sync(0xffffffffu, want);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    while (m[e]) {
+      const int src = __ffs(m[e]) - 1;
+      m[e] &= m[e] - 1;
+      const float v = __shfl_sync(0xffffffffu, acc[e], src);
+      const int id = id0 + (src >> 2) + 8 * (e >> 1);
+      uint2* L = lists + (2 * (src & 3) + (e & 1)) * kTopK;
+      const uint2 cur = lane < kTopK ? L[lane] : make_uint2(0u, 0u);
+      const bool ahead = lane < kTopK && better(__uint_as_float(cur.x), (int)cur.y, v, id);
+      const int pos = __popc(__ballot_sync(0xffffffffu, ahead));  // entries that stay ahead (a prefix)
+      __syncwarp();
+      if (pos < kTopK) {
+        if (lane >= pos && lane < kTopK - 1) L[lane + 1] = cur;
+        if (lane == pos) L[pos] = make_uint2(__float_as_uint(v), (unsigned)id);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);  // bytes in registers: release before the math
-      bf16_step<1, 2>(wv, Xs, stride, s * 128, 1, acc, lane);
-    }
-    if (dead || tile >= total) continue;
-    if (tile >= vt) {
-      const int c0 = (tile - vt) * 16;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 2 * t + (e & 1);
-        if (r < p.rows) p.z[(size_t)r * p.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
-      }
-    } else {
-      const int id0 = tile * 16;
-      bool want = false;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 2 * t + (e & 1);
-        if (r < p.rows && better(acc[0][e], id0 + g + 8 * (e >> 1), lv[r * kTopK + kTopK - 1], li[r * kTopK + kTopK - 1]))
-          want = true;
-      }
-      unsigned m = __ballot_sync(0xffffffffu, want);
-      while (m) {
-        const int l = __ffs(m) - 1;
-        if (lane == l) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = 2 * t + (e & 1);
-            if (r < p.rows) topk_insert(lv + r * kTopK, li + r * kTopK, acc[0][e], id0 + g + 8 * (e >> 1));
-          }
-        }
-        __syncwarp();
-        m &= m - 1;
-      }
     }
   }
-  consumers_sync<kConsumers * 32>();
-  // merge the 8 warp lists of each row
-  for (int r = warp; r < p.rows; r += kConsumers) {
-    float v[4];
-    int id[4];
+}
+
+// Merge the 16 warp lists of each row into the CTA's list (lane: warp lane/2, entries
+// 8*(lane&1) .. +7) -> cand_val/cand_id[part][row][16].
+DEVI void merge_warp_lists(const uint2* lists, int rows, float* cand_val, int32_t* cand_id, int part, int warp,
+                           int nwarps, int lane) {
+  for (int r = warp; r < rows; r += nwarps) {
+    float v[8];
+    int id[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int src = ((lane >> 2) * 8 + r) * kTopK + (lane & 3) * 4 + i;
-      v[i] = lv_all[src];
-      id[i] = li_all[src];
+    for (int i = 0; i < 8; ++i) {
+      const uint2 e = lists[((lane >> 1) * 8 + r) * kTopK + (lane & 1) * 8 + i];
+      v[i] = __uint_as_float(e.x);
+      id[i] = (int)e.y;
     }
-    for (int k = 0; k < kTopK; ++k) {
+    for (int kk = 0; kk < kTopK; ++kk) {
       int bi = 0;
 #pragma unroll
-      for (int i = 1; i < 4; ++i)
+      for (int i = 1; i < 8; ++i)
         if (better(v[i], id[i], v[bi], id[bi])) bi = i;
       float bv = v[0];
       int bid = id[0];
 #pragma unroll
-      for (int i = 1; i < 4; ++i)
+      for (int i = 1; i < 8; ++i)
         if (i == bi) { bv = v[i]; bid = id[i]; }
       int bl = lane;
 #pragma unroll
@@ -537,17 +464,119 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_slmhead(SLmParams p) {
         if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) { bv = ov; bid = oid; bl = ol; }
       }
       if (lane == 0) {
-        const size_t o = ((size_t)blockIdx.x * p.rows + r) * kTopK + k;
-        p.cand_val[o] = bv;
-        p.cand_id[o] = bid;
+        const size_t o = ((size_t)part * rows + r) * kTopK + kk;
+        cand_val[o] = bv;
+        cand_id[o] = bid;
       }
       if (lane == bl) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 8; ++i)
           if (i == bi) { v[i] = -INFINITY; id[i] = 0x7fffffff; }
       }
     }
   }
+}
+
+struct SLmParams {
+  const uint8_t* W;  // prepared bf16 records of [lm_head; sel_proj]
+  int V, R, H;
+  const uint16_t* X;  // final-normed rows [rows][H]
+  int rows;
+  float* z;           // [rows][R]
+  float* cand_val;    // [gridDim.x][rows][16]
+  int32_t* cand_id;
+  int* err;
+};
+
+constexpr int kHeadSlot = kHeadTiles * 2048;  // one record step: 32 KB
+constexpr int kHeadNS = 3;
+
+__global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kHeadNS];
+  __shared__ __align__(8) uint64_t empty[kHeadNS];
+  __shared__ __align__(8) uint64_t xbar;
+  constexpr int NC = kGemvConsumers * 32;
+  const int H = p.H, stride = H * 2 + 64;
+  uint8_t* ring = smem;
+  uint8_t* Xs = smem + kHeadNS * kHeadSlot;
+  uint2* lists = reinterpret_cast<uint2*>(Xs + 8 * stride);  // [16 warps][8 rows][16]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int half = warp >> 3, wt = warp & 7;
+  const int vt = p.V / 16, total = vt + p.R / 16, S = H / 64;
+  const int nrec = (total + kHeadTiles - 1) / kHeadTiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kHeadNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGemvConsumers);
+    }
+    mbar_init(&xbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  if (warp == kGemvConsumers) {
+    if (lane != 0) return;
+    int cnt = 0;
+    for (int rec = blockIdx.x; rec < nrec; rec += gridDim.x)
+      for (int s = 0; s < S; ++s) {
+        const int slot = cnt % kHeadNS, round = cnt / kHeadNS;
+        if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
+          set_err(p.err, DFLASH2_DEV_TIMEOUT);
+          return;
+        }
+        mbar_expect_tx(&full[slot], kHeadSlot);
+        bulk_g2s(ring + slot * kHeadSlot, p.W + ((size_t)rec * S + s) * kHeadSlot, kHeadSlot, &full[slot]);
+        ++cnt;
+      }
+    return;
+  }
+
+  for (int i = threadIdx.x; i < kGemvConsumers * 8 * kTopK; i += NC)
+    lists[i] = make_uint2(__float_as_uint(-INFINITY), 0x7fffffffu);
+  pdl_wait();
+  uint32_t xph = 0;
+  stage_x_chunk<NC>(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
+  uint2* my = lists + warp * 8 * kTopK;
+  int cnt = 0;
+  bool dead = false;
+  for (int rec = blockIdx.x; rec < nrec; rec += gridDim.x) {
+    const int tile = rec * kHeadTiles + half * 8 + wt;
+    float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
+    for (int s = 0; s < S; ++s) {
+      const int slot = cnt % kHeadNS;
+      if (!dead && !mbar_wait_sleep_bounded(&full[slot], (cnt / kHeadNS) & 1)) {
+        set_err(p.err, DFLASH2_DEV_TIMEOUT);
+        dead = true;
+      }
+      ++cnt;
+      if (dead) continue;
+      const uint8_t* sb = ring + slot * kHeadSlot + (half * 8 + wt) * 2048;
+      uint4 wv[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        wv[2 * j] = lds_slot(sb + j * 1024 + lane * 16);
+        wv[2 * j + 1] = lds_slot(sb + j * 1024 + 512 + lane * 16);
+      }
+      bf16_step<1, 2>(wv, Xs, stride, s * 128, 1, acc, lane);
+      slot_release(&empty[slot], wv[0].x ^ wv[1].x ^ wv[2].x ^ wv[3].x, lane);
+    }
+    if (dead || tile >= total) continue;
+    if (tile >= vt) {
+      const int c0 = (tile - vt) * 16;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = 2 * t + (e & 1);
+        if (r < p.rows) p.z[(size_t)r * p.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
+      }
+    } else {
+      offer_tile(my, acc[0], tile * 16, p.rows, lane);
+    }
+  }
+  consumers_sync<NC>();
+  merge_warp_lists(lists, p.rows, p.cand_val, p.cand_id, blockIdx.x, warp, kGemvConsumers, lane);
 }
 
 }  // namespace dfl

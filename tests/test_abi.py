@@ -40,7 +40,7 @@ def test_strerror_and_sizes(lib):
     H, F, HQ, HKV = d.hidden, d.ffn, d.n_q * 128, d.n_kv * 128
     mats = H * d.n_taps * H + d.layers * (HQ * H + 2 * HKV * H + H * HQ + 3 * F * H)
     dyn = d.layers * 2 * (H // 4) * H * 2
-    head = -(-(d.vocab + d.rank) // 128) * 128 * H * 2  # output head + selector projection, whole 8-tile groups
+    head = -(-(d.vocab + d.rank) // 256) * 256 * H * 2  # output head + selector projection, whole 16-tile records
     # prepared copy: the Q4_K matrices keep their size, bf16 matrices and the output head theirs
     assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144 + dyn + head
     full = binding.config(inputs.FULL)
