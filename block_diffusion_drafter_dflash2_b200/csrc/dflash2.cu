@@ -32,7 +32,7 @@ struct Plan {
   GemvPlan fc, dc, qkv, o, gu, dn;
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
   bool persistent;
-  size_t psmem, off_cfv, off_cfi, off_ssp;
+  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau;
   int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
   bool lm_stream;
   size_t lm_smem;
@@ -69,9 +69,10 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   const int ring = ns * slot;
   const int per_unit = g.R * unitK * 2;
   const int extra = kGemvConsumers * 1024 + kConsumers * 32 * g.NT * 4 * 4;  // per-warp scale tables, set reduction
+  const int sums = q4 ? g.R * 8 * 4 : 0;  // Q4: activation sums per staged unit (8 sub-blocks x R rows)
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
-  g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
+  g.kc_units = std::max(1, std::min(g.U, budget / (per_unit + sums)));
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra + (size_t)sums * g.kc_units;
   return g;
 }
 
@@ -89,6 +90,7 @@ GemvPlan plan_gemv_persistent(int tiles, int rows, int K, bool q4, int nsm) {
   g.P = (int)std::min<long long>(nsm, g.W);  // every CTA in [0, P) owns at least one unit
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
   g.kc_units = std::max(1, std::min(g.U, (kPXBytes - 64 * g.R) / (g.R * unitK * 2)));
+  if (q4) g.kc_units = std::max(1, std::min(g.kc_units, kPSumBytes / (g.R * 8 * 4)));  // activation sums fit
   if (g.kc_units < g.U && g.kc_units > 1) g.kc_units &= ~1;  // whole slots (two units each) per chunk
   g.smem = 0;
   return g;
@@ -153,7 +155,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.persistent = B == 1 && p.Bk <= 8 && p.QVP == 32 && 8 * (p.H * 2 + 64) <= kPXBytes &&
                  (size_t)(p.MT * 16 + 2 * kAttnKeys) * kAttnStride * 2 <= (size_t)kPXBytes;
   p.psmem = (size_t)kPNS * kPSlot + kPXBytes + (size_t)kGemvConsumers * 128 * 8 + (size_t)kConsumers * 32 * 8 * 4 +
-            (size_t)kGemvConsumers * 64 * 4;
+            (size_t)kPSumBytes;
   if (p.persistent) {
     p.pfc = plan_gemv_persistent(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
     p.pdc = plan_gemv_persistent((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
@@ -207,6 +209,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_cfv = take((size_t)p.lm_rows * kTopK * 4);
   p.off_cfi = take((size_t)p.lm_rows * kTopK * 4);
   p.off_ssp = take((size_t)(p.H / 128) * 4 * p.Mb * 4);
+  p.off_tau = take((size_t)p.lm_rows * kTopK * kTopK * 4);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
@@ -582,6 +585,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     S.cand_id = at<int32_t>(ws, P.off_ci);
     S.cand_fval = at<float>(ws, P.off_cfv);
     S.cand_fid = at<int32_t>(ws, P.off_cfi);
+    S.tau = at<float>(ws, P.off_tau);
     S.h = h;
     S.ssp = at<float>(ws, P.off_ssp);
     S.gbar = reinterpret_cast<unsigned*>(ctr + P.ctr_total - 1);
@@ -591,9 +595,9 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     S.dbg_final_h = dbg ? dbg->final_h : nullptr;
     {
       SelParams& sp = S.sel;
-      sp.cand_val = S.cand_fval;
-      sp.cand_id = S.cand_fid;
-      sp.nparts = 1;
+      sp.cand_val = S.cand_val;  // the CTAs' lists: one part per CTA of the launch
+      sp.cand_id = S.cand_id;
+      sp.nparts = P.nsm;
       sp.rows_total = P.D;
       sp.z = zbuf;
       sp.R = P.R;
@@ -939,7 +943,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     sp.dbg_logit = dbg ? dbg->cand_logit : nullptr;
     sp.err = err;
     if (sp.dbg_cand && !sp.dbg_logit) sp.dbg_cand = nullptr;
-    CK(launch_pdl(k_selector, dim3(batch), dim3(256), 0, s, sp));
+    float* tau = at<float>(ws, P.off_tau);
+    float* clg = at<float>(ws, P.off_cfv);
+    int32_t* cdg = at<int32_t>(ws, P.off_cfi);
+    CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), 0, s, sp, tau, clg, cdg));
+    CK(launch_pdl(k_sel_viterbi, dim3(batch), dim3(32), 0, s, sp, (const float*)tau, (const float*)clg,
+                  (const int32_t*)cdg));
   }
   return DFLASH2_OK;
 }
@@ -1005,8 +1014,8 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   const Plan P = make_plan(c, batch);
   if (P.persistent && persistent_ready(P)) return 1;
   // embed, fc GEMV, fc norm | per layer: norm, W_dc GEMV, dynconv, QKV GEMV, attention, combine,
-  // W_o GEMV, norm, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector
-  return 3 + 10 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 1;
+  // W_o GEMV, norm, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
+  return 3 + 10 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

@@ -29,6 +29,7 @@ constexpr int kPNS = 3;
 constexpr int kPThreads = kGemvThreads;     // 16 consumer warps + 1 producer warp
 constexpr int kPNC = kGemvConsumers * 32;   // consumer threads
 constexpr int kPXBytes = 82944;             // activation staging (8 rows x 5120 bf16 + padding); attention buffers
+constexpr int kPSumBytes = 5120;            // combine weights [16][64] floats / Q4 activation sums
 constexpr long long kBarrierSpin = 1ll << 24;
 constexpr unsigned long long kBarrierNs = 2000000000ull;  // 2 s
 
@@ -70,6 +71,7 @@ struct StepParams {
   int32_t* cand_id;
   float* cand_fval;         // merged [D][16]
   int32_t* cand_fid;
+  float* tau;               // selector transition scores [D][16][16]
   SelParams sel;
   float* h;
   float* ssp;               // sums of squares of h: [H/128 column groups][4 quarters][Mb]
@@ -193,7 +195,7 @@ struct PState {
   float2* coef;     // [16 warps][128]
   float* red;       // [8][32][8]
   float* rs;        // [16] row scales
-  float* wsh;       // [16 warps][64] attention-combine weights
+  float* wsh;       // [16 warps][64] attention-combine weights; Q4 activation sums during products (5 KB)
   int* row_ok;      // [64]
   int cnt;
   uint32_t xph, aph;
@@ -336,6 +338,10 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
         } else {
           stage_computed<R>(pg, S, k0, nk, stride, st);
         }
+        if (Q4) {
+          x_sums<kPNC>(st.Xs, stride, R, nk, st.wsh);  // the combine-weight region, free during products
+          consumers_sync<kPNC>();
+        }
         staged = true;
       }
       for (int k = 0; k < cu; k += kPUnits) {
@@ -352,7 +358,7 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
             for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
             sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
           }
-          if (have && ntact > 0) q4_unit<NT>(q, sc, coef, st.Xs, stride, (u - base) * 512, ntact, acc, lane);
+          if (have && ntact > 0) q4_unit<NT>(q, sc, coef, st.Xs, stride, (u - base) * 512, st.wsh, ntact, acc, lane);
           slot_release(&st.empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
         } else {
           uint4 wv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -506,26 +512,6 @@ __device__ __noinline__ void consume_head(const StepParams& S, PState& st) {
   merge_warp_lists(lists, D, S.cand_val, S.cand_id, c, warp, kGemvConsumers, lane);
 }
 
-// Row r's final top-16 from the CTAs' lists (warp 0 of CTA r), into cand_fval/cand_fid.
-__device__ __noinline__ void merge_row(const StepParams& S, int r, PState& st) {
-  constexpr int kCap = 1024;
-  float* sv = reinterpret_cast<float*>(st.Xs);
-  int* si = reinterpret_cast<int*>(st.Xs) + kCap;
-  int* n = reinterpret_cast<int*>(st.Xs) + 2 * kCap;
-  float* ov = reinterpret_cast<float*>(st.Xs) + 2 * kCap + 32;
-  int* oi = reinterpret_cast<int*>(st.Xs) + 2 * kCap + 64;
-  merge_lists_row(S.cand_val, S.cand_id, gridDim.x, S.D, r, sv, si, kCap, n, ov, oi);
-  const int lane = threadIdx.x & 31;
-  if (lane < kTopK) {
-    S.cand_fval[r * kTopK + lane] = ov[lane];
-    S.cand_fid[r * kTopK + lane] = oi[lane];
-    if (S.sel.dbg_cand) {
-      S.sel.dbg_cand[r * kTopK + lane] = oi[lane];
-      S.sel.dbg_logit[r * kTopK + lane] = ov[lane];
-    }
-  }
-}
-
 // Context row c = RMSNorm(fc output row c; fc_norm), or zero past the request's new rows; one
 // CTA, the row's loads issued together (kB float4 per consumer thread cover H <= 8192).
 __device__ __noinline__ void ctx_row(const StepParams& S, int c, PState& st) {
@@ -577,8 +563,10 @@ __global__ void __launch_bounds__(kPThreads, 1) k_step_persistent(const __grid_c
   __shared__ __align__(8) uint64_t xbar, abar;
   __shared__ float rs[16];
   __shared__ int row_ok[kAttnKeys];
-  __shared__ int cand_s[kMaxD][kTopK];
-  __shared__ float cl_s[kMaxD][kTopK];
+  __shared__ int cand_s[2][kTopK];  // selector: candidates of rows t - 1 and t
+  __shared__ float cl_s[2][kTopK];
+  __shared__ int src_s[kTopK];
+  __shared__ int sel_n[2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPNS; ++s) {
@@ -690,27 +678,36 @@ __global__ void __launch_bounds__(kPThreads, 1) k_step_persistent(const __grid_c
   }
   consume_head(S, st);
   grid_sync(S.gbar, epoch, S.err);
-  if (c < S.D && warp == 0) merge_row(S, c, st);
-  grid_sync(S.gbar, epoch, S.err);
-  if (c == 0) {
-    const int D = S.D;
-    if (threadIdx.x < D * kTopK) {
-      const int t = threadIdx.x / kTopK, k = threadIdx.x % kTopK;
-      const float v = __ldcg(S.cand_fval + threadIdx.x);
-      int id = __ldcg(S.cand_fid + threadIdx.x);
-      if (!isfinite(v)) set_err(S.err, DFLASH2_DEV_NONFINITE);
-      if (id < 0 || id >= S.V) {
-        set_err(S.err, DFLASH2_DEV_NONFINITE);
-        id = 0;
+  // A6: CTA t < D: final candidates of rows t and t - 1, then the transition scores tau_t
+  if (c < S.D) {
+    const int t = c;
+    float* sv = reinterpret_cast<float*>(st.Xs) + warp * 1024;
+    int* si = reinterpret_cast<int*>(st.Xs) + warp * 1024 + 512;
+    if (warp == 0 || (warp == 1 && t > 0)) selector_row(S.sel, t - warp, sv, si, &sel_n[warp], cl_s[1 - warp], cand_s[1 - warp]);
+    consumers_sync<kPNC>();
+    if (threadIdx.x < kTopK) {
+      S.cand_fval[t * kTopK + threadIdx.x] = cl_s[1][threadIdx.x];
+      S.cand_fid[t * kTopK + threadIdx.x] = cand_s[1][threadIdx.x];
+      if (S.sel.dbg_cand) {
+        S.sel.dbg_cand[t * kTopK + threadIdx.x] = cand_s[1][threadIdx.x];
+        S.sel.dbg_logit[t * kTopK + threadIdx.x] = cl_s[1][threadIdx.x];
       }
-      cand_s[t][k] = id;
-      cl_s[t][k] = v;
+      if (t == 0) {
+        if (threadIdx.x == 0) {
+          const int a = S.block_tokens[0];
+          src_s[0] = (a < 0 || a >= S.V) ? 0 : a;
+        }
+      } else {
+        src_s[threadIdx.x] = cand_s[0][threadIdx.x];
+      }
     }
     consumers_sync<kPNC>();
-    float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(st.Xs);
-    float(*Wj)[kTopK] = reinterpret_cast<float(*)[kTopK]>(st.Xs + kTopK * kMaxR * 4);
-    selector_core<kPNC>(S.sel, 0, cand_s, cl_s, As, Wj);
+    float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(st.Xs + 8192);
+    float(*Wj)[kTopK] = reinterpret_cast<float(*)[kTopK]>(st.Xs + 8192 + kTopK * kMaxR * 4);
+    selector_tau<kPNC>(S.sel, 0, t, src_s, t == 0 ? 1 : kTopK, cand_s[1], As, Wj, S.tau + (size_t)t * kTopK * kTopK);
   }
+  grid_sync(S.gbar, epoch, S.err);
+  if (c == 0 && warp == 0) selector_viterbi(S.sel, 0, S.cand_fval, S.cand_fid, S.tau);
 }
 
 }  // namespace dfl

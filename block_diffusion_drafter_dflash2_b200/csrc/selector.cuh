@@ -35,91 +35,6 @@ struct SelParams {
   int* err;
 };
 
-// Transition scores and the Viterbi path of request b from its merged candidates (cand, cl in
-// shared memory), run by the first NTHR threads (named barrier 1).  As, Wj: shared scratch of
-// 16 x 256 floats each.  Writes out_path / out_scores and advances seq_len[b].
-template <int NTHR>
-DEVI void selector_core(const SelParams& p, int b, int (*cand)[kTopK], float (*cl)[kTopK], float (*As)[kMaxR],
-                        float (*Wj)[kTopK]) {
-  __shared__ float tau[kTopK][kTopK];
-  __shared__ float delta[kMaxD][kTopK];
-  __shared__ int bp[kMaxD][kTopK];
-  __shared__ int src_ids[kTopK];
-  const int D = p.Bk - 1, R = p.R;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 2. per position: transition scores tau_t, then one Viterbi step in warp 0
-  //    (lane j of warp 0 holds delta_t(j))
-  float d = 0.f;
-  for (int t = 0; t < D; ++t) {
-    const int nsrc = t == 0 ? 1 : kTopK;
-    if (threadIdx.x < kTopK) {
-      int a = t == 0 ? p.block_tokens[b * p.Bk] : cand[t - 1][threadIdx.x];
-      if (a < 0 || a >= p.V) a = 0;
-      src_ids[threadIdx.x] = a;
-    }
-    consumers_sync<NTHR>();
-    const float* zt = p.z + (size_t)(b * D + t) * R;
-    const int R8 = R / 8;
-    for (int i = threadIdx.x; i < kTopK * R8; i += NTHR) {
-      const int j = i / R8, r = (i % R8) * 8;
-      const uint4 bv = *reinterpret_cast<const uint4*>(p.cb_b + (size_t)cand[t][j] * R + r);
-      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        Wj[r + 2 * e][j] = __ldcg(zt + r + 2 * e) * bf2f(bw[e] & 0xffff);
-        Wj[r + 2 * e + 1][j] = __ldcg(zt + r + 2 * e + 1) * bf2f(bw[e] >> 16);
-      }
-      if (j < nsrc) {
-        const uint4 av = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          As[j][r + 2 * e] = bf2f(aw[e] & 0xffff);
-          As[j][r + 2 * e + 1] = bf2f(aw[e] >> 16);
-        }
-      }
-    }
-    consumers_sync<NTHR>();
-    {
-      const int i = threadIdx.x / kTopK, j = threadIdx.x % kTopK;
-      if (i < nsrc) {
-        float s = 0.f;
-        for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[r][j], s);
-        tau[i][j] = s;
-      }
-    }
-    consumers_sync<NTHR>();
-    if (warp == 0) {
-      const int j = lane & 15;
-      int bi = 0;
-      if (t == 0) {
-        d = cl[0][j] + tau[0][j];
-      } else {
-        float best = 0.f;
-        bi = -1;
-        for (int i = 0; i < kTopK; ++i) {
-          const float s = __shfl_sync(0xffffffffu, d, i) + tau[i][j];
-          if (bi < 0 || s > best) { best = s; bi = i; }
-        }
-        d = cl[t][j] + best;
-      }
-      if (lane < kTopK) { delta[t][j] = d; bp[t][j] = bi; }
-    }
-  }
-  consumers_sync<NTHR>();
-  if (threadIdx.x == 0) {
-    int jj = 0;
-    for (int i = 1; i < kTopK; ++i)
-      if (delta[D - 1][i] > delta[D - 1][jj]) jj = i;
-    for (int t = D - 1; t >= 0; --t) {
-      p.out_path[b * D + t] = cand[t][jj];
-      p.out_scores[b * D + t] = delta[t][jj];
-      jj = bp[t][jj];
-    }
-    p.seq_len[b] += p.n_new[b];
-  }
-}
-
 // Final top-16 of one drafted row from `nparts` sorted partial lists ([part][rows_total][16]),
 // by one warp.  T0 = max(best 16th entry of a list, 16th best list head) bounds the final 16th
 // from below (either way at least 16 entries reach it), so only list prefixes >= T0 are
@@ -237,46 +152,157 @@ DEVI void merge_lists_row(const float* cv, const int32_t* ci, int nparts, int ro
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(256) k_selector(SelParams p) {
+// Transition scores of position t of request b, tau[i][j] = sum_r A[src_i][r] z_t[r] B[cand_j][r]
+// for sources i < nsrc (t = 0: the block's first token; t > 0: the candidates of t-1), by the
+// first NTHR (>= 256) threads (named barrier 1).  As, Wj: shared scratch of 16 x 256 floats each.
+template <int NTHR>
+DEVI void selector_tau(const SelParams& p, int b, int t, const int* src_ids, int nsrc, const int* cand_t,
+                       float (*As)[kMaxR], float (*Wj)[kTopK], float* tau) {
+  const int D = p.Bk - 1, R = p.R, R8 = R / 8;
+  const float* zt = p.z + (size_t)(b * D + t) * R;
+  for (int i = threadIdx.x; i < kTopK * R8; i += NTHR) {
+    const int j = i / R8, r = (i % R8) * 8;
+    const uint4 bv = *reinterpret_cast<const uint4*>(p.cb_b + (size_t)cand_t[j] * R + r);
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      Wj[r + 2 * e][j] = __ldcg(zt + r + 2 * e) * bf2f(bw[e] & 0xffff);
+      Wj[r + 2 * e + 1][j] = __ldcg(zt + r + 2 * e + 1) * bf2f(bw[e] >> 16);
+    }
+    if (j < nsrc) {
+      const uint4 av = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
+      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        As[j][r + 2 * e] = bf2f(aw[e] & 0xffff);
+        As[j][r + 2 * e + 1] = bf2f(aw[e] >> 16);
+      }
+    }
+  }
+  consumers_sync<NTHR>();
+  const int i = threadIdx.x / kTopK, j = threadIdx.x % kTopK;
+  if (i < nsrc) {
+    float s = 0.f;
+    for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[r][j], s);
+    tau[i * kTopK + j] = s;
+  }
+}
+
+// Viterbi over the D positions of request b by one warp (lane j < 16 holds delta_t(j)):
+//   delta_0(j) = cl_0(j) + tau_0(0, j),  delta_t(j) = cl_t(j) + max_i (delta_{t-1}(i) + tau_t(i, j)),
+// first maximum on ties (smallest i; at the end smallest j).  Writes the path and its running
+// scores and advances seq_len[b] by n_new[b].  cl/cand: [D][16], tau: [D][16][16] (global).
+DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int32_t* cand, const float* tau) {
+  const int lane = threadIdx.x & 31, j = lane & 15, D = p.Bk - 1;
+  float d = 0.f;
+  float dl[kMaxD];
+  int bp[kMaxD];
+#pragma unroll
+  for (int t = 0; t < kMaxD; ++t) {
+    dl[t] = 0.f;
+    bp[t] = 0;
+    if (t >= D) continue;
+    const float* tt = tau + (size_t)t * kTopK * kTopK;
+    const float c = __ldcg(cl + t * kTopK + j);
+    if (t == 0) {
+      d = c + __ldcg(tt + j);
+    } else {
+      float best = 0.f;
+      int bi = -1;
+      for (int i = 0; i < kTopK; ++i) {
+        const float sc = __shfl_sync(0xffffffffu, d, i) + __ldcg(tt + i * kTopK + j);
+        if (bi < 0 || sc > best) { best = sc; bi = i; }
+      }
+      d = c + best;
+      bp[t] = bi;
+    }
+    dl[t] = d;
+  }
+  int jj = 0;
+  float bestd = __shfl_sync(0xffffffffu, d, 0);
+  for (int i = 1; i < kTopK; ++i) {
+    const float v = __shfl_sync(0xffffffffu, d, i);
+    if (v > bestd) { bestd = v; jj = i; }
+  }
+#pragma unroll
+  for (int t = kMaxD - 1; t >= 0; --t) {
+    if (t >= D) continue;
+    const float sc = __shfl_sync(0xffffffffu, dl[t], jj);
+    const int prev = __shfl_sync(0xffffffffu, bp[t], jj);
+    if (lane == 0) {
+      p.out_path[b * D + t] = __ldcg(cand + t * kTopK + jj);
+      p.out_scores[b * D + t] = sc;
+    }
+    jj = prev;
+  }
+  if (lane == 0) p.seq_len[b] += p.n_new[b];
+}
+
+// Final candidates of row (b, t) from the CTA lists into cl/cand (shared), ids outside [0, V)
+// (and non-finite logits) flagged and replaced by 0.  One warp; sv/si: >= 512 entries each.
+DEVI void selector_row(const SelParams& p, int row, float* sv, int* si, int* surv, float* cl, int* cand) {
+  merge_lists_row(p.cand_val, p.cand_id, p.nparts, p.rows_total, row, sv, si, 512, surv, cl, cand);
+  __syncwarp();
+  const int lane = threadIdx.x & 31;
+  if (lane < kTopK) {
+    if (!isfinite(cl[lane])) set_err(p.err, DFLASH2_DEV_NONFINITE);
+    if (cand[lane] < 0 || cand[lane] >= p.V) {
+      set_err(p.err, DFLASH2_DEV_NONFINITE);
+      cand[lane] = 0;
+    }
+  }
+  __syncwarp();
+}
+
+// One CTA per (position t, request b): final candidates of rows t (and t-1, the sources), then
+// tau_t -> tau_g[b][t]; row t's candidates -> cl_g/cand_g (and the debug outputs).
+__global__ void __launch_bounds__(256) k_sel_tau(SelParams p, float* tau_g, float* cl_g, int32_t* cand_g) {
   pdl_trigger();
   pdl_wait();
-  const int b = blockIdx.x, D = p.Bk - 1;
-  const int warp = threadIdx.x >> 5;
-  __shared__ int cand[kMaxD][kTopK];
-  __shared__ float cl[kMaxD][kTopK];
-  // phase 1: per-lane merge lists [warps][32][16] (values, then ids); phase 2: codebook rows
+  const int t = blockIdx.x, b = blockIdx.y, D = p.Bk - 1, warp = threadIdx.x >> 5;
+  __shared__ int cand[2][kTopK];
+  __shared__ float cl[2][kTopK];
+  __shared__ int src[kTopK];
+  __shared__ int surv[2];
   __shared__ __align__(16) float big[2 * kTopK * kMaxR];
   float(*As)[kMaxR] = reinterpret_cast<float(*)[kMaxR]>(big);
   float(*Wj)[kTopK] = reinterpret_cast<float(*)[kTopK]>(big + kTopK * kMaxR);  // [r][j]: conflict-free reads
-
-  // 1. merge the CTA lists of each drafted position into the final top-16
-  constexpr int kCap = 512;
-  __shared__ int surv_n[kWarps];
-  for (int t = warp; t < D; t += kWarps) {
-    float* sv = big + warp * kCap;
-    int* si = reinterpret_cast<int*>(big + kWarps * kCap) + warp * kCap;
-    merge_lists_row(p.cand_val, p.cand_id, p.nparts, p.rows_total, b * D + t, sv, si, kCap, &surv_n[warp], cl[t],
-                    cand[t]);
+  // warp 0: row t; warp 1: row t - 1 (the sources), each in its own part of `big`
+  if (warp == 0 || (warp == 1 && t > 0)) {
+    float* sv = big + warp * 1024;
+    int* si = reinterpret_cast<int*>(big + warp * 1024 + 512);
+    selector_row(p, b * D + t - warp, sv, si, &surv[warp], cl[1 - warp], cand[1 - warp]);
   }
   __syncthreads();
-  if (threadIdx.x < D * kTopK) {
-    const int t = threadIdx.x / kTopK, k = threadIdx.x % kTopK;
-    const float v = cl[t][k];
-    int id = cand[t][k];
-    if (!isfinite(v)) set_err(p.err, DFLASH2_DEV_NONFINITE);
-    if (id < 0 || id >= p.V) {
-      set_err(p.err, DFLASH2_DEV_NONFINITE);
-      cand[t][k] = 0;
+  if (threadIdx.x < kTopK) {
+    const size_t o = (size_t)(b * D + t) * kTopK + threadIdx.x;
+    cl_g[o] = cl[1][threadIdx.x];
+    cand_g[o] = cand[1][threadIdx.x];
+    if (p.dbg_cand) {
+      p.dbg_cand[o] = cand[1][threadIdx.x];
+      p.dbg_logit[o] = cl[1][threadIdx.x];
+    }
+    if (t == 0) {
+      if (threadIdx.x == 0) {
+        int a = p.block_tokens[b * p.Bk];
+        src[0] = (a < 0 || a >= p.V) ? 0 : a;
+      }
+    } else {
+      src[threadIdx.x] = cand[0][threadIdx.x];
     }
   }
   __syncthreads();
+  selector_tau<256>(p, b, t, src, t == 0 ? 1 : kTopK, cand[1], As, Wj, tau_g + (size_t)(b * D + t) * kTopK * kTopK);
+}
 
-  selector_core<256>(p, b, cand, cl, As, Wj);
-  if (p.dbg_cand && threadIdx.x < D * kTopK) {
-    const int t = threadIdx.x / kTopK, k = threadIdx.x % kTopK;
-    p.dbg_cand[(b * D + t) * kTopK + k] = cand[t][k];
-    p.dbg_logit[(b * D + t) * kTopK + k] = cl[t][k];
-  }
+// One warp per request: the Viterbi path over the D positions.
+__global__ void __launch_bounds__(32) k_sel_viterbi(SelParams p, const float* tau_g, const float* cl_g,
+                                                    const int32_t* cand_g) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, D = p.Bk - 1;
+  selector_viterbi(p, b, cl_g + (size_t)b * D * kTopK, cand_g + (size_t)b * D * kTopK,
+                   tau_g + (size_t)b * D * kTopK * kTopK);
 }
 
 }  // namespace dfl
