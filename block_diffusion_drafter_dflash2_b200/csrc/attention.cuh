@@ -3,10 +3,11 @@
 // Work split (flash-decoding): one CTA per (request, kv head, chunk of 64 cache
 // keys = 4 pages) plus one CTA for the block's own keys.  The query vectors of
 // a kv head's group (G query heads x Bk block rows, padded to 16-row mma
-// tiles) attend to the chunk; each warp owns 16 query vectors.  K and V rows of
-// the chunk are brought into shared memory by the TMA engine (1-D bulk copies,
-// 256 bytes per row into a padded 272-byte stride, completion on an mbarrier
-// with a bounded wait).  Scores and P.V use mma.sync m16n8k16; softmax
+// tiles) attend to the chunk; each math warp owns 16 query vectors.  K and V
+// rows of the chunk are loaded into shared memory (272-byte padded stride) by
+// every thread of the CTA with 16-byte L2 loads, all issued before any store
+// (64 rows of 256 bytes as one bulk copy per row cost more in copy-engine
+// overhead than they move).  Scores and P.V use mma.sync m16n8k16; softmax
 // statistics are fp32.  A combine kernel merges the chunk partials.
 //
 // Visibility (FastFlowLM card, "Draft" row: sliding window 2048): block row t
@@ -42,11 +43,10 @@ DEVI void attn_geometry(const AttnParams& p, int b, long long& Lb, long long& cs
 
 // One chunk item (request b, kv head kvh, chunk c) processed by the first NTHR threads of the CTA
 // (named barrier 1); warps 0..MT-1 do the math.  buf: (MT*16 + 2*64) * 272 bytes of shared memory;
-// bar: an initialised mbarrier whose phase `phase` tracks across items; row_ok: 64 ints.
+// row_ok: 64 ints.
 // Returns without touching anything when the chunk lies outside the request's window.
 template <int MT, int NTHR>
-DEVI void attn_item(const AttnParams& p, int c, int kvh, int b, uint8_t* buf, uint64_t* bar, uint32_t& phase,
-                    int* row_ok) {
+DEVI void attn_item(const AttnParams& p, int c, int kvh, int b, uint8_t* buf, int* row_ok) {
   uint16_t* Qs = reinterpret_cast<uint16_t*>(buf);
   uint16_t* Ks = Qs + MT * 16 * kAttnStride;
   uint16_t* Vs = Ks + kAttnKeys * kAttnStride;
@@ -113,49 +113,42 @@ DEVI void attn_item(const AttnParams& p, int c, int kvh, int b, uint8_t* buf, ui
     if (threadIdx.x < kAttnKeys) row_ok[threadIdx.x] = threadIdx.x < p.Bk;
     consumers_sync<NTHR>();
   } else {
-    if (warp == 0) {
-      fence_proxy_async();  // cache rows written by earlier kernels/CTAs are read by the bulk copies
-      int ok[2];
-      int32_t pg[2];
+    // the chunk's 64 cache keys (4 pages) with 16-byte L2 loads by every thread, all issued before
+    // any store; keys past the request's length or on unmapped pages read as zero and are masked
+    constexpr int kVec = kAttnKeys * 16;  // 16-byte vectors per K (or V) chunk
+    constexpr int kPerKV = (kVec + NTHR - 1) / NTHR;
+    uint4 kr[kPerKV], vr[kPerKV];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int kk = lane + 32 * h;
+    for (int k = 0; k < kPerKV; ++k) {
+      const int i = threadIdx.x + k * NTHR, kk = i >> 4, v = i & 15;
+      kr[k] = vr[k] = make_uint4(0, 0, 0, 0);
+      if (i < kVec) {
         const long long j = key0 + kk;
-        ok[h] = 0;
-        pg[h] = -1;
+        bool ok = false;
         if (j < Lb) {
           const int lp = (int)(j / kPage);
-          pg[h] = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
-          if (pg[h] >= 0 && pg[h] < p.num_pages) ok[h] = 1;
-          else set_err(p.err, DFLASH2_DEV_PAGE);
+          const int32_t pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+          ok = pg >= 0 && pg < p.num_pages;
+          if (ok) {
+            const size_t off = (((size_t)pg * p.nkv + kvh) * kPage + j % kPage) * kHeadDim + v * 8;
+            kr[k] = __ldcg(reinterpret_cast<const uint4*>(p.kc + off));
+            vr[k] = __ldcg(reinterpret_cast<const uint4*>(p.vc + off));
+          } else if (v == 0) {
+            set_err(p.err, DFLASH2_DEV_PAGE);
+          }
         }
-        row_ok[kk] = ok[h];
+        if (v == 0) row_ok[kk] = ok;
       }
-      const int nvalid = __popc(__ballot_sync(0xffffffffu, ok[0])) + __popc(__ballot_sync(0xffffffffu, ok[1]));
-      if (lane == 0) mbar_expect_tx(bar, (uint32_t)nvalid * 2u * kHeadDim * 2u);
-      __syncwarp();
+    }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int kk = lane + 32 * h;
-        if (ok[h]) {
-          const long long j = key0 + kk;
-          const size_t off = (((size_t)pg[h] * p.nkv + kvh) * kPage + j % kPage) * kHeadDim;
-          bulk_g2s(Ks + kk * kAttnStride, p.kc + off, kHeadDim * 2, bar);
-          bulk_g2s(Vs + kk * kAttnStride, p.vc + off, kHeadDim * 2, bar);
-        } else {
-          uint4* kr = reinterpret_cast<uint4*>(Ks + kk * kAttnStride);
-          uint4* vr = reinterpret_cast<uint4*>(Vs + kk * kAttnStride);
-          for (int v = 0; v < 16; ++v) kr[v] = vr[v] = make_uint4(0, 0, 0, 0);
-        }
+    for (int k = 0; k < kPerKV; ++k) {
+      const int i = threadIdx.x + k * NTHR, kk = i >> 4, v = i & 15;
+      if (i < kVec) {
+        *reinterpret_cast<uint4*>(Ks + kk * kAttnStride + v * 8) = kr[k];
+        *reinterpret_cast<uint4*>(Vs + kk * kAttnStride + v * 8) = vr[k];
       }
     }
     consumers_sync<NTHR>();
-    const bool ok = mbar_wait_sleep_bounded(bar, phase);
-    phase ^= 1u;
-    if (!ok) {
-      if (threadIdx.x == 0) set_err(p.err, DFLASH2_DEV_TIMEOUT);
-      return;
-    }
   }
   if (warp >= MT) return;
 
@@ -246,20 +239,15 @@ DEVI void attn_item(const AttnParams& p, int c, int kvh, int b, uint8_t* buf, ui
 }
 
 
-template <int MT>  // 16-row query tiles per CTA (= warps)
-__global__ void __launch_bounds__(MT * 32) k_attn_chunk(AttnParams p) {
+constexpr int kAttnThreads = 256;  // loaders; the first MT warps also do the math
+
+template <int MT>  // 16-row query tiles per CTA (= math warps)
+__global__ void __launch_bounds__(kAttnThreads) k_attn_chunk(AttnParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bar;
   __shared__ int row_ok[kAttnKeys];
   pdl_trigger();
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
   pdl_wait();
-  uint32_t phase = 0;
-  attn_item<MT, MT * 32>(p, blockIdx.x, blockIdx.y, blockIdx.z, smem, &bar, phase, row_ok);
+  attn_item<MT, kAttnThreads>(p, blockIdx.x, blockIdx.y, blockIdx.z, smem, row_ok);
 }
 
 // One warp per (request, kv head, query vector): merge the chunk partials -> o bf16 [Mb][nq][128].

@@ -69,10 +69,9 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   const int ring = ns * slot;
   const int per_unit = g.R * unitK * 2;
   const int extra = kGemvConsumers * 1024 + kConsumers * 32 * g.NT * 4 * 4;  // per-warp scale tables, set reduction
-  const int sums = q4 ? g.R * 8 * 4 : 0;  // Q4: activation sums per staged unit (8 sub-blocks x R rows)
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
-  g.kc_units = std::max(1, std::min(g.U, budget / (per_unit + sums)));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra + (size_t)sums * g.kc_units;
+  g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
   return g;
 }
 
@@ -90,7 +89,6 @@ GemvPlan plan_gemv_persistent(int tiles, int rows, int K, bool q4, int nsm) {
   g.P = (int)std::min<long long>(nsm, g.W);  // every CTA in [0, P) owns at least one unit
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
   g.kc_units = std::max(1, std::min(g.U, (kPXBytes - 64 * g.R) / (g.R * unitK * 2)));
-  if (q4) g.kc_units = std::max(1, std::min(g.kc_units, kPSumBytes / (g.R * 8 * 4)));  // activation sums fit
   if (g.kc_units < g.U && g.kc_units > 1) g.kc_units &= ~1;  // whole slots (two units each) per chunk
   g.smem = 0;
   return g;
@@ -155,7 +153,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.persistent = B == 1 && p.Bk <= 8 && p.QVP == 32 && 8 * (p.H * 2 + 64) <= kPXBytes &&
                  (size_t)(p.MT * 16 + 2 * kAttnKeys) * kAttnStride * 2 <= (size_t)kPXBytes;
   p.psmem = (size_t)kPNS * kPSlot + kPXBytes + (size_t)kGemvConsumers * 128 * 8 + (size_t)kConsumers * 32 * 8 * 4 +
-            (size_t)kPSumBytes;
+            (size_t)kPWshBytes;
   if (p.persistent) {
     p.pfc = plan_gemv_persistent(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
     p.pdc = plan_gemv_persistent((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
@@ -342,7 +340,7 @@ cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(MT * 32), smem, s, ap);
+  return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(kAttnThreads), smem, s, ap);
 }
 
 int fail(cudaError_t e) { return e == cudaSuccess ? DFLASH2_OK : DFLASH2_ERR_CUDA; }

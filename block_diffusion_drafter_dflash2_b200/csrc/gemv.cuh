@@ -46,36 +46,17 @@ struct QkvEpi {
   int* err;
 };
 
-// Column sums of the staged activations per 32-wide sub-block, the X of y += D*S - M*X below:
-// xsum[b * R + r] = sum over the sub-block b of row r (bf16 values, fp32 sum), for the nk staged
-// columns of rows [0, R).  Computed once per staged chunk and shared by every warp.
-template <int NTHR>
-DEVI void x_sums(const uint8_t* Xs, int stride, int R, int nk, float* xsum) {
-  const int nsb = nk / 32;
-  for (int i = threadIdx.x; i < R * nsb; i += NTHR) {
-    const int r = i % R, b = i / R;
-    const uint4* x = reinterpret_cast<const uint4*>(Xs + r * stride + b * 64);
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 v = x[k];
-      s += bf2f(v.x & 0xffff) + bf2f(v.x >> 16) + bf2f(v.y & 0xffff) + bf2f(v.y >> 16) + bf2f(v.z & 0xffff) +
-           bf2f(v.z >> 16) + bf2f(v.w & 0xffff) + bf2f(v.w >> 16);
-    }
-    xsum[b * R + r] = s;
-  }
-}
-
 // One Q4_K group unit (16 rows x 256 k of one tile) against NT 8-row activation tiles.
 // q: the lane's 64 bytes of 4-bit codes (mma fragment order), sc: its feature's scale record.
 // Per 32-wide sub-block j: S = sum (128 + q) x by mma on the codes with the 0x4300 exponent
-// (bf16 128 + q exactly), then y += D*S - M*X with D = d*sc_j, M = dmin*m_j + 128*D and X the
-// sub-block's activation sum from xsum (R = 8 * NT rows per sub-block entry).
+// (bf16 128 + q exactly), X = sum x by an mma with all-ones weights, then
+// y += D*S - M*X with D = d*sc_j, M = dmin*m_j + 128*D.
 template <int NT>
 DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8_t* Xs, int stride, int kbyte,
-                  const float* xsum, int ntact, float (&acc)[NT][4], int lane) {
-  constexpr int R = NT * 8;
+                  int ntact, float (&acc)[NT][4], int lane) {
   const int g = lane >> 2, t = lane & 3;
+  // A = 1.0 in every slot: the mma then yields X_j = sum_k x_k (bf16 x, fp32 accumulate) per row
+  const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
   {
     // lane decodes (d*sc_j, dmin*m_j + 128*d*sc_j) of feature lane/2, sub-blocks 4*(lane&1) .. +3
     const int f = lane >> 1, jb = (lane & 1) * 4;
@@ -92,7 +73,6 @@ DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8
     }
     __syncwarp();
   }
-  const float* xs_unit = xsum + (kbyte / 512) * 8 * R;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t w0 = (j & 1) ? q[j >> 1].z : q[j >> 1].x;
@@ -111,15 +91,16 @@ DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8
     for (int nt = 0; nt < NT; ++nt) {
       if (nt < ntact) {
         const uint4 bx = *reinterpret_cast<const uint4*>(Xs + (nt * 8 + g) * stride + kbyte + j * 64 + t * 16);
-        const float2 xv = *reinterpret_cast<const float2*>(xs_unit + j * R + nt * 8 + 2 * t);
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, xs[4] = {0.f, 0.f, 0.f, 0.f};
         mma16816(s, a0, bx.x, bx.y);
         mma16816(s, a1, bx.z, bx.w);
+        mma16816(xs, ones, bx.x, bx.y);
+        mma16816(xs, ones, bx.z, bx.w);
         // acc += D * S - M * X, two accumulators per packed FMA
         float2 a01 = make_float2(acc[nt][0], acc[nt][1]), a23 = make_float2(acc[nt][2], acc[nt][3]);
-        a01 = ffma2(make_float2(-cg.y, -cg.y), xv, a01);
+        a01 = ffma2(make_float2(-cg.y, -cg.y), make_float2(xs[0], xs[1]), a01);
         a01 = ffma2(make_float2(cg.x, cg.x), make_float2(s[0], s[1]), a01);
-        a23 = ffma2(make_float2(-ch.y, -ch.y), xv, a23);
+        a23 = ffma2(make_float2(-ch.y, -ch.y), make_float2(xs[2], xs[3]), a23);
         a23 = ffma2(make_float2(ch.x, ch.x), make_float2(s[2], s[3]), a23);
         acc[nt][0] = a01.x;
         acc[nt][1] = a01.y;

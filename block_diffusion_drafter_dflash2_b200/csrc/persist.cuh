@@ -29,7 +29,7 @@ constexpr int kPNS = 3;
 constexpr int kPThreads = kGemvThreads;     // 16 consumer warps + 1 producer warp
 constexpr int kPNC = kGemvConsumers * 32;   // consumer threads
 constexpr int kPXBytes = 82944;             // activation staging (8 rows x 5120 bf16 + padding); attention buffers
-constexpr int kPSumBytes = 5120;            // combine weights [16][64] floats / Q4 activation sums
+constexpr int kPWshBytes = 4096;            // attention-combine weights [16 warps][64] floats
 constexpr long long kBarrierSpin = 1ll << 24;
 constexpr unsigned long long kBarrierNs = 2000000000ull;  // 2 s
 
@@ -195,7 +195,7 @@ struct PState {
   float2* coef;     // [16 warps][128]
   float* red;       // [8][32][8]
   float* rs;        // [16] row scales
-  float* wsh;       // [16 warps][64] attention-combine weights; Q4 activation sums during products (5 KB)
+  float* wsh;       // [16 warps][64] attention-combine weights
   int* row_ok;      // [64]
   int cnt;
   uint32_t xph, aph;
@@ -338,10 +338,6 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
         } else {
           stage_computed<R>(pg, S, k0, nk, stride, st);
         }
-        if (Q4) {
-          x_sums<kPNC>(st.Xs, stride, R, nk, st.wsh);  // the combine-weight region, free during products
-          consumers_sync<kPNC>();
-        }
         staged = true;
       }
       for (int k = 0; k < cu; k += kPUnits) {
@@ -358,7 +354,7 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
             for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
             sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
           }
-          if (have && ntact > 0) q4_unit<NT>(q, sc, coef, st.Xs, stride, (u - base) * 512, st.wsh, ntact, acc, lane);
+          if (have && ntact > 0) q4_unit<NT>(q, sc, coef, st.Xs, stride, (u - base) * 512, ntact, acc, lane);
           slot_release(&st.empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
         } else {
           uint4 wv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -657,8 +653,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_step_persistent(const __grid_c
       ap.kc = L.kc;
       ap.vc = L.vc;
       const int nitems = ap.nkv * (ap.NC + 1);
-      for (int it = c; it < nitems; it += P) attn_item<2, kPNC>(ap, it % (ap.NC + 1), it / (ap.NC + 1), 0, st.Xs,
-                                                                st.abar, st.aph, st.row_ok);
+      for (int it = c; it < nitems; it += P) attn_item<2, kPNC>(ap, it % (ap.NC + 1), it / (ap.NC + 1), 0, st.Xs, st.row_ok);
       grid_sync(S.gbar, epoch, S.err);
       const int G = ap.nq / ap.nkv, nw = ap.nkv * G * ap.Bk;
       for (int it = c * kGemvConsumers + warp; it < nw; it += P * kGemvConsumers)

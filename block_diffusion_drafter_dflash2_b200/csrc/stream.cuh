@@ -218,7 +218,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
   const int stride = p.kc_units * RC::kUnitK * 2 + 64;
   float2* coef_all = reinterpret_cast<float2*>(Xs + R * stride);                // [16 warps][128]
   float* red = reinterpret_cast<float*>(coef_all + kGemvConsumers * 128);       // [8][32][NT*4]
-  float* xsum = red + kConsumers * 32 * NT * 4;                                  // Q4: [kc_units * 8][R]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int set = warp / kConsumers, wt = warp % kConsumers;
 
@@ -292,19 +291,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
           if (staged_mz != mz) {
             stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx, p.ldx, stage_rows, R, p.U * RC::kUnitK * 2, Xs, stride, &xbar,
                               xph, p.err);
-            if (Q4) {
-              x_sums<NC>(Xs, stride, R, p.U * RC::kUnitK, xsum);
-              consumers_sync<NC>();
-            }
             staged_mz = mz;
           }
         } else {
           stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R,
                             cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err);
-          if (Q4) {
-            x_sums<NC>(Xs, stride, R, cu * RC::kUnitK, xsum);
-            consumers_sync<NC>();
-          }
         }
         for (int u = c0; u < c0 + cu; ++u) {
           const int slot = cnt % RC::kNS;
@@ -325,7 +316,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
             const uint4 sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
-            q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, xsum, ntact, acc, lane);
+            q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane);
             slot_release(&empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
           } else {
             uint4 wv[4];
