@@ -30,6 +30,19 @@ from block_diffusion_drafter_dflash2_b200 import accounting, inputs  # noqa: E40
 NOMINAL_HBM_GBS = 8000.0
 
 
+def head_traffic_ratio():
+    """DRAM bytes per algorithmic byte of the streaming LM-head kernel, from the committed ncu
+    summary of its small-case capture (None if the summary is missing)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_k_slmhead_prof_small.md")) as f:
+            for line in f:
+                if line.startswith("dram bytes per algorithmic byte:"):
+                    return float(line.split(":")[1])
+    except OSError:
+        pass
+    return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -275,11 +288,15 @@ def main():
     byt = accounting.step_bytes(dims, L_after, [Bk] * B)
     hbm, peak_kind = peaks()
     nk = dr.step_kernels()
+    traffic = None
     if nk == 1:  # the whole step is one persistent kernel: its bytes are the step's
         rk_name, rk_bytes = "k_step_persistent (whole block step, one cooperative launch)", byt["total"]
     else:
         rk_name = "k_slmhead / k_lmhead_topk (LM head + streaming top-16 + selector projection)"
         rk_bytes = accounting.lmhead_bytes(dims, B * D)
+        ratio = head_traffic_ratio() if B * D <= 8 else None  # captured for the streaming kernel
+        if ratio is not None:
+            traffic = ratio * rk_bytes  # small-case capture scaled by the launch's bytes
     rk_gbs = rk_bytes / (lm_ms * 1e-3) / 1e9
     value = ws / (ms_max * 1e-3)  # draft steps/s over all ranks (one step = a rank's whole batch)
     line = {
@@ -303,7 +320,7 @@ def main():
                      "frac_of_8tbs": byt["total"] / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                      "frac_of_measured": byt["total"] / (ms_max * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind},
         "roofline": {"kernel": rk_name, "bound": "hbm",
-                     "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm, "traffic": None,
+                     "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm, "traffic": traffic,
                      "algorithmic_bytes": rk_bytes, "avg_launch_ms": lm_ms, "peak_kind": peak_kind},
         "e2e": {"value": ws / (e2e_ms * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

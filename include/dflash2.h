@@ -154,10 +154,11 @@ size_t dflash2_prepared_size(const dflash2_config *cfg);
  * (device, 16-byte aligned, dst_bytes >= dflash2_prepared_size): the 8 tiles of 16 rows
  * of each column group interleaved per K unit (Q4_K: 256-wide super-blocks, codes in
  * mma fragment order; bf16: 64-wide steps), gate and up interleaved 4 + 4 tiles per
- * group, and the output head followed by the selector projection as one matrix padded
- * to whole groups.  Values are not changed: the prepared copy holds the same bits,
- * reordered.  Fills `out` (host struct) with `src`'s pointers except the streamed
- * matrices, which point into dst (wu aliases wg); out->prepared = 1.  The embedding
+ * group, and the output head followed by the selector projection as one matrix in
+ * records of 16 tiles per 64-wide step (32 KB), padded to whole records.  Values are not
+ * changed: the prepared copy holds the same bits, reordered.  Fills `out` (host struct)
+ * with `src`'s pointers except the streamed matrices, which point into dst (wu aliases
+ * wg; lm_head and sel_proj both point at the combined head); out->prepared = 1.  The embedding
  * table, norms, static taps and codebooks stay where they are.  Asynchronous on `stream`. */
 int dflash2_prepare_weights(const dflash2_config *cfg, const dflash2_weights *src, void *dst,
                             size_t dst_bytes, dflash2_weights *out, void *stream);
