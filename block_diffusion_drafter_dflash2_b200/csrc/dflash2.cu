@@ -279,6 +279,15 @@ struct Epi {
   uint16_t* act = nullptr;
   int F = 0;
   QkvEpi qkv{};
+  // RMSNorm folding (see SGemvParams): residual epilogues write hw and ssp; consumers scale by rs
+  float* ssp = nullptr;
+  int ssp_rows = 0;
+  uint16_t* hw = nullptr;
+  const uint16_t* hw_w = nullptr;
+  int hw_ld = 0;
+  const float* rs_in = nullptr;
+  int rs_H = 0;
+  float eps = 0.f;
 };
 
 SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X, int ldx,
@@ -306,6 +315,14 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   prm.act = e.act;
   prm.F = e.F;
   prm.qkv = e.qkv;
+  prm.ssp = e.ssp;
+  prm.ssp_rows = e.ssp_rows;
+  prm.hw = e.hw;
+  prm.hw_w = e.hw_w;
+  prm.hw_ld = e.hw_ld;
+  prm.rs_in = e.rs_in;
+  prm.rs_H = e.rs_H;
+  prm.eps = e.eps;
   prm.err = err;
   return prm;
 }
@@ -723,8 +740,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
     return DFLASH2_OK;
   }
-  // A1: block rows from the shared embedding table
-  CK(launch_pdl(k_embed, dim3(Mb), dim3(256), 0, s, in->block_tokens, w->embed, h, H, P.V, err));
+  // A1: block rows from the shared embedding table (+ the first RMSNorm's inputs: h * ln1 and the
+  // rows' sums of squares; every RMSNorm before a product is folded the same way: the residual
+  // epilogues write bf16(h * w) and sums of squares, the product scales its outputs per row)
+  float* ssp = at<float>(ws, P.off_ssp);
+  CK(launch_pdl(k_embed, dim3(Mb), dim3(256), 0, s, in->block_tokens, w->embed, h, H, P.V, err, xb, w->layer[0].ln1,
+                ssp, Mb));
   if (dbg && dbg->hidden) CK(cudaMemcpyAsync(dbg->hidden, h, hbytes, cudaMemcpyDeviceToDevice, s));
 
   // A2: context rows = RMSNorm_fc(W_fc . concat(taps)); fc output staged in xf
@@ -753,19 +774,9 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   for (int l = 0; l < c->layers; ++l) {
     const dflash2_layer_weights& L = w->layer[l];
     int* lctr = ctr + P.ctr_fc + (size_t)l * P.ctr_per_layer;
-    // A3a: x = RMSNorm(h; ln1), g = W_dc x, y = dynconv(x, g)
+    // A3a: x = RMSNorm(h; ln1), g = W_dc x (operand xb = bf16(h * ln1), outputs scaled by the row
+    // scale), y = dynconv(x, g)
     {
-      NormParams np{};
-      np.in = h;
-      np.w = L.ln1;
-      np.eps = c->rms_eps;
-      np.H = H;
-      np.out_bf = xb;
-      np.ldob = H;
-      np.out_f = xf;
-      np.mode = 0;
-      np.Bk = P.Bk;
-      CK(launch_norm(np, Mb, s));
       if (dbg && dbg->hidden && l > 0)
         CK(cudaMemcpyAsync(dbg->hidden + (size_t)l * Mb * H, h, hbytes, cudaMemcpyDeviceToDevice, s));
       GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
@@ -773,9 +784,13 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       e.mode = EPI_STORE;
       e.y = gbuf;
       e.ldy = H / 2;
+      e.rs_in = ssp;
+      e.ssp_rows = Mb;
+      e.rs_H = H;
+      e.eps = c->rms_eps;
       CK(launch_gemv(P.dc, false, &seg, 1, false, xb, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err, s));
-      CK(launch_pdl(k_dynconv, dim3(Mb, (H / 4 + 255) / 256), dim3(256), 0, s, (const float*)xf, (const float*)gbuf,
-                    L.dc_s0, L.dc_s1, H, P.Bk, yb));
+      CK(launch_pdl(k_dynconv, dim3(Mb, (H / 4 + 255) / 256), dim3(256), 0, s, (const float*)h, (const float*)ssp, Mb,
+                    L.ln1, c->rms_eps, (const float*)gbuf, L.dc_s0, L.dc_s1, H, P.Bk, yb));
     }
     // A3b+c: q from the block rows; k, v from block + context rows (stacked: each matrix read once);
     // the last CTA of each head applies q/k RMSNorm + RoPE and appends context K/V to the cache
@@ -827,17 +842,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       e.mode = EPI_RESID;
       e.y = h;
       e.ldy = H;
+      e.hw = xb;  // bf16(h * ln2) and sums of squares for the gate/up product
+      e.hw_w = L.ln2;
+      e.hw_ld = H;
+      e.ssp = ssp;
+      e.ssp_rows = Mb;
       CK(launch_gemv(P.o, P.q4, &seg, 1, false, ob, P.HQ, Mb, part, H, Mb, lctr + P.ctr_layer[2], e, err, s));
-      NormParams np{};
-      np.in = h;
-      np.w = L.ln2;
-      np.eps = c->rms_eps;
-      np.H = H;
-      np.out_bf = xb;
-      np.ldob = H;
-      np.mode = 0;
-      np.Bk = P.Bk;
-      CK(launch_norm(np, Mb, s));
     }
     // A3f: h += W_d (silu(W_g x2) * W_u x2); gate and up tiles paired per CTA so the SwiGLU is fused
     {
@@ -846,12 +856,23 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       e.mode = EPI_SWIGLU;
       e.act = act;
       e.F = P.F;
+      e.rs_in = ssp;
+      e.ssp_rows = Mb;
+      e.rs_H = H;
+      e.eps = c->rms_eps;
       CK(launch_gemv(P.gu, P.q4, segs, 2, true, xb, H, Mb, part, 2 * P.F, Mb, lctr + P.ctr_layer[3], e, err, s));
       GemvSeg seg{(const uint8_t*)L.wd, H / 16, Mb, 0};
       Epi e2;
       e2.mode = EPI_RESID;
       e2.y = h;
       e2.ldy = H;
+      if (l + 1 < c->layers) {  // bf16(h * ln1') and sums of squares for the next layer
+        e2.hw = xb;
+        e2.hw_w = w->layer[l + 1].ln1;
+        e2.hw_ld = H;
+        e2.ssp = ssp;
+        e2.ssp_rows = Mb;
+      }
       CK(launch_gemv(P.dn, P.q4, &seg, 1, false, act, P.F, Mb, part, H, Mb, lctr + P.ctr_layer[4], e2, err, s));
     }
   }
@@ -1011,9 +1032,9 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   if (!cfg_ok(c) || batch < 1) return 0;
   const Plan P = make_plan(c, batch);
   if (P.persistent && persistent_ready(P)) return 1;
-  // embed, fc GEMV, fc norm | per layer: norm, W_dc GEMV, dynconv, QKV GEMV, attention, combine,
-  // W_o GEMV, norm, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
-  return 3 + 10 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
+  // embed, fc GEMV, fc norm | per layer: W_dc GEMV, dynconv, QKV GEMV, attention, combine, W_o GEMV,
+  // gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
+  return 3 + 8 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

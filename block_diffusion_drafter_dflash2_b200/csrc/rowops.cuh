@@ -6,22 +6,37 @@
 namespace dfl {
 
 // h[r] = E[block_tokens[r]] (fp32); ids outside [0, V) flag DFLASH2_DEV_TOKEN and read row 0.
+// Also the first RMSNorm's inputs: hw[r] = bf16(h[r] * w) and the row's sums of squares per
+// 32-column quarter, ssp[q][ldr] (the consumer applies the row scale).
 __global__ void k_embed(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E, float* __restrict__ h,
-                        int H, int V, int* err) {
+                        int H, int V, int* err, uint16_t* __restrict__ hw, const uint16_t* __restrict__ w,
+                        float* __restrict__ ssp, int ldr) {
   pdl_trigger();
   pdl_wait();
-  const int r = blockIdx.x;
+  const int r = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int id = tok[r];
   if (id < 0 || id >= V) {
     if (threadIdx.x == 0) set_err(err, DFLASH2_DEV_TOKEN);
     id = 0;
   }
-  const uint4* e = reinterpret_cast<const uint4*>(E + (size_t)id * H);
+  const uint16_t* erow = E + (size_t)id * H;
+  const uint4* e = reinterpret_cast<const uint4*>(erow);
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const uint4 v = e[c];
+    const uint4 v = e[c], wv = reinterpret_cast<const uint4*>(w)[c];
     float4* o = reinterpret_cast<float4*>(h + (size_t)r * H + c * 8);
     o[0] = make_float4(bf2f(v.x & 0xffff), bf2f(v.x >> 16), bf2f(v.y & 0xffff), bf2f(v.y >> 16));
     o[1] = make_float4(bf2f(v.z & 0xffff), bf2f(v.z >> 16), bf2f(v.w & 0xffff), bf2f(v.w >> 16));
+    const uint32_t vv[4] = {v.x, v.y, v.z, v.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      out[k] = pack_bf2(bf2f(vv[k] & 0xffff) * bf2f(ww[k] & 0xffff), bf2f(vv[k] >> 16) * bf2f(ww[k] >> 16));
+    reinterpret_cast<uint4*>(hw + (size_t)r * H)[c] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  for (int q = warp; q < H / 32; q += blockDim.x >> 5) {
+    const float v = bf2f(erow[q * 32 + lane]);
+    const float s = warp_sum(v * v);
+    if (lane == 0) ssp[(size_t)q * ldr + r] = s;
   }
 }
 
@@ -104,24 +119,40 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
   }
 }
 
-// y_t[c] = (s0[c] + tanh g_t[c/4]) x_t[c] + (s1[c] + tanh g_t[H/4 + c/4]) x_{t-1}[c], x_{-1} = 0.
-// Thread = 4 channels sharing one gate pair; grid (rows, H/1024).
-__global__ void k_dynconv(const float* __restrict__ xf, const float* __restrict__ g, const uint16_t* __restrict__ s0,
-                          const uint16_t* __restrict__ s1, int H, int Bk, uint16_t* __restrict__ y) {
+// y_t[c] = (s0[c] + tanh g_t[c/4]) x_t[c] + (s1[c] + tanh g_t[H/4 + c/4]) x_{t-1}[c], x_{-1} = 0,
+// with x = RMSNorm(h; w) formed here from the residual rows and their quarter-column sums of
+// squares ssp[q][ldr].  Thread = 4 channels sharing one gate pair; grid (rows, H/1024).
+__global__ void k_dynconv(const float* __restrict__ hres, const float* __restrict__ ssp, int ldr,
+                          const uint16_t* __restrict__ w, float eps, const float* __restrict__ g,
+                          const uint16_t* __restrict__ s0, const uint16_t* __restrict__ s1, int H, int Bk,
+                          uint16_t* __restrict__ y) {
+  __shared__ float rs2[2];
   pdl_trigger();
   pdl_wait();
-  const int r = blockIdx.x, t = r % Bk, G = H / 4;
-  const int q = blockIdx.y * blockDim.x + threadIdx.x;
-  if (q >= G) return;
-  const float a0 = tanhf(g[(size_t)r * (H / 2) + q]), a1 = tanhf(g[(size_t)r * (H / 2) + G + q]);
-  const float4 xc = reinterpret_cast<const float4*>(xf + (size_t)r * H)[q];
-  const float4 xp = t > 0 ? reinterpret_cast<const float4*>(xf + (size_t)(r - 1) * H)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint2 w0 = *reinterpret_cast<const uint2*>(s0 + 4 * q), w1 = *reinterpret_cast<const uint2*>(s1 + 4 * q);
-  const float y0 = (bf2f(w0.x & 0xffff) + a0) * xc.x + (bf2f(w1.x & 0xffff) + a1) * xp.x;
-  const float y1 = (bf2f(w0.x >> 16) + a0) * xc.y + (bf2f(w1.x >> 16) + a1) * xp.y;
-  const float y2 = (bf2f(w0.y & 0xffff) + a0) * xc.z + (bf2f(w1.y & 0xffff) + a1) * xp.z;
-  const float y3 = (bf2f(w0.y >> 16) + a0) * xc.w + (bf2f(w1.y >> 16) + a1) * xp.w;
-  *reinterpret_cast<uint2*>(y + (size_t)r * H + 4 * q) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
+  const int r = blockIdx.x, t = r % Bk, G = H / 4, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 2) {  // row scales of rows r (warp 0) and r - 1 (warp 1)
+    const int rr = r - warp;
+    float q = 0.f;
+    if (warp == 0 || t > 0)
+      for (int i = lane; i < H / 32; i += 32) q += ssp[(size_t)i * ldr + rr];
+    q = warp_sum(q);
+    if (lane == 0) rs2[warp] = (warp == 0 || t > 0) ? rsqrtf(q / H + eps) : 0.f;
+  }
+  __syncthreads();
+  const int qi = blockIdx.y * blockDim.x + threadIdx.x;
+  if (qi >= G) return;
+  const float a0 = tanhf(g[(size_t)r * (H / 2) + qi]), a1 = tanhf(g[(size_t)r * (H / 2) + G + qi]);
+  const float4 hc = reinterpret_cast<const float4*>(hres + (size_t)r * H)[qi];
+  const float4 hp = t > 0 ? reinterpret_cast<const float4*>(hres + (size_t)(r - 1) * H)[qi] : make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint2 wv = *reinterpret_cast<const uint2*>(w + 4 * qi);
+  const uint2 w0 = *reinterpret_cast<const uint2*>(s0 + 4 * qi), w1 = *reinterpret_cast<const uint2*>(s1 + 4 * qi);
+  const float n0 = bf2f(wv.x & 0xffff), n1 = bf2f(wv.x >> 16), n2 = bf2f(wv.y & 0xffff), n3 = bf2f(wv.y >> 16);
+  const float rc = rs2[0], rp = rs2[1];
+  const float y0 = (bf2f(w0.x & 0xffff) + a0) * (hc.x * rc * n0) + (bf2f(w1.x & 0xffff) + a1) * (hp.x * rp * n0);
+  const float y1 = (bf2f(w0.x >> 16) + a0) * (hc.y * rc * n1) + (bf2f(w1.x >> 16) + a1) * (hp.y * rp * n1);
+  const float y2 = (bf2f(w0.y & 0xffff) + a0) * (hc.z * rc * n2) + (bf2f(w1.y & 0xffff) + a1) * (hp.z * rp * n2);
+  const float y3 = (bf2f(w0.y >> 16) + a0) * (hc.w * rc * n3) + (bf2f(w1.y >> 16) + a1) * (hp.w * rp * n3);
+  *reinterpret_cast<uint2*>(y + (size_t)r * H + 4 * qi) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
 }
 
 __global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,

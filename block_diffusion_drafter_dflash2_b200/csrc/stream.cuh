@@ -88,8 +88,31 @@ struct SGemvParams {
   QkvEpi qkv;
   float* ssp;         // EPI_RESID: per-row sums of squares of the new rows, or null
   int ssp_rows;       // row stride of ssp: [column group][quarter][ssp_rows]
+  // RMSNorm folded into the products.  EPI_RESID with hw: also hw = bf16(h_new * hw_w) (the next
+  // norm's weight applied, its row scale not); the consumer of hw (EPI_STORE / EPI_SWIGLU with
+  // rs_in) multiplies its outputs by the row scale rs = 1/sqrt(mean(h^2) + eps) from rs_in, the
+  // quarter-column sums of squares the residual epilogue left.
+  uint16_t* hw;
+  const uint16_t* hw_w;
+  int hw_ld;
+  const float* rs_in;
+  int rs_H;
+  float eps;
   int* err;
 };
+
+// Row scales of rows [mz, mz + rows) from quarter-column sums of squares (ssp layout
+// [H/128][4][ldr]) into s_rs[0 .. rows); warp r handles row r.  Consumer threads (barrier 1).
+DEVI void rows_scale(const float* ssp, int ldr, int H, float eps, int mz, int rows, float* s_rs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nq = (H >> 7) * 4;
+  for (int r = warp; r < rows; r += kGemvConsumers) {
+    float q = 0.f;
+    for (int i = lane; i < nq; i += 32) q += __ldcg(ssp + (size_t)i * ldr + mz + r);
+    q = warp_sum(q);
+    if (lane == 0) s_rs[r] = rsqrtf(q / H + eps);
+  }
+  consumers_sync<kGemvConsumers * 32>();
+}
 
 // Owner CTA of global position x when [0, W) is cut into P ranges [c*W/P, (c+1)*W/P).
 DEVI long long sk_owner(long long x, long long W, long long P) { return ((x + 1) * P + W - 1) / W - 1; }
@@ -130,24 +153,47 @@ DEVI int sk_rows(const SGemvParams& p, int si, int mz, int R) {
   return r > R ? R : (r < 0 ? 0 : r);
 }
 
+// Sum of the split-K partials of one output in piece order (deterministic); the loads go out in
+// batches of 8 before they are added, so a fix-up costs one or two L2 round trips, not npieces.
 DEVI float sum_pieces(const SGemvParams& p, int npieces, int row, int col) {
   const float* b = p.part + (size_t)row * p.ldo + col;
   float v = 0.f;
-  for (int s = 0; s < npieces; ++s) v += __ldcg(b + (size_t)s * p.piece_stride);
+  for (int s0 = 0; s0 < npieces; s0 += 8) {
+    float x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = s0 + k < npieces ? __ldcg(b + (size_t)(s0 + k) * p.piece_stride) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v += x[k];
+  }
   return v;
 }
 
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   const int tid = threadIdx.x, nthr = kGemvConsumers * 32, warp = tid >> 5, lane = tid & 31;
+  __shared__ float s_rs[64];
   if (p.paired) {
     const int f0 = grp * 64;
     const int rows = sk_rows(p, 0, mz, R);
-    for (int i = tid; i < rows * 64; i += nthr) {
-      const int r = i >> 6, f = f0 + (i & 63);
-      const float gv = sum_pieces(p, npieces, mz + r, p.seg[0].out_col + f);
-      const float uv = sum_pieces(p, npieces, mz + r, p.seg[1].out_col + f);
-      p.act[(size_t)(mz + r) * p.F + f] = f2bf(gv / (1.f + __expf(-gv)) * uv);
+    if (p.rs_in) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
+    // two outputs per thread per round: all their partial loads are in flight together
+    for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
+      float gv[2], uv[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
+        const bool ok = i < rows * 64;
+        gv[k] = ok ? sum_pieces(p, npieces, mz + r, p.seg[0].out_col + f) : 0.f;
+        uv[k] = ok ? sum_pieces(p, npieces, mz + r, p.seg[1].out_col + f) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
+        if (i >= rows * 64) continue;
+        const float sc = p.rs_in ? s_rs[r] : 1.f;
+        const float g = gv[k] * sc, u = uv[k] * sc;
+        p.act[(size_t)(mz + r) * p.F + f] = f2bf(g / (1.f + __expf(-g)) * u);
+      }
     }
     return;
   }
@@ -156,6 +202,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   if (tile0 < 0) return;
   const int col0 = p.seg[si].out_col + tile0 * 16;
   const int rows = sk_rows(p, si, mz, R);
+  if (p.rs_in && p.epi == EPI_STORE) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
   if (p.epi == EPI_QKV) {
     const int head = tile0 / 8;
     for (int r = warp; r < rows; r += kGemvConsumers) {
@@ -167,19 +214,34 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
     }
     return;
   }
-  for (int i = tid; i < rows * 128; i += nthr) {
-    const int r = i >> 7, c = col0 + (i & 127);
-    const float v = sum_pieces(p, npieces, mz + r, c);
-    float* y = p.y + (size_t)(mz + r) * p.ldy + c;
-    if (p.epi == EPI_RESID) {
-      const float nv = __ldcg(y) + v;  // L2 read: another CTA may have written it
-      *y = nv;
-      if (p.ssp) {  // sum of squares of this warp's 32 columns of the new row, for the next RMSNorm
-        const float q = warp_sum(nv * nv);
-        if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
+  // four outputs per thread per round: all their partial loads (and the residual reads) are in
+  // flight together before any store
+  for (int i0 = tid; i0 < rows * 128; i0 += 4 * nthr) {
+    float v[4], old[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = i0 + k * nthr, r = i >> 7, c = col0 + (i & 127);
+      const bool ok = i < rows * 128;
+      v[k] = ok ? sum_pieces(p, npieces, mz + r, c) : 0.f;
+      // L2 read: another CTA may have written the residual row
+      old[k] = ok && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)(mz + r) * p.ldy + c) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = i0 + k * nthr, r = i >> 7, c = col0 + (i & 127);
+      if (i >= rows * 128) break;  // warp-uniform: rows * 128 is a multiple of 32
+      float* y = p.y + (size_t)(mz + r) * p.ldy + c;
+      if (p.epi == EPI_RESID) {
+        const float nv = old[k] + v[k];
+        *y = nv;
+        if (p.hw) p.hw[(size_t)(mz + r) * p.hw_ld + c] = f2bf(nv * bf2f(p.hw_w[c]));
+        if (p.ssp) {  // sum of squares of this warp's 32 columns of the new row, for the next RMSNorm
+          const float q = warp_sum(nv * nv);
+          if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
+        }
+      } else {
+        *y = p.rs_in ? v[k] * s_rs[r] : v[k];
       }
-    } else {
-      *y = v;
     }
   }
 }
