@@ -32,13 +32,13 @@ struct Plan {
   GemvPlan fc, dc, qkv, o, gu, dn;
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
   bool persistent;
-  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau;
+  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart;
   int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
   bool lm_stream;
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
       off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
-  size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_total;
+  size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_head, ctr_total;
   size_t off_s_taps, off_s_nnew, off_s_btok, off_s_tgt, off_s_path, off_s_scores, off_s_acc, off_s_emit;
   size_t step_bytes, total;
 };
@@ -141,7 +141,7 @@ Plan make_plan(const dflash2_config* c, int B) {
     p.lm_NT = 1;
     p.lm_rows_per_pass = 8;
     p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
-    p.lm_nparts = std::min(p.nsm, (lm_tiles + kHeadTiles - 1) / kHeadTiles);
+    p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
   } else {
     p.lm_NT = 2;
     p.lm_rows_per_pass = 16;
@@ -208,6 +208,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_cfi = take((size_t)p.lm_rows * kTopK * 4);
   p.off_ssp = take((size_t)(p.H / 128) * 4 * p.Mb * 4);
   p.off_tau = take((size_t)p.lm_rows * kTopK * kTopK * 4);
+  p.off_hpart = take(p.lm_stream ? (size_t)p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4 : 0);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
@@ -220,7 +221,8 @@ Plan make_plan(const dflash2_config* c, int B) {
     acc += nctr(*lp[i]);
   }
   p.ctr_per_layer = acc;
-  p.ctr_total = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer + 1;  // + the persistent step's grid barrier
+  p.ctr_head = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;  // the streaming head's record tickets
+  p.ctr_total = p.ctr_head + (size_t)(lm_tiles + kHeadTiles - 1) / kHeadTiles + 1;  // + the persistent grid barrier
   p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
   p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
@@ -912,6 +914,8 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       lp.z = zbuf;
       lp.cand_val = at<float>(ws, P.off_cv);
       lp.cand_id = at<int32_t>(ws, P.off_ci);
+      lp.part = at<float>(ws, P.off_hpart);
+      lp.counters = ctr + P.ctr_head;
       lp.err = err;
       CK(launch_pdl(k_slmhead, dim3(P.lm_nparts), dim3(kGemvThreads), P.lm_smem, s, lp));
     } else {

@@ -494,30 +494,18 @@ DEVI void offer_tile(uint2* lists, const float (&acc)[4], int id0, int rows, int
   }
 }
 
-// Merge the 16 warp lists of each row into the CTA's list (lane: warp lane/2, entries
-// 8*(lane&1) .. +7) -> cand_val/cand_id[part][row][16].
+// Merge the 16 warp lists of each row into the CTA's list -> cand_val/cand_id[part][row][16].
+// Lane l owns a sorted run of 8 entries (warp list l/2, entries 8*(l&1) .. +7) and a read position;
+// each round the warp picks the best run head (ties: lower lane) and that lane advances.
 DEVI void merge_warp_lists(const uint2* lists, int rows, float* cand_val, int32_t* cand_id, int part, int warp,
                            int nwarps, int lane) {
   for (int r = warp; r < rows; r += nwarps) {
-    float v[8];
-    int id[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint2 e = lists[((lane >> 1) * 8 + r) * kTopK + (lane & 1) * 8 + i];
-      v[i] = __uint_as_float(e.x);
-      id[i] = (int)e.y;
-    }
+    const uint2* run = lists + ((lane >> 1) * 8 + r) * kTopK + (lane & 1) * 8;
+    int pos = 0;
     for (int kk = 0; kk < kTopK; ++kk) {
-      int bi = 0;
-#pragma unroll
-      for (int i = 1; i < 8; ++i)
-        if (better(v[i], id[i], v[bi], id[bi])) bi = i;
-      float bv = v[0];
-      int bid = id[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i)
-        if (i == bi) { bv = v[i]; bid = id[i]; }
-      int bl = lane;
+      const uint2 e = pos < 8 ? run[pos] : make_uint2(__float_as_uint(-INFINITY), 0x7fffffffu);
+      float bv = __uint_as_float(e.x);
+      int bid = (int)e.y, bl = lane;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -530,11 +518,7 @@ DEVI void merge_warp_lists(const uint2* lists, int rows, float* cand_val, int32_
         cand_val[o] = bv;
         cand_id[o] = bid;
       }
-      if (lane == bl) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i == bi) { v[i] = -INFINITY; id[i] = 0x7fffffff; }
-      }
+      if (lane == bl) ++pos;
     }
   }
 }
@@ -547,17 +531,24 @@ struct SLmParams {
   float* z;           // [rows][R]
   float* cand_val;    // [gridDim.x][rows][16]
   int32_t* cand_id;
+  float* part;        // split records' partial accumulators [gridDim.x][2][16 warps][32 lanes][4]
+  int* counters;      // [records] arrival tickets, zero before the launch (the last arrival re-zeroes)
   int* err;
 };
 
 constexpr int kHeadSlot = kHeadTiles * 2048;  // one record step: 32 KB
 constexpr int kHeadNS = 3;
 
+// Work split: stream-K over (record, K step) units, CTA c taking [c*W/P, (c+1)*W/P) of the
+// W = records * (H/64) steps, so every SM streams the same number of bytes.  A record cut between
+// CTAs leaves each owner's accumulators in `part`; the last owner to arrive (arrival ticket, no
+// waiting) adds them in owner order (deterministic) and offers the tile's logits.
 __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kHeadNS];
   __shared__ __align__(8) uint64_t empty[kHeadNS];
   __shared__ __align__(8) uint64_t xbar;
+  __shared__ int s_last;
   constexpr int NC = kGemvConsumers * 32;
   const int H = p.H, stride = H * 2 + 64;
   uint8_t* ring = smem;
@@ -567,6 +558,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
   const int half = warp >> 3, wt = warp & 7;
   const int vt = p.V / 16, total = vt + p.R / 16, S = H / 64;
   const int nrec = (total + kHeadTiles - 1) / kHeadTiles;
+  const long long W = (long long)nrec * S, P = gridDim.x, c = blockIdx.x;
+  const long long x0 = c * W / P, x1 = (c + 1) * W / P;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kHeadNS; ++s) {
@@ -580,19 +573,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
   pdl_trigger();
 
   if (warp == kGemvConsumers) {
+    // ---- producer: this CTA's range of record steps is one contiguous stretch of the head ----
     if (lane != 0) return;
     int cnt = 0;
-    for (int rec = blockIdx.x; rec < nrec; rec += gridDim.x)
-      for (int s = 0; s < S; ++s) {
-        const int slot = cnt % kHeadNS, round = cnt / kHeadNS;
-        if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
-          set_err(p.err, DFLASH2_DEV_TIMEOUT);
-          return;
-        }
-        mbar_expect_tx(&full[slot], kHeadSlot);
-        bulk_g2s(ring + slot * kHeadSlot, p.W + ((size_t)rec * S + s) * kHeadSlot, kHeadSlot, &full[slot]);
-        ++cnt;
+    for (long long x = x0; x < x1; ++x) {
+      const int slot = cnt % kHeadNS, round = cnt / kHeadNS;
+      if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
+        set_err(p.err, DFLASH2_DEV_TIMEOUT);
+        return;
       }
+      mbar_expect_tx(&full[slot], kHeadSlot);
+      bulk_g2s(ring + slot * kHeadSlot, p.W + (size_t)x * kHeadSlot, kHeadSlot, &full[slot]);
+      ++cnt;
+    }
     return;
   }
 
@@ -604,10 +597,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
   uint2* my = lists + warp * 8 * kTopK;
   int cnt = 0;
   bool dead = false;
-  for (int rec = blockIdx.x; rec < nrec; rec += gridDim.x) {
+  const int rec_first = (int)(x0 / S);
+  for (long long x = x0; x < x1;) {
+    const int rec = (int)(x / S), s0 = (int)(x % S);
+    const int s1 = (x1 - x) < (long long)(S - s0) ? s0 + (int)(x1 - x) : S;
     const int tile = rec * kHeadTiles + half * 8 + wt;
     float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-    for (int s = 0; s < S; ++s) {
+    for (int s = s0; s < s1; ++s) {
       const int slot = cnt % kHeadNS;
       if (!dead && !mbar_wait_sleep_bounded(&full[slot], (cnt / kHeadNS) & 1)) {
         set_err(p.err, DFLASH2_DEV_TIMEOUT);
@@ -625,7 +621,45 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
       bf16_step<1, 2>(wv, Xs, stride, s * 128, 1, acc, lane);
       slot_release(&empty[slot], wv[0].x ^ wv[1].x ^ wv[2].x ^ wv[3].x, lane);
     }
-    if (dead || tile >= total) continue;
+    x += s1 - s0;
+    bool have = true;
+    if (s0 > 0 || s1 < S) {
+      // a record cut between CTAs: owners first..last of its steps
+      const long long ux = (long long)rec * S;
+      const long long first = sk_owner(ux, W, P), last = sk_owner(ux + S - 1, W, P);
+      const int k = rec == rec_first ? 0 : 1;
+      float4* mine = reinterpret_cast<float4*>(p.part) + ((c * 2 + k) * kGemvConsumers + warp) * 32 + lane;
+      *mine = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+      __threadfence();
+      consumers_sync<NC>();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(p.counters + rec, 1);
+        s_last = prev == (int)(last - first);
+        if (s_last) p.counters[rec] = 0;
+      }
+      consumers_sync<NC>();
+      have = s_last != 0;
+      if (have) {
+        __threadfence();
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        for (long long o = first; o <= last; ++o) {
+          float4 v;
+          if (o == c) {
+            v = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+          } else {
+            const int ko = rec == (int)((o * W / P) / S) ? 0 : 1;
+            v = __ldcg(reinterpret_cast<const float4*>(p.part) + ((o * 2 + ko) * kGemvConsumers + warp) * 32 + lane);
+          }
+          a[0] += v.x;
+          a[1] += v.y;
+          a[2] += v.z;
+          a[3] += v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][e] = a[e];
+      }
+    }
+    if (!have || dead || tile >= total) continue;
     if (tile >= vt) {
       const int c0 = (tile - vt) * 16;
 #pragma unroll
