@@ -290,6 +290,10 @@ struct Epi {
   const float* rs_in = nullptr;
   int rs_H = 0;
   float eps = 0.f;
+  const float* dyn_h = nullptr;
+  const uint16_t *dyn_w = nullptr, *dyn_s0 = nullptr, *dyn_s1 = nullptr;
+  uint16_t* dyn_y = nullptr;
+  int Bk = 1;
 };
 
 SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X, int ldx,
@@ -325,6 +329,12 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   prm.rs_in = e.rs_in;
   prm.rs_H = e.rs_H;
   prm.eps = e.eps;
+  prm.dyn_h = e.dyn_h;
+  prm.dyn_w = e.dyn_w;
+  prm.dyn_s0 = e.dyn_s0;
+  prm.dyn_s1 = e.dyn_s1;
+  prm.dyn_y = e.dyn_y;
+  prm.Bk = e.Bk;
   prm.err = err;
   return prm;
 }
@@ -503,7 +513,12 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
     O.wg = O.wu = d;
     d += 2 * bytes(F, H, q4);
     O.wd = prep(S.wd, H, F, q4);
-    O.dc_w = (const uint16_t*)prep(S.dc_w, 2 * (H / 4), H, false);
+    // the convolution's gate generators a0 | a1 interleaved 4 + 4 tiles per group (both gates of a
+    // channel group in one CTA's fix-up); dc_w points at the pair
+    place(S.dc_w, H / 4, H, false, PrepPlace{0, 4, 0, 8});
+    place(S.dc_w + (size_t)(H / 4) * H, H / 4, H, false, PrepPlace{0, 4, 4, 8});
+    O.dc_w = (const uint16_t*)d;
+    d += bytes(2 * (H / 4), H, false);
   }
   // the output head and the selector projection as one [V + R, H] matrix in records of 16 tiles
   // (32 KB per 64-wide step: one bulk copy feeds two 8-tile column groups), padded to whole records
@@ -651,12 +666,13 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       Q.kc = kv->k[l];
       Q.vc = kv->v[l];
       {  // A3a: g = W_dc RMSNorm(h; ln1), operand computed in the staging
-        GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
+        GemvSeg segs[2] = {{(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, 0},
+                           {(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, H / 4}};  // a0 | a1 paired
         Epi e;
         e.mode = EPI_STORE;
         e.y = gbuf;
         e.ldy = H / 2;
-        Q.dc.g = sgemv_params(P.pdc, &seg, 1, false, nullptr, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err);
+        Q.dc.g = sgemv_params(P.pdc, segs, 2, true, nullptr, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err);
         Q.dc.P = P.pdc.P;
         Q.dc.q4 = 0;
         Q.dc.stage = STG_NORM;
@@ -781,18 +797,22 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     {
       if (dbg && dbg->hidden && l > 0)
         CK(cudaMemcpyAsync(dbg->hidden + (size_t)l * Mb * H, h, hbytes, cudaMemcpyDeviceToDevice, s));
-      GemvSeg seg{(const uint8_t*)L.dc_w, (H / 2) / 16, Mb, 0};
+      // gate generators a0 | a1 paired per group; the fix-up applies the row scale, tanh and the
+      // two-tap convolution of its 256 channels and writes y (bf16) for the q/k/v product
+      GemvSeg segs[2] = {{(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, 0}, {(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, H / 4}};
       Epi e;
-      e.mode = EPI_STORE;
-      e.y = gbuf;
-      e.ldy = H / 2;
+      e.mode = EPI_DYNCONV;
       e.rs_in = ssp;
       e.ssp_rows = Mb;
       e.rs_H = H;
       e.eps = c->rms_eps;
-      CK(launch_gemv(P.dc, false, &seg, 1, false, xb, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err, s));
-      CK(launch_pdl(k_dynconv, dim3(Mb, (H / 4 + 255) / 256), dim3(256), 0, s, (const float*)h, (const float*)ssp, Mb,
-                    L.ln1, c->rms_eps, (const float*)gbuf, L.dc_s0, L.dc_s1, H, P.Bk, yb));
+      e.dyn_h = h;
+      e.dyn_w = L.ln1;
+      e.dyn_s0 = L.dc_s0;
+      e.dyn_s1 = L.dc_s1;
+      e.dyn_y = yb;
+      e.Bk = P.Bk;
+      CK(launch_gemv(P.dc, false, segs, 2, true, xb, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err, s));
     }
     // A3b+c: q from the block rows; k, v from block + context rows (stacked: each matrix read once);
     // the last CTA of each head applies q/k RMSNorm + RoPE and appends context K/V to the cache
@@ -1036,9 +1056,9 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   if (!cfg_ok(c) || batch < 1) return 0;
   const Plan P = make_plan(c, batch);
   if (P.persistent && persistent_ready(P)) return 1;
-  // embed, fc GEMV, fc norm | per layer: W_dc GEMV, dynconv, QKV GEMV, attention, combine, W_o GEMV,
-  // gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
-  return 3 + 8 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
+  // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention, combine,
+  // W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
+  return 3 + 7 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

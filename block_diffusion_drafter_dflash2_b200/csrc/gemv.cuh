@@ -29,7 +29,7 @@ struct GemvSeg {
   int out_col;       // first output column
 };
 
-enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3 };
+enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_DYNCONV = 4 };
 
 // Fused epilogue of the q|k|v projection: per-head q/k RMSNorm, RoPE at the absolute
 // position, block rows -> qb/kb/vb, context rows (t < n_new) -> the layer's paged cache.

@@ -1,5 +1,4 @@
-// Row-wise kernels of the block step: embedding gather, RMSNorm, two-tap
-// dynamic convolution, greedy acceptance.
+// Row-wise kernels of the block step: embedding gather, RMSNorm, greedy acceptance.
 #pragma once
 #include "common.cuh"
 
@@ -117,42 +116,6 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
     if (ob) *reinterpret_cast<uint2*>(ob + 4 * c) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
     if (of) of[c] = make_float4(y0, y1, y2, y3);
   }
-}
-
-// y_t[c] = (s0[c] + tanh g_t[c/4]) x_t[c] + (s1[c] + tanh g_t[H/4 + c/4]) x_{t-1}[c], x_{-1} = 0,
-// with x = RMSNorm(h; w) formed here from the residual rows and their quarter-column sums of
-// squares ssp[q][ldr].  Thread = 4 channels sharing one gate pair; grid (rows, H/1024).
-__global__ void k_dynconv(const float* __restrict__ hres, const float* __restrict__ ssp, int ldr,
-                          const uint16_t* __restrict__ w, float eps, const float* __restrict__ g,
-                          const uint16_t* __restrict__ s0, const uint16_t* __restrict__ s1, int H, int Bk,
-                          uint16_t* __restrict__ y) {
-  __shared__ float rs2[2];
-  pdl_trigger();
-  pdl_wait();
-  const int r = blockIdx.x, t = r % Bk, G = H / 4, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < 2) {  // row scales of rows r (warp 0) and r - 1 (warp 1)
-    const int rr = r - warp;
-    float q = 0.f;
-    if (warp == 0 || t > 0)
-      for (int i = lane; i < H / 32; i += 32) q += ssp[(size_t)i * ldr + rr];
-    q = warp_sum(q);
-    if (lane == 0) rs2[warp] = (warp == 0 || t > 0) ? rsqrtf(q / H + eps) : 0.f;
-  }
-  __syncthreads();
-  const int qi = blockIdx.y * blockDim.x + threadIdx.x;
-  if (qi >= G) return;
-  const float a0 = tanhf(g[(size_t)r * (H / 2) + qi]), a1 = tanhf(g[(size_t)r * (H / 2) + G + qi]);
-  const float4 hc = reinterpret_cast<const float4*>(hres + (size_t)r * H)[qi];
-  const float4 hp = t > 0 ? reinterpret_cast<const float4*>(hres + (size_t)(r - 1) * H)[qi] : make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint2 wv = *reinterpret_cast<const uint2*>(w + 4 * qi);
-  const uint2 w0 = *reinterpret_cast<const uint2*>(s0 + 4 * qi), w1 = *reinterpret_cast<const uint2*>(s1 + 4 * qi);
-  const float n0 = bf2f(wv.x & 0xffff), n1 = bf2f(wv.x >> 16), n2 = bf2f(wv.y & 0xffff), n3 = bf2f(wv.y >> 16);
-  const float rc = rs2[0], rp = rs2[1];
-  const float y0 = (bf2f(w0.x & 0xffff) + a0) * (hc.x * rc * n0) + (bf2f(w1.x & 0xffff) + a1) * (hp.x * rp * n0);
-  const float y1 = (bf2f(w0.x >> 16) + a0) * (hc.y * rc * n1) + (bf2f(w1.x >> 16) + a1) * (hp.y * rp * n1);
-  const float y2 = (bf2f(w0.y & 0xffff) + a0) * (hc.z * rc * n2) + (bf2f(w1.y & 0xffff) + a1) * (hp.z * rp * n2);
-  const float y3 = (bf2f(w0.y >> 16) + a0) * (hc.w * rc * n3) + (bf2f(w1.y >> 16) + a1) * (hp.w * rp * n3);
-  *reinterpret_cast<uint2*>(y + (size_t)r * H + 4 * qi) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
 }
 
 __global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,

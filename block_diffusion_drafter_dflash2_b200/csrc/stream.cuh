@@ -98,6 +98,12 @@ struct SGemvParams {
   const float* rs_in;
   int rs_H;
   float eps;
+  // EPI_DYNCONV (paired gate generators a0 | a1 of the two-tap convolution): y_t = (s0 + tanh a0)
+  // x_t + (s1 + tanh a1) x_{t-1} with x = RMSNorm(h; dyn_w) formed from the residual rows dyn_h
+  const float* dyn_h;
+  const uint16_t *dyn_w, *dyn_s0, *dyn_s1;
+  uint16_t* dyn_y;  // bf16 [rows][rs_H]
+  int Bk;
   int* err;
 };
 
@@ -171,11 +177,13 @@ DEVI float sum_pieces(const SGemvParams& p, int npieces, int row, int col) {
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   const int tid = threadIdx.x, nthr = kGemvConsumers * 32, warp = tid >> 5, lane = tid & 31;
-  __shared__ float s_rs[64];
+  __shared__ float s_rs[72];
   if (p.paired) {
     const int f0 = grp * 64;
     const int rows = sk_rows(p, 0, mz, R);
-    if (p.rs_in) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
+    // the convolution's x_{t-1} of the group's first row may be the previous row group's last
+    const int pre = p.epi == EPI_DYNCONV && mz > 0 ? 1 : 0;
+    if (p.rs_in) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
     // two outputs per thread per round: all their partial loads are in flight together
     for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
       float gv[2], uv[2];
@@ -190,9 +198,33 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
       for (int k = 0; k < 2; ++k) {
         const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
         if (i >= rows * 64) continue;
-        const float sc = p.rs_in ? s_rs[r] : 1.f;
+        const float sc = p.rs_in ? s_rs[pre + r] : 1.f;
         const float g = gv[k] * sc, u = uv[k] * sc;
-        p.act[(size_t)(mz + r) * p.F + f] = f2bf(g / (1.f + __expf(-g)) * u);
+        if (p.epi == EPI_SWIGLU) {
+          p.act[(size_t)(mz + r) * p.F + f] = f2bf(g / (1.f + __expf(-g)) * u);
+        } else if (p.epi == EPI_STORE) {
+          p.y[(size_t)(mz + r) * p.ldy + p.seg[0].out_col + f] = g;
+          p.y[(size_t)(mz + r) * p.ldy + p.seg[1].out_col + f] = u;
+        } else {  // EPI_DYNCONV: channels 4f .. 4f + 3 of block row mz + r, gates (g, u) of that row
+          const int row = mz + r, t = row % p.Bk, H = p.rs_H;
+          const float a0 = tanhf(g), a1 = tanhf(u), rc = s_rs[pre + r];
+          const float4 hc = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)row * H + 4 * f));
+          float4 hp = make_float4(0.f, 0.f, 0.f, 0.f);
+          float rp = 0.f;
+          if (t > 0) {
+            hp = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)(row - 1) * H + 4 * f));
+            rp = s_rs[pre + r - 1];
+          }
+          const uint2 wv = *reinterpret_cast<const uint2*>(p.dyn_w + 4 * f);
+          const uint2 e0 = *reinterpret_cast<const uint2*>(p.dyn_s0 + 4 * f);
+          const uint2 e1 = *reinterpret_cast<const uint2*>(p.dyn_s1 + 4 * f);
+          const float n0 = bf2f(wv.x & 0xffff), n1 = bf2f(wv.x >> 16), n2 = bf2f(wv.y & 0xffff), n3 = bf2f(wv.y >> 16);
+          const float y0 = (bf2f(e0.x & 0xffff) + a0) * (hc.x * rc * n0) + (bf2f(e1.x & 0xffff) + a1) * (hp.x * rp * n0);
+          const float y1 = (bf2f(e0.x >> 16) + a0) * (hc.y * rc * n1) + (bf2f(e1.x >> 16) + a1) * (hp.y * rp * n1);
+          const float y2 = (bf2f(e0.y & 0xffff) + a0) * (hc.z * rc * n2) + (bf2f(e1.y & 0xffff) + a1) * (hp.z * rp * n2);
+          const float y3 = (bf2f(e0.y >> 16) + a0) * (hc.w * rc * n3) + (bf2f(e1.y >> 16) + a1) * (hp.w * rp * n3);
+          *reinterpret_cast<uint2*>(p.dyn_y + (size_t)row * H + 4 * f) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
+        }
       }
     }
     return;
