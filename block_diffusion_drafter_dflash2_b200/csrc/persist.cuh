@@ -406,18 +406,14 @@ __device__ __noinline__ void consume_gemv_t(const PGemv& pg, const StepParams& S
         }
       }
     }
-    __threadfence();
     consumers_sync<kPNC>();
     if (threadIdx.x == 0) {
-      const int prev = atomicAdd(p.counters + gidx, 1);
+      const int prev = ticket_acq_rel(p.counters + gidx);
       s_last = prev == npieces - 1;
       if (s_last) p.counters[gidx] = 0;
     }
     consumers_sync<kPNC>();
-    if (s_last && ntact > 0) {
-      __threadfence();
-      fixup_group(p, grp, R, npieces);
-    }
+    if (s_last && ntact > 0) fixup_group(p, grp, R, npieces);
     x += ub - ua;
   }
 }

@@ -120,6 +120,15 @@ DEVI void rows_scale(const float* ssp, int ldr, int H, float eps, int mz, int ro
   consumers_sync<kGemvConsumers * 32>();
 }
 
+// Arrival ticket of a split-K group, taken by thread 0 right after a CTA barrier: the acq_rel
+// atomic releases the CTA's partial stores (ordered before it by the barrier) and acquires the
+// earlier arrivals', so the last arrival can read every partial after its next barrier.
+DEVI int ticket_acq_rel(int* ctr) {
+  int prev;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
+  return prev;
+}
+
 // Owner CTA of global position x when [0, W) is cut into P ranges [c*W/P, (c+1)*W/P).
 DEVI long long sk_owner(long long x, long long W, long long P) { return ((x + 1) * P + W - 1) / W - 1; }
 
@@ -175,15 +184,20 @@ DEVI float sum_pieces(const SGemvParams& p, int npieces, int row, int col) {
 }
 
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
-DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
+// rs_pre: row scales of rows [0, rows) computed at the kernel's start (single row group), or null.
+DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, const float* rs_pre = nullptr) {
   const int tid = threadIdx.x, nthr = kGemvConsumers * 32, warp = tid >> 5, lane = tid & 31;
   __shared__ float s_rs[72];
+  const float* rsv = s_rs;
   if (p.paired) {
     const int f0 = grp * 64;
     const int rows = sk_rows(p, 0, mz, R);
     // the convolution's x_{t-1} of the group's first row may be the previous row group's last
     const int pre = p.epi == EPI_DYNCONV && mz > 0 ? 1 : 0;
-    if (p.rs_in) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
+    if (p.rs_in) {
+      if (rs_pre && mz == 0) rsv = rs_pre;
+      else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
+    }
     // two outputs per thread per round: all their partial loads are in flight together
     for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
       float gv[2], uv[2];
@@ -198,7 +212,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
       for (int k = 0; k < 2; ++k) {
         const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
         if (i >= rows * 64) continue;
-        const float sc = p.rs_in ? s_rs[pre + r] : 1.f;
+        const float sc = p.rs_in ? rsv[pre + r] : 1.f;
         const float g = gv[k] * sc, u = uv[k] * sc;
         if (p.epi == EPI_SWIGLU) {
           p.act[(size_t)(mz + r) * p.F + f] = f2bf(g / (1.f + __expf(-g)) * u);
@@ -207,13 +221,13 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
           p.y[(size_t)(mz + r) * p.ldy + p.seg[1].out_col + f] = u;
         } else {  // EPI_DYNCONV: channels 4f .. 4f + 3 of block row mz + r, gates (g, u) of that row
           const int row = mz + r, t = row % p.Bk, H = p.rs_H;
-          const float a0 = tanhf(g), a1 = tanhf(u), rc = s_rs[pre + r];
+          const float a0 = tanhf(g), a1 = tanhf(u), rc = rsv[pre + r];
           const float4 hc = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)row * H + 4 * f));
           float4 hp = make_float4(0.f, 0.f, 0.f, 0.f);
           float rp = 0.f;
           if (t > 0) {
             hp = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)(row - 1) * H + 4 * f));
-            rp = s_rs[pre + r - 1];
+            rp = rsv[pre + r - 1];
           }
           const uint2 wv = *reinterpret_cast<const uint2*>(p.dyn_w + 4 * f);
           const uint2 e0 = *reinterpret_cast<const uint2*>(p.dyn_s0 + 4 * f);
@@ -234,7 +248,10 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
   if (tile0 < 0) return;
   const int col0 = p.seg[si].out_col + tile0 * 16;
   const int rows = sk_rows(p, si, mz, R);
-  if (p.rs_in && p.epi == EPI_STORE) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
+  if (p.rs_in && p.epi == EPI_STORE) {
+    if (rs_pre && mz == 0) rsv = rs_pre;
+    else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
+  }
   if (p.epi == EPI_QKV) {
     const int head = tile0 / 8;
     for (int r = warp; r < rows; r += kGemvConsumers) {
@@ -272,7 +289,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces) {
           if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
         }
       } else {
-        *y = p.rs_in ? v[k] * s_rs[r] : v[k];
+        *y = p.rs_in ? v[k] * rsv[r] : v[k];
       }
     }
   }
@@ -358,6 +375,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
 
   // ---- consumers: ring slot k is consumed by warp set (k & 1) ----
   pdl_wait();  // activations and the partial/ticket buffers come from earlier kernels
+  // a folded RMSNorm's row scales, computed now (off the fix-up's critical path) when all rows
+  // form one row group
+  __shared__ float s_rs0[64];
+  const bool rs_early = p.rs_in && p.rows <= 64;
+  if (rs_early) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, 0, p.rows, s_rs0);
   float2* coef = coef_all + warp * 128;
   int cnt = 0, staged_mz = -1;
   uint32_t xph = 0;
@@ -463,18 +485,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
     }
     // split-K: the last CTA of this column group to arrive sums the partials in range order
     // (deterministic) and runs the epilogue; nobody waits
-    __threadfence();
     consumers_sync<NC>();
     if (threadIdx.x == 0) {
-      const int prev = atomicAdd(p.counters + gidx, 1);
+      const int prev = ticket_acq_rel(p.counters + gidx);
       s_last = prev == npieces - 1;
       if (s_last) p.counters[gidx] = 0;
     }
     consumers_sync<NC>();
-    if (s_last && ntact > 0) {
-      __threadfence();
-      sk_fixup(p, grp, mz, R, npieces);
-    }
+    if (s_last && ntact > 0) sk_fixup(p, grp, mz, R, npieces, rs_early ? s_rs0 : nullptr);
     x += ub - ua;
   }
 }
@@ -662,17 +680,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
       const int k = rec == rec_first ? 0 : 1;
       float4* mine = reinterpret_cast<float4*>(p.part) + ((c * 2 + k) * kGemvConsumers + warp) * 32 + lane;
       *mine = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-      __threadfence();
       consumers_sync<NC>();
       if (threadIdx.x == 0) {
-        const int prev = atomicAdd(p.counters + rec, 1);
+        const int prev = ticket_acq_rel(p.counters + rec);
         s_last = prev == (int)(last - first);
         if (s_last) p.counters[rec] = 0;
       }
       consumers_sync<NC>();
       have = s_last != 0;
       if (have) {
-        __threadfence();
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         for (long long o = first; o <= last; ++o) {
           float4 v;
