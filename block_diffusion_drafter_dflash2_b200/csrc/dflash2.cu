@@ -32,7 +32,7 @@ struct Plan {
   GemvPlan fc, dc, qkv, o, gu, dn;
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
   bool persistent;
-  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart;
+  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
   int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
   bool lm_stream;
   size_t lm_smem;
@@ -208,6 +208,8 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_cfi = take((size_t)p.lm_rows * kTopK * 4);
   p.off_ssp = take((size_t)(p.H / 128) * 4 * p.Mb * 4);
   p.off_tau = take((size_t)p.lm_rows * kTopK * kTopK * 4);
+  p.off_rope = take((size_t)2 * p.Mb * 64 * 8);
+  p.off_rpage = take((size_t)p.Mb * 8);
   p.off_hpart = take(p.lm_stream ? (size_t)p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4 : 0);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
@@ -762,8 +764,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   // rows' sums of squares; every RMSNorm before a product is folded the same way: the residual
   // epilogues write bf16(h * w) and sums of squares, the product scales its outputs per row)
   float* ssp = at<float>(ws, P.off_ssp);
+  float2* rope = at<float2>(ws, P.off_rope);
+  int2* rpage = at<int2>(ws, P.off_rpage);
+  RopeInit ri{kv->seq_len, in->n_new, kv->page_table, kv->max_pages, kv->num_pages, P.Bk, Mb,
+              log2((double)c->rope_theta), rope, rpage};
   CK(launch_pdl(k_embed, dim3(Mb), dim3(256), 0, s, in->block_tokens, w->embed, h, H, P.V, err, xb, w->layer[0].ln1,
-                ssp, Mb));
+                ssp, Mb, ri));
   if (dbg && dbg->hidden) CK(cudaMemcpyAsync(dbg->hidden, h, hbytes, cudaMemcpyDeviceToDevice, s));
 
   // A2: context rows = RMSNorm_fc(W_fc . concat(taps)); fc output staged in xf
@@ -842,6 +848,8 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       q.page_table = kv->page_table;
       q.max_pages = kv->max_pages;
       q.num_pages = kv->num_pages;
+      q.rope = rope;  // positions and cache slots of this step, from the embedding kernel
+      q.rpage = rpage;
       q.err = err;
       CK(launch_gemv(P.qkv, P.q4, segs, 3, false, yb, H, 2 * Mb, part, ldo, 2 * Mb, lctr + P.ctr_layer[1], e, err, s));
     }

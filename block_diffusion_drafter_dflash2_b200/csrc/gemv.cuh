@@ -43,8 +43,24 @@ struct QkvEpi {
   uint16_t *kc, *vc;       // [pages][nkv][16][128]
   const int32_t* page_table;
   int max_pages, num_pages;
+  // Optional per-step tables (null: computed here): rope[row][j] = (cos, sin) of row's position
+  // times theta^(-2j/128), rows [0, Mb) block rows then [Mb, 2Mb) context rows; rpage[ctx row] =
+  // (page, slot) of its cache position, page -2 for rows past n_new, -1 for an unmapped page.
+  const float2* rope;
+  const int2* rpage;
   int* err;
 };
+
+// RoPE angle of position pos for frequency j: pos * theta^(-2j/128) reduced modulo 2 pi in double,
+// then sin/cos in fp32.
+DEVI float2 rope_cs(long long pos, int j, double log2_theta) {
+  const double inv = exp2(-(2.0 * j / kHeadDim) * log2_theta);
+  double a = (double)pos * inv;
+  a -= 6.283185307179586 * rint(a / 6.283185307179586);
+  float sn, cs;
+  sincosf((float)a, &sn, &cs);
+  return make_float2(cs, sn);
+}
 
 // One Q4_K group unit (16 rows x 256 k of one tile) against NT 8-row activation tiles.
 // q: the lane's 64 bytes of 4-bit codes (mma fragment order), sc: its feature's scale record.
@@ -137,8 +153,18 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
   const bool ctx = row >= e.Mb;
   const int rr = ctx ? row - e.Mb : row;
   const int b = rr / e.Bk, t = rr % e.Bk;
-  const int L0 = e.seq_len[b], nn = e.n_new[b];
-  if (ctx && t >= nn) return;
+  int L0 = 0, nn = 0;
+  int2 dstpg = make_int2(0, 0);
+  if (e.rope) {
+    if (ctx) {
+      dstpg = e.rpage[rr];
+      if (dstpg.x == -2) return;  // past the request's new rows
+    }
+  } else {
+    L0 = e.seq_len[b];
+    nn = e.n_new[b];
+    if (ctx && t >= nn) return;
+  }
   float x[4] = {xin[0], xin[1], xin[2], xin[3]};
   const int dims[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
   if (kind < 2) {
@@ -150,15 +176,10 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
     const long long pos = ctx ? (long long)L0 + t : (long long)L0 + nn + t;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      // angle pos * theta^(-2i/128) reduced modulo 2 pi in double, rotated in fp32
-      const double inv = exp2(-(2.0 * dims[i] / kHeadDim) * e.log2_theta);
-      double a = (double)pos * inv;
-      a -= 6.283185307179586 * rint(a / 6.283185307179586);
-      float sn, cs;
-      sincosf((float)a, &sn, &cs);
+      const float2 c = e.rope ? e.rope[(size_t)row * 64 + dims[i]] : rope_cs(pos, dims[i], e.log2_theta);
       const float x0 = x[i], x1 = x[i + 2];
-      x[i] = x0 * cs - x1 * sn;
-      x[i + 2] = x1 * cs + x0 * sn;
+      x[i] = x0 * c.x - x1 * c.y;
+      x[i + 2] = x1 * c.x + x0 * c.y;
     }
   }
   uint16_t* dst;
@@ -167,14 +188,17 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
     const int nh = kind == 0 ? e.nq : e.nkv;
     dst = base + ((size_t)row * nh + head) * kHeadDim;
   } else {
-    const long long pos = (long long)L0 + t;
-    const int lp = (int)(pos / kPage);
-    const int pg = lp < e.max_pages ? e.page_table[(size_t)b * e.max_pages + lp] : -1;
-    if (pg < 0 || pg >= e.num_pages) {
+    if (!e.rope) {
+      const long long pos = (long long)L0 + t;
+      const int lp = (int)(pos / kPage);
+      const int pg = lp < e.max_pages ? e.page_table[(size_t)b * e.max_pages + lp] : -1;
+      dstpg = make_int2(pg >= 0 && pg < e.num_pages ? pg : -1, (int)(pos % kPage));
+    }
+    if (dstpg.x < 0) {
       if (lane == 0) set_err(e.err, DFLASH2_DEV_PAGE);
       return;
     }
-    dst = (kind == 1 ? e.kc : e.vc) + (((size_t)pg * e.nkv + head) * kPage + pos % kPage) * kHeadDim;
+    dst = (kind == 1 ? e.kc : e.vc) + (((size_t)dstpg.x * e.nkv + head) * kPage + dstpg.y) * kHeadDim;
   }
   *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf2(x[0], x[1]);
   *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf2(x[2], x[3]);

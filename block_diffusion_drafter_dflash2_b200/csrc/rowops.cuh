@@ -1,18 +1,45 @@
 // Row-wise kernels of the block step: embedding gather, RMSNorm, greedy acceptance.
 #pragma once
 #include "common.cuh"
+#include "gemv.cuh"
 
 namespace dfl {
 
 // h[r] = E[block_tokens[r]] (fp32); ids outside [0, V) flag DFLASH2_DEV_TOKEN and read row 0.
 // Also the first RMSNorm's inputs: hw[r] = bf16(h[r] * w) and the row's sums of squares per
 // 32-column quarter, ssp[q][ldr] (the consumer applies the row scale).
+// Per-step RoPE tables (QkvEpi::rope / rpage), filled by the embedding kernel: CTA r does block
+// row r and context row r.
+struct RopeInit {
+  const int32_t *seq_len, *n_new, *page_table;
+  int max_pages, num_pages, Bk, Mb;
+  double log2_theta;
+  float2* rope;
+  int2* rpage;
+};
+
 __global__ void k_embed(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E, float* __restrict__ h,
                         int H, int V, int* err, uint16_t* __restrict__ hw, const uint16_t* __restrict__ w,
-                        float* __restrict__ ssp, int ldr) {
+                        float* __restrict__ ssp, int ldr, RopeInit ri) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (ri.rope && threadIdx.x < 128) {
+    const int b = r / ri.Bk, t = r % ri.Bk, j = threadIdx.x & 63;
+    const long long L0 = ri.seq_len[b], nn = ri.n_new[b];
+    const bool ctxrow = threadIdx.x >= 64;
+    const long long pos = ctxrow ? L0 + t : L0 + nn + t;
+    ri.rope[((size_t)(ctxrow ? ri.Mb + r : r)) * 64 + j] = rope_cs(pos, j, ri.log2_theta);
+    if (ctxrow && j == 0) {
+      int2 d = make_int2(-2, 0);
+      if (t < nn) {
+        const int lp = (int)(pos / kPage);
+        const int pg = lp < ri.max_pages ? ri.page_table[(size_t)b * ri.max_pages + lp] : -1;
+        d = make_int2(pg >= 0 && pg < ri.num_pages ? pg : -1, (int)(pos % kPage));
+      }
+      ri.rpage[r] = d;
+    }
+  }
   int id = tok[r];
   if (id < 0 || id >= V) {
     if (threadIdx.x == 0) set_err(err, DFLASH2_DEV_TOKEN);

@@ -297,9 +297,16 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
 
 // Bring rows [0, nrows) of an X chunk (row stride ldx elements, `bytes` per row) into Xs (row
 // stride `stride` bytes) with bulk copies on xbar; rows [nrows, R) are zeroed.  Consumer threads.
+// Work done while a staging copy is in flight: a folded RMSNorm's row scales (once).
+struct StageRs {
+  const SGemvParams* p;
+  float* s_rs;
+  bool pending;
+};
+
 template <int NTHR>
 DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes, uint8_t* Xs, int stride,
-                        uint64_t* xbar, uint32_t& xph, int* err) {
+                        uint64_t* xbar, uint32_t& xph, int* err, StageRs* rs = nullptr) {
   consumers_sync<NTHR>();  // every consumer is done with the previous chunk
   if (threadIdx.x == 0) {
     mbar_expect_tx(xbar, (uint32_t)(nrows * bytes));
@@ -309,7 +316,12 @@ DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes,
     const int r = nrows + i / (bytes / 16), v = i % (bytes / 16);
     *reinterpret_cast<uint4*>(Xs + r * stride + v * 16) = make_uint4(0, 0, 0, 0);
   }
-  consumers_sync<NTHR>();
+  if (rs && rs->pending) {  // (rows_scale ends with the consumer barrier)
+    rows_scale(rs->p->rs_in, rs->p->ssp_rows, rs->p->rs_H, rs->p->eps, 0, rs->p->rows, rs->s_rs);
+    rs->pending = false;
+  } else {
+    consumers_sync<NTHR>();
+  }
   if (!mbar_wait_sleep_bounded(xbar, xph) && threadIdx.x == 0) set_err(err, DFLASH2_DEV_TIMEOUT);
   xph ^= 1u;
 }
@@ -379,7 +391,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
   // form one row group
   __shared__ float s_rs0[64];
   const bool rs_early = p.rs_in && p.rows <= 64;
-  if (rs_early) rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, 0, p.rows, s_rs0);
+  StageRs srs{&p, s_rs0, rs_early};  // computed while the first activation copy is in flight
   float2* coef = coef_all + warp * 128;
   int cnt = 0, staged_mz = -1;
   uint32_t xph = 0;
@@ -406,12 +418,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
           base = 0;
           if (staged_mz != mz) {
             stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx, p.ldx, stage_rows, R, p.U * RC::kUnitK * 2, Xs, stride, &xbar,
-                              xph, p.err);
+                              xph, p.err, &srs);
             staged_mz = mz;
           }
         } else {
           stage_x_chunk<NC>(p.X + (size_t)mz * p.ldx + (size_t)c0 * RC::kUnitK, p.ldx, stage_rows, R,
-                            cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err);
+                            cu * RC::kUnitK * 2, Xs, stride, &xbar, xph, p.err, &srs);
         }
         for (int u = c0; u < c0 + cu; ++u) {
           const int slot = cnt % RC::kNS;
