@@ -315,3 +315,302 @@ __global__ void k_attn_combine(AttnParams p, uint16_t* __restrict__ ob) {
 }
 
 }  // namespace dfl
+
+namespace dfl {
+
+// ---------------------------------------------------------------------------
+// Sliding-window attention of one (request, kv head) on a cluster of 8 CTAs, merge included.
+// The keys seen by the block's queries are the cache window [cs, Lb) followed by the block's own
+// Bk keys; CTA r of the cluster takes keys [r*KC, (r+1)*KC) of that sequence.  Its warps split
+// them into 4 quarters (warp = quarter * MT + query tile): S = Q K^T and P.V on mma.sync with a
+// quarter-local softmax, the quarters merged in shared memory into the CTA's (m, l, o), then the 8
+// CTAs' partials merged over distributed shared memory, each CTA finishing 1/8 of the query
+// vectors.  The merge order is fixed, so the result does not depend on timing.
+//
+// Cache rows below seq_len were written by earlier steps and are not touched during this one,
+// so they are fetched (cp.async) before waiting on the previous kernel; the rows that kernel
+// writes (this step's context rows, the block's keys and the queries) are fetched after.
+constexpr int kClusterCtas = 8;
+
+DEVI void cp_async16(void* dst, const void* src, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(pred ? 16 : 0)
+               : "memory");
+}
+DEVI void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+DEVI uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+DEVI void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared-memory address of `p` in CTA `rank` of the cluster
+DEVI uint32_t cluster_map(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+DEVI float ld_cluster_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+DEVI float2 ld_cluster_f32x2(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
+  return v;
+}
+
+constexpr int kClRedStride = kHeadDim + 8;  // floats per row of the quarter partials (bank spread)
+
+// Dynamic shared memory of k_attn_cluster: queries + KC key rows + KC value rows, bf16, padded rows.
+constexpr size_t attn_cluster_smem(int MT, int KC) { return (size_t)(MT * 16 + 2 * KC) * kAttnStride * 2; }
+
+template <int MT, int NTK>  // MT 16-row query tiles; NTK 8-key tiles per warp quarter (KC = 32*NTK keys per CTA)
+__global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint16_t* __restrict__ ob) {
+  constexpr int NT = MT * 128, kQv = MT * 16, KC = 32 * NTK, KQ = 8 * NTK, kQpc = kQv / kClusterCtas;
+  static_assert(MT <= 2 && NTK % 2 == 0, "shape");
+  static_assert(MT * 4 * 16 * kClRedStride * 4 <= 2 * KC * kAttnStride * 2, "quarter partials fit over K/V");
+  static_assert(kQpc * 64 == NT, "one output pair per thread in the cluster merge");
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int row_ok[KC];  // 0 masked, 1 cache key (window applies), 2 block key
+  __shared__ int pgs[KC / kPage];
+  __shared__ float red_m[MT * 4][16], red_l[MT * 4][16];
+  __shared__ float cm[kQv], cl[kQv];
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* Ks = Qs + kQv * kAttnStride;
+  uint16_t* Vs = Ks + KC * kAttnStride;
+  float* red_o = reinterpret_cast<float*>(Ks);  // [MT*4 warps][16][kClRedStride] after the math
+  pdl_trigger();
+  const uint32_t r = cluster_rank();
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.nq / p.nkv, nqv = G * p.Bk;
+  // step inputs (no kernel of this step writes them)
+  const long long S0 = p.seq_len[b];
+  const long long Lb = S0 + p.n_new[b];
+  long long s0 = Lb - p.W + 1;
+  if (s0 < 0) s0 = 0;
+  const long long cs = (s0 / kPage) * kPage;
+  const long long ncache = Lb - cs;
+  const long long k0 = (long long)r * KC;  // cs + k0 is page aligned (KC is a multiple of kPage)
+
+  for (int i = threadIdx.x; i < KC / kPage; i += NT) {
+    int pg = -1;
+    if (k0 + (long long)i * kPage < ncache) {
+      const long long lp = (cs + k0) / kPage + i;
+      pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+      if (pg >= p.num_pages) pg = -1;
+    }
+    pgs[i] = pg;
+  }
+  __syncthreads();
+  // ---- before the wait: cache rows of earlier steps; rows past everything read as zero ----
+  for (int i = threadIdx.x; i < KC * 16; i += NT) {
+    const int kk = i >> 4, v = i & 15;
+    const long long kg = k0 + kk;
+    bool mine = false, ok = false;
+    const uint16_t *ksrc = p.kc, *vsrc = p.vc;
+    if (kg < ncache) {
+      const long long j = cs + kg;
+      if (j < S0) {
+        mine = true;
+        const int pg = pgs[kk / kPage];
+        ok = pg >= 0;
+        if (ok) {
+          const size_t off = (((size_t)pg * p.nkv + kvh) * kPage + j % kPage) * kHeadDim + v * 8;
+          ksrc += off;
+          vsrc += off;
+        } else if (v == 0) {
+          set_err(p.err, DFLASH2_DEV_PAGE);
+        }
+      }
+    } else if (kg - ncache >= p.Bk) {
+      mine = true;  // past the block's keys: masked, zero-filled
+    }
+    if (mine) {
+      cp_async16(Ks + kk * kAttnStride + v * 8, ksrc, ok);
+      cp_async16(Vs + kk * kAttnStride + v * 8, vsrc, ok);
+      if (v == 0) row_ok[kk] = ok ? 1 : 0;
+    }
+  }
+  pdl_wait();  // queries, the block's keys and this step's context rows come from the QKV kernel
+  for (int i = threadIdx.x; i < KC * 16; i += NT) {
+    const int kk = i >> 4, v = i & 15;
+    const long long kg = k0 + kk;
+    bool mine = false, ok = false;
+    int type = 0;
+    const uint16_t *ksrc = p.kc, *vsrc = p.vc;
+    if (kg < ncache) {
+      const long long j = cs + kg;
+      if (j >= S0) {
+        mine = true;
+        const int pg = pgs[kk / kPage];
+        ok = pg >= 0;
+        type = ok ? 1 : 0;
+        if (ok) {
+          const size_t off = (((size_t)pg * p.nkv + kvh) * kPage + j % kPage) * kHeadDim + v * 8;
+          ksrc += off;
+          vsrc += off;
+        } else if (v == 0) {
+          set_err(p.err, DFLASH2_DEV_PAGE);
+        }
+      }
+    } else if (kg - ncache < p.Bk) {
+      mine = ok = true;
+      type = 2;
+      const size_t off = ((size_t)(b * p.Bk + (int)(kg - ncache)) * p.nkv + kvh) * kHeadDim + v * 8;
+      ksrc = p.kb + off;
+      vsrc = p.vb + off;
+    }
+    if (mine) {
+      cp_async16(Ks + kk * kAttnStride + v * 8, ksrc, ok);
+      cp_async16(Vs + kk * kAttnStride + v * 8, vsrc, ok);
+      if (v == 0) row_ok[kk] = type;
+    }
+  }
+  for (int i = threadIdx.x; i < kQv * 16; i += NT) {
+    const int qv = i >> 4, v = i & 15;
+    const bool ok = qv < nqv;
+    const uint16_t* src = p.qb;
+    if (ok) src += ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim + v * 8;
+    cp_async16(Qs + qv * kAttnStride + v * 8, src, ok);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // ---- warp (qt, kq): 16 query vectors x KQ keys ----
+  const int qt = warp % MT, kq = warp / MT, g = lane >> 2, t4 = lane & 3;
+  float s[NTK][4];
+#pragma unroll
+  for (int n = 0; n < NTK; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  const uint16_t* Qw = Qs + qt * 16 * kAttnStride;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t a[4];
+    ldmatrix_x4(a, Qw + (lane & 15) * kAttnStride + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+    for (int n = 0; n < NTK; ++n) {
+      uint32_t b0, b1;
+      ldmatrix_x2(b0, b1, Ks + (kq * KQ + n * 8 + (lane & 7)) * kAttnStride + ks * 16 + ((lane >> 3) & 1) * 8);
+      mma16816(s[n], a, b0, b1);
+    }
+  }
+  float mrow[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int n = 0; n < NTK; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int qv = qt * 16 + g + 8 * (e >> 1);
+      const int kk = kq * KQ + n * 8 + 2 * t4 + (e & 1);
+      const int type = row_ok[kk];
+      bool vis = qv < nqv && type != 0;
+      if (vis && type == 1) vis = cs + k0 + kk >= Lb + qv / G - p.W + 1;
+      const float v = vis ? s[n][e] * p.scale_log2 : -INFINITY;
+      s[n][e] = v;
+      mrow[e >> 1] = fmaxf(mrow[e >> 1], v);
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 1));
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 2));
+  }
+  float lrow[2] = {0.f, 0.f};
+#pragma unroll
+  for (int n = 0; n < NTK; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = mrow[e >> 1];
+      const float pv = m == -INFINITY ? 0.f : exp2f(s[n][e] - m);
+      s[n][e] = pv;
+      lrow[e >> 1] += pv;
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+  }
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < NTK / 2; ++kk) {
+    uint32_t a[4];
+    a[0] = pack_bf2(s[2 * kk][0], s[2 * kk][1]);
+    a[1] = pack_bf2(s[2 * kk][2], s[2 * kk][3]);
+    a[2] = pack_bf2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+    a[3] = pack_bf2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      uint32_t b0, b1;
+      ldmatrix_x2_trans(b0, b1, Vs + (kq * KQ + kk * 16 + (lane & 15)) * kAttnStride + n * 8);
+      mma16816(o[n], a, b0, b1);
+    }
+  }
+  __syncthreads();  // K/V are no longer read: their space takes the quarter partials
+  {
+    float* ro = red_o + (size_t)warp * 16 * kClRedStride;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = g + 8 * h;
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2*>(ro + row * kClRedStride + n * 8 + 2 * t4) = make_float2(o[n][2 * h], o[n][2 * h + 1]);
+      if (t4 == 0) {
+        red_m[warp][row] = mrow[h];
+        red_l[warp][row] = lrow[h];
+      }
+    }
+  }
+  __syncthreads();
+  // ---- merge the quarters; the CTA's o lands in quarter 0's rows (row qv of red_o) ----
+  for (int i = threadIdx.x; i < kQv * kHeadDim; i += NT) {
+    const int qv = i / kHeadDim, d = i % kHeadDim, qtt = qv / 16, row = qv % 16;
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) M = fmaxf(M, red_m[q * MT + qtt][row]);
+    float O = 0.f, L = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int wq = q * MT + qtt;
+      const float wgt = M == -INFINITY ? 0.f : exp2f(red_m[wq][row] - M);
+      O += wgt * red_o[((size_t)wq * 16 + row) * kClRedStride + d];
+      L += wgt * red_l[wq][row];
+    }
+    red_o[(size_t)qv * kClRedStride + d] = O;  // only this thread reads or writes this element
+    if (d == 0) {
+      cm[qv] = M;
+      cl[qv] = L;
+    }
+  }
+  cluster_sync_all();
+  // ---- merge the cluster's 8 partials: this CTA finishes query vectors r*kQpc .. +kQpc-1 ----
+  {
+    const int qv = (int)r * kQpc + threadIdx.x / 64, d = (threadIdx.x % 64) * 2;
+    float mc[kClusterCtas], M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kClusterCtas; ++c) {
+      mc[c] = ld_cluster_f32(cluster_map(cm + qv, c));
+      M = fmaxf(M, mc[c]);
+    }
+    float L = 0.f;
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kClusterCtas; ++c) {
+      const float wgt = mc[c] == -INFINITY ? 0.f : exp2f(mc[c] - M);
+      L += wgt * ld_cluster_f32(cluster_map(cl + qv, c));
+      const float2 v = ld_cluster_f32x2(cluster_map(red_o + (size_t)qv * kClRedStride + d, c));
+      acc.x += wgt * v.x;
+      acc.y += wgt * v.y;
+    }
+    if (qv < nqv) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      uint16_t* dst = ob + ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim + d;
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf2(acc.x * inv, acc.y * inv);
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
+}
+
+}  // namespace dfl

@@ -28,6 +28,7 @@ struct GemvPlan {
 
 struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
+  int attn_ntk;  // > 0: attention as one cluster kernel with 32*attn_ntk keys per CTA; 0: chunks + merge kernel
   bool q4;
   GemvPlan fc, dc, qkv, o, gu, dn;
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
@@ -128,6 +129,17 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.QVP = (p.QV + 15) / 16 * 16;
   p.MT = p.QVP / 16;
   p.NC = (c->window + kPage - 2 + kAttnKeys - 1) / kAttnKeys;
+  {
+    // the cluster's 8 CTAs cover the window's keys (page aligned) and the block's keys
+    const int need = (c->window + kPage - 2 + p.Bk + kClusterCtas - 1) / kClusterCtas;
+    p.attn_ntk = 0;
+    if (p.MT <= 2)
+      for (int ntk : {4, 8, 10, 12})
+        if (32 * ntk >= need) {
+          p.attn_ntk = ntk;
+          break;
+        }
+  }
   p.fc = plan_gemv(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
   p.dc = plan_gemv((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
   p.qkv = plan_gemv((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
@@ -372,6 +384,42 @@ cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
     attr = true;
   }
   return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(kAttnThreads), smem, s, ap);
+}
+
+template <int MT, int NTK>
+cudaError_t launch_attn_cluster_t(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
+  static bool attr = false;
+  const size_t smem = attn_cluster_smem(MT, 32 * NTK);
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_cluster<MT, NTK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kClusterCtas, ap.nkv, P.B);
+  cfg.blockDim = dim3(MT * 128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kClusterCtas;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_attn_cluster<MT, NTK>, ap, ob);
+}
+
+template <int MT>
+cudaError_t launch_attn_cluster_mt(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
+  switch (P.attn_ntk) {
+    case 4: return launch_attn_cluster_t<MT, 4>(P, ap, ob, s);
+    case 8: return launch_attn_cluster_t<MT, 8>(P, ap, ob, s);
+    case 10: return launch_attn_cluster_t<MT, 10>(P, ap, ob, s);
+    default: return launch_attn_cluster_t<MT, 12>(P, ap, ob, s);
+  }
 }
 
 int fail(cudaError_t e) { return e == cudaSuccess ? DFLASH2_OK : DFLASH2_ERR_CUDA; }
@@ -857,13 +905,18 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     {
       ap.kc = kv->k[l];
       ap.vc = kv->v[l];
-      switch (P.MT) {
-        case 1: CK(launch_attn_t<1>(P, ap, s)); break;
-        case 2: CK(launch_attn_t<2>(P, ap, s)); break;
-        case 3: CK(launch_attn_t<3>(P, ap, s)); break;
-        default: CK(launch_attn_t<4>(P, ap, s)); break;
+      if (P.attn_ntk > 0) {
+        if (P.MT == 1) CK(launch_attn_cluster_mt<1>(P, ap, ob, s));
+        else CK(launch_attn_cluster_mt<2>(P, ap, ob, s));
+      } else {
+        switch (P.MT) {
+          case 1: CK(launch_attn_t<1>(P, ap, s)); break;
+          case 2: CK(launch_attn_t<2>(P, ap, s)); break;
+          case 3: CK(launch_attn_t<3>(P, ap, s)); break;
+          default: CK(launch_attn_t<4>(P, ap, s)); break;
+        }
+        CK(launch_pdl(k_attn_combine, dim3((P.QV + 3) / 4, c->n_kv, batch), dim3(128), 0, s, ap, ob));
       }
-      CK(launch_pdl(k_attn_combine, dim3((P.QV + 3) / 4, c->n_kv, batch), dim3(128), 0, s, ap, ob));
     }
     // A3e: h += W_o o (residual added by the last CTA of each column group)
     {
@@ -1064,9 +1117,10 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   if (!cfg_ok(c) || batch < 1) return 0;
   const Plan P = make_plan(c, batch);
   if (P.persistent && persistent_ready(P)) return 1;
-  // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention, combine,
-  // W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head pass(es), selector (tau, Viterbi)
-  return 3 + 7 * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
+  // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention (+ a merge
+  // kernel when the merge is not fused in), W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head
+  // pass(es), selector (tau, Viterbi)
+  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {
