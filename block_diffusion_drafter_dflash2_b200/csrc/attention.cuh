@@ -15,6 +15,8 @@
 // cache key j is visible iff max(0, p - W + 1) <= j < Lb; all block keys are
 // visible to all block rows.
 #pragma once
+#include <climits>
+
 #include "common.cuh"
 
 namespace dfl {
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
   __shared__ int row_ok[KC];  // 0 masked, 1 cache key (window applies), 2 block key
   __shared__ int pgs[KC / kPage];
   __shared__ float red_m[MT * 4][16], red_l[MT * 4][16];
-  __shared__ float cm[kQv], cl[kQv];
+  __shared__ float cm[kQv], cl[kQv], qw[kQv][4];
   uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
   uint16_t* Ks = Qs + kQv * kAttnStride;
   uint16_t* Vs = Ks + KC * kAttnStride;
@@ -395,10 +397,20 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
   const long long cs = (s0 / kPage) * kPage;
   const long long ncache = Lb - cs;
   const long long k0 = (long long)r * KC;  // cs + k0 is page aligned (KC is a multiple of kPage)
+  // this CTA's rows: [0, o_end) cache rows of earlier steps, [o_end, c_end) this step's context
+  // rows, [c_end, b_end) the block's keys, [b_end, KC) nothing (masked, zero)
+  auto clampkc = [](long long x) { return (int)(x < 0 ? 0 : (x > KC ? KC : x)); };
+  const int o_end = clampkc(S0 - cs - k0), c_end = clampkc(ncache - k0), b_end = clampkc(ncache + p.Bk - k0);
+  const int u0 = (int)(k0 - ncache);  // block key of row kk: kk + u0
+  constexpr int RP = NT / 16;          // rows per pass (16 lanes per row)
+  const int v = threadIdx.x & 15, slot = threadIdx.x >> 4;
+  const size_t page_stride = (size_t)p.nkv * kPage * kHeadDim;
+  const uint16_t* kc0 = p.kc + (size_t)kvh * kPage * kHeadDim + v * 8;
+  const uint16_t* vc0 = p.vc + (size_t)kvh * kPage * kHeadDim + v * 8;
 
   for (int i = threadIdx.x; i < KC / kPage; i += NT) {
     int pg = -1;
-    if (k0 + (long long)i * kPage < ncache) {
+    if (i * kPage < c_end) {
       const long long lp = (cs + k0) / kPage + i;
       pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
       if (pg >= p.num_pages) pg = -1;
@@ -406,72 +418,34 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
     pgs[i] = pg;
   }
   __syncthreads();
+  // one cache row: 16 lanes, 16 bytes each; an unmapped page reads as zero and flags the error
+  auto cache_row = [&](int kk) {
+    const int pg = pgs[kk / kPage];
+    const bool ok = pg >= 0;
+    const size_t off = ok ? (size_t)pg * page_stride + (size_t)(kk % kPage) * kHeadDim : 0;
+    cp_async16(Ks + kk * kAttnStride + v * 8, kc0 + off, ok);
+    cp_async16(Vs + kk * kAttnStride + v * 8, vc0 + off, ok);
+    if (v == 0) {
+      row_ok[kk] = ok ? 1 : 0;
+      if (!ok) set_err(p.err, DFLASH2_DEV_PAGE);
+    }
+  };
   // ---- before the wait: cache rows of earlier steps; rows past everything read as zero ----
-  for (int i = threadIdx.x; i < KC * 16; i += NT) {
-    const int kk = i >> 4, v = i & 15;
-    const long long kg = k0 + kk;
-    bool mine = false, ok = false;
-    const uint16_t *ksrc = p.kc, *vsrc = p.vc;
-    if (kg < ncache) {
-      const long long j = cs + kg;
-      if (j < S0) {
-        mine = true;
-        const int pg = pgs[kk / kPage];
-        ok = pg >= 0;
-        if (ok) {
-          const size_t off = (((size_t)pg * p.nkv + kvh) * kPage + j % kPage) * kHeadDim + v * 8;
-          ksrc += off;
-          vsrc += off;
-        } else if (v == 0) {
-          set_err(p.err, DFLASH2_DEV_PAGE);
-        }
-      }
-    } else if (kg - ncache >= p.Bk) {
-      mine = true;  // past the block's keys: masked, zero-filled
-    }
-    if (mine) {
-      cp_async16(Ks + kk * kAttnStride + v * 8, ksrc, ok);
-      cp_async16(Vs + kk * kAttnStride + v * 8, vsrc, ok);
-      if (v == 0) row_ok[kk] = ok ? 1 : 0;
-    }
+  for (int kk = slot; kk < o_end; kk += RP) cache_row(kk);
+  for (int kk = b_end + slot; kk < KC; kk += RP) {
+    cp_async16(Ks + kk * kAttnStride + v * 8, p.kc, false);
+    cp_async16(Vs + kk * kAttnStride + v * 8, p.vc, false);
+    if (v == 0) row_ok[kk] = 0;
   }
   pdl_wait();  // queries, the block's keys and this step's context rows come from the QKV kernel
-  for (int i = threadIdx.x; i < KC * 16; i += NT) {
-    const int kk = i >> 4, v = i & 15;
-    const long long kg = k0 + kk;
-    bool mine = false, ok = false;
-    int type = 0;
-    const uint16_t *ksrc = p.kc, *vsrc = p.vc;
-    if (kg < ncache) {
-      const long long j = cs + kg;
-      if (j >= S0) {
-        mine = true;
-        const int pg = pgs[kk / kPage];
-        ok = pg >= 0;
-        type = ok ? 1 : 0;
-        if (ok) {
-          const size_t off = (((size_t)pg * p.nkv + kvh) * kPage + j % kPage) * kHeadDim + v * 8;
-          ksrc += off;
-          vsrc += off;
-        } else if (v == 0) {
-          set_err(p.err, DFLASH2_DEV_PAGE);
-        }
-      }
-    } else if (kg - ncache < p.Bk) {
-      mine = ok = true;
-      type = 2;
-      const size_t off = ((size_t)(b * p.Bk + (int)(kg - ncache)) * p.nkv + kvh) * kHeadDim + v * 8;
-      ksrc = p.kb + off;
-      vsrc = p.vb + off;
-    }
-    if (mine) {
-      cp_async16(Ks + kk * kAttnStride + v * 8, ksrc, ok);
-      cp_async16(Vs + kk * kAttnStride + v * 8, vsrc, ok);
-      if (v == 0) row_ok[kk] = type;
-    }
+  for (int kk = o_end + slot; kk < c_end; kk += RP) cache_row(kk);
+  for (int kk = c_end + slot; kk < b_end; kk += RP) {
+    const size_t off = ((size_t)(b * p.Bk + kk + u0) * p.nkv + kvh) * kHeadDim + v * 8;
+    cp_async16(Ks + kk * kAttnStride + v * 8, p.kb + off, true);
+    cp_async16(Vs + kk * kAttnStride + v * 8, p.vb + off, true);
+    if (v == 0) row_ok[kk] = 2;
   }
-  for (int i = threadIdx.x; i < kQv * 16; i += NT) {
-    const int qv = i >> 4, v = i & 15;
+  for (int qv = slot; qv < kQv; qv += RP) {
     const bool ok = qv < nqv;
     const uint16_t* src = p.qb;
     if (ok) src += ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim + v * 8;
@@ -497,20 +471,28 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
       mma16816(s[n], a, b0, b1);
     }
   }
+  // key kk (cache) is inside the window of block row t iff t <= tmax0 + kk
+  const int tmax0 = (int)(cs + k0 - Lb + p.W - 1);
+  int trow[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int qv = qt * 16 + g + 8 * h;
+    trow[h] = qv < nqv ? qv / G : INT_MAX;  // INT_MAX: padding vector, sees nothing
+  }
   float mrow[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-  for (int n = 0; n < NTK; ++n)
+  for (int n = 0; n < NTK; ++n) {
+    const int kb0 = kq * KQ + n * 8 + 2 * t4;
+    const int ty[2] = {row_ok[kb0], row_ok[kb0 + 1]};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int qv = qt * 16 + g + 8 * (e >> 1);
-      const int kk = kq * KQ + n * 8 + 2 * t4 + (e & 1);
-      const int type = row_ok[kk];
-      bool vis = qv < nqv && type != 0;
-      if (vis && type == 1) vis = cs + k0 + kk >= Lb + qv / G - p.W + 1;
-      const float v = vis ? s[n][e] * p.scale_log2 : -INFINITY;
-      s[n][e] = v;
-      mrow[e >> 1] = fmaxf(mrow[e >> 1], v);
+      const int h = e >> 1, type = ty[e & 1];
+      const bool vis = trow[h] != INT_MAX && (type == 2 || (type == 1 && trow[h] <= tmax0 + kb0 + (e & 1)));
+      const float x = vis ? s[n][e] * p.scale_log2 : -INFINITY;
+      s[n][e] = x;
+      mrow[h] = fmaxf(mrow[h], x);
     }
+  }
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 1));
@@ -565,24 +547,29 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
   }
   __syncthreads();
   // ---- merge the quarters; the CTA's o lands in quarter 0's rows (row qv of red_o) ----
-  for (int i = threadIdx.x; i < kQv * kHeadDim; i += NT) {
-    const int qv = i / kHeadDim, d = i % kHeadDim, qtt = qv / 16, row = qv % 16;
+  if (threadIdx.x < kQv) {
+    const int qv = threadIdx.x, qtt = qv / 16, row = qv % 16;
     float M = -INFINITY;
 #pragma unroll
     for (int q = 0; q < 4; ++q) M = fmaxf(M, red_m[q * MT + qtt][row]);
-    float O = 0.f, L = 0.f;
+    float L = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int wq = q * MT + qtt;
       const float wgt = M == -INFINITY ? 0.f : exp2f(red_m[wq][row] - M);
-      O += wgt * red_o[((size_t)wq * 16 + row) * kClRedStride + d];
+      qw[qv][q] = wgt;
       L += wgt * red_l[wq][row];
     }
+    cm[qv] = M;
+    cl[qv] = L;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kQv * kHeadDim; i += NT) {
+    const int qv = i / kHeadDim, d = i % kHeadDim, qtt = qv / 16, row = qv % 16;
+    float O = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) O += qw[qv][q] * red_o[((size_t)(q * MT + qtt) * 16 + row) * kClRedStride + d];
     red_o[(size_t)qv * kClRedStride + d] = O;  // only this thread reads or writes this element
-    if (d == 0) {
-      cm[qv] = M;
-      cl[qv] = L;
-    }
   }
   cluster_sync_all();
   // ---- merge the cluster's 8 partials: this CTA finishes query vectors r*kQpc .. +kQpc-1 ----
