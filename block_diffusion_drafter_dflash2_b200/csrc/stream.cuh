@@ -129,6 +129,25 @@ DEVI int ticket_acq_rel(int* ctr) {
   return prev;
 }
 
+// Arrival of a non-designated split-K piece: a release reduction, after a CTA barrier that orders
+// the CTA's partial stores before it; nobody waits for it to complete.
+DEVI void arrive_release(int* ctr) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+// The designated CTA of a split-K group waits (bounded) until the other npieces - 1 pieces have
+// arrived, with acquire loads, then rearms the counter.  False when the limit expired.
+DEVI bool await_pieces(int* ctr, int others) {
+  for (long long i = 0; i < (kWaitLimit >> 4); ++i) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= others) {
+      *ctr = 0;
+      return true;
+    }
+  }
+  return false;
+}
+
 // Owner CTA of global position x when [0, W) is cut into P ranges [c*W/P, (c+1)*W/P).
 DEVI long long sk_owner(long long x, long long W, long long P) { return ((x + 1) * P + W - 1) / W - 1; }
 
@@ -495,16 +514,22 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
         }
       }
     }
-    // split-K: the last CTA of this column group to arrive sums the partials in range order
-    // (deterministic) and runs the epilogue; nobody waits
+    // split-K: the owner of the group's first unit (it reaches the group last, at the end of its
+    // range, unless the whole group lies inside it) sums the partials in range order
+    // (deterministic) and runs the epilogue; the other owners post their arrival and go on
     consumers_sync<NC>();
-    if (threadIdx.x == 0) {
-      const int prev = ticket_acq_rel(p.counters + gidx);
-      s_last = prev == npieces - 1;
-      if (s_last) p.counters[gidx] = 0;
+    if (c != first) {
+      if (threadIdx.x == 0) arrive_release(p.counters + gidx);
+    } else {
+      bool go = true;  // a group inside this range has no other pieces
+      if (npieces > 1) {
+        if (threadIdx.x == 0) s_last = await_pieces(p.counters + gidx, npieces - 1);
+        consumers_sync<NC>();
+        go = s_last != 0;
+        if (!go && threadIdx.x == 0) set_err(p.err, DFLASH2_DEV_TIMEOUT);
+      }
+      if (go && ntact > 0) sk_fixup(p, grp, mz, R, npieces, rs_early ? s_rs0 : nullptr);
     }
-    consumers_sync<NC>();
-    if (s_last && ntact > 0) sk_fixup(p, grp, mz, R, npieces, rs_early ? s_rs0 : nullptr);
     x += ub - ua;
   }
 }
