@@ -285,7 +285,7 @@ cudaError_t launch_sgemv_t(const GemvPlan& g, const SGemvParams& prm, cudaStream
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kGemvThreads), g.smem, s, prm);
+  return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kSGemvThreads), g.smem, s, prm);
 }
 
 struct Epi {

@@ -39,6 +39,7 @@ constexpr int kConsumers = 8;                          // consumer warps of the 
 constexpr int kGemvSets = 2;                           // GEMV: two warp sets alternate ring slots
 constexpr int kGemvConsumers = kGemvSets * kConsumers;
 constexpr int kGemvThreads = (kGemvConsumers + 1) * 32;
+constexpr int kSGemvThreads = (kGemvConsumers + 2) * 32;  // streamed GEMV: + a watcher warp
 
 template <bool Q4>
 struct Ring;
@@ -134,16 +135,14 @@ DEVI int ticket_acq_rel(int* ctr) {
 DEVI void arrive_release(int* ctr) {
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
 }
-// The designated CTA of a split-K group waits (bounded) until the other npieces - 1 pieces have
-// arrived, with acquire loads, then rearms the counter.  False when the limit expired.
-DEVI bool await_pieces(int* ctr, int others) {
+// Wait (bounded) until the other `others` pieces of a split-K group have arrived, with acquire
+// loads; false when the limit expired.
+DEVI bool await_pieces(const int* ctr, int others) {
   for (long long i = 0; i < (kWaitLimit >> 4); ++i) {
     int v;
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    if (v >= others) {
-      *ctr = 0;
-      return true;
-    }
+    if (v >= others) return true;
+    __nanosleep(128);
   }
   return false;
 }
@@ -346,7 +345,7 @@ DEVI void stage_x_chunk(const uint16_t* X, int ldx, int nrows, int R, int bytes,
 }
 
 template <int NT, bool Q4>
-__global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
+__global__ void __launch_bounds__(kSGemvThreads, 1) k_sgemv(SGemvParams p) {
   using RC = Ring<Q4>;
   constexpr int R = NT * 8;
   constexpr int NC = kGemvConsumers * 32;
@@ -354,6 +353,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
   __shared__ __align__(8) uint64_t full[RC::kNS];
   __shared__ __align__(8) uint64_t empty[RC::kNS];
   __shared__ __align__(8) uint64_t xbar;
+  __shared__ __align__(8) uint64_t seen;  // the watcher saw the other pieces of the last group
   __shared__ int s_last;
   uint8_t* ring = smem;
   uint8_t* Xs = smem + RC::kNS * RC::kSlot;
@@ -369,12 +369,27 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
       mbar_init(&empty[s], kConsumers);  // the 8 warps of the set that owns the slot
     }
     mbar_init(&xbar, 1);
+    mbar_init(&seen, 1);
     fence_mbar_init();
   }
   __syncthreads();
   pdl_trigger();
   const long long P = gridDim.x, c = blockIdx.x;
   const long long x0 = c * p.W / P, x1 = (c + 1) * p.W / P;
+
+  if (warp == kGemvConsumers + 1) {
+    // ---- watcher: when this CTA fixes up the group its range ends in, wait for that group's
+    // other pieces now, so the consumers find them arrived when they get there ----
+    if (lane != 0 || x1 <= x0) return;
+    const long long gstart = (x1 - 1) / p.U * p.U;
+    const int gidx = (int)(gstart / p.U);
+    const long long first = sk_owner(gstart, p.W, P);
+    const int npieces = (int)(sk_owner(gstart + p.U - 1, p.W, P) - first + 1);
+    if (c != first || npieces < 2) return;
+    s_last = await_pieces(p.counters + gidx, npieces - 1) ? 1 : 0;
+    mbar_arrive(&seen);  // (release: orders the flag and the acquired arrivals before the consumers)
+    return;
+  }
 
   if (warp == kGemvConsumers) {
     // ---- producer: weights only, so it may run ahead of the previous kernel ----
@@ -522,11 +537,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_sgemv(SGemvParams p) {
       if (threadIdx.x == 0) arrive_release(p.counters + gidx);
     } else {
       bool go = true;  // a group inside this range has no other pieces
-      if (npieces > 1) {
-        if (threadIdx.x == 0) s_last = await_pieces(p.counters + gidx, npieces - 1);
-        consumers_sync<NC>();
-        go = s_last != 0;
+      if (npieces > 1) {  // the group this range ends in: the watcher waited for its pieces
+        go = mbar_wait_bounded(&seen, 0) && s_last != 0;
         if (!go && threadIdx.x == 0) set_err(p.err, DFLASH2_DEV_TIMEOUT);
+        if (threadIdx.x == 0) p.counters[gidx] = 0;  // every piece has arrived: rearm
       }
       if (go && ntact > 0) sk_fixup(p, grp, mz, R, npieces, rs_early ? s_rs0 : nullptr);
     }
