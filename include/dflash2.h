@@ -230,9 +230,9 @@ int dflash2_device_error(const void *workspace, int32_t *out_bits, void *stream)
  * most 8 runs as ONE persistent cooperative kernel (one CTA per SM, grid
  * barriers between dependent operations) when the device supports cooperative
  * launch and the environment variable DFLASH2_PERSISTENT is "1"; otherwise
- * the step is a sequence of kernels (six per layer; seven when the attention merge runs as a
- * kernel of its own, which the plan picks for more than 32 query vectors per kv head or a
- * window above 3954 keys).
+ * the step is a sequence of kernels (six per layer; seven when the attention chunks are merged by
+ * a kernel of their own, which the plan picks for more than 32 query vectors per kv head or when
+ * window + block size exceeds 3058 keys).
  * 0 on an invalid config or batch. */
 int32_t dflash2_step_kernels(const dflash2_config *cfg, int32_t batch);
 

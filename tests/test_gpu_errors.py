@@ -59,7 +59,8 @@ def test_unmapped_append_page_sets_page_bit(tiny):
 def test_misaligned_taps_are_rejected(tiny):
     wl, dr = tiny
     st = inputs.make_state(wl, "cuda")
-    bad = torch.zeros(st["taps"].numel() + 8, dtype=torch.bfloat16, device="cuda")[1:].view(st["taps"].shape)
+    n = st["taps"].numel()
+    bad = torch.zeros(n + 8, dtype=torch.bfloat16, device="cuda")[1:1 + n].view(st["taps"].shape)  # 2-byte offset
     with pytest.raises(binding.DFlash2Error, match="ALIGN"):
         dr.draft_step({"taps": bad, "n_new": st["n_new"], "block_tokens": st["block_tokens"]}, st,
                       torch.zeros((1, 7), dtype=torch.int32, device="cuda"),
