@@ -201,6 +201,31 @@ DEVI float sum_pieces(const SGemvParams& p, int npieces, int row, int col) {
   return v;
 }
 
+// Split-K sums of up to 4 outputs (row[k], col[k]; ok[k] false: 0), each in piece order (the same
+// additions as sum_pieces); the loads of a round of 4 pieces for all 4 outputs go out together, so
+// a fix-up thread pays one L2 round trip per 4 pieces rather than one per output.
+DEVI void sum_pieces4(const SGemvParams& p, int npieces, const int (&row)[4], const int (&col)[4],
+                      const bool (&ok)[4], float (&v)[4]) {
+  const float* b[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    b[k] = p.part + (size_t)row[k] * p.ldo + col[k];
+    v[k] = 0.f;
+  }
+  for (int s0 = 0; s0 < npieces; s0 += 4) {
+    float x[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        x[k][j] = ok[k] && s0 + j < npieces ? __ldcg(b[k] + (size_t)(s0 + j) * p.piece_stride) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[k] += x[k][j];
+  }
+}
+
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 // rs_pre: row scales of rows [0, rows) computed at the kernel's start (single row group), or null.
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, const float* rs_pre = nullptr) {
@@ -219,12 +244,24 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     // two outputs per thread per round: all their partial loads are in flight together
     for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
       float gv[2], uv[2];
+      {
+        int rw[4], cl[4];
+        bool okk[4];
+        float sv[4];
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
-        const bool ok = i < rows * 64;
-        gv[k] = ok ? sum_pieces(p, npieces, mz + r, p.seg[0].out_col + f) : 0.f;
-        uv[k] = ok ? sum_pieces(p, npieces, mz + r, p.seg[1].out_col + f) : 0.f;
+        for (int k = 0; k < 2; ++k) {
+          const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
+          okk[2 * k] = okk[2 * k + 1] = i < rows * 64;
+          rw[2 * k] = rw[2 * k + 1] = mz + r;
+          cl[2 * k] = p.seg[0].out_col + f;
+          cl[2 * k + 1] = p.seg[1].out_col + f;
+        }
+        sum_pieces4(p, npieces, rw, cl, okk, sv);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          gv[k] = sv[2 * k];
+          uv[k] = sv[2 * k + 1];
+        }
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -274,9 +311,10 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     const int head = tile0 / 8;
     for (int r = warp; r < rows; r += kGemvConsumers) {
       float x[4];
-      const int dims[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) x[i] = sum_pieces(p, npieces, mz + r, col0 + dims[i]);
+      const int rw[4] = {mz + r, mz + r, mz + r, mz + r};
+      const int cl[4] = {col0 + 2 * lane, col0 + 2 * lane + 1, col0 + 64 + 2 * lane, col0 + 65 + 2 * lane};
+      const bool okk[4] = {true, true, true, true};
+      sum_pieces4(p, npieces, rw, cl, okk, x);
       qkv_head_row(p.qkv, si, head, mz + r, x, lane);
     }
     return;
@@ -285,13 +323,19 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
   // flight together before any store
   for (int i0 = tid; i0 < rows * 128; i0 += 4 * nthr) {
     float v[4], old[4];
+    {
+      int rw[4], cl[4];
+      bool okk[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = i0 + k * nthr, r = i >> 7, c = col0 + (i & 127);
-      const bool ok = i < rows * 128;
-      v[k] = ok ? sum_pieces(p, npieces, mz + r, c) : 0.f;
-      // L2 read: another CTA may have written the residual row
-      old[k] = ok && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)(mz + r) * p.ldy + c) : 0.f;
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k * nthr;
+        rw[k] = mz + (i >> 7);
+        cl[k] = col0 + (i & 127);
+        okk[k] = i < rows * 128;
+        // L2 read: another CTA may have written the residual row
+        old[k] = okk[k] && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)rw[k] * p.ldy + cl[k]) : 0.f;
+      }
+      sum_pieces4(p, npieces, rw, cl, okk, v);
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
