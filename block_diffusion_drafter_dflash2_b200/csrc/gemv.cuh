@@ -149,7 +149,37 @@ DEVI void bf16_step(const uint4 (&w)[2 * NJ], const uint8_t* Xs, int stride, int
 }
 
 // q/k RMSNorm + RoPE of one head of one row (lane holds dims 2L, 2L+1, 64+2L, 65+2L), then store.
-DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float (&xin)[4], int lane) {
+// Operands of one (kind, row) epilogue that do not depend on the product, when the per-step
+// tables are in use: the context row's cache slot, the q/k norm weights and the RoPE factors of
+// this lane's dimensions.  Loaded before the split-K partials so that all come back together.
+struct QkvPre {
+  int2 dstpg;
+  float w[4];
+  float2 cs[2];
+};
+
+DEVI QkvPre qkv_prefetch(const QkvEpi& e, int kind, int row, int lane) {
+  QkvPre q;
+  q.dstpg = make_int2(0, 0);
+  q.w[0] = q.w[1] = q.w[2] = q.w[3] = 1.f;
+  q.cs[0] = q.cs[1] = make_float2(1.f, 0.f);
+  if (!e.rope) return q;
+  if (row >= e.Mb) q.dstpg = e.rpage[row - e.Mb];
+  if (kind < 2) {
+    const uint16_t* w = kind == 0 ? e.qn : e.kn;
+    q.w[0] = bf2f(w[2 * lane]);
+    q.w[1] = bf2f(w[2 * lane + 1]);
+    q.w[2] = bf2f(w[64 + 2 * lane]);
+    q.w[3] = bf2f(w[65 + 2 * lane]);
+    q.cs[0] = e.rope[(size_t)row * 64 + 2 * lane];
+    q.cs[1] = e.rope[(size_t)row * 64 + 2 * lane + 1];
+  }
+  return q;
+}
+
+// pre: qkv_prefetch of the same (kind, row).
+DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float (&xin)[4], int lane,
+                       const QkvPre& pre) {
   const bool ctx = row >= e.Mb;
   const int rr = ctx ? row - e.Mb : row;
   const int b = rr / e.Bk, t = rr % e.Bk;
@@ -157,7 +187,7 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
   int2 dstpg = make_int2(0, 0);
   if (e.rope) {
     if (ctx) {
-      dstpg = e.rpage[rr];
+      dstpg = pre.dstpg;
       if (dstpg.x == -2) return;  // past the request's new rows
     }
   } else {
@@ -172,11 +202,11 @@ DEVI void qkv_head_row(const QkvEpi& e, int kind, int head, int row, const float
     const float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
     const float rs = rsqrtf(ss / kHeadDim + e.eps);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = x[i] * rs * bf2f(w[dims[i]]);
+    for (int i = 0; i < 4; ++i) x[i] = x[i] * rs * (e.rope ? pre.w[i] : bf2f(w[dims[i]]));
     const long long pos = ctx ? (long long)L0 + t : (long long)L0 + nn + t;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const float2 c = e.rope ? e.rope[(size_t)row * 64 + dims[i]] : rope_cs(pos, dims[i], e.log2_theta);
+      const float2 c = e.rope ? pre.cs[i] : rope_cs(pos, dims[i], e.log2_theta);
       const float x0 = x[i], x1 = x[i + 2];
       x[i] = x0 * c.x - x1 * c.y;
       x[i + 2] = x1 * c.x + x0 * c.y;

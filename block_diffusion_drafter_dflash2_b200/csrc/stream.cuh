@@ -314,15 +314,16 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
       const int rw[4] = {mz + r, mz + r, mz + r, mz + r};
       const int cl[4] = {col0 + 2 * lane, col0 + 2 * lane + 1, col0 + 64 + 2 * lane, col0 + 65 + 2 * lane};
       const bool okk[4] = {true, true, true, true};
+      const QkvPre pre = qkv_prefetch(p.qkv, si, mz + r, lane);  // in flight with the partial loads
       sum_pieces4(p, npieces, rw, cl, okk, x);
-      qkv_head_row(p.qkv, si, head, mz + r, x, lane);
+      qkv_head_row(p.qkv, si, head, mz + r, x, lane, pre);
     }
     return;
   }
   // four outputs per thread per round: all their partial loads (and the residual reads) are in
   // flight together before any store
   for (int i0 = tid; i0 < rows * 128; i0 += 4 * nthr) {
-    float v[4], old[4];
+    float v[4], old[4], hwf[4];
     {
       int rw[4], cl[4];
       bool okk[4];
@@ -334,6 +335,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
         okk[k] = i < rows * 128;
         // L2 read: another CTA may have written the residual row
         old[k] = okk[k] && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)rw[k] * p.ldy + cl[k]) : 0.f;
+        hwf[k] = okk[k] && p.epi == EPI_RESID && p.hw ? bf2f(p.hw_w[cl[k]]) : 0.f;
       }
       sum_pieces4(p, npieces, rw, cl, okk, v);
     }
@@ -345,7 +347,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
       if (p.epi == EPI_RESID) {
         const float nv = old[k] + v[k];
         *y = nv;
-        if (p.hw) p.hw[(size_t)(mz + r) * p.hw_ld + c] = f2bf(nv * bf2f(p.hw_w[c]));
+        if (p.hw) p.hw[(size_t)(mz + r) * p.hw_ld + c] = f2bf(nv * hwf[k]);
         if (p.ssp) {  // sum of squares of this warp's 32 columns of the new row, for the next RMSNorm
           const float q = warp_sum(nv * nv);
           if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
