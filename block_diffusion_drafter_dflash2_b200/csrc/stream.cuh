@@ -244,6 +244,8 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     // two outputs per thread per round: all their partial loads are in flight together
     for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
       float gv[2], uv[2];
+      float4 hc[2], hp[2];
+      uint2 wv[2], e0[2], e1[2];
       {
         int rw[4], cl[4];
         bool okk[4];
@@ -255,6 +257,17 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
           rw[2 * k] = rw[2 * k + 1] = mz + r;
           cl[2 * k] = p.seg[0].out_col + f;
           cl[2 * k + 1] = p.seg[1].out_col + f;
+          // the convolution's operands go out with the partial loads
+          hc[k] = hp[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          wv[k] = e0[k] = e1[k] = make_uint2(0, 0);
+          if (okk[2 * k] && p.epi == EPI_DYNCONV) {
+            const int row = mz + r, H = p.rs_H;
+            hc[k] = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)row * H + 4 * f));
+            if (row % p.Bk > 0) hp[k] = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)(row - 1) * H + 4 * f));
+            wv[k] = *reinterpret_cast<const uint2*>(p.dyn_w + 4 * f);
+            e0[k] = *reinterpret_cast<const uint2*>(p.dyn_s0 + 4 * f);
+            e1[k] = *reinterpret_cast<const uint2*>(p.dyn_s1 + 4 * f);
+          }
         }
         sum_pieces4(p, npieces, rw, cl, okk, sv);
 #pragma unroll
@@ -277,21 +290,14 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
         } else {  // EPI_DYNCONV: channels 4f .. 4f + 3 of block row mz + r, gates (g, u) of that row
           const int row = mz + r, t = row % p.Bk, H = p.rs_H;
           const float a0 = tanhf(g), a1 = tanhf(u), rc = rsv[pre + r];
-          const float4 hc = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)row * H + 4 * f));
-          float4 hp = make_float4(0.f, 0.f, 0.f, 0.f);
-          float rp = 0.f;
-          if (t > 0) {
-            hp = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)(row - 1) * H + 4 * f));
-            rp = rsv[pre + r - 1];
-          }
-          const uint2 wv = *reinterpret_cast<const uint2*>(p.dyn_w + 4 * f);
-          const uint2 e0 = *reinterpret_cast<const uint2*>(p.dyn_s0 + 4 * f);
-          const uint2 e1 = *reinterpret_cast<const uint2*>(p.dyn_s1 + 4 * f);
-          const float n0 = bf2f(wv.x & 0xffff), n1 = bf2f(wv.x >> 16), n2 = bf2f(wv.y & 0xffff), n3 = bf2f(wv.y >> 16);
-          const float y0 = (bf2f(e0.x & 0xffff) + a0) * (hc.x * rc * n0) + (bf2f(e1.x & 0xffff) + a1) * (hp.x * rp * n0);
-          const float y1 = (bf2f(e0.x >> 16) + a0) * (hc.y * rc * n1) + (bf2f(e1.x >> 16) + a1) * (hp.y * rp * n1);
-          const float y2 = (bf2f(e0.y & 0xffff) + a0) * (hc.z * rc * n2) + (bf2f(e1.y & 0xffff) + a1) * (hp.z * rp * n2);
-          const float y3 = (bf2f(e0.y >> 16) + a0) * (hc.w * rc * n3) + (bf2f(e1.y >> 16) + a1) * (hp.w * rp * n3);
+          const float rp = t > 0 ? rsv[pre + r - 1] : 0.f;
+          const float4 c4 = hc[k], p4 = hp[k];
+          const uint2 w2 = wv[k], s0 = e0[k], s1 = e1[k];
+          const float n0 = bf2f(w2.x & 0xffff), n1 = bf2f(w2.x >> 16), n2 = bf2f(w2.y & 0xffff), n3 = bf2f(w2.y >> 16);
+          const float y0 = (bf2f(s0.x & 0xffff) + a0) * (c4.x * rc * n0) + (bf2f(s1.x & 0xffff) + a1) * (p4.x * rp * n0);
+          const float y1 = (bf2f(s0.x >> 16) + a0) * (c4.y * rc * n1) + (bf2f(s1.x >> 16) + a1) * (p4.y * rp * n1);
+          const float y2 = (bf2f(s0.y & 0xffff) + a0) * (c4.z * rc * n2) + (bf2f(s1.y & 0xffff) + a1) * (p4.z * rp * n2);
+          const float y3 = (bf2f(s0.y >> 16) + a0) * (c4.w * rc * n3) + (bf2f(s1.y >> 16) + a1) * (p4.w * rp * n3);
           *reinterpret_cast<uint2*>(p.dyn_y + (size_t)row * H + 4 * f) = make_uint2(pack_bf2(y0, y1), pack_bf2(y2, y3));
         }
       }
