@@ -39,7 +39,7 @@ struct Plan {
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
       off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
-  size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_head, ctr_total;
+  size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_head, ctr_sel, ctr_total;
   size_t off_s_taps, off_s_nnew, off_s_btok, off_s_tgt, off_s_path, off_s_scores, off_s_acc, off_s_emit;
   size_t step_bytes, total;
 };
@@ -236,7 +236,8 @@ Plan make_plan(const dflash2_config* c, int B) {
   }
   p.ctr_per_layer = acc;
   p.ctr_head = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;  // the streaming head's record tickets
-  p.ctr_total = p.ctr_head + (size_t)(lm_tiles + kHeadTiles - 1) / kHeadTiles + 1;  // + the persistent grid barrier
+  p.ctr_sel = p.ctr_head + (size_t)(lm_tiles + kHeadTiles - 1) / kHeadTiles;  // selector arrival tickets
+  p.ctr_total = p.ctr_sel + (size_t)B + 1;                                      // + the persistent grid barrier
   p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
   p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
@@ -1050,9 +1051,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     float* tau = at<float>(ws, P.off_tau);
     float* clg = at<float>(ws, P.off_cfv);
     int32_t* cdg = at<int32_t>(ws, P.off_cfi);
-    CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), 0, s, sp, tau, clg, cdg));
-    CK(launch_pdl(k_sel_viterbi, dim3(batch), dim3(32), 0, s, sp, (const float*)tau, (const float*)clg,
-                  (const int32_t*)cdg));
+    CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), 0, s, sp, tau, clg, cdg, ctr + P.ctr_sel));
   }
   return DFLASH2_OK;
 }
@@ -1119,8 +1118,8 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   if (P.persistent && persistent_ready(P)) return 1;
   // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention (+ a merge
   // kernel when the merge is not fused in), W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head
-  // pass(es), selector (tau, Viterbi)
-  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 2;
+  // pass(es), selector (transition scores, the last CTA of a request runs its Viterbi path)
+  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 1;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

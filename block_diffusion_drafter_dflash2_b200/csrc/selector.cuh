@@ -44,14 +44,22 @@ struct SelParams {
 DEVI void merge_lists_row(const float* cv, const int32_t* ci, int nparts, int rows_total, int row, float* sv, int* si,
                           int cap, int* surv, float* out_v, int* out_id) {
   const int lane = threadIdx.x & 31;
+  // the lane's first 8 lists (parts lane, lane + 32, ...): their heads stay in registers (fully
+  // unrolled, no local memory) and all 16 loads go out together
   float T0 = -INFINITY;
   float heads[8];
-  int nh = 0;
-  for (int part = lane; part < nparts; part += 32) {
-    const size_t o = ((size_t)part * rows_total + row) * kTopK;
-    T0 = fmaxf(T0, __ldcg(cv + o + kTopK - 1));
-    if (nh < 8) heads[nh++] = __ldcg(cv + o);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int part = lane + 32 * q;
+    heads[q] = -INFINITY;
+    if (part < nparts) {
+      const size_t o = ((size_t)part * rows_total + row) * kTopK;
+      T0 = fmaxf(T0, __ldcg(cv + o + kTopK - 1));
+      heads[q] = __ldcg(cv + o);
+    }
   }
+  for (int part = lane + 256; part < nparts; part += 32)
+    T0 = fmaxf(T0, __ldcg(cv + ((size_t)part * rows_total + row) * kTopK + kTopK - 1));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) T0 = fmaxf(T0, __shfl_xor_sync(0xffffffffu, T0, o));
   if (nparts <= 8 * 32) {
@@ -60,30 +68,76 @@ DEVI void merge_lists_row(const float* cv, const int32_t* ci, int nparts, int ro
     for (int k = 0; k < kTopK; ++k) {
       float lb = -INFINITY;
       int li_ = -1;
-      for (int i = 0; i < nh; ++i)
-        if (heads[i] > lb) { lb = heads[i]; li_ = i; }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (heads[q] > lb) {
+          lb = heads[q];
+          li_ = q;
+        }
       float m = lb;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       const unsigned who = __ballot_sync(0xffffffffu, li_ >= 0 && lb == m);
-      if (who && lane == __ffs(who) - 1) heads[li_] = -INFINITY;
+      if (who && lane == __ffs(who) - 1) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q == li_) heads[q] = -INFINITY;
+      }
       hb = m;
     }
     T0 = fmaxf(T0, hb);
   }
   if (lane == 0) *surv = 0;
   __syncwarp();
-  for (int part = lane; part < nparts; part += 32) {
-    const size_t o = ((size_t)part * rows_total + row) * kTopK;
-    for (int k = 0; k < kTopK; ++k) {
-      const float v = __ldcg(cv + o + k);
-      if (!(v >= T0)) break;  // lists are sorted
-      const int slot = atomicAdd(surv, 1);
-      if (slot < cap) {
-        sv[slot] = v;
-        si[slot] = __ldcg(ci + o + k);
+  // survivors: each sorted list contributes a prefix >= T0.  The lane's lists (at most 8) are read
+  // 4 entries at a time, all of them together, so a round costs one L2 round trip; the ids of the
+  // survivors are fetched afterwards in one batch (si holds the entry's offset until then).
+  {
+    unsigned live = 0;  // bit q: the lane's list q may continue
+    int nq = 0;
+    for (int part = lane; part < nparts && nq < 8; part += 32) live |= 1u << nq++;
+    for (int k0 = 0; k0 < kTopK && __any_sync(0xffffffffu, live != 0); k0 += 4) {
+      float4 v4[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (live >> q & 1u)
+          v4[q] = __ldcg(reinterpret_cast<const float4*>(cv + ((size_t)(lane + 32 * q) * rows_total + row) * kTopK + k0));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (!(live >> q & 1u)) continue;
+        const float e4[4] = {v4[q].x, v4[q].y, v4[q].z, v4[q].w};
+        const size_t o = ((size_t)(lane + 32 * q) * rows_total + row) * kTopK + k0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (!(e4[e] >= T0)) {  // lists are sorted: this one is done
+            live &= ~(1u << q);
+            break;
+          }
+          const int slot = atomicAdd(surv, 1);
+          if (slot < cap) {
+            sv[slot] = e4[e];
+            si[slot] = (int)(o + e);
+          }
+        }
       }
     }
+    // more than 8 lists per lane (over 256 parts): the rest one entry at a time
+    for (int part = lane + 256; part < nparts; part += 32) {
+      const size_t o = ((size_t)part * rows_total + row) * kTopK;
+      for (int k = 0; k < kTopK; ++k) {
+        const float v = __ldcg(cv + o + k);
+        if (!(v >= T0)) break;
+        const int slot = atomicAdd(surv, 1);
+        if (slot < cap) {
+          sv[slot] = v;
+          si[slot] = (int)(o + k);
+        }
+      }
+    }
+    __syncwarp();
+    const int ns = min(*surv, cap);
+#pragma unroll 4
+    for (int i = lane; i < ns; i += 32) si[i] = __ldcg(ci + si[i]);
   }
   __syncwarp();
   const int n = *surv;
@@ -182,9 +236,12 @@ DEVI void selector_tau(const SelParams& p, int b, int t, const int* src_ids, int
   consumers_sync<NTHR>();
   const int i = threadIdx.x / kTopK, j = threadIdx.x % kTopK;
   if (i < nsrc) {
-    float s = 0.f;
-    for (int r = 0; r < R; ++r) s = fmaf(As[i][r], Wj[r][j], s);
-    tau[i * kTopK + j] = s;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains, added in a fixed order
+    for (int r = 0; r < R; r += 4) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s4[e] = fmaf(As[i][r + e], Wj[r + e][j], s4[e]);
+    }
+    tau[i * kTopK + j] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
 }
 
@@ -192,7 +249,11 @@ DEVI void selector_tau(const SelParams& p, int b, int t, const int* src_ids, int
 //   delta_0(j) = cl_0(j) + tau_0(0, j),  delta_t(j) = cl_t(j) + max_i (delta_{t-1}(i) + tau_t(i, j)),
 // first maximum on ties (smallest i; at the end smallest j).  Writes the path and its running
 // scores and advances seq_len[b] by n_new[b].  cl/cand: [D][16], tau: [D][16][16] (global).
+// SH: cl/cand/tau are in shared memory (plain loads); otherwise global, written by other CTAs (L2).
+template <bool SH = false>
 DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int32_t* cand, const float* tau) {
+  auto ldf = [](const float* a) { return SH ? *a : __ldcg(a); };
+  auto ldi = [](const int32_t* a) { return SH ? *a : __ldcg(a); };
   const int lane = threadIdx.x & 31, j = lane & 15, D = p.Bk - 1;
   float d = 0.f;
   float dl[kMaxD];
@@ -203,14 +264,14 @@ DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int
     bp[t] = 0;
     if (t >= D) continue;
     const float* tt = tau + (size_t)t * kTopK * kTopK;
-    const float c = __ldcg(cl + t * kTopK + j);
+    const float c = ldf(cl + t * kTopK + j);
     if (t == 0) {
-      d = c + __ldcg(tt + j);
+      d = c + ldf(tt + j);
     } else {
       float best = 0.f;
       int bi = -1;
       for (int i = 0; i < kTopK; ++i) {
-        const float sc = __shfl_sync(0xffffffffu, d, i) + __ldcg(tt + i * kTopK + j);
+        const float sc = __shfl_sync(0xffffffffu, d, i) + ldf(tt + i * kTopK + j);
         if (bi < 0 || sc > best) { best = sc; bi = i; }
       }
       d = c + best;
@@ -230,7 +291,7 @@ DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int
     const float sc = __shfl_sync(0xffffffffu, dl[t], jj);
     const int prev = __shfl_sync(0xffffffffu, bp[t], jj);
     if (lane == 0) {
-      p.out_path[b * D + t] = __ldcg(cand + t * kTopK + jj);
+      p.out_path[b * D + t] = ldi(cand + t * kTopK + jj);
       p.out_scores[b * D + t] = sc;
     }
     jj = prev;
@@ -255,8 +316,11 @@ DEVI void selector_row(const SelParams& p, int row, float* sv, int* si, int* sur
 }
 
 // One CTA per (position t, request b): final candidates of rows t (and t-1, the sources), then
-// tau_t -> tau_g[b][t]; row t's candidates -> cl_g/cand_g (and the debug outputs).
-__global__ void __launch_bounds__(256) k_sel_tau(SelParams p, float* tau_g, float* cl_g, int32_t* cand_g) {
+// tau_t -> tau_g[b][t]; row t's candidates -> cl_g/cand_g (and the debug outputs).  The last of a
+// request's D CTAs to finish (arrival ticket per request, acq_rel; rearmed by it) runs the
+// request's Viterbi path.
+__global__ void __launch_bounds__(256) k_sel_tau(SelParams p, float* tau_g, float* cl_g, int32_t* cand_g,
+                                                 int* tickets) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x, b = blockIdx.y, D = p.Bk - 1, warp = threadIdx.x >> 5;
@@ -293,16 +357,29 @@ __global__ void __launch_bounds__(256) k_sel_tau(SelParams p, float* tau_g, floa
   }
   __syncthreads();
   selector_tau<256>(p, b, t, src, t == 0 ? 1 : kTopK, cand[1], As, Wj, tau_g + (size_t)(b * D + t) * kTopK * kTopK);
-}
-
-// One warp per request: the Viterbi path over the D positions.
-__global__ void __launch_bounds__(32) k_sel_viterbi(SelParams p, const float* tau_g, const float* cl_g,
-                                                    const int32_t* cand_g) {
-  pdl_trigger();
-  pdl_wait();
-  const int b = blockIdx.x, D = p.Bk - 1;
-  selector_viterbi(p, b, cl_g + (size_t)b * D * kTopK, cand_g + (size_t)b * D * kTopK,
-                   tau_g + (size_t)b * D * kTopK * kTopK);
+  __shared__ int s_last;
+  __syncthreads();  // this CTA's tau, cl and cand stores precede its arrival
+  if (threadIdx.x == 0) {
+    int prev;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;" : "=r"(prev) : "l"(tickets + b) : "memory");
+    s_last = prev == D - 1;
+    if (s_last) tickets[b] = 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  // the request's scores and candidates into shared memory in one round trip, then the path
+  float* tau_s = big;                                        // [D][16][16]
+  float* cl_s = big + kMaxD * kTopK * kTopK;                 // [D][16]
+  int* cd_s = reinterpret_cast<int*>(cl_s + kMaxD * kTopK);  // [D][16]
+  const float* tb = tau_g + (size_t)b * D * kTopK * kTopK;
+  for (int i = threadIdx.x; i < D * kTopK * kTopK / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(tau_s)[i] = __ldcg(reinterpret_cast<const float4*>(tb) + i);
+  for (int i = threadIdx.x; i < D * kTopK; i += blockDim.x) {
+    cl_s[i] = __ldcg(cl_g + (size_t)b * D * kTopK + i);
+    cd_s[i] = __ldcg(cand_g + (size_t)b * D * kTopK + i);
+  }
+  __syncthreads();
+  if (warp == 0) selector_viterbi<true>(p, b, cl_s, cd_s, tau_s);
 }
 
 }  // namespace dfl
