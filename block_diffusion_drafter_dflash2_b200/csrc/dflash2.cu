@@ -1051,7 +1051,14 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     float* tau = at<float>(ws, P.off_tau);
     float* clg = at<float>(ws, P.off_cfv);
     int32_t* cdg = at<int32_t>(ws, P.off_cfi);
-    CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), 0, s, sp, tau, clg, cdg, ctr + P.ctr_sel));
+    // The CTAs are few and latency-bound: reserve (unused) dynamic shared memory so that each gets
+    // an SM of its own instead of several landing on the first SM the output head frees.
+    static bool sel_attr = false;
+    if (!sel_attr) {
+      CK(cudaFuncSetAttribute(k_sel_tau, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSpreadSmem));
+      sel_attr = true;
+    }
+    CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), kSelSpreadSmem, s, sp, tau, clg, cdg, ctr + P.ctr_sel));
   }
   return DFLASH2_OK;
 }

@@ -16,6 +16,7 @@
 namespace dfl {
 
 constexpr int kMaxD = 15;
+constexpr int kSelSpreadSmem = 160 * 1024;  // dynamic shared memory reserved per selector CTA (one per SM)
 constexpr int kMaxR = 256;
 
 struct SelParams {
