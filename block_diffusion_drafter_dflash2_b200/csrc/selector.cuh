@@ -11,9 +11,18 @@
 //   delta_t(j) = u_t(j) + max_i (delta_{t-1}(i) + tau_t(c_{t-1,i} -> c_tj)),
 // smaller candidate index on ties.  fp32 throughout.
 #pragma once
+#include <climits>
+
 #include "common.cuh"
 
 namespace dfl {
+
+// Integer keys that order like the floats (no NaN): a warp max/min of floats in one redux.
+DEVI int order_key(float f) {
+  const int k = __float_as_int(f);
+  return k >= 0 ? k : k ^ 0x7fffffff;
+}
+DEVI float key_float(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
 
 constexpr int kMaxD = 15;
 constexpr int kSelSpreadSmem = 160 * 1024;  // dynamic shared memory reserved per selector CTA (one per SM)
@@ -64,29 +73,30 @@ DEVI void merge_lists_row(const float* cv, const int32_t* ci, int nparts, int ro
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) T0 = fmaxf(T0, __shfl_xor_sync(0xffffffffu, T0, o));
   if (nparts <= 8 * 32) {
-    // 16th largest head: 16 rounds of a warp max, removing one occurrence each time
-    float hb = -INFINITY;
+    // 16th largest head: 16 rounds of a warp max (one redux on order-preserving integer keys),
+    // removing one occurrence each time
+    int hk[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hk[q] = order_key(heads[q]);
+    int hb = INT_MIN;
     for (int k = 0; k < kTopK; ++k) {
-      float lb = -INFINITY;
-      int li_ = -1;
+      int lb = INT_MIN, li_ = -1;
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (heads[q] > lb) {
-          lb = heads[q];
+        if (hk[q] > lb) {
+          lb = hk[q];
           li_ = q;
         }
-      float m = lb;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int m = __reduce_max_sync(0xffffffffu, lb);
       const unsigned who = __ballot_sync(0xffffffffu, li_ >= 0 && lb == m);
       if (who && lane == __ffs(who) - 1) {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          if (q == li_) heads[q] = -INFINITY;
+          if (q == li_) hk[q] = INT_MIN;
       }
       hb = m;
     }
-    T0 = fmaxf(T0, hb);
+    if (hb != INT_MIN) T0 = fmaxf(T0, key_float(hb));
   }
   if (lane == 0) *surv = 0;
   __syncwarp();
@@ -142,23 +152,44 @@ DEVI void merge_lists_row(const float* cv, const int32_t* ci, int nparts, int ro
   }
   __syncwarp();
   const int n = *surv;
+  if (n <= 64) {
+    // few survivors (the usual case): each one's rank is the number of survivors better than it
+    // (ids are distinct, so ranks are), and the 16 best go straight to their places
+    if (lane < kTopK) {
+      out_v[lane] = -INFINITY;
+      out_id[lane] = 0x7fffffff;
+    }
+    __syncwarp();
+    for (int e = lane; e < n; e += 32) {
+      const float v = sv[e];
+      const int id = si[e];
+      int rank = 0;
+      for (int i = 0; i < n; ++i) rank += better(sv[i], si[i], v, id) ? 1 : 0;
+      if (rank < kTopK) {
+        out_v[rank] = v;
+        out_id[rank] = id;
+      }
+    }
+    __syncwarp();
+    return;
+  }
   if (n <= cap) {
     for (int k = 0; k < kTopK; ++k) {
       float bv = -INFINITY;
       int bid = 0x7fffffff, bslot = -1;
       for (int i = lane; i < n; i += 32)
         if (better(sv[i], si[i], bv, bid)) { bv = sv[i]; bid = si[i]; bslot = i; }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-        const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
-        if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && os > bslot)) { bv = ov; bid = oid; bslot = os; }
-      }
+      // best value (redux on order-preserving keys), then the smallest id among its holders
+      const int mk = __reduce_max_sync(0xffffffffu, order_key(bv));
+      const int mid = __reduce_min_sync(0xffffffffu, order_key(bv) == mk ? bid : 0x7fffffff);
+      const unsigned who = __ballot_sync(0xffffffffu, order_key(bv) == mk && bid == mid && bslot >= 0);
       if (lane == 0) {
-        out_id[k] = bid;
-        out_v[k] = bv;
-        if (bslot >= 0) { sv[bslot] = -INFINITY; si[bslot] = 0x7fffffff; }
+        out_id[k] = mid;
+        out_v[k] = key_float(mk);
+      }
+      if (who && lane == __ffs(who) - 1) {
+        sv[bslot] = -INFINITY;
+        si[bslot] = 0x7fffffff;
       }
       __syncwarp();
     }
