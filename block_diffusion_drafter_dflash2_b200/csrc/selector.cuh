@@ -246,18 +246,34 @@ DEVI void selector_tau(const SelParams& p, int b, int t, const int* src_ids, int
                        float (*As)[kMaxR], float (*Wj)[kTopK], float* tau) {
   const int D = p.Bk - 1, R = p.R, R8 = R / 8;
   const float* zt = p.z + (size_t)(b * D + t) * R;
-  for (int i = threadIdx.x; i < kTopK * R8; i += NTHR) {
-    const int j = i / R8, r = (i % R8) * 8;
-    const uint4 bv = *reinterpret_cast<const uint4*>(p.cb_b + (size_t)cand_t[j] * R + r);
-    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+  // every thread issues the loads of all its items (codebook rows are random HBM rows) before
+  // converting any of them
+  constexpr int kIt = (kTopK * (kMaxR / 8) + NTHR - 1) / NTHR;
+  uint4 bv[kIt], av[kIt];
+  float4 z0[kIt], z1[kIt];
+#pragma unroll
+  for (int k = 0; k < kIt; ++k) {
+    const int i = threadIdx.x + k * NTHR, j = i / R8, r = (i % R8) * 8;
+    if (i < kTopK * R8) {
+      bv[k] = *reinterpret_cast<const uint4*>(p.cb_b + (size_t)cand_t[j] * R + r);
+      z0[k] = __ldcg(reinterpret_cast<const float4*>(zt + r));
+      z1[k] = __ldcg(reinterpret_cast<const float4*>(zt + r + 4));
+      if (j < nsrc) av[k] = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kIt; ++k) {
+    const int i = threadIdx.x + k * NTHR, j = i / R8, r = (i % R8) * 8;
+    if (i >= kTopK * R8) continue;
+    const uint32_t bw[4] = {bv[k].x, bv[k].y, bv[k].z, bv[k].w};
+    const float zz[8] = {z0[k].x, z0[k].y, z0[k].z, z0[k].w, z1[k].x, z1[k].y, z1[k].z, z1[k].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      Wj[r + 2 * e][j] = __ldcg(zt + r + 2 * e) * bf2f(bw[e] & 0xffff);
-      Wj[r + 2 * e + 1][j] = __ldcg(zt + r + 2 * e + 1) * bf2f(bw[e] >> 16);
+      Wj[r + 2 * e][j] = zz[2 * e] * bf2f(bw[e] & 0xffff);
+      Wj[r + 2 * e + 1][j] = zz[2 * e + 1] * bf2f(bw[e] >> 16);
     }
     if (j < nsrc) {
-      const uint4 av = *reinterpret_cast<const uint4*>(p.cb_a + (size_t)src_ids[j] * R + r);
-      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+      const uint32_t aw[4] = {av[k].x, av[k].y, av[k].z, av[k].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         As[j][r + 2 * e] = bf2f(aw[e] & 0xffff);
@@ -300,12 +316,15 @@ DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int
     if (t == 0) {
       d = c + ldf(tt + j);
     } else {
-      float best = 0.f;
-      int bi = -1;
-      for (int i = 0; i < kTopK; ++i) {
-        const float sc = __shfl_sync(0xffffffffu, d, i) + ldf(tt + i * kTopK + j);
-        if (bi < 0 || sc > best) { best = sc; bi = i; }
-      }
+      // all 16 shuffles and loads go out together; the first maximum wins
+      float sc[kTopK];
+#pragma unroll
+      for (int i = 0; i < kTopK; ++i) sc[i] = __shfl_sync(0xffffffffu, d, i) + ldf(tt + i * kTopK + j);
+      float best = sc[0];
+      int bi = 0;
+#pragma unroll
+      for (int i = 1; i < kTopK; ++i)
+        if (sc[i] > best) { best = sc[i]; bi = i; }
       d = c + best;
       bp[t] = bi;
     }
