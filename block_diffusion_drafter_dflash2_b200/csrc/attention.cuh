@@ -369,21 +369,23 @@ constexpr int kClRedStride = kHeadDim + 8;  // floats per row of the quarter par
 // Dynamic shared memory of k_attn_cluster: queries + KC key rows + KC value rows, bf16, padded rows.
 constexpr size_t attn_cluster_smem(int MT, int KC) { return (size_t)(MT * 16 + 2 * KC) * kAttnStride * 2; }
 
-template <int MT, int NTK>  // MT 16-row query tiles; NTK 8-key tiles per warp quarter (KC = 32*NTK keys per CTA)
-__global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint16_t* __restrict__ ob) {
-  constexpr int NT = MT * 128, kQv = MT * 16, KC = 32 * NTK, KQ = 8 * NTK, kQpc = kQv / kClusterCtas;
-  static_assert(MT <= 2 && NTK % 2 == 0, "shape");
-  static_assert(MT * 4 * 16 * kClRedStride * 4 <= 2 * KC * kAttnStride * 2, "quarter partials fit over K/V");
-  static_assert(kQpc * 64 == NT, "one output pair per thread in the cluster merge");
+// MT 16-row query tiles; KG key groups (warp = group * MT + tile); NTK 8-key tiles per group
+// (KC = KG * 8 * NTK keys per CTA).
+template <int MT, int NTK, int KG = 4>
+__global__ void __launch_bounds__(MT * KG * 32, 1) k_attn_cluster(AttnParams p, uint16_t* __restrict__ ob) {
+  constexpr int NT = MT * KG * 32, kQv = MT * 16, KQ = 8 * NTK, KC = KG * KQ, kQpc = kQv / kClusterCtas;
+  static_assert(MT <= 2 && NTK % 2 == 0 && KC % kPage == 0, "shape");
+  static_assert(MT * KG * 16 * kClRedStride * 4 <= 2 * KC * kAttnStride * 2, "group partials fit over K/V");
+  static_assert(kQpc >= 1 && kQpc * 64 <= NT, "one output pair per thread in the cluster merge");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int row_ok[KC];  // 0 masked, 1 cache key (window applies), 2 block key
   __shared__ int pgs[KC / kPage];
-  __shared__ float red_m[MT * 4][16], red_l[MT * 4][16];
-  __shared__ float cm[kQv], cl[kQv], qw[kQv][4];
+  __shared__ float red_m[MT * KG][16], red_l[MT * KG][16];
+  __shared__ float cm[kQv], cl[kQv], qw[kQv][KG];
   uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
   uint16_t* Ks = Qs + kQv * kAttnStride;
   uint16_t* Vs = Ks + KC * kAttnStride;
-  float* red_o = reinterpret_cast<float*>(Ks);  // [MT*4 warps][16][kClRedStride] after the math
+  float* red_o = reinterpret_cast<float*>(Ks);  // [MT*KG warps][16][kClRedStride] after the math
   pdl_trigger();
   const uint32_t r = cluster_rank();
   const int kvh = blockIdx.y, b = blockIdx.z;
@@ -551,10 +553,10 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
     const int qv = threadIdx.x, qtt = qv / 16, row = qv % 16;
     float M = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) M = fmaxf(M, red_m[q * MT + qtt][row]);
+    for (int q = 0; q < KG; ++q) M = fmaxf(M, red_m[q * MT + qtt][row]);
     float L = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < KG; ++q) {
       const int wq = q * MT + qtt;
       const float wgt = M == -INFINITY ? 0.f : exp2f(red_m[wq][row] - M);
       qw[qv][q] = wgt;
@@ -568,12 +570,12 @@ __global__ void __launch_bounds__(MT * 128, 1) k_attn_cluster(AttnParams p, uint
     const int qv = i / kHeadDim, d = i % kHeadDim, qtt = qv / 16, row = qv % 16;
     float O = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) O += qw[qv][q] * red_o[((size_t)(q * MT + qtt) * 16 + row) * kClRedStride + d];
+    for (int q = 0; q < KG; ++q) O += qw[qv][q] * red_o[((size_t)(q * MT + qtt) * 16 + row) * kClRedStride + d];
     red_o[(size_t)qv * kClRedStride + d] = O;  // only this thread reads or writes this element
   }
   cluster_sync_all();
   // ---- merge the cluster's 8 partials: this CTA finishes query vectors r*kQpc .. +kQpc-1 ----
-  {
+  if (threadIdx.x < kQpc * 64) {
     const int qv = (int)r * kQpc + threadIdx.x / 64, d = (threadIdx.x % 64) * 2;
     float mc[kClusterCtas], M = -INFINITY;
 #pragma unroll

@@ -28,7 +28,8 @@ struct GemvPlan {
 
 struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
-  int attn_ntk;  // > 0: attention as one cluster kernel with 32*attn_ntk keys per CTA; 0: chunks + merge kernel
+  int attn_ntk;  // > 0: attention as one cluster kernel, attn_kg key groups of 8*attn_ntk keys per CTA; 0: chunks + merge
+  int attn_kg;
   bool q4;
   GemvPlan fc, dc, qkv, o, gu, dn;
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
@@ -133,12 +134,24 @@ Plan make_plan(const dflash2_config* c, int B) {
     // the cluster's 8 CTAs cover the window's keys (page aligned) and the block's keys
     const int need = (c->window + kPage - 2 + p.Bk + kClusterCtas - 1) / kClusterCtas;
     p.attn_ntk = 0;
-    if (p.MT <= 2)
-      for (int ntk : {4, 8, 10, 12})
+    p.attn_kg = 4;
+    if (p.MT <= 2) {
+      for (int ntk : {4, 8})
         if (32 * ntk >= need) {
           p.attn_ntk = ntk;
           break;
         }
+      if (!p.attn_ntk && 6 * 48 >= need) {  // 6 key groups of 48 keys: 12 warps per CTA
+        p.attn_ntk = 6;
+        p.attn_kg = 6;
+      }
+      if (!p.attn_ntk)
+        for (int ntk : {10, 12})
+          if (32 * ntk >= need) {
+            p.attn_ntk = ntk;
+            break;
+          }
+    }
   }
   p.fc = plan_gemv(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
   p.dc = plan_gemv((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
@@ -387,18 +400,18 @@ cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
   return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(kAttnThreads), smem, s, ap);
 }
 
-template <int MT, int NTK>
+template <int MT, int NTK, int KG>
 cudaError_t launch_attn_cluster_t(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
   static bool attr = false;
-  const size_t smem = attn_cluster_smem(MT, 32 * NTK);
+  const size_t smem = attn_cluster_smem(MT, KG * 8 * NTK);
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_cluster<MT, NTK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_cluster<MT, NTK, KG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kClusterCtas, ap.nkv, P.B);
-  cfg.blockDim = dim3(MT * 128);
+  cfg.blockDim = dim3(MT * KG * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute at[2];
@@ -410,16 +423,17 @@ cudaError_t launch_attn_cluster_t(const Plan& P, const AttnParams& ap, uint16_t*
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k_attn_cluster<MT, NTK>, ap, ob);
+  return cudaLaunchKernelEx(&cfg, k_attn_cluster<MT, NTK, KG>, ap, ob);
 }
 
 template <int MT>
 cudaError_t launch_attn_cluster_mt(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
+  if (P.attn_kg == 6) return launch_attn_cluster_t<MT, 6, 6>(P, ap, ob, s);
   switch (P.attn_ntk) {
-    case 4: return launch_attn_cluster_t<MT, 4>(P, ap, ob, s);
-    case 8: return launch_attn_cluster_t<MT, 8>(P, ap, ob, s);
-    case 10: return launch_attn_cluster_t<MT, 10>(P, ap, ob, s);
-    default: return launch_attn_cluster_t<MT, 12>(P, ap, ob, s);
+    case 4: return launch_attn_cluster_t<MT, 4, 4>(P, ap, ob, s);
+    case 8: return launch_attn_cluster_t<MT, 8, 4>(P, ap, ob, s);
+    case 10: return launch_attn_cluster_t<MT, 10, 4>(P, ap, ob, s);
+    default: return launch_attn_cluster_t<MT, 12, 4>(P, ap, ob, s);
   }
 }
 
