@@ -52,6 +52,15 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_sustained_tflops():
+    """Measured sustained dense bf16 rate (the step is long), else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1400.0, "fallback"
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
@@ -287,6 +296,8 @@ def main():
     L_after = [int(v) + Bk for v in inputs.context_lengths(wl)]
     byt = accounting.step_bytes(dims, L_after, [Bk] * B)
     hbm, peak_kind = peaks()
+    tpk, tpk_kind = bf16_sustained_tflops()
+    flops = accounting.step_flops(dims, B)
     nk = dr.step_kernels()
     traffic = None
     if nk == 1:  # the whole step is one persistent kernel: its bytes are the step's
@@ -319,6 +330,11 @@ def main():
         "step_hbm": {"algorithmic_bytes": byt["total"], "achieved_gbs": byt["total"] / (ms_max * 1e-3) / 1e9,
                      "frac_of_8tbs": byt["total"] / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                      "frac_of_measured": byt["total"] / (ms_max * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind},
+        # the matrix products as a contraction (the bound of the 64-request workload), against the
+        # measured sustained bf16 dense rate
+        "step_tensor": {"flops": flops, "achieved_tflops": flops / (ms_max * 1e-3) / 1e12, "peak_tflops": tpk,
+                        "frac": flops / (ms_max * 1e-3) / 1e12 / tpk, "peak_kind": tpk_kind,
+                        "path": "mma.sync m16n8k16 streaming engine"},
         "roofline": {"kernel": rk_name, "bound": "hbm",
                      "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm, "traffic": traffic,
                      "algorithmic_bytes": rk_bytes, "avg_launch_ms": lm_ms, "peak_kind": peak_kind},

@@ -35,7 +35,7 @@ struct Plan {
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
   bool persistent;
   size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
-  int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows;
+  int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows, lm_groups;
   bool lm_stream;
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
@@ -161,7 +161,10 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.dn = plan_gemv(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
   p.lm_rows = B * p.D;
   const int lm_tiles = p.V / 16 + p.R / 16;
-  p.lm_stream = p.lm_rows <= 8;
+  // the streaming head takes any number of rows in groups of 8 (one launch, CTAs per group and
+  // vocabulary part); the 16-row pass kernel below stays as the fallback
+  p.lm_stream = true;
+  p.lm_groups = (p.lm_rows + 7) / 8;
   if (p.lm_stream) {
     p.lm_NT = 1;
     p.lm_rows_per_pass = 8;
@@ -235,7 +238,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_tau = take((size_t)p.lm_rows * kTopK * kTopK * 4);
   p.off_rope = take((size_t)2 * p.Mb * 64 * 8);
   p.off_rpage = take((size_t)p.Mb * 8);
-  p.off_hpart = take(p.lm_stream ? (size_t)p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4 : 0);
+  p.off_hpart = take(p.lm_stream ? (size_t)p.lm_groups * p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4 : 0);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
@@ -249,7 +252,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   }
   p.ctr_per_layer = acc;
   p.ctr_head = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;  // the streaming head's record tickets
-  p.ctr_sel = p.ctr_head + (size_t)(lm_tiles + kHeadTiles - 1) / kHeadTiles;  // selector arrival tickets
+  p.ctr_sel = p.ctr_head + (size_t)p.lm_groups * ((lm_tiles + kHeadTiles - 1) / kHeadTiles);  // selector tickets
   p.ctr_total = p.ctr_sel + (size_t)B + 1;                                      // + the persistent grid barrier
   p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
@@ -1013,7 +1016,8 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       lp.part = at<float>(ws, P.off_hpart);
       lp.counters = ctr + P.ctr_head;
       lp.err = err;
-      CK(launch_pdl(k_slmhead, dim3(P.lm_nparts), dim3(kGemvThreads), P.lm_smem, s, lp));
+      lp.groups = P.lm_groups;
+      CK(launch_pdl(k_slmhead, dim3(P.lm_nparts * P.lm_groups), dim3(kGemvThreads), P.lm_smem, s, lp));
     } else {
       for (int pass = 0; pass < P.lm_passes; ++pass) {
         LmParams lp{};

@@ -650,8 +650,10 @@ DEVI void offer_tile(uint2* lists, const float (&acc)[4], int id0, int rows, int
 // Merge the 16 warp lists of each row into the CTA's list -> cand_val/cand_id[part][row][16].
 // Lane l owns a sorted run of 8 entries (warp list l/2, entries 8*(l&1) .. +7) and a read position;
 // each round the warp picks the best run head (ties: lower lane) and that lane advances.
+// rows_total / row0: the output lists are [part][rows_total][16], this CTA's rows start at row0.
 DEVI void merge_warp_lists(const uint2* lists, int rows, float* cand_val, int32_t* cand_id, int part, int warp,
-                           int nwarps, int lane) {
+                           int nwarps, int lane, int rows_total = -1, int row0 = 0) {
+  if (rows_total < 0) rows_total = rows;
   for (int r = warp; r < rows; r += nwarps) {
     const uint2* run = lists + ((lane >> 1) * 8 + r) * kTopK + (lane & 1) * 8;
     int pos = 0;
@@ -667,7 +669,7 @@ DEVI void merge_warp_lists(const uint2* lists, int rows, float* cand_val, int32_
         if (better(ov, oid, bv, bid) || (ov == bv && oid == bid && ol < bl)) { bv = ov; bid = oid; bl = ol; }
       }
       if (lane == 0) {
-        const size_t o = ((size_t)part * rows + r) * kTopK + kk;
+        const size_t o = ((size_t)part * rows_total + row0 + r) * kTopK + kk;
         cand_val[o] = bv;
         cand_id[o] = bid;
       }
@@ -680,12 +682,13 @@ struct SLmParams {
   const uint8_t* W;  // prepared bf16 records of [lm_head; sel_proj]
   int V, R, H;
   const uint16_t* X;  // final-normed rows [rows][H]
-  int rows;
+  int rows;           // all rows; groups of 8 (row group g: rows 8g .. 8g + 7)
+  int groups;         // row groups: CTA b works on vocabulary part b / groups for row group b % groups
   float* z;           // [rows][R]
-  float* cand_val;    // [gridDim.x][rows][16]
+  float* cand_val;    // [parts][rows][16]
   int32_t* cand_id;
-  float* part;        // split records' partial accumulators [gridDim.x][2][16 warps][32 lanes][4]
-  int* counters;      // [records] arrival tickets, zero before the launch (the last arrival re-zeroes)
+  float* part;        // split records' partial accumulators [groups][parts][2][16 warps][32 lanes][4]
+  int* counters;      // [groups][records] arrival tickets, zero before the launch (the last arrival re-zeroes)
   int* err;
 };
 
@@ -711,7 +714,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
   const int half = warp >> 3, wt = warp & 7;
   const int vt = p.V / 16, total = vt + p.R / 16, S = H / 64;
   const int nrec = (total + kHeadTiles - 1) / kHeadTiles;
-  const long long W = (long long)nrec * S, P = gridDim.x, c = blockIdx.x;
+  // row group g of vocabulary part c: the groups of one part are neighbours in launch order, so
+  // they stream the same records at about the same time (HBM once, L2 for the others)
+  const int G = p.groups, grp = blockIdx.x % G, row0 = grp * 8;
+  const int rows = p.rows - row0 < 8 ? p.rows - row0 : 8;
+  const long long W = (long long)nrec * S, P = gridDim.x / G, c = blockIdx.x / G;
+  float* part_g = p.part + (size_t)grp * P * 2 * kGemvConsumers * 32 * 4;
+  int* ctr_g = p.counters + (size_t)grp * nrec;
   const long long x0 = c * W / P, x1 = (c + 1) * W / P;
 
   if (threadIdx.x == 0) {
@@ -746,7 +755,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
     lists[i] = make_uint2(__float_as_uint(-INFINITY), 0x7fffffffu);
   pdl_wait();
   uint32_t xph = 0;
-  stage_x_chunk<NC>(p.X, H, p.rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
+  stage_x_chunk<NC>(p.X + (size_t)row0 * H, H, rows, 8, H * 2, Xs, stride, &xbar, xph, p.err);
   uint2* my = lists + warp * 8 * kTopK;
   int cnt = 0;
   bool dead = false;
@@ -781,13 +790,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
       const long long ux = (long long)rec * S;
       const long long first = sk_owner(ux, W, P), last = sk_owner(ux + S - 1, W, P);
       const int k = rec == rec_first ? 0 : 1;
-      float4* mine = reinterpret_cast<float4*>(p.part) + ((c * 2 + k) * kGemvConsumers + warp) * 32 + lane;
+      float4* mine = reinterpret_cast<float4*>(part_g) + ((c * 2 + k) * kGemvConsumers + warp) * 32 + lane;
       *mine = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
       consumers_sync<NC>();
       if (threadIdx.x == 0) {
-        const int prev = ticket_acq_rel(p.counters + rec);
+        const int prev = ticket_acq_rel(ctr_g + rec);
         s_last = prev == (int)(last - first);
-        if (s_last) p.counters[rec] = 0;
+        if (s_last) ctr_g[rec] = 0;
       }
       consumers_sync<NC>();
       have = s_last != 0;
@@ -799,7 +808,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
             v = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
           } else {
             const int ko = rec == (int)((o * W / P) / S) ? 0 : 1;
-            v = __ldcg(reinterpret_cast<const float4*>(p.part) + ((o * 2 + ko) * kGemvConsumers + warp) * 32 + lane);
+            v = __ldcg(reinterpret_cast<const float4*>(part_g) + ((o * 2 + ko) * kGemvConsumers + warp) * 32 + lane);
           }
           a[0] += v.x;
           a[1] += v.y;
@@ -816,14 +825,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = 2 * t + (e & 1);
-        if (r < p.rows) p.z[(size_t)r * p.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
+        if (r < rows) p.z[(size_t)(row0 + r) * p.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
       }
     } else {
-      offer_tile(my, acc[0], tile * 16, p.rows, lane);
+      offer_tile(my, acc[0], tile * 16, rows, lane);
     }
   }
   consumers_sync<NC>();
-  merge_warp_lists(lists, p.rows, p.cand_val, p.cand_id, blockIdx.x, warp, kGemvConsumers, lane);
+  merge_warp_lists(lists, rows, p.cand_val, p.cand_id, (int)c, warp, kGemvConsumers, lane, p.rows, row0);
 }
 
 }  // namespace dfl
