@@ -303,7 +303,7 @@ def main():
     if nk == 1:  # the whole step is one persistent kernel: its bytes are the step's
         rk_name, rk_bytes = "k_step_persistent (whole block step, one cooperative launch)", byt["total"]
     else:
-        rk_name = "k_slmhead / k_lmhead_topk (LM head + streaming top-16 + selector projection)"
+        rk_name = "k_slmhead (LM head + streaming top-16 + selector projection)"
         rk_bytes = accounting.lmhead_bytes(dims, B * D)
         ratio = head_traffic_ratio() if B * D <= 8 else None  # captured for the streaming kernel
         if ratio is not None:

@@ -11,7 +11,6 @@
 
 namespace dfl {
 
-constexpr int kWarps = 8;             // warps per CTA of the streaming GEMV / LM-head kernels
 constexpr int kUnit = 256;            // K granularity of the streaming GEMV (one Q4_K super-block)
 constexpr int kQ4Bytes = 2304;        // prepared Q4_K tile x super-block: 2048 B codes + 256 B scales
 constexpr int kTopK = 16;

@@ -10,7 +10,6 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemv.cuh"
-#include "lmhead.cuh"
 #include "rowops.cuh"
 #include "persist.cuh"
 #include "selector.cuh"
@@ -35,8 +34,7 @@ struct Plan {
   GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
   bool persistent;
   size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
-  int lm_NT, lm_rows_per_pass, lm_passes, lm_nparts, lm_rows, lm_groups;
-  bool lm_stream;
+  int lm_nparts, lm_rows, lm_groups;
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
       off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
@@ -161,22 +159,11 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.dn = plan_gemv(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
   p.lm_rows = B * p.D;
   const int lm_tiles = p.V / 16 + p.R / 16;
-  // the streaming head takes any number of rows in groups of 8 (one launch, CTAs per group and
-  // vocabulary part); the 16-row pass kernel below stays as the fallback
-  p.lm_stream = true;
+  // the streaming head takes any number of rows in groups of 8 (one launch, a CTA per group and
+  // vocabulary part)
   p.lm_groups = (p.lm_rows + 7) / 8;
-  if (p.lm_stream) {
-    p.lm_NT = 1;
-    p.lm_rows_per_pass = 8;
-    p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
-    p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
-  } else {
-    p.lm_NT = 2;
-    p.lm_rows_per_pass = 16;
-    p.lm_smem = (size_t)16 * (p.H * 2 + 64) + (size_t)kWarps * 16 * kTopK * 8;
-    p.lm_nparts = std::min(p.nsm, (lm_tiles + kWarps - 1) / kWarps);
-  }
-  p.lm_passes = (p.lm_rows + p.lm_rows_per_pass - 1) / p.lm_rows_per_pass;
+  p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
+  p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
   // one request with a block of <= 8: the whole step runs as one persistent launch
   p.persistent = B == 1 && p.Bk <= 8 && p.QVP == 32 && 8 * (p.H * 2 + 64) <= kPXBytes &&
                  (size_t)(p.MT * 16 + 2 * kAttnKeys) * kAttnStride * 2 <= (size_t)kPXBytes;
@@ -238,7 +225,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_tau = take((size_t)p.lm_rows * kTopK * kTopK * 4);
   p.off_rope = take((size_t)2 * p.Mb * 64 * 8);
   p.off_rpage = take((size_t)p.Mb * 8);
-  p.off_hpart = take(p.lm_stream ? (size_t)p.lm_groups * p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4 : 0);
+  p.off_hpart = take((size_t)p.lm_groups * p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
@@ -997,7 +984,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   // A5: LM head + streaming top-16 (+ selector projection)
   {
     if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
-    if (P.lm_stream) {
+    {
       static bool attr = false;
       if (!attr) {
         CK(cudaFuncSetAttribute(k_slmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit - kStaticSmem));
@@ -1018,28 +1005,6 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       lp.err = err;
       lp.groups = P.lm_groups;
       CK(launch_pdl(k_slmhead, dim3(P.lm_nparts * P.lm_groups), dim3(kGemvThreads), P.lm_smem, s, lp));
-    } else {
-      for (int pass = 0; pass < P.lm_passes; ++pass) {
-        LmParams lp{};
-        lp.W = (const uint8_t*)w->lm_head;
-        lp.V = P.V;
-        lp.R = P.R;
-        lp.H = H;
-        lp.row_base = pass * P.lm_rows_per_pass;
-        lp.X = hn + (size_t)lp.row_base * H;
-        lp.rows = std::min(P.lm_rows_per_pass, P.lm_rows - lp.row_base);
-        lp.rows_total = P.lm_rows;
-        lp.z = zbuf;
-        lp.cand_val = at<float>(ws, P.off_cv);
-        lp.cand_id = at<int32_t>(ws, P.off_ci);
-        static bool attr = false;
-        if (!attr) {
-          CK(cudaFuncSetAttribute(k_lmhead_topk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit - kStaticSmem));
-          attr = true;
-        }
-        k_lmhead_topk<2><<<P.lm_nparts, kWarps * 32, P.lm_smem, s>>>(lp);
-        CK(cudaGetLastError());
-      }
     }
     if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
     if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
@@ -1144,7 +1109,7 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention (+ a merge
   // kernel when the merge is not fused in), W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head
   // pass(es), selector (transition scores, the last CTA of a request runs its Viterbi path)
-  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + (P.lm_stream ? 1 : P.lm_passes) + 1;
+  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + 1 + 1;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

@@ -31,7 +31,6 @@
 // order — deterministic — and runs the epilogue.
 #pragma once
 #include "gemv.cuh"
-#include "lmhead.cuh"
 
 namespace dfl {
 
