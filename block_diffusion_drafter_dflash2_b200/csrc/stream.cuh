@@ -692,7 +692,7 @@ struct SLmParams {
 };
 
 constexpr int kHeadSlot = kHeadTiles * 2048;  // one record step: 32 KB
-constexpr int kHeadNS = 3;
+constexpr int kHeadNS = 4;
 
 // Work split: stream-K over (record, K step) units, CTA c taking [c*W/P, (c+1)*W/P) of the
 // W = records * (H/64) steps, so every SM streams the same number of bytes.  A record cut between
