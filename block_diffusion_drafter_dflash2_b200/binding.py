@@ -196,15 +196,18 @@ class Drafter:
 
     def spec_step_host(self, state: dict, taps_h, n_new_h, block_tokens_h, target_h, path_h, scores_h, accepted_h,
                        emitted_h, stream=None, kv: Optional[KV] = None) -> int:
-        """Host-buffer round trip (inputs copied in, outputs copied back, stream synchronised)."""
+        """Host-buffer round trip (inputs in, outputs back, stream synchronised); returns the device
+        error bits.  With page-locked buffers the library's kernels read and write them in place."""
         kvs = kv if kv is not None else kv_struct(state)
-        dev_err = C.c_int32(0)
+        if getattr(self, "_err_h", None) is None:
+            self._err_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+        self._err_h.zero_()
         rc = self.lib.dflash2_spec_step_host(
             C.byref(self.cfg), C.byref(self.w), C.byref(kvs), self.batch, _ptr(taps_h), _ptr(n_new_h),
             _ptr(block_tokens_h), _ptr(target_h), _ptr(path_h), _ptr(scores_h), _ptr(accepted_h), _ptr(emitted_h),
-            C.addressof(dev_err), _ptr(self.workspace), self.ws_bytes, _stream(stream))
+            _ptr(self._err_h), _ptr(self.workspace), self.ws_bytes, _stream(stream))
         check(rc, "spec_step_host")
-        return dev_err.value
+        return int(self._err_h[0])
 
     def step_kernels(self) -> int:
         """Kernels one draft_step launches (1: the whole step is one persistent kernel)."""

@@ -96,6 +96,18 @@ GemvPlan plan_gemv_persistent(int tiles, int rows, int K, bool q4, int nsm) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Device address of a page-locked host buffer (under unified addressing every page-locked
+// allocation is mapped into the device's address space), or null for pageable or misaligned memory.
+void* host_mapped(const void* h) {
+  if (!h || ((uintptr_t)h & 3u)) return nullptr;
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, h) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 bool cfg_ok(const dflash2_config* c) {
   if (!c) return false;
   const long long HQ = (long long)c->n_q * c->head_dim;
@@ -1083,21 +1095,47 @@ int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, co
   cudaStream_t s = (cudaStream_t)stream;
   const size_t Mb = P.Mb;
   CK(cudaMemcpyAsync(at<void>(ws, P.off_s_taps), taps_h, Mb * P.T * P.H * 2, cudaMemcpyHostToDevice, s));
-  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_nnew), n_new_h, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
-  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_btok), block_tokens_h, Mb * 4, cudaMemcpyHostToDevice, s));
-  CK(cudaMemcpyAsync(at<void>(ws, P.off_s_tgt), target_h, Mb * 4, cudaMemcpyHostToDevice, s));
+  // While the taps copy runs: when every small buffer is page-locked, kernels read and write them
+  // in place (one gather kernel and the acceptance kernel) instead of eight small copies.
+  void* const small_h[] = {(void*)n_new_h, (void*)block_tokens_h, (void*)target_h, path_h, scores_h, accepted_h,
+                           emitted_h, dev_err};
+  void* small_d[8] = {};
+  bool direct = true;
+  for (int i = 0; i < (dev_err ? 8 : 7) && direct; ++i) {
+    small_d[i] = host_mapped(small_h[i]);
+    direct = small_d[i] != nullptr;
+  }
+  if (direct) {
+    k_stage_host_inputs<<<1, 256, 0, s>>>((const int32_t*)small_d[0], (const int32_t*)small_d[1],
+                                         (const int32_t*)small_d[2], batch, (int)Mb, at<int32_t>(ws, P.off_s_nnew),
+                                         at<int32_t>(ws, P.off_s_btok), at<int32_t>(ws, P.off_s_tgt));
+    CK(cudaGetLastError());
+  } else {
+    CK(cudaMemcpyAsync(at<void>(ws, P.off_s_nnew), n_new_h, (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(at<void>(ws, P.off_s_btok), block_tokens_h, Mb * 4, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(at<void>(ws, P.off_s_tgt), target_h, Mb * 4, cudaMemcpyHostToDevice, s));
+  }
   dflash2_inputs in{at<uint16_t>(ws, P.off_s_taps), at<int32_t>(ws, P.off_s_nnew), at<int32_t>(ws, P.off_s_btok)};
   int rc = dflash2_draft_step(c, w, &in, kv, batch, at<int32_t>(ws, P.off_s_path), at<float>(ws, P.off_s_scores), ws,
                               ws_bytes, nullptr, stream);
   if (rc) return rc;
-  rc = dflash2_accept(at<int32_t>(ws, P.off_s_path), at<int32_t>(ws, P.off_s_tgt), batch, P.Bk,
-                      at<int32_t>(ws, P.off_s_acc), at<int32_t>(ws, P.off_s_emit), stream);
-  if (rc) return rc;
-  CK(cudaMemcpyAsync(path_h, at<void>(ws, P.off_s_path), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
-  CK(cudaMemcpyAsync(scores_h, at<void>(ws, P.off_s_scores), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
-  CK(cudaMemcpyAsync(accepted_h, at<void>(ws, P.off_s_acc), (size_t)batch * 4, cudaMemcpyDeviceToHost, s));
-  CK(cudaMemcpyAsync(emitted_h, at<void>(ws, P.off_s_emit), Mb * 4, cudaMemcpyDeviceToHost, s));
-  if (dev_err) CK(cudaMemcpyAsync(dev_err, at<void>(ws, P.off_err), 4, cudaMemcpyDeviceToHost, s));
+  if (direct) {
+    const int n = std::max(batch * P.D, batch);
+    k_accept_to_host<<<(n + 127) / 128, 128, 0, s>>>(
+        at<int32_t>(ws, P.off_s_path), at<float>(ws, P.off_s_scores), at<int32_t>(ws, P.off_s_tgt), batch, P.Bk,
+        at<int>(ws, P.off_err), (int32_t*)small_d[3], (float*)small_d[4], (int32_t*)small_d[5], (int32_t*)small_d[6],
+        (int32_t*)small_d[7]);
+    CK(cudaGetLastError());
+  } else {
+    rc = dflash2_accept(at<int32_t>(ws, P.off_s_path), at<int32_t>(ws, P.off_s_tgt), batch, P.Bk,
+                        at<int32_t>(ws, P.off_s_acc), at<int32_t>(ws, P.off_s_emit), stream);
+    if (rc) return rc;
+    CK(cudaMemcpyAsync(path_h, at<void>(ws, P.off_s_path), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(scores_h, at<void>(ws, P.off_s_scores), (size_t)batch * P.D * 4, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(accepted_h, at<void>(ws, P.off_s_acc), (size_t)batch * 4, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(emitted_h, at<void>(ws, P.off_s_emit), Mb * 4, cudaMemcpyDeviceToHost, s));
+    if (dev_err) CK(cudaMemcpyAsync(dev_err, at<void>(ws, P.off_err), 4, cudaMemcpyDeviceToHost, s));
+  }
   CK(cudaStreamSynchronize(s));
   return DFLASH2_OK;
 }

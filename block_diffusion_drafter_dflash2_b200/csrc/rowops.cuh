@@ -145,15 +145,50 @@ __global__ void __launch_bounds__(256) k_norm(NormParams p) {
   }
 }
 
-__global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,
+// Greedy acceptance of request b: the longest prefix on which draft and target agree, then the
+// emitted tokens (accepted drafts, the target's token after them, -1 padding).
+DEVI void accept_request(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int b, int Bk,
                          int32_t* __restrict__ accepted, int32_t* __restrict__ emitted) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= B) return;
   const int D = Bk - 1;
   int n = 0;
   while (n < D && draft[b * D + n] == target[b * Bk + n]) ++n;
   accepted[b] = n;
   for (int i = 0; i < Bk; ++i) emitted[b * Bk + i] = i < n ? draft[b * D + i] : (i == n ? target[b * Bk + n] : -1);
+}
+
+__global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,
+                         int32_t* __restrict__ accepted, int32_t* __restrict__ emitted) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) accept_request(draft, target, b, Bk, accepted, emitted);
+}
+
+// Host-buffer round, page-locked buffers (device-addressable): the small inputs (n_new [B], block
+// tokens and targets [Mb]) gathered into the workspace by one kernel instead of three copies.
+__global__ void k_stage_host_inputs(const int32_t* __restrict__ n_new_h, const int32_t* __restrict__ btok_h,
+                                    const int32_t* __restrict__ tgt_h, int B, int Mb, int32_t* __restrict__ n_new,
+                                    int32_t* __restrict__ btok, int32_t* __restrict__ tgt) {
+  pdl_trigger();
+  for (int i = threadIdx.x; i < B; i += blockDim.x) n_new[i] = n_new_h[i];
+  for (int i = threadIdx.x; i < Mb; i += blockDim.x) {
+    btok[i] = btok_h[i];
+    tgt[i] = tgt_h[i];
+  }
+}
+
+// ... and the round's results written straight to them: the draft path and scores [B][Bk-1], the
+// acceptance (accepted [B], emitted [B][Bk]) and, when err_h is set, the device error word.
+__global__ void k_accept_to_host(const int32_t* __restrict__ draft, const float* __restrict__ scores,
+                                 const int32_t* __restrict__ target, int B, int Bk, const int* __restrict__ err,
+                                 int32_t* __restrict__ path_h, float* __restrict__ scores_h,
+                                 int32_t* __restrict__ accepted_h, int32_t* __restrict__ emitted_h,
+                                 int32_t* __restrict__ err_h) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B * (Bk - 1)) {
+    path_h[i] = draft[i];
+    scores_h[i] = scores[i];
+  }
+  if (i < B) accept_request(draft, target, i, Bk, accepted_h, emitted_h);
+  if (i == 0 && err_h) *err_h = *err;
 }
 
 }  // namespace dfl

@@ -211,10 +211,14 @@ int dflash2_accept(const int32_t *draft, const int32_t *target, int32_t batch, i
 /* A whole speculative draft round with HOST buffers: copies taps, n_new,
  * block_tokens and target (host, same layouts as above) into the workspace,
  * runs dflash2_draft_step and dflash2_accept, copies path, scores, accepted and
- * emitted back to host memory and synchronizes `stream`.  Page-locked host
- * buffers make the copies asynchronous.  Weights and the KV cache stay on the
- * device.  Returns the first error; device error bits are returned in
- * *dev_err (host) when dev_err is not NULL. */
+ * emitted back to host memory and synchronizes `stream`.  Weights and the KV
+ * cache stay on the device.  When n_new, block_tokens, target, the four
+ * outputs and dev_err (if given) are all page-locked and 4-byte aligned, the
+ * library's kernels read and write them in place (the device-mapped view of
+ * page-locked memory) instead of issuing eight small copies; otherwise they are
+ * copied.  taps is always copied (asynchronously when page-locked).  Returns
+ * the first error; device error bits are returned in *dev_err (host) when
+ * dev_err is not NULL. */
 int dflash2_spec_step_host(const dflash2_config *cfg, const dflash2_weights *w, const dflash2_kv *kv,
                            int32_t batch, const uint16_t *taps_h, const int32_t *n_new_h,
                            const int32_t *block_tokens_h, const int32_t *target_h, int32_t *path_h,

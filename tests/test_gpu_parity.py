@@ -117,6 +117,43 @@ def test_steps_chain_and_device_state_advances():
     parity.check_request(run2, hw_t, hw, 0)
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_buffer_round_matches_device_step(pinned):
+    """The host-buffer round returns the device step's path and scores bit for bit and the oracle's
+    acceptance: page-locked buffers (read and written in place by the kernels) and pageable ones
+    (copied)."""
+    import dataclasses
+    from block_diffusion_drafter_dflash2_b200.binding import Drafter
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], batch=3, ctx_lo=1, ctx_hi=200, target_mode="first_mismatch")
+    w, _, _ = weights_for(wl)
+    B, D = wl.batch, wl.dims.block - 1
+    dr = Drafter(wl.dims, w, B)
+    st_dev, st_host = inputs.make_state(wl, "cuda"), inputs.make_state(wl, "cuda")
+    path = torch.full((B, D), -7, dtype=torch.int32, device="cuda")
+    scores = torch.full((B, D), float("nan"), dtype=torch.float32, device="cuda")
+    dr.draft_step({"taps": st_dev["taps"], "n_new": st_dev["n_new"], "block_tokens": st_dev["block_tokens"]}, st_dev,
+                  path, scores)
+    torch.cuda.synchronize()
+    assert dr.device_error() == 0
+    target = inputs.make_targets(wl, path).cpu()
+
+    def host(t):
+        t = t.cpu().clone()
+        return t.pin_memory() if pinned else t
+
+    ins = [host(st_host[k]) for k in ("taps", "n_new", "block_tokens")] + [host(target)]
+    outs = [host(torch.full(shape, -5, dtype=dt)) for shape, dt in
+            (((B, D), torch.int32), ((B, D), torch.float32), ((B,), torch.int32), ((B, wl.dims.block), torch.int32))]
+    assert all(t.is_pinned() == pinned for t in ins + outs)
+    derr = dr.spec_step_host(st_host, *ins, *outs)
+    assert derr == 0
+    assert torch.equal(outs[0], path.cpu())
+    assert torch.equal(outs[1].view(torch.int32), scores.cpu().view(torch.int32))
+    o_acc, o_em = oracle.accept(path.cpu(), target)
+    assert np.array_equal(outs[2].numpy(), o_acc) and np.array_equal(outs[3].numpy(), o_em)
+    assert torch.equal(st_host["seq_len"], st_dev["seq_len"])
+
+
 @pytest.mark.slow
 def test_full_b1_persistent(monkeypatch):
     """The full single-request step as one persistent kernel."""
