@@ -69,6 +69,13 @@ def test_null_arguments_are_rejected(lib):
     assert lib.dflash2_accept(None, None, 1, 8, None, None, None) == -1
     out = C.c_int32()
     assert lib.dflash2_device_error(None, C.byref(out), None) == -1
+    # the host-buffer round validates its host pointers, batch and workspace before any CUDA call
+    h = [C.c_int32() for _ in range(8)]
+    ptrs = [C.addressof(v) for v in h]
+    assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 1, None, *ptrs[1:8], None, None, 0,
+                                      None) == -1
+    assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 0, *ptrs, None, ptrs[0], 0, None) == -1
+    assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 1, *ptrs, None, None, 0, None) == -1
 
 
 def test_unprepared_q4k_weights_are_rejected(lib):
