@@ -46,7 +46,7 @@ class Weights(C.Structure):
 
 
 class Trace(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in ("hidden", "ctx", "final_h", "cand", "cand_logit", "z")]
+    _fields_ = [(n, C.c_void_p) for n in ("hidden", "ctx", "final_h", "cand", "cand_logit", "z", "q0", "k0")]
 
 
 _lib = None
@@ -278,6 +278,8 @@ def draft_request(dims, hw: HostWeights, taps_b, n_new: int, btok_b, k_cache, v_
             "cand": np.zeros((D, K), np.int32),
             "cand_logit": np.zeros((D, K)),
             "z": np.zeros((D, R)),
+            "q0": np.zeros((Bk, dims.n_q * dims.head_dim)),
+            "k0": np.zeros((Bk, dims.n_kv * dims.head_dim)),
         }
         trs = Trace(*[_p(tr[n]) for n, _ in Trace._fields_])
     ds = dims_struct(dims)

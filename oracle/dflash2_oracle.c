@@ -74,6 +74,8 @@ typedef struct {
   int32_t *cand;      /* [block-1][topk] */
   double *cand_logit; /* [block-1][topk] */
   double *z;          /* [block-1][rank] */
+  double *q0;         /* [block][n_q*head_dim]: layer 0 block queries after q-norm and RoPE */
+  double *k0;         /* [block][n_kv*head_dim]: layer 0 block keys after k-norm and RoPE */
 } orc_trace;
 
 /* ------------------------------------------------------------------ */
@@ -506,6 +508,10 @@ int orc_draft_request(const orc_dims *c, const orc_weights *w, const uint16_t *t
         memcpy(v, nrm, sizeof(double) * hd);
         orc_rope(v, hd, Lb + t, c->rope_theta);
       }
+    }
+    if (l == 0 && tr) {
+      if (tr->q0) memcpy(tr->q0, q, sizeof(double) * (size_t)Bk * HQ);
+      if (tr->k0) memcpy(tr->k0, kb, sizeof(double) * (size_t)Bk * HKV);
     }
     /* context rows: K/V of this layer appended to its cache at L0..Lb-1 */
     for (int i = 0; i < n_new && err == ORC_OK; ++i) {

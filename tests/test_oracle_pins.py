@@ -4,6 +4,7 @@ Each test fixes the oracle to something other than itself, chosen so that a
 plausible slip (a dropped term, a wrong sign or index, a transposed operand)
 fails at least one of them.
 """
+import dataclasses
 import itertools
 import json
 import os
@@ -302,6 +303,69 @@ def test_attention_short_context_sees_all():
     assert err == 0 and np.allclose(o[:, :128], vis.mean(0), atol=1e-12)
 
 
+def _brute_attention(d, q, kb, vb, kc, vc, pt, Lb):
+    """Attention from its textbook definition, one (block row, query head) at a time: collect
+    the keys the row may see (cache positions inside the window, looked up page by page, then
+    every block key), scores q.k / sqrt(head_dim), softmax, weighted sum of the values."""
+    hd, grp = d.head_dim, d.n_q // d.n_kv
+    o = np.zeros_like(q)
+    for t in range(d.block):
+        p = Lb + t
+        j0 = max(0, p - d.window + 1)
+        for h in range(d.n_q):
+            kvh = h // grp
+            keys = [bits_to_f64(kc[pt[j // 16], kvh, j % 16]) for j in range(j0, Lb)]
+            vals = [bits_to_f64(vc[pt[j // 16], kvh, j % 16]) for j in range(j0, Lb)]
+            keys += [kb[u, kvh * hd:(kvh + 1) * hd] for u in range(d.block)]
+            vals += [vb[u, kvh * hd:(kvh + 1) * hd] for u in range(d.block)]
+            s = np.array([float(np.dot(q[t, h * hd:(h + 1) * hd], k)) for k in keys]) / np.sqrt(hd)
+            w = np.exp(s - s.max())
+            w /= w.sum()
+            o[t, h * hd:(h + 1) * hd] = sum(wi * v for wi, v in zip(w, vals))
+    return o
+
+
+@pytest.mark.parametrize("window,L0,n_new", [(40, 70, 5), (4096, 20, 3), (17, 33, 6)])
+def test_attention_matches_brute_force_softmax(window, L0, n_new):
+    """Random, non-degenerate queries (scores of order one, so neither uniform nor saturated),
+    GQA groups of 2, a shuffled page table and the window cutting through pages: every output
+    element equals the brute-force softmax attention."""
+    d, q, kb, vb, kc, vc, pt, Lb = _attn_setup(window=window, L0=L0, n_new=n_new)
+    err, o = oracle.attention(d, q, kb, vb, kc, vc, pt, Lb)
+    assert err == 0
+    want = _brute_attention(d, q, kb, vb, kc, vc, pt, Lb)
+    assert np.allclose(o, want, rtol=0, atol=1e-12)
+    s = q[0, :128] @ kb[:, :128].T / np.sqrt(128)
+    assert 0.3 < s.std() < 3.0  # the case exercises the softmax away from its limits
+
+
+def test_attention_softmax_scale_closed_form():
+    """Two visible keys (a one-token window leaves only the block's two keys) along one axis:
+    the weights are exp(a c_u / sqrt(128)) normalised, so with c_0 - c_1 = sqrt(128) ln 3 the
+    head with a = 1 returns 3/4 of value 0 and 1/4 of value 1, the head with a = 2 returns
+    9/10 and 1/10.  Any other score scale (1/128, none) moves these numbers."""
+    d = inputs.Dims(layers=1, hidden=256, ffn=256, n_q=2, n_kv=1, head_dim=128, window=1, vocab=64,
+                    n_taps=1, block=2, topk=4, rank=4)
+    hd = 128
+    kc = bf16_bits(rng.standard_normal((1, 1, 16, hd)))
+    vc = bf16_bits(rng.standard_normal((1, 1, 16, hd)))
+    pt = np.zeros(1, np.int32)
+    q = np.zeros((2, 2 * hd))
+    q[:, 0] = 1.0
+    q[:, hd] = 2.0
+    kb = np.zeros((2, hd))
+    kb[0, 0] = 0.5 + np.sqrt(128.0) * np.log(3.0)
+    kb[1, 0] = 0.5
+    vb = np.zeros((2, hd))
+    vb[0, 1] = 1.0
+    vb[1, 2] = 1.0
+    err, o = oracle.attention(d, q, kb, vb, kc, vc, pt, 3)
+    assert err == 0
+    for t in range(2):
+        assert np.allclose(o[t, [1, 2]], [0.75, 0.25], atol=1e-12)
+        assert np.allclose(o[t, [hd + 1, hd + 2]], [0.9, 0.1], atol=1e-12)
+
+
 # ------------------------------------------------------------------ top-k
 
 def test_topk_matches_full_sort_with_ties():
@@ -487,6 +551,114 @@ def test_step_with_zero_output_projections_keeps_embeddings():
     for t in range(1, d.block):
         want = oracle.rmsnorm(E[bt[t]], w["final_norm"], d.rms_eps)
         assert np.allclose(tr["final_h"][t - 1], want, atol=1e-12)
+
+
+def _bf16_layers_tiny():
+    d = dataclasses.replace(inputs.TINY, wfmt=1)
+    return dataclasses.replace(inputs.WORKLOADS["tiny"], dims=d)
+
+
+# (gate a, up b) per MLP channel j: the channel's gate row is a/H, its up row b/H, so on a row of
+# ones the gate is a*c and the up value b*c (c = 1/sqrt(1 + eps), the RMSNorm of a constant row)
+_MLP_CASES = [(40.0, 0.5), (-40.0, 3.0), (0.0, 5.0), (1.0, 1.0), (1.5, 1.0), (-1.5, 1.0), (2.5, -2.0)]
+
+
+def test_mlp_branch_gate_goes_through_silu():
+    """One layer with W_o = 0 (attention adds nothing), embeddings of ones and ln2 = 1, so the MLP
+    sees a constant row; W_d copies channel j of the SwiGLU product back onto hidden unit j.
+    Saturated gates fix the roles (SiLU on W_g's output, multiplying W_u's): gate +40 passes the
+    up value through (x sigma(x) -> x), gate -40 blocks it, gate 0 gives exactly 0; the pair
+    +-1.5 pins silu(x) - silu(-x) = x; gate 1 gives sigma(1) = 1 / (1 + e^-1)."""
+    wl = _bf16_layers_tiny()
+    d = wl.dims
+    H, F = d.hidden, d.ffn
+
+    def mut(w):
+        w["embed"].fill_(1.0)
+        L = w["layers"][0]
+        L["wo"].zero_()
+        L["ln2"].fill_(1.0)
+        wg = torch.zeros(F, H)
+        wu = torch.zeros(F, H)
+        wd = torch.zeros(H, F)
+        for j, (a, b) in enumerate(_MLP_CASES):
+            wg[j] = a / H
+            wu[j] = b / H
+            wd[j, j] = 1.0
+        L["wg"] = wg.to(torch.bfloat16)
+        L["wu"] = wu.to(torch.bfloat16)
+        L["wd"] = wd.to(torch.bfloat16)
+        assert torch.equal(L["wg"].float(), wg) and torch.equal(L["wu"].float(), wu)  # exact in bf16
+
+    w, st, kc, vc, (err, path, scores, sl, tr) = _tiny_step(wl=wl, mutate=mut)
+    assert err == 0
+    c = 1.0 / np.sqrt(1.0 + d.rms_eps)
+    h0, h1 = tr["hidden"][0], tr["hidden"][1]
+    assert np.all(h0 == 1.0)
+    for t in range(d.block):
+        y = h1[t] - 1.0
+        assert abs(y[0] - 40 * c * 0.5 * c) <= 1e-9              # open gate: u passes
+        assert abs(y[1]) <= 1e-12                                  # closed gate: nothing
+        assert y[2] == 0.0                                         # silu(0) = 0
+        assert abs(y[3] - 0.7310585786300049) <= 1e-5              # sigma(1), the logistic function
+        assert abs((y[4] - y[5]) - 1.5 * c * c) <= 1e-12           # silu(x) - silu(-x) = x
+        assert y[6] < 0 and abs(y[6] / (-2.0 * c) - 2.5 * c / (1 + np.exp(-2.5 * c))) <= 1e-12
+        assert np.all(y[len(_MLP_CASES):] == 0.0)
+
+
+def _angle_mod_pi(x0, x1):
+    return np.mod(np.arctan2(x1, x0), np.pi)
+
+
+def _pos_mod_pi(p):
+    return np.mod(float(p), np.pi)
+
+
+def test_qk_norm_precedes_rope_at_absolute_positions():
+    """Query head 0 and key head 0 of layer 0 carry one nonzero input dimension (dim 0, the sum
+    of the row); q/k-norm weights differ between dim 0 and its RoPE partner dim 64.  Norm first,
+    then rotation: the pair (0, 64) has amplitude qn[0] * sqrt(128) and angle = position (mod pi,
+    the sign of the sum being unknown) with frequency theta^0 = 1.  Rotation first would give
+    amplitudes mixed from qn[0] and qn[64] and a different angle.  Block rows sit at Lb + t
+    (queries and block keys); context rows are appended to the cache at L0 + i."""
+    wl = _bf16_layers_tiny()
+    d = wl.dims
+
+    def mut(w):
+        L = w["layers"][0]
+        for n in ("wq", "wk"):
+            L[n].zero_()
+            L[n][0] = 1.0
+        L["qn"].fill_(1.0)
+        L["qn"][0], L["qn"][64] = 1.5, 0.5
+        L["kn"].fill_(1.0)
+        L["kn"][0], L["kn"][64] = 0.75, 1.25
+
+    w, st, kc, vc, (err, path, scores, sl, tr) = _tiny_step(wl=wl, mutate=mut)
+    assert err == 0
+    L0, n = int(st["seq_len"][0]), int(st["n_new"][0])
+    Lb = L0 + n
+    hd = d.head_dim
+    for name, trace, wt in (("q", tr["q0"], 1.5), ("k", tr["k0"], 0.75)):
+        for t in range(d.block):
+            v = trace[t]
+            others = np.ones(v.size, bool)
+            others[[0, 64]] = False
+            assert np.all(v[others] == 0.0), name
+            assert abs(np.hypot(v[0], v[64]) - wt * np.sqrt(hd)) <= 1e-3, (name, t)
+            diff = abs(_angle_mod_pi(v[0], v[64]) - _pos_mod_pi(Lb + t))
+            assert min(diff, np.pi - diff) <= 1e-9, (name, t)
+    # context keys in the cache (bf16): position L0 + i, amplitude kn[0] * sqrt(128)
+    pt = oracle._np(st["page_table"][0])
+    for i in range(n):
+        pos = L0 + i
+        row = bits_to_f64(kc[0][pt[pos // 16], 0, pos % 16])
+        others = np.ones(hd, bool)
+        others[[0, 64]] = False
+        assert np.all(row[others] == 0.0)
+        assert abs(np.hypot(row[0], row[64]) - 0.75 * np.sqrt(hd)) <= 0.75 * np.sqrt(hd) * 2 ** -7
+        diff = abs(_angle_mod_pi(row[0], row[64]) - _pos_mod_pi(pos))
+        assert min(diff, np.pi - diff) <= 2 ** -6, i
 
 
 def test_step_ignores_cache_outside_window():
