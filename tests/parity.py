@@ -4,7 +4,12 @@ the same seeded inputs, compare.
 Tolerances (the drafter's bf16-activation path against the fp64 oracle):
   * continuous tensors (hidden states, context rows, final rows, appended cache
     rows, candidate logits end to end): max |gpu - oracle| / max |oracle| <= 2e-2
-    over the compared tensor;
+    per row (per head vector for the cache rows), so an error confined to one row
+    or head cannot hide under another row's larger values;
+  * the selector's end-to-end path: the oracle's own path equals the GPU's, or the
+    oracle scores the GPU's path within the bound the 2e-2 logit tolerance allows
+    (twice the per-position tolerance, summed over the positions);
+  * top-16 ids of every row are distinct;
   * stage-wise (the oracle fed the GPU's own bf16 operands, so only fp32
     accumulation order differs): logits and selector projection within 1e-3
     relative; top-16 ids identical except where the oracle's logits of the
@@ -25,10 +30,16 @@ STAGE_TOL = 1e-3
 
 
 def maxrel(g, o) -> float:
+    """Worst row of max |g - o| / max |o| (each row normalised by its own largest oracle value;
+    the last axis is the row)."""
     g = np.asarray(g, np.float64)
     o = np.asarray(o, np.float64)
-    den = float(np.max(np.abs(o))) if o.size else 1.0
-    return float(np.max(np.abs(g - o)) / max(den, 1e-30)) if o.size else 0.0
+    if not o.size:
+        return 0.0
+    g = g.reshape(-1, o.shape[-1])
+    o = o.reshape(-1, o.shape[-1])
+    den = np.maximum(np.max(np.abs(o), axis=1), 1e-30)
+    return float(np.max(np.max(np.abs(g - o), axis=1) / den))
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
@@ -98,6 +109,11 @@ def host_weights(weights: dict) -> tuple:
 
 def check_topk_row(g_ids, g_vals, o_ids, o_vals, o_at_g) -> None:
     """Top-16 of one row: GPU ids/logits against the oracle's, fed the same bf16 operand."""
+    assert len(set(np.asarray(g_ids).tolist())) == len(g_ids), ("duplicate candidate ids", g_ids)
+    # the GPU's own order: logit descending, smaller id first among equal logits
+    for i in range(len(g_ids) - 1):
+        assert g_vals[i] > g_vals[i + 1] or (g_vals[i] == g_vals[i + 1] and g_ids[i] < g_ids[i + 1]), \
+            ("GPU list out of order", g_ids, g_vals)
     assert np.max(np.abs(g_vals - o_at_g) / np.maximum(1.0, np.abs(o_at_g))) <= STAGE_TOL, (g_vals, o_at_g)
     if np.array_equal(g_ids, o_ids):
         return
@@ -147,7 +163,7 @@ def check_request(run: dict, hw_t: dict, hw: oracle.HostWeights, b: int, check_s
             ot = np.transpose(o_, (0, 2, 1, 3))
             bt = np.transpose(before, (0, 2, 1, 3))
             assert np.array_equal(gt[~new], bt[~new]), "GPU wrote outside the appended rows"
-            if n:
+            if n:  # [rows][head][dim]: one tolerance per head vector
                 r = maxrel(oracle.bf16_to_f64(gt[new]), oracle.bf16_to_f64(ot[new]))
                 report[f"cache{l}"] = max(report.get(f"cache{l}", 0.0), r)
                 assert r <= TOL, report
@@ -187,8 +203,43 @@ def check_request(run: dict, hw_t: dict, hw: oracle.HostWeights, b: int, check_s
     assert report["cand_logit_e2e"] <= TOL, report
     # seq_len advanced by n_new
     assert int(run["state"]["seq_len"][b]) == int(run["seq_before"][b]) + n
+    # the oracle's own end-to-end path against the GPU's: equal, or the oracle scores both paths
+    # within the bound the end-to-end logit tolerance allows
     report["oracle_path_equal_gpu_path"] = bool(np.array_equal(o_path, g_path))
+    if not report["oracle_path_equal_gpu_path"]:
+        margin, bound = e2e_path_margin(hw_t, tr, x0, o_path, g_path)
+        report["e2e_path_margin"], report["e2e_path_bound"] = margin, bound
+        assert margin <= bound, ("end-to-end path differs beyond the logit tolerance", o_path, g_path, margin, bound)
     return report
+
+
+def e2e_path_margin(hw_t: dict, tr: dict, x0: int, o_path, g_path):
+    """The oracle's score of its own path minus its score of the GPU's path (both in the oracle's
+    fp64 logits and transitions), and the largest gap the 2e-2 end-to-end tolerance permits:
+    a path's score moves by at most TOL * (max |logit| + max |transition|) per position, and
+    the GPU maximised its own scores, so the oracle's two scores differ by at most twice that
+    summed over the positions."""
+    lm, A, Bc = hw_t["lm_head"], hw_t["cb_a"], hw_t["cb_b"]
+    fh, z = tr["final_h"], tr["z"]
+    D = fh.shape[0]
+
+    def rows(t, ids):
+        return oracle.bf16_to_f64(oracle._np(t[torch.as_tensor(np.asarray(ids, np.int64))]))
+
+    def score(path):
+        prev = np.concatenate([[x0], path[:-1]])
+        lg = np.einsum("th,th->t", rows(lm, path), fh)
+        tau = np.einsum("tr,tr,tr->t", rows(A, prev), z, rows(Bc, path))
+        return float(lg.sum() + tau.sum())
+
+    cand = tr["cand"]
+    bound = 0.0
+    for t in range(D):
+        lmax = float(np.max(np.abs(tr["cand_logit"][t])))
+        srcs = [x0] if t == 0 else cand[t - 1]
+        tmax = float(np.max(np.abs(rows(A, srcs) * z[t]) @ np.abs(rows(Bc, cand[t])).T))
+        bound += 2.0 * TOL * (lmax + tmax)
+    return score(np.asarray(o_path)) - score(np.asarray(g_path)), bound
 
 
 def check_accept(run: dict) -> None:

@@ -50,7 +50,8 @@ def test_static_scratch_step_matches_workspace_step(name):
             outs.append((path.cpu(), scores.cpu()))
         (pa, sa), (pb, sb) = outs
         assert torch.equal(pa, pb), (call, pa, pb)
-        assert torch.allclose(sa, sb, rtol=2e-2, atol=1e-3), (call, sa, sb)
+        # same kernels, same data, deterministic split-K fix-ups: the scores agree bit for bit
+        assert torch.equal(sa.view(torch.int32), sb.view(torch.int32)), (call, sa, sb)
         assert torch.equal(st_a["seq_len"], st_b["seq_len"])
         for l in range(d.layers):
             assert torch.equal(st_a["k_cache"][l], st_b["k_cache"][l])
