@@ -31,16 +31,21 @@ NOMINAL_HBM_GBS = 8000.0
 
 
 def head_traffic_ratio():
-    """DRAM bytes per algorithmic byte of the streaming LM-head kernel, from the committed ncu
-    summary of its small-case capture (None if the summary is missing)."""
+    """DRAM bytes per algorithmic byte of the streaming LM-head kernel, from the machine-readable
+    summary of its small-case ncu capture; None when the summary is missing or the kernel's source
+    has changed since the capture (the counters then describe another kernel)."""
+    import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "ncu_k_slmhead_prof_small.md")) as f:
-            for line in f:
-                if line.startswith("dram bytes per algorithmic byte:"):
-                    return float(line.split(":")[1])
-    except OSError:
-        pass
-    return None
+        with open(os.path.join(ROOT, "profiles", "ncu_k_slmhead_prof_small.json")) as f:
+            cap = json.load(f)
+        with open(os.path.join(ROOT, "block_diffusion_drafter_dflash2_b200", "csrc", "stream.cuh")) as f:
+            src = f.read()
+    except (OSError, ValueError):
+        return None
+    i = src.find("__global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead")
+    if i < 0 or hashlib.sha256(src[i:].encode()).hexdigest() != cap.get("kernel_source_sha256"):
+        return None
+    return float(cap["dram_bytes_per_algorithmic_byte"])
 
 
 def peaks():
@@ -166,6 +171,15 @@ def host_copy_weights(w: dict):
     return hw_t, oracle.HostWeights(hw_t)
 
 
+def bench_config(wl, ws: int) -> dict:
+    """The workload description both arms print."""
+    d = wl.dims
+    return {"workload": wl.name, "requests_per_gpu": wl.batch, "context": wl.ctx_lo, "block": d.block,
+            "layers": d.layers, "hidden": d.hidden, "vocab": d.vocab,
+            "parallelism": f"replicas x{ws} (requests sharded, no collective)",
+            "l2": "inputs larger than L2 (3.7 GB of weights streamed per step)"}
+
+
 def run_reference(args, ws, rank):
     """The reference arm: the CPU oracle as it stands, timed on the host cores (rank 0 only)."""
     if rank != 0:
@@ -177,17 +191,19 @@ def run_reference(args, ws, rank):
     hw_t, hw = host_copy_weights(w)
     del w
     st_h = host_state_for_request0(st)
-    for _ in range(min(args.warmup, 1)):
+    # one untimed oracle step (each takes seconds on the host cores; the timed steps are bounded by
+    # --ref-budget-s): the line reports the warm-up it ran
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
         oracle_step_time(wl, hw_t, hw, st_h, 0.0, 1)
     times, cores = oracle_step_time(wl, hw_t, hw, st_h, args.ref_budget_s, args.steps)
     per = sum(times) / len(times)
     value = 1.0 / per
     line = {
         "impl": "reference", "metric": "DFlash2 draft steps/s (8-token block)", "value": value,
-        "unit": "steps/s", "n_gpus": ws, "steps": len(times), "warmup": args.warmup, "ms_per_step": per * 1e3,
+        "unit": "steps/s", "n_gpus": ws, "steps": len(times), "warmup": warm, "ms_per_step": per * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "context": wl.ctx_lo, "block": wl.dims.block,
-                   "description": wl.description},
+        "config": bench_config(wl, ws),
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
                          "sample": f"{len(times)} full block steps of request 0 (fp64 C oracle, OpenMP)"},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -300,14 +316,11 @@ def main():
     flops = accounting.step_flops(dims, B)
     nk = dr.step_kernels()
     traffic = None
-    if nk == 1:  # the whole step is one persistent kernel: its bytes are the step's
-        rk_name, rk_bytes = "k_step_persistent (whole block step, one cooperative launch)", byt["total"]
-    else:
-        rk_name = "k_slmhead (LM head + streaming top-16 + selector projection)"
-        rk_bytes = accounting.lmhead_bytes(dims, B * D)
-        ratio = head_traffic_ratio() if B * D <= 8 else None  # captured for the streaming kernel
-        if ratio is not None:
-            traffic = ratio * rk_bytes  # small-case capture scaled by the launch's bytes
+    rk_name = "k_slmhead (LM head + streaming top-16 + selector projection)"
+    rk_bytes = accounting.lmhead_bytes(dims, B * D)
+    ratio = head_traffic_ratio() if B * D <= 8 else None  # captured for the streaming kernel
+    if ratio is not None:
+        traffic = ratio * rk_bytes  # small-case capture scaled by the launch's bytes
     rk_gbs = rk_bytes / (lm_ms * 1e-3) / 1e9
     value = ws / (ms_max * 1e-3)  # draft steps/s over all ranks (one step = a rank's whole batch)
     line = {
@@ -323,10 +336,8 @@ def main():
         "vs_baseline": None,
         "dtype": "q4k/bf16 weights, bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded N(0,0.02) weights quantised to Q4_K, bf16 LM head/codebooks, N(0,1) taps and KV)",
-        "config": {"workload": wl.name, "requests_per_gpu": B, "context": wl.ctx_lo, "block": Bk,
-                   "layers": dims.layers, "hidden": dims.hidden, "vocab": dims.vocab,
-                   "parallelism": f"replicas x{ws} (requests sharded, no collective)",
-                   "l2": "inputs larger than L2 (3.7 GB of weights streamed per step)"},
+        "config": bench_config(wl, ws),
+        "request_steps_per_s": value * B,
         "step_hbm": {"algorithmic_bytes": byt["total"], "achieved_gbs": byt["total"] / (ms_max * 1e-3) / 1e9,
                      "frac_of_8tbs": byt["total"] / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                      "frac_of_measured": byt["total"] / (ms_max * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind},

@@ -210,7 +210,7 @@ class Drafter:
         return int(self._err_h[0])
 
     def step_kernels(self) -> int:
-        """Kernels one draft_step launches (1: the whole step is one persistent kernel)."""
+        """Kernels one draft_step launches."""
         return int(self.lib.dflash2_step_kernels(C.byref(self.cfg), self.batch))
 
     def device_error(self, stream=None) -> int:

@@ -391,7 +391,8 @@ __global__ void __launch_bounds__(MT * KG * 32, 1) k_attn_cluster(AttnParams p, 
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.nq / p.nkv, nqv = G * p.Bk;
-  // step inputs (no kernel of this step writes them)
+  // step inputs: no kernel of this step writes them, and the step's opening memsets order every
+  // earlier writer (host staging, the previous round's acceptance) before this launch
   const long long S0 = p.seq_len[b];
   const long long Lb = S0 + p.n_new[b];
   long long s0 = Lb - p.W + 1;

@@ -11,7 +11,6 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "rowops.cuh"
-#include "persist.cuh"
 #include "selector.cuh"
 #include "stream.cuh"
 
@@ -31,9 +30,7 @@ struct Plan {
   int attn_kg;
   bool q4;
   GemvPlan fc, dc, qkv, o, gu, dn;
-  GemvPlan pfc, pdc, pqkv, po, pgu, pdn;  // persistent single-launch step (batch 1)
-  bool persistent;
-  size_t psmem, off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
+  size_t off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
   int lm_nparts, lm_rows, lm_groups;
   size_t lm_smem;
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
@@ -72,25 +69,6 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
   g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
-  return g;
-}
-
-// Plan of one streamed product inside the persistent step: every SM takes part (P = #SMs) and the
-// activations live in the fixed staging region of that kernel.
-GemvPlan plan_gemv_persistent(int tiles, int rows, int K, bool q4, int nsm) {
-  GemvPlan g;
-  g.R = rows <= 8 ? 8 : 16;
-  g.NT = g.R / 8;
-  g.mgroups = 1;
-  g.groups = (tiles + kConsumers - 1) / kConsumers;
-  const int unitK = q4 ? 256 : 64;
-  g.U = K / unitK;
-  g.W = (long long)g.groups * g.U;
-  g.P = (int)std::min<long long>(nsm, g.W);  // every CTA in [0, P) owns at least one unit
-  g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
-  g.kc_units = std::max(1, std::min(g.U, (kPXBytes - 64 * g.R) / (g.R * unitK * 2)));
-  if (g.kc_units < g.U && g.kc_units > 1) g.kc_units &= ~1;  // whole slots (two units each) per chunk
-  g.smem = 0;
   return g;
 }
 
@@ -176,20 +154,6 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.lm_groups = (p.lm_rows + 7) / 8;
   p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
   p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
-  // one request with a block of <= 8: the whole step runs as one persistent launch
-  p.persistent = B == 1 && p.Bk <= 8 && p.QVP == 32 && 8 * (p.H * 2 + 64) <= kPXBytes &&
-                 (size_t)(p.MT * 16 + 2 * kAttnKeys) * kAttnStride * 2 <= (size_t)kPXBytes;
-  p.psmem = (size_t)kPNS * kPSlot + kPXBytes + (size_t)kGemvConsumers * 128 * 8 + (size_t)kConsumers * 32 * 8 * 4 +
-            (size_t)kPWshBytes;
-  if (p.persistent) {
-    p.pfc = plan_gemv_persistent(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
-    p.pdc = plan_gemv_persistent((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
-    p.pqkv = plan_gemv_persistent((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
-    p.po = plan_gemv_persistent(p.H / 16, p.Mb, p.HQ, p.q4, p.nsm);
-    p.pgu = plan_gemv_persistent(2 * p.F / 16, p.Mb, p.H, p.q4, p.nsm);
-    p.pdn = plan_gemv_persistent(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
-  }
-
   auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.max_pieces * rows * ldo * 4; };
   size_t part = 0;
   part = std::max(part, part_bytes(p.fc, p.Mb, p.H));
@@ -198,15 +162,6 @@ Plan make_plan(const dflash2_config* c, int B) {
   part = std::max(part, part_bytes(p.o, p.Mb, p.H));
   part = std::max(part, part_bytes(p.gu, p.Mb, 2 * p.F));
   part = std::max(part, part_bytes(p.dn, p.Mb, p.H));
-  if (p.persistent) {
-    part = std::max(part, part_bytes(p.pfc, p.Mb, p.H));
-    part = std::max(part, part_bytes(p.pdc, p.Mb, p.H / 2));
-    part = std::max(part, part_bytes(p.pqkv, 2 * p.Mb, p.HQ + 2 * p.HKV));
-    part = std::max(part, part_bytes(p.po, p.Mb, p.H));
-    part = std::max(part, part_bytes(p.pgu, p.Mb, 2 * p.F));
-    part = std::max(part, part_bytes(p.pdn, p.Mb, p.H));
-  }
-
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t r = o;
@@ -228,7 +183,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_ob = take((size_t)p.Mb * p.HQ * 2);
   p.off_act = take((size_t)p.Mb * p.F * 2);
   p.off_hn = take((size_t)std::max(p.lm_rows, 1) * p.H * 2);
-  const size_t nlists = (size_t)std::max(p.lm_nparts, p.persistent ? p.nsm : 0);
+  const size_t nlists = (size_t)p.lm_nparts;
   p.off_cv = take(nlists * p.lm_rows * kTopK * 4);
   p.off_ci = take(nlists * p.lm_rows * kTopK * 4);
   p.off_cfv = take((size_t)p.lm_rows * kTopK * 4);
@@ -252,7 +207,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.ctr_per_layer = acc;
   p.ctr_head = p.ctr_fc + (size_t)c->layers * p.ctr_per_layer;  // the streaming head's record tickets
   p.ctr_sel = p.ctr_head + (size_t)p.lm_groups * ((lm_tiles + kHeadTiles - 1) / kHeadTiles);  // selector tickets
-  p.ctr_total = p.ctr_sel + (size_t)B + 1;                                      // + the persistent grid barrier
+  p.ctr_total = p.ctr_sel + (size_t)B;
   p.off_ctr = take(p.ctr_total * 4);
   p.step_bytes = o;
   p.off_s_taps = take((size_t)p.Mb * p.T * p.H * 2);
@@ -274,6 +229,24 @@ T* at(void* ws, size_t off) {
 
 bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
+constexpr int kMaxDevices = 64;
+
+// Opt kernel k into `bytes` of dynamic shared memory on the current device.  CUDA keeps this
+// attribute per device, so it is recorded per device in `done` (one array per kernel); host
+// threads that race here set the same value, which is harmless.
+template <typename... KArgs>
+cudaError_t smem_optin(void (*k)(KArgs...), int bytes, std::atomic<int>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire) == bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done[dev].store(bytes, std::memory_order_release);
+  return cudaSuccess;
+}
+
 // Launch with programmatic dependent launch: the kernel may start while the previous kernel on
 // the stream drains; every kernel launched this way calls griddepcontrol.wait before it touches
 // data written by earlier kernels.
@@ -294,13 +267,9 @@ cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, 
 
 template <int NT, bool Q4>
 cudaError_t launch_sgemv_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_sgemv<NT, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemLimit - kStaticSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<int> attr[kMaxDevices];
+  const cudaError_t e = smem_optin(k_sgemv<NT, Q4>, kSmemLimit - kStaticSmem, attr);
+  if (e != cudaSuccess) return e;
   return launch_pdl(k_sgemv<NT, Q4>, dim3(g.P), dim3(kSGemvThreads), g.smem, s, prm);
 }
 
@@ -392,25 +361,19 @@ cudaError_t launch_norm(const NormParams& np, int rows, cudaStream_t s) {
 
 template <int MT>
 cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
-  static bool attr = false;
+  static std::atomic<int> attr[kMaxDevices];
   const size_t smem = (size_t)(MT * 16 + 2 * kAttnKeys) * kAttnStride * 2;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_chunk<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t e = smem_optin(k_attn_chunk<MT>, (int)smem, attr);
+  if (e != cudaSuccess) return e;
   return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(kAttnThreads), smem, s, ap);
 }
 
 template <int MT, int NTK, int KG>
 cudaError_t launch_attn_cluster_t(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
-  static bool attr = false;
+  static std::atomic<int> attr[kMaxDevices];
   const size_t smem = attn_cluster_smem(MT, KG * 8 * NTK);
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_cluster<MT, NTK, KG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t e = smem_optin(k_attn_cluster<MT, NTK, KG>, (int)smem, attr);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kClusterCtas, ap.nkv, P.B);
   cfg.blockDim = dim3(MT * KG * 32);
@@ -466,6 +429,15 @@ int check_weights(const dflash2_config* c, const dflash2_weights* w) {
   return DFLASH2_OK;
 }
 
+int check_kv(const dflash2_config* c, const dflash2_kv* kv) {
+  if (!kv || !kv->page_table || !kv->seq_len || kv->max_pages < 1 || kv->num_pages < 1) return DFLASH2_ERR_ARG;
+  for (int l = 0; l < c->layers; ++l) {
+    if (!kv->k[l] || !kv->v[l]) return DFLASH2_ERR_ARG;
+    if (!aligned16(kv->k[l]) || !aligned16(kv->v[l])) return DFLASH2_ERR_ALIGN;
+  }
+  return DFLASH2_OK;
+}
+
 // Scratch of the allocation-free entry point: file-scope device memory, present on every GPU
 // that loads this library for the life of the process.
 static __device__ __align__(256) uint8_t g_static_scratch[DFLASH2_STATIC_SCRATCH_BYTES];
@@ -473,7 +445,6 @@ static __device__ __align__(256) uint8_t g_static_scratch[DFLASH2_STATIC_SCRATCH
 // Device address of g_static_scratch on the current device, looked up once per device.  (The
 // symbol's name in host code is only a host-side stand-in, not a device address.)
 void* static_scratch(cudaError_t* err) {
-  constexpr int kMaxDevices = 64;
   static std::atomic<void*> cache[kMaxDevices];
   int dev = 0;
   *err = cudaGetDevice(&dev);
@@ -488,31 +459,6 @@ void* static_scratch(cudaError_t* err) {
   if (*err != cudaSuccess) return nullptr;
   cache[dev].store(p, std::memory_order_release);
   return p;
-}
-
-// The persistent step needs its shared memory opted in and one CTA of it resident on every SM
-// (cooperative launch); checked once per device.
-bool persistent_ready(const Plan& P) {
-  const char* env = getenv("DFLASH2_PERSISTENT");  // opt in with "1" (the kernel sequence is the default)
-  if (!env || env[0] != '1') return false;
-  constexpr int kMaxDevices = 64;
-  static std::atomic<int> state[kMaxDevices];  // 0 unknown, 1 ready, 2 not available
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  int st = state[dev].load(std::memory_order_acquire);
-  if (st == 0) {
-    int coop = 0, nb = 0;
-    st = 2;
-    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
-        cudaFuncSetAttribute(k_step_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.psmem) ==
-            cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_step_persistent, kPThreads, P.psmem) == cudaSuccess &&
-        nb >= 1)
-      st = 1;
-    cudaGetLastError();
-    state[dev].store(st, std::memory_order_release);
-  }
-  return st == 1;
 }
 
 }  // namespace
@@ -606,13 +552,9 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   if (batch < 1 || !in || !kv || !out_path || !out_scores || !ws) return DFLASH2_ERR_ARG;
   int rc = check_weights(c, w);
   if (rc) return rc;
-  if (!in->taps || !in->n_new || !in->block_tokens || !kv->page_table || !kv->seq_len || kv->max_pages < 1 ||
-      kv->num_pages < 1)
-    return DFLASH2_ERR_ARG;
-  for (int l = 0; l < c->layers; ++l) {
-    if (!kv->k[l] || !kv->v[l]) return DFLASH2_ERR_ARG;
-    if (!aligned16(kv->k[l]) || !aligned16(kv->v[l])) return DFLASH2_ERR_ALIGN;
-  }
+  if (!in->taps || !in->n_new || !in->block_tokens) return DFLASH2_ERR_ARG;
+  rc = check_kv(c, kv);
+  if (rc) return rc;
   if (!aligned16(in->taps) || ((uintptr_t)ws & 255u)) return DFLASH2_ERR_ALIGN;
   const Plan P = make_plan(c, batch);
   if (ws_bytes < P.step_bytes) return DFLASH2_ERR_WORKSPACE;
@@ -655,176 +597,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
 
   float* gbuf = at<float>(ws, P.off_g);
   int* ctr = at<int>(ws, P.off_ctr);
+  // These two memsets are full stream barriers: every earlier operation on the stream (the host
+  // round's staging kernel, the previous round's acceptance writing n_new and block tokens) has
+  // finished before the step's first kernel, so the kernels below may read the step inputs before
+  // their programmatic-launch wait.
   CK(cudaMemsetAsync(err, 0, 4, s));
   CK(cudaMemsetAsync(ctr, 0, P.ctr_total * 4, s));
-  if (P.persistent && persistent_ready(P)) {
-    if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
-    StepParams S;
-    memset(&S, 0, sizeof(S));
-    S.layers = c->layers;
-    S.Bk = P.Bk;
-    S.Mb = Mb;
-    S.H = H;
-    S.D = P.D;
-    S.V = P.V;
-    S.R = P.R;
-    S.eps = c->rms_eps;
-    S.block_tokens = in->block_tokens;
-    S.embed = w->embed;
-    S.fc_norm = w->fc_norm;
-    S.fcout = xf;
-    S.ctx = ctx;
-    S.n_new = in->n_new;
-    S.ap = ap;
-    S.ob = ob;
-    S.head = (const uint8_t*)w->lm_head;
-    S.final_norm = w->final_norm;
-    S.z = zbuf;
-    S.cand_val = at<float>(ws, P.off_cv);
-    S.cand_id = at<int32_t>(ws, P.off_ci);
-    S.cand_fval = at<float>(ws, P.off_cfv);
-    S.cand_fid = at<int32_t>(ws, P.off_cfi);
-    S.tau = at<float>(ws, P.off_tau);
-    S.h = h;
-    S.ssp = at<float>(ws, P.off_ssp);
-    S.gbar = reinterpret_cast<unsigned*>(ctr + P.ctr_total - 1);
-    S.err = err;
-    S.dbg_hidden = dbg ? dbg->hidden : nullptr;
-    S.dbg_ctx = dbg ? dbg->ctx : nullptr;
-    S.dbg_final_h = dbg ? dbg->final_h : nullptr;
-    {
-      SelParams& sp = S.sel;
-      sp.cand_val = S.cand_val;  // the CTAs' lists: one part per CTA of the launch
-      sp.cand_id = S.cand_id;
-      sp.nparts = P.nsm;
-      sp.rows_total = P.D;
-      sp.z = zbuf;
-      sp.R = P.R;
-      sp.V = P.V;
-      sp.Bk = P.Bk;
-      sp.cb_a = w->cb_a;
-      sp.cb_b = w->cb_b;
-      sp.block_tokens = in->block_tokens;
-      sp.out_path = out_path;
-      sp.out_scores = out_scores;
-      sp.seq_len = kv->seq_len;
-      sp.n_new = in->n_new;
-      sp.dbg_cand = dbg ? dbg->cand : nullptr;
-      sp.dbg_logit = dbg ? dbg->cand_logit : nullptr;
-      sp.err = err;
-      if (sp.dbg_cand && !sp.dbg_logit) sp.dbg_cand = nullptr;
-    }
-    // A2: fc over the taps (operand copied), output to xf
-    {
-      GemvSeg seg{(const uint8_t*)w->fc, H / 16, Mb, 0};
-      Epi e;
-      e.mode = EPI_STORE;
-      e.y = xf;
-      e.ldy = H;
-      S.fc.g = sgemv_params(P.pfc, &seg, 1, false, in->taps, P.T * H, Mb, part, H, Mb, ctr, e, err);
-      S.fc.P = P.pfc.P;
-      S.fc.q4 = P.q4;
-      S.fc.stage = STG_COPY;
-    }
-    for (int l = 0; l < c->layers; ++l) {
-      const dflash2_layer_weights& L = w->layer[l];
-      int* lctr = ctr + P.ctr_fc + (size_t)l * P.ctr_per_layer;
-      PLayer& Q = S.L[l];
-      Q.kc = kv->k[l];
-      Q.vc = kv->v[l];
-      {  // A3a: g = W_dc RMSNorm(h; ln1), operand computed in the staging
-        GemvSeg segs[2] = {{(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, 0},
-                           {(const uint8_t*)L.dc_w, (H / 4) / 16, Mb, H / 4}};  // a0 | a1 paired
-        Epi e;
-        e.mode = EPI_STORE;
-        e.y = gbuf;
-        e.ldy = H / 2;
-        Q.dc.g = sgemv_params(P.pdc, segs, 2, true, nullptr, H, Mb, part, H / 2, Mb, lctr + P.ctr_layer[0], e, err);
-        Q.dc.P = P.pdc.P;
-        Q.dc.q4 = 0;
-        Q.dc.stage = STG_NORM;
-        Q.dc.nw = L.ln1;
-      }
-      {  // A3b+c: q|k|v of [dynconv rows; context rows], the dynconv computed in the staging
-        const int ldo = P.HQ + 2 * P.HKV;
-        GemvSeg segs[3] = {{(const uint8_t*)L.wq, P.HQ / 16, Mb, 0},
-                           {(const uint8_t*)L.wk, P.HKV / 16, 2 * Mb, P.HQ},
-                           {(const uint8_t*)L.wv, P.HKV / 16, 2 * Mb, P.HQ + P.HKV}};
-        Epi e;
-        e.mode = EPI_QKV;
-        QkvEpi& q = e.qkv;
-        q.qn = L.qn;
-        q.kn = L.kn;
-        q.eps = c->rms_eps;
-        q.log2_theta = log2((double)c->rope_theta);
-        q.Bk = P.Bk;
-        q.nq = c->n_q;
-        q.nkv = c->n_kv;
-        q.Mb = Mb;
-        q.seq_len = kv->seq_len;
-        q.n_new = in->n_new;
-        q.qb = qb;
-        q.kb = kb;
-        q.vb = vb;
-        q.kc = kv->k[l];
-        q.vc = kv->v[l];
-        q.page_table = kv->page_table;
-        q.max_pages = kv->max_pages;
-        q.num_pages = kv->num_pages;
-        q.err = err;
-        Q.qkv.g = sgemv_params(P.pqkv, segs, 3, false, nullptr, H, 2 * Mb, part, ldo, 2 * Mb, lctr + P.ctr_layer[1], e, err);
-        Q.qkv.P = P.pqkv.P;
-        Q.qkv.q4 = P.q4;
-        Q.qkv.stage = STG_DYNCONV;
-        Q.qkv.nw = L.ln1;
-        Q.qkv.gdc = gbuf;
-        Q.qkv.s0 = L.dc_s0;
-        Q.qkv.s1 = L.dc_s1;
-        Q.qkv.ctx = ctx;
-      }
-      {  // A3e: h += W_o o
-        GemvSeg seg{(const uint8_t*)L.wo, H / 16, Mb, 0};
-        Epi e;
-        e.mode = EPI_RESID;
-        e.y = h;
-        e.ldy = H;
-        Q.o.g = sgemv_params(P.po, &seg, 1, false, ob, P.HQ, Mb, part, H, Mb, lctr + P.ctr_layer[2], e, err);
-        Q.o.g.ssp = S.ssp;  // sums of squares of the new h for the gate/up RMSNorm
-        Q.o.g.ssp_rows = Mb;
-        Q.o.P = P.po.P;
-        Q.o.q4 = P.q4;
-        Q.o.stage = STG_COPY;
-      }
-      {  // A3f: act = SwiGLU of gate|up over RMSNorm(h; ln2) (computed in the staging); h += W_d act
-        GemvSeg segs[2] = {{(const uint8_t*)L.wg, P.F / 16, Mb, 0}, {(const uint8_t*)L.wg, P.F / 16, Mb, P.F}};
-        Epi e;
-        e.mode = EPI_SWIGLU;
-        e.act = act;
-        e.F = P.F;
-        Q.gu.g = sgemv_params(P.pgu, segs, 2, true, nullptr, H, Mb, part, 2 * P.F, Mb, lctr + P.ctr_layer[3], e, err);
-        Q.gu.P = P.pgu.P;
-        Q.gu.q4 = P.q4;
-        Q.gu.stage = STG_NORM;
-        Q.gu.nw = L.ln2;
-        GemvSeg seg{(const uint8_t*)L.wd, H / 16, Mb, 0};
-        Epi e2;
-        e2.mode = EPI_RESID;
-        e2.y = h;
-        e2.ldy = H;
-        Q.dn.g = sgemv_params(P.pdn, &seg, 1, false, act, P.F, Mb, part, H, Mb, lctr + P.ctr_layer[4], e2, err);
-        Q.dn.g.ssp = S.ssp;  // ... for the next layer's RMSNorm or the final norm
-        Q.dn.g.ssp_rows = Mb;
-        Q.dn.P = P.pdn.P;
-        Q.dn.q4 = P.q4;
-        Q.dn.stage = STG_COPY;
-      }
-    }
-    void* args[] = {&S};
-    CK(cudaLaunchCooperativeKernel((const void*)k_step_persistent, dim3(P.nsm), dim3(kPThreads), args, P.psmem, s));
-    if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
-    if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
-    return DFLASH2_OK;
-  }
   // A1: block rows from the shared embedding table (+ the first RMSNorm's inputs: h * ln1 and the
   // rows' sums of squares; every RMSNorm before a product is folded the same way: the residual
   // epilogues write bf16(h * w) and sums of squares, the product scales its outputs per row)
@@ -997,11 +775,8 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   {
     if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
     {
-      static bool attr = false;
-      if (!attr) {
-        CK(cudaFuncSetAttribute(k_slmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit - kStaticSmem));
-        attr = true;
-      }
+      static std::atomic<int> attr[kMaxDevices];
+      CK(smem_optin(k_slmhead, kSmemLimit - kStaticSmem, attr));
       SLmParams lp{};
       lp.W = (const uint8_t*)w->lm_head;
       lp.V = P.V;
@@ -1048,11 +823,8 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     int32_t* cdg = at<int32_t>(ws, P.off_cfi);
     // The CTAs are few and latency-bound: reserve (unused) dynamic shared memory so that each gets
     // an SM of its own instead of several landing on the first SM the output head frees.
-    static bool sel_attr = false;
-    if (!sel_attr) {
-      CK(cudaFuncSetAttribute(k_sel_tau, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSpreadSmem));
-      sel_attr = true;
-    }
+    static std::atomic<int> sel_attr[kMaxDevices];
+    CK(smem_optin(k_sel_tau, kSelSpreadSmem, sel_attr));
     CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), kSelSpreadSmem, s, sp, tau, clg, cdg, ctr + P.ctr_sel));
   }
   return DFLASH2_OK;
@@ -1090,6 +862,13 @@ int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, co
   if (batch < 1 || !taps_h || !n_new_h || !block_tokens_h || !target_h || !path_h || !scores_h || !accepted_h ||
       !emitted_h || !ws)
     return DFLASH2_ERR_ARG;
+  // everything the step checks is checked before the first copy or launch, so a rejected call
+  // leaves no queued work reading the caller's host buffers
+  int rc = check_weights(c, w);
+  if (rc) return rc;
+  rc = check_kv(c, kv);
+  if (rc) return rc;
+  if ((uintptr_t)ws & 255u) return DFLASH2_ERR_ALIGN;
   const Plan P = make_plan(c, batch);
   if (ws_bytes < P.total) return DFLASH2_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
@@ -1116,9 +895,12 @@ int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, co
     CK(cudaMemcpyAsync(at<void>(ws, P.off_s_tgt), target_h, Mb * 4, cudaMemcpyHostToDevice, s));
   }
   dflash2_inputs in{at<uint16_t>(ws, P.off_s_taps), at<int32_t>(ws, P.off_s_nnew), at<int32_t>(ws, P.off_s_btok)};
-  int rc = dflash2_draft_step(c, w, &in, kv, batch, at<int32_t>(ws, P.off_s_path), at<float>(ws, P.off_s_scores), ws,
-                              ws_bytes, nullptr, stream);
-  if (rc) return rc;
+  rc = dflash2_draft_step(c, w, &in, kv, batch, at<int32_t>(ws, P.off_s_path), at<float>(ws, P.off_s_scores), ws,
+                          ws_bytes, nullptr, stream);
+  if (rc) {
+    cudaStreamSynchronize(s);  // queued copies may still read the caller's host buffers
+    return rc;
+  }
   if (direct) {
     const int n = std::max(batch * P.D, batch);
     k_accept_to_host<<<(n + 127) / 128, 128, 0, s>>>(
@@ -1143,7 +925,6 @@ int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, co
 int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   if (!cfg_ok(c) || batch < 1) return 0;
   const Plan P = make_plan(c, batch);
-  if (P.persistent && persistent_ready(P)) return 1;
   // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention (+ a merge
   // kernel when the merge is not fused in), W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head
   // pass(es), selector (transition scores, the last CTA of a request runs its Viterbi path)

@@ -167,7 +167,6 @@ __global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __res
 __global__ void k_stage_host_inputs(const int32_t* __restrict__ n_new_h, const int32_t* __restrict__ btok_h,
                                     const int32_t* __restrict__ tgt_h, int B, int Mb, int32_t* __restrict__ n_new,
                                     int32_t* __restrict__ btok, int32_t* __restrict__ tgt) {
-  pdl_trigger();
   for (int i = threadIdx.x; i < B; i += blockDim.x) n_new[i] = n_new_h[i];
   for (int i = threadIdx.x; i < Mb; i += blockDim.x) {
     btok[i] = btok_h[i];

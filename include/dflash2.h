@@ -130,8 +130,7 @@ typedef struct dflash2_inputs {
  *   LM head's operand); cand: int32 and cand_logit: fp32 [batch*(block-1)][16];
  *   z: fp32 [batch*(block-1)][rank] selector projection.
  * ev_lm_begin / ev_lm_end: cudaEvent_t (as void*) recorded on `stream` around
- *   the LM-head + top-16 kernel, or, when the step runs as one persistent kernel
- *   (dflash2_step_kernels() == 1), around that kernel. */
+ *   the LM-head + top-16 kernel. */
 typedef struct dflash2_debug {
   float *hidden;
   uint16_t *ctx;
@@ -230,13 +229,10 @@ int dflash2_spec_step_host(const dflash2_config *cfg, const dflash2_weights *w, 
 int dflash2_device_error(const void *workspace, int32_t *out_bits, void *stream);
 
 /* Kernels one dflash2_draft_step call launches for `batch` requests on the
- * current device (memsets not counted).  A single request with a block of at
- * most 8 runs as ONE persistent cooperative kernel (one CTA per SM, grid
- * barriers between dependent operations) when the device supports cooperative
- * launch and the environment variable DFLASH2_PERSISTENT is "1"; otherwise
- * the step is a sequence of kernels (six per layer; seven when the attention chunks are merged by
- * a kernel of their own, which the plan picks for more than 32 query vectors per kv head or when
- * window + block size exceeds 3058 keys).
+ * current device (memsets not counted): embedding, fc product, fc norm, six per
+ * layer (seven when the attention chunks are merged by a kernel of their own,
+ * which the plan picks for more than 32 query vectors per kv head or when
+ * window + block size exceeds 3058 keys), final norm, output head, selector.
  * 0 on an invalid config or batch. */
 int32_t dflash2_step_kernels(const dflash2_config *cfg, int32_t batch);
 

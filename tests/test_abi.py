@@ -90,7 +90,6 @@ def test_unprepared_q4k_weights_are_rejected(lib):
 
 
 def test_step_kernel_count_without_a_device(lib):
-    # no GPU here: the persistent single-kernel step is unavailable, so the step is the kernel sequence
     cfg = binding.config(inputs.TINY)
     # embed, fc, fc norm | 7 per layer | final norm, LM head, selector tau + Viterbi
     assert lib.dflash2_step_kernels(C.byref(cfg), 1) == 3 + 6 * inputs.TINY.layers + 1 + 1 + 1
