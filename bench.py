@@ -316,12 +316,22 @@ def main():
     flops = accounting.step_flops(dims, B)
     nk = dr.step_kernels()
     traffic = None
-    rk_name = "k_slmhead (LM head + streaming top-16 + selector projection)"
     rk_bytes = accounting.lmhead_bytes(dims, B * D)
-    ratio = head_traffic_ratio() if B * D <= 8 else None  # captured for the streaming kernel
-    if ratio is not None:
-        traffic = ratio * rk_bytes  # small-case capture scaled by the launch's bytes
     rk_gbs = rk_bytes / (lm_ms * 1e-3) / 1e9
+    if B * D <= 8:
+        rk_name = "k_slmhead (LM head + streaming top-16 + selector projection)"
+        ratio = head_traffic_ratio()  # captured for the streaming kernel
+        if ratio is not None:
+            traffic = ratio * rk_bytes  # small-case capture scaled by the launch's bytes
+        roof = {"bound": "hbm", "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm}
+    else:
+        rk_name = "k_umma_head (tcgen05 LM head + top-16 + selector projection)"
+        hflops = accounting.lmhead_flops(dims, B * D)
+        tf = hflops / (lm_ms * 1e-3) / 1e12
+        if B * D >= 128:  # a dense contraction: the tensor pipe bounds it
+            roof = {"bound": "tensor", "achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk}
+        else:
+            roof = {"bound": "hbm", "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm}
     value = ws / (ms_max * 1e-3)  # draft steps/s over all ranks (one step = a rank's whole batch)
     line = {
         "metric": "DFlash2 draft steps/s (8-token block)",
@@ -345,10 +355,11 @@ def main():
         # measured sustained bf16 dense rate
         "step_tensor": {"flops": flops, "achieved_tflops": flops / (ms_max * 1e-3) / 1e12, "peak_tflops": tpk,
                         "frac": flops / (ms_max * 1e-3) / 1e12 / tpk, "peak_kind": tpk_kind,
-                        "path": "mma.sync m16n8k16 streaming engine"},
-        "roofline": {"kernel": rk_name, "bound": "hbm",
-                     "achieved": rk_gbs, "peak": hbm, "unit": "GB/s", "frac": rk_gbs / hbm, "traffic": traffic,
-                     "algorithmic_bytes": rk_bytes, "avg_launch_ms": lm_ms, "peak_kind": peak_kind},
+                        "path": ("tcgen05 (TMEM) products above 64 block rows" if B * Bk > 64 else
+                                 "mma.sync m16n8k16 streaming engine")},
+        "roofline": {"kernel": rk_name, **roof, "traffic": traffic, "algorithmic_bytes": rk_bytes,
+                     "avg_launch_ms": lm_ms,
+                     "peak_kind": peak_kind if roof["bound"] == "hbm" else f"{tpk_kind} sustained bf16"},
         "e2e": {"value": ws / (e2e_ms * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": accounting.launches_per_step(dims, B, nk) * K,

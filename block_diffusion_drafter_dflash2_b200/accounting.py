@@ -42,6 +42,11 @@ def lmhead_bytes(dims: Dims, rows: int) -> float:
     return (dims.vocab + dims.rank) * dims.hidden * 2.0 + rows * dims.hidden * 2.0
 
 
+def lmhead_flops(dims: Dims, rows: int) -> float:
+    """2 x multiply-adds of one output-head launch (head and selector projection) over `rows`."""
+    return 2.0 * rows * (dims.vocab + dims.rank) * dims.hidden
+
+
 def step_flops(dims: Dims, batch: int) -> float:
     """2 x multiply-adds of the matrices applied (block rows, context rows, drafted rows)."""
     H, F, T, R, V = dims.hidden, dims.ffn, dims.n_taps, dims.rank, dims.vocab

@@ -55,9 +55,13 @@ class Debug(C.Structure):
                                           "ev_lm_end")]
 
 
+class InputsMut(C.Structure):
+    _fields_ = [("taps", C.c_void_p), ("n_new", C.c_void_p), ("block_tokens", C.c_void_p)]
+
+
 EXPORTS = ("dflash2_workspace_size", "dflash2_prepared_size", "dflash2_prepare_weights", "dflash2_draft_step",
-           "dflash2_draft_step_static", "dflash2_accept", "dflash2_spec_step_host", "dflash2_device_error",
-           "dflash2_step_kernels", "dflash2_strerror")
+           "dflash2_draft_step_static", "dflash2_accept", "dflash2_accept_sampled", "dflash2_accept_chain", "dflash2_spec_round",
+           "dflash2_spec_step_host", "dflash2_device_error", "dflash2_step_kernels", "dflash2_strerror")
 
 _lib = None
 
@@ -83,6 +87,11 @@ def load(path: str = LIB_PATH):
                                               C.POINTER(KV), C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
                                               C.POINTER(Debug), C.c_void_p]
     lib.dflash2_accept.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
+    lib.dflash2_accept_sampled.argtypes = [C.c_void_p] * 5 + [C.c_int32] * 3 + [C.c_void_p] * 3
+    lib.dflash2_accept_chain.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32] + [C.c_void_p] * 5
+    lib.dflash2_spec_round.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(InputsMut), C.POINTER(KV),
+                                       C.c_int32, C.c_void_p, C.c_void_p, C.c_int32] + [C.c_void_p] * 5 + \
+        [C.c_size_t, C.c_void_p]
     lib.dflash2_spec_step_host.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(KV), C.c_int32] + \
         [C.c_void_p] * 9 + [C.c_void_p, C.c_size_t, C.c_void_p]
     lib.dflash2_device_error.argtypes = [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]
@@ -193,6 +202,30 @@ class Drafter:
                stream=None):
         check(self.lib.dflash2_accept(_ptr(draft), _ptr(target), self.batch, self.dims.block, _ptr(accepted),
                                       _ptr(emitted), _stream(stream)), "accept")
+
+    def accept_sampled(self, draft, p_target, u_accept, u_sample, accepted, emitted, q_draft=None, stream=None):
+        """Exact rejection-sampling acceptance (sampled decoding)."""
+        check(self.lib.dflash2_accept_sampled(_ptr(draft), _ptr(p_target), _ptr(q_draft), _ptr(u_accept),
+                                              _ptr(u_sample), self.batch, self.dims.block, int(p_target.shape[-1]),
+                                              _ptr(accepted), _ptr(emitted), _stream(stream)), "accept_sampled")
+
+    def accept_chain(self, draft, target, mask_id: int, accepted, emitted, n_new_next, block_tokens_next,
+                     stream=None):
+        """Acceptance plus the next round's n_new and block tokens, on the device."""
+        check(self.lib.dflash2_accept_chain(_ptr(draft), _ptr(target), self.batch, self.dims.block, int(mask_id),
+                                            _ptr(accepted), _ptr(emitted), _ptr(n_new_next),
+                                            _ptr(block_tokens_next), _stream(stream)), "accept_chain")
+
+    def spec_round(self, inputs: dict, state: dict, prev_path, target, mask_id: int, accepted, emitted, out_path,
+                   out_scores, stream=None, kv: Optional[KV] = None):
+        """Chained acceptance of the previous draft, then the next draft step; inputs["n_new"] and
+        inputs["block_tokens"] are overwritten with the next round's values on the device."""
+        ins = InputsMut(inputs["taps"].data_ptr(), inputs["n_new"].data_ptr(), inputs["block_tokens"].data_ptr())
+        kvs = kv if kv is not None else kv_struct(state)
+        check(self.lib.dflash2_spec_round(C.byref(self.cfg), C.byref(self.w), C.byref(ins), C.byref(kvs),
+                                          self.batch, _ptr(prev_path), _ptr(target), int(mask_id), _ptr(accepted),
+                                          _ptr(emitted), _ptr(out_path), _ptr(out_scores), _ptr(self.workspace),
+                                          self.ws_bytes, _stream(stream)), "spec_round")
 
     def spec_step_host(self, state: dict, taps_h, n_new_h, block_tokens_h, target_h, path_h, scores_h, accepted_h,
                        emitted_h, stream=None, kv: Optional[KV] = None) -> int:

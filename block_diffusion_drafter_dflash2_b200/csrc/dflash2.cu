@@ -11,8 +11,10 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "rowops.cuh"
+#include "sampling.cuh"
 #include "selector.cuh"
 #include "stream.cuh"
+#include "umma.cuh"
 
 using namespace dfl;
 
@@ -22,7 +24,13 @@ struct GemvPlan {
   int NT = 1, R = 8, groups = 1, mgroups = 1, U = 1, P = 1, kc_units = 1, max_pieces = 1;
   long long W = 1;
   size_t smem = 0;
+  bool umma = false;  // tensor-core (tcgen05) product + fix-up instead of the streaming engine
+  int rows = 0, K = 0;
 };
+
+// Above this many activation rows a product runs on the tcgen05 tensor cores (k_umma): the
+// streaming engine would need several 64-row groups, each re-reading the weights.
+constexpr int kUmmaMinRows = 65;
 
 struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
@@ -33,6 +41,9 @@ struct Plan {
   size_t off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
   int lm_nparts, lm_rows, lm_groups;
   size_t lm_smem;
+  bool lm_umma;                  // output head on the tensor cores (k_umma_head)
+  int lm_uP, lm_unrt, lm_unrec;  // its grid, row tiles of 256 and head records
+  int sel_parts;                 // candidate lists per row the selector merges
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
       off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
   size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_head, ctr_sel, ctr_total;
@@ -53,6 +64,22 @@ constexpr int kStaticSmem = 2048;  // mbarriers and flags of the streaming kerne
 // tiles: 16-row tiles over all segments; paired: gate/up (groups = tiles / 8 still, 4 + 4 tiles each)
 GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   GemvPlan g;
+  g.rows = rows;
+  g.K = K;
+  if (rows >= kUmmaMinRows) {
+    g.umma = true;
+    g.R = kUmmaRows;
+    g.NT = 8;
+    g.mgroups = (rows + kUmmaRows - 1) / kUmmaRows;
+    g.groups = (tiles + kConsumers - 1) / kConsumers;
+    g.U = K / (q4 ? Ring<true>::kUnitK : Ring<false>::kUnitK);
+    g.W = (long long)g.groups * g.mgroups * g.U;
+    g.P = (int)std::min<long long>(nsm, g.W);
+    g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
+    g.kc_units = g.U;
+    g.smem = kUmmaSmem;
+    return g;
+  }
   g.R = rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
   g.NT = g.R / 8;
   g.mgroups = g.R == 64 ? (rows + 63) / 64 : 1;
@@ -154,6 +181,12 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.lm_groups = (p.lm_rows + 7) / 8;
   p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
   p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
+  // more than one group of 8 drafted rows: the head is a dense contraction on the tensor cores
+  p.lm_umma = p.lm_rows > 8;
+  p.lm_unrt = (p.lm_rows + 255) / 256;
+  p.lm_unrec = (lm_tiles + kHeadTiles - 1) / kHeadTiles;
+  p.lm_uP = std::max(1, p.nsm / p.lm_unrt) * p.lm_unrt;
+  p.sel_parts = p.lm_umma ? p.lm_uP / p.lm_unrt : p.lm_nparts;
   auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.max_pieces * rows * ldo * 4; };
   size_t part = 0;
   part = std::max(part, part_bytes(p.fc, p.Mb, p.H));
@@ -183,7 +216,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_ob = take((size_t)p.Mb * p.HQ * 2);
   p.off_act = take((size_t)p.Mb * p.F * 2);
   p.off_hn = take((size_t)std::max(p.lm_rows, 1) * p.H * 2);
-  const size_t nlists = (size_t)p.lm_nparts;
+  const size_t nlists = (size_t)std::max(p.lm_nparts, p.sel_parts);
   p.off_cv = take(nlists * p.lm_rows * kTopK * 4);
   p.off_ci = take(nlists * p.lm_rows * kTopK * 4);
   p.off_cfv = take((size_t)p.lm_rows * kTopK * 4);
@@ -338,10 +371,64 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   return prm;
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no link against the
+// driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !ptr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  f = reinterpret_cast<EncodeTiledFn>(ptr);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
+
+// Tensor map of a bf16 activation matrix [rows][ldx] (K valid columns): boxes of 64 columns x 256
+// rows, 128-byte swizzle (the tcgen05 K-major operand layout); rows past the end read as zero.
+cudaError_t make_act_tmap(CUtensorMap* tm, const uint16_t* X, int K, int ldx, int rows) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kUmmaRows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = f(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Tensor-core product (stream-K pieces into the partial buffer) and its fix-up kernel (piece sums
+// in order + the product's epilogue), both with programmatic dependent launch.
+template <bool Q4>
+cudaError_t launch_umma_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_t s) {
+  static std::atomic<int> attr[kMaxDevices];
+  cudaError_t e = smem_optin(k_umma<Q4>, kUmmaSmem, attr);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tm;
+  e = make_act_tmap(&tm, prm.X, g.K, prm.ldx, prm.rows);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(k_umma<Q4>, dim3(g.P), dim3(kUmmaThreads), (size_t)kUmmaSmem, s, tm, prm);
+  if (e != cudaSuccess) return e;
+  const int fix_blocks = prm.groups * ((prm.rows + 63) / 64);
+  return launch_pdl(k_umma_fixup, dim3(fix_blocks), dim3(kGemvConsumers * 32), 0, s, prm, g.P);
+}
+
 cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X,
                         int ldx, int rows, float* part, int ldo, int out_rows, int* counters, const Epi& e, int* err,
                         cudaStream_t s) {
   const SGemvParams prm = sgemv_params(g, segs, nseg, paired, X, ldx, rows, part, ldo, out_rows, counters, e, err);
+  if (g.umma) return q4 ? launch_umma_t<true>(g, prm, s) : launch_umma_t<false>(g, prm, s);
   switch (g.NT * 2 + (q4 ? 1 : 0)) {
     case 2: return launch_sgemv_t<1, false>(g, prm, s);
     case 3: return launch_sgemv_t<1, true>(g, prm, s);
@@ -774,7 +861,25 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
   // A5: LM head + streaming top-16 (+ selector projection)
   {
     if (dbg && dbg->ev_lm_begin) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_begin, s));
-    {
+    if (P.lm_umma) {
+      static std::atomic<int> uattr[kMaxDevices];
+      CK(smem_optin(k_umma_head, kUHeadSmem, uattr));
+      CUtensorMap tm;
+      CK(make_act_tmap(&tm, hn, H, H, P.lm_rows));
+      UHeadParams hp{};
+      hp.W = (const uint8_t*)w->lm_head;
+      hp.V = P.V;
+      hp.R = P.R;
+      hp.H = H;
+      hp.rows = P.lm_rows;
+      hp.nrec = P.lm_unrec;
+      hp.nrt = P.lm_unrt;
+      hp.z = zbuf;
+      hp.cand_val = at<float>(ws, P.off_cv);
+      hp.cand_id = at<int32_t>(ws, P.off_ci);
+      hp.err = err;
+      CK(launch_pdl(k_umma_head, dim3(P.lm_uP), dim3(kUmmaThreads), (size_t)kUHeadSmem, s, tm, hp));
+    } else {
       static std::atomic<int> attr[kMaxDevices];
       CK(smem_optin(k_slmhead, kSmemLimit - kStaticSmem, attr));
       SLmParams lp{};
@@ -801,7 +906,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     SelParams sp{};
     sp.cand_val = at<float>(ws, P.off_cv);
     sp.cand_id = at<int32_t>(ws, P.off_ci);
-    sp.nparts = P.lm_nparts;
+    sp.nparts = P.sel_parts;
     sp.rows_total = P.lm_rows;
     sp.z = zbuf;
     sp.R = P.R;
@@ -852,6 +957,49 @@ int dflash2_accept(const int32_t* draft, const int32_t* target, int32_t batch, i
   if (!draft || !target || !accepted || !emitted || batch < 1 || block < 2) return DFLASH2_ERR_ARG;
   k_accept<<<(batch + 127) / 128, 128, 0, (cudaStream_t)stream>>>(draft, target, batch, block, accepted, emitted);
   return fail(cudaGetLastError());
+}
+
+int dflash2_accept_sampled(const int32_t* draft, const float* p_target, const float* q_draft, const float* u_accept,
+                           const uint32_t* u_sample, int32_t batch, int32_t block, int32_t vocab, int32_t* accepted,
+                           int32_t* emitted, void* stream) {
+  if (!draft || !p_target || !u_accept || !u_sample || !accepted || !emitted || batch < 1 || block < 2 || vocab < 1)
+    return DFLASH2_ERR_ARG;
+  k_accept_sampled<<<batch, kSampThreads, 0, (cudaStream_t)stream>>>(draft, p_target, q_draft, u_accept, u_sample,
+                                                                     block, vocab, accepted, emitted);
+  return fail(cudaGetLastError());
+}
+
+int dflash2_accept_chain(const int32_t* draft, const int32_t* target, int32_t batch, int32_t block, int32_t mask_id,
+                         int32_t* accepted, int32_t* emitted, int32_t* n_new_next, int32_t* block_tokens_next,
+                         void* stream) {
+  if (!draft || !target || !accepted || !emitted || !n_new_next || !block_tokens_next || batch < 1 || block < 2 ||
+      mask_id < 0)
+    return DFLASH2_ERR_ARG;
+  k_accept_chain<<<(batch + 127) / 128, 128, 0, (cudaStream_t)stream>>>(draft, target, batch, block, mask_id, accepted,
+                                                                        emitted, n_new_next, block_tokens_next);
+  return fail(cudaGetLastError());
+}
+
+int dflash2_spec_round(const dflash2_config* c, const dflash2_weights* w, dflash2_inputs_mut* in, const dflash2_kv* kv,
+                       int32_t batch, const int32_t* prev_path, const int32_t* target, int32_t mask_id,
+                       int32_t* accepted, int32_t* emitted, int32_t* out_path, float* out_scores, void* ws,
+                       size_t ws_bytes, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (!in || !in->taps || !in->n_new || !in->block_tokens || !prev_path || !target || !accepted || !emitted ||
+      !out_path || !out_scores || !ws || batch < 1 || mask_id < 0 || mask_id >= c->vocab)
+    return DFLASH2_ERR_ARG;
+  // the step's own checks, before anything is queued
+  int rc = check_weights(c, w);
+  if (rc) return rc;
+  rc = check_kv(c, kv);
+  if (rc) return rc;
+  if (!aligned16(in->taps) || ((uintptr_t)ws & 255u)) return DFLASH2_ERR_ALIGN;
+  if (ws_bytes < make_plan(c, batch).step_bytes) return DFLASH2_ERR_WORKSPACE;
+  rc = dflash2_accept_chain(prev_path, target, batch, c->block, mask_id, accepted, emitted, in->n_new,
+                            in->block_tokens, stream);
+  if (rc) return rc;
+  const dflash2_inputs ci{in->taps, in->n_new, in->block_tokens};
+  return dflash2_draft_step(c, w, &ci, kv, batch, out_path, out_scores, ws, ws_bytes, nullptr, stream);
 }
 
 int dflash2_spec_step_host(const dflash2_config* c, const dflash2_weights* w, const dflash2_kv* kv, int32_t batch,
@@ -928,7 +1076,12 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   // embed, fc GEMV, fc norm | per layer: W_dc GEMV (+ convolution), QKV GEMV, attention (+ a merge
   // kernel when the merge is not fused in), W_o GEMV, gate/up GEMV, W_d GEMV | final norm, LM head
   // pass(es), selector (transition scores, the last CTA of a request runs its Viterbi path)
-  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + 1 + 1;
+  // (a tensor-core product is two kernels: the product and its fix-up)
+  const GemvPlan* gp[6] = {&P.dc, &P.qkv, &P.o, &P.gu, &P.dn, &P.fc};
+  int extra = 0;
+  for (int i = 0; i < 5; ++i) extra += gp[i]->umma ? c->layers : 0;
+  extra += P.fc.umma ? 1 : 0;
+  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + 1 + 1 + extra;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

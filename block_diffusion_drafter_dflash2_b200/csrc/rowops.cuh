@@ -162,6 +162,22 @@ __global__ void k_accept(const int32_t* __restrict__ draft, const int32_t* __res
   if (b < B) accept_request(draft, target, b, Bk, accepted, emitted);
 }
 
+// Acceptance that also writes the next round's draft inputs: n_new_next[b] = accepted + 1 (the
+// accepted drafted tokens and the target's own token become the next context rows) and the next
+// block = [target[b][accepted], mask_id, ...].  One thread per request; the next-round buffers may
+// be the step's own n_new / block_tokens (the step that read them has finished on this stream).
+__global__ void k_accept_chain(const int32_t* __restrict__ draft, const int32_t* __restrict__ target, int B, int Bk,
+                               int32_t mask_id, int32_t* __restrict__ accepted, int32_t* __restrict__ emitted,
+                               int32_t* __restrict__ n_new_next, int32_t* __restrict__ btok_next) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  accept_request(draft, target, b, Bk, accepted, emitted);
+  const int n = accepted[b];
+  n_new_next[b] = n + 1;
+  btok_next[(size_t)b * Bk] = target[(size_t)b * Bk + n];
+  for (int i = 1; i < Bk; ++i) btok_next[(size_t)b * Bk + i] = mask_id;
+}
+
 // Host-buffer round, page-locked buffers (device-addressable): the small inputs (n_new [B], block
 // tokens and targets [Mb]) gathered into the workspace by one kernel instead of three copies.
 __global__ void k_stage_host_inputs(const int32_t* __restrict__ n_new_h, const int32_t* __restrict__ btok_h,

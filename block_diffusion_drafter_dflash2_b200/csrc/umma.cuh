@@ -1,0 +1,560 @@
+// Batched layer products on the 5th-generation tensor cores (tcgen05 / TMEM).
+//
+// When the step carries many block rows (many requests), a layer product is a dense
+// contraction: Y[row][feature] = sum_k X[row][k] W[feature][k] with a few hundred rows.  The
+// streaming mma.sync engine (stream.cuh) re-reads its activation fragments from shared memory
+// for every weight fragment, so there it is bound by shared-memory operand traffic; this kernel
+// feeds the tensor cores from shared-memory descriptors instead and accumulates in TMEM.
+//
+// One CTA per SM (stream-K over the same (column group, row chunk, K unit) plane as the
+// streaming engine, so the split-K pieces, their order and the fix-up epilogues are shared):
+//  * warp 0, one thread: TMA (cp.async.bulk.tensor, no multicast) of the activation tile
+//    [256 rows][64 k] bf16 into a 128-byte-swizzled K-major stage;
+//  * warps 4-7: weight producers.  They read the prepared records of the column group (128
+//    features = 8 tiles of 16, the layout of dflash2_prepare_weights) straight from global
+//    memory and write the [128 features][64 k] bf16 operand into the same swizzled K-major
+//    layout.  Q4_K codes become bf16 128+q with one LOP3 (0x4300 | q), widen exactly to fp32,
+//    and w = (128+q) * (d sc_j) - (dmin m_j + 128 d sc_j) is formed by a packed fp32 fused
+//    multiply-add and rounded once to bf16 (the only rounding of a weight; rounding the
+//    sub-block scale or min to bf16 first would bias all 32 weights of a sub-block alike);
+//    bf16 weights are moved as they are.  After the K range of a
+//    piece they read the accumulator back (tcgen05.ld) and store the fp32 partial;
+//  * warp 1: allocates 256 TMEM columns; one thread issues tcgen05.mma (kind::f16, bf16 x bf16
+//    -> fp32, M = 128 features, N = 256 rows, K = 16) and commits each stage back to the
+//    producers and each finished piece to the epilogue.
+// Every mbarrier wait is bounded; an expired wait sets DFLASH2_DEV_TIMEOUT and the waiting role
+// skips its remaining work, so the CTA still exits and frees its TMEM.
+#pragma once
+#include <cuda.h>
+
+#include "stream.cuh"
+
+namespace dfl {
+
+constexpr int kUmmaRows = 256;                     // activation rows per tile (MMA N)
+constexpr int kUmmaStages = 4;
+constexpr int kUmmaABytes = 128 * 128;             // [128 features][64 k] bf16
+constexpr int kUmmaBBytes = kUmmaRows * 128;       // [256 rows][64 k] bf16
+constexpr int kUmmaThreads = 256;
+constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + 1024;  // + alignment slack
+constexpr int kUmmaTmemCols = 256;
+
+// ---- tcgen05 / TMA wrappers (one instruction each) ----
+DEVI void tmem_alloc(uint32_t* dst_smem, int cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(cols)
+               : "memory");
+}
+DEVI void tmem_relinquish() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory"); }
+DEVI void tmem_dealloc(uint32_t taddr, int cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+DEVI void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, fp32 accumulate)
+DEVI void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32*(w%4) ..)
+DEVI void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+DEVI void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Generic-proxy shared-memory writes made visible to the async proxy (the tensor cores).
+DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 2-D tiled TMA load (no multicast): box at (x elements along K, y rows) of the tensor map.
+DEVI void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand stored as 8-row x 128-byte swizzled atoms
+// (rows 128 bytes apart, 8-row groups 1024 bytes apart): start address, leading offset 16 B,
+// stride offset 1024 B, descriptor version 1, layout SWIZZLE_128B.
+DEVI uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N = 256, M = 128.
+constexpr uint32_t kUmmaIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kUmmaRows >> 3) << 17) |
+                                ((uint32_t)(128 >> 4) << 24);
+
+// Byte offset of the 16-byte chunk c (k = 8c .. 8c+7) of row m in a 128-byte-swizzled stage.
+DEVI uint32_t sw128_off(int m, int c) { return (uint32_t)(m * 128 + ((c ^ (m & 7)) << 4)); }
+
+DEVI bool wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, int* err) {
+  if (dead) return false;
+  if (!mbar_wait_bounded(bar, parity)) {
+    set_err(err, DFLASH2_DEV_TIMEOUT);
+    dead = true;
+    return false;
+  }
+  return true;
+}
+
+// (D, C) of sub-block j from a canonical 16-byte Q4_K scale record: D = d*sc_j and
+// C = -(dmin*m_j + 128*D), so that w = (128 + q)*D + C.  d*sc_j and dmin*m_j are exact in fp32
+// (an fp16 times a 6-bit integer); C carries one fp32 rounding, 2^-17 of a quantisation step.
+DEVI float2 q4_scale_dc(const uint4 sc, int j) {
+  const float d = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
+  const float dm = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
+  const unsigned long long scp = (unsigned long long)sc.y | ((unsigned long long)(sc.z & 0xffffu) << 32);
+  const unsigned long long mp = (unsigned long long)(sc.z >> 16) | ((unsigned long long)sc.w << 16);
+  const float D = d * (float)((scp >> (6 * j)) & 63u), M = dm * (float)((mp >> (6 * j)) & 63u);
+  return make_float2(D, -fmaf(128.f, D, M));
+}
+
+// bf16 pair (128 + q0, 128 + q1) -> the two weights in fp32 (exact widening, one fused
+// multiply-add each on the packed pair), rounded once to a bf16 pair.
+DEVI uint32_t q4_pair(uint32_t v, float2 dc) {
+  const float2 x = make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+  const float2 w = ffma2(x, make_float2(dc.x, dc.x), make_float2(dc.y, dc.y));
+  return pack_bf2(w.x, w.y);
+}
+
+// One row's 8 consecutive weights from two code words (nibble slots of the prepared record: word
+// bits 4s hold slot s; row g takes slots 0,4 | 2,6 with shifts 0 | 8, row g+8 the same with an
+// extra shift of 4), dequantised to 4 bf16 pairs.
+DEVI uint4 q4_chunk(uint32_t w0, uint32_t w1, int rs, float2 dc) {
+  const uint32_t k128 = 0x43004300u;  // bf16 pair (128, 128)
+  const uint32_t a = ((w0 >> rs) & 0x000F000Fu) | k128, b = ((w0 >> (rs + 8)) & 0x000F000Fu) | k128;
+  const uint32_t c = ((w1 >> rs) & 0x000F000Fu) | k128, d = ((w1 >> (rs + 8)) & 0x000F000Fu) | k128;
+  return make_uint4(q4_pair(a, dc), q4_pair(b, dc), q4_pair(c, dc), q4_pair(d, dc));
+}
+
+template <bool Q4>
+__global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t xfull[kUmmaStages], afull[kUmmaStages], sempty[kUmmaStages];
+  __shared__ __align__(8) uint64_t accfull, accempty;
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* As = smem;                              // [stages][128 x 128 B]
+  uint8_t* Bs = smem + kUmmaStages * kUmmaABytes;  // [stages][256 x 128 B]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kSub = Q4 ? 4 : 1;  // 64-wide stages per prepared K unit
+  constexpr int kUnitK = Q4 ? 256 : 64;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kUmmaStages; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&afull[s], 4);
+      mbar_init(&sempty[s], 1);
+    }
+    mbar_init(&accfull, 1);
+    mbar_init(&accempty, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kUmmaTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  pdl_trigger();
+  const long long P = gridDim.x, c = blockIdx.x;
+  const long long x0 = c * p.W / P, x1 = (c + 1) * p.W / P;
+
+  if (warp == 0) {
+    // ---- activation producer (TMA) ----
+    if (lane == 0) {
+      pdl_wait();  // the activations come from the previous kernel
+      bool dead = false;
+      int cnt = 0;
+      for (long long x = x0; x < x1 && !dead;) {
+        const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
+        const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        int si;
+        sk_tile(p, grp, 0, si);
+        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
+          for (int u = ua; u < ub && !dead; ++u)
+            for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
+              const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
+              if (round > 0 && !wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err)) break;
+              mbar_expect_tx(&xfull[s], kUmmaBBytes);
+              tma_load_2d(Bs + s * kUmmaBBytes, &tmx, u * kUnitK + sub * 64, mz, &xfull[s]);
+            }
+        }
+        x += ub - ua;
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      bool dead = false;
+      int cnt = 0, piece = 0;
+      for (long long x = x0; x < x1 && !dead;) {
+        const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
+        const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        int si;
+        sk_tile(p, grp, 0, si);
+        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
+          if (piece > 0 && !wait_or_die(&accempty, (piece - 1) & 1, dead, p.err)) break;
+          tc_fence_after();
+          bool first = true;
+          for (int u = ua; u < ub && !dead; ++u)
+            for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
+              const int s = cnt % kUmmaStages;
+              const uint32_t par = (cnt / kUmmaStages) & 1;
+              if (!wait_or_die(&xfull[s], par, dead, p.err) || !wait_or_die(&afull[s], par, dead, p.err)) break;
+              tc_fence_after();
+              const uint64_t ad = sw128_desc(smem_u32(As + s * kUmmaABytes));
+              const uint64_t bd = sw128_desc(smem_u32(Bs + s * kUmmaBBytes));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes inside the swizzled rows
+                tc_mma(tmem, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (first && kk == 0) ? 0u : 1u);
+              first = false;
+              tc_commit(&sempty[s]);  // the stage is free once these MMAs have read it
+            }
+          if (!dead) tc_commit(&accfull);  // the piece's accumulator is complete
+          ++piece;
+        }
+        x += ub - ua;
+      }
+    }
+  } else if (warp >= 4) {
+    // ---- weight producers, then the piece epilogue ----
+    const int dw = warp - 4, g = lane >> 2, t = lane & 3;
+    bool dead = false, waited = false;
+    int cnt = 0, piece = 0;
+    for (long long x = x0; x < x1;) {
+      const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
+      const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
+      const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+      int si0;
+      sk_tile(p, grp, 0, si0);
+      if (sk_rows(p, si0, mz, kUmmaRows) > 0) {
+        const uint8_t* src = sk_group_src<Q4>(p, grp);
+        for (int u = ua; u < ub; ++u) {
+          const uint8_t* rec[2];
+          uint4 code[2][kSub], scl[2][2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            rec[h] = src + (size_t)u * Ring<Q4>::kSlot + (size_t)(2 * dw + h) * Ring<Q4>::kUnitBytes;
+            if (Q4) {  // the unit's codes and the scale records of rows g, g+8 of this warp's tiles
+#pragma unroll
+              for (int q = 0; q < kSub; ++q) code[h][q] = ldg_stream(rec[h] + (q * 32 + lane) * 16);
+              scl[h][0] = __ldg(reinterpret_cast<const uint4*>(rec[h] + 2048 + g * 16));
+              scl[h][1] = __ldg(reinterpret_cast<const uint4*>(rec[h] + 2048 + (g + 8) * 16));
+            }
+          }
+#pragma unroll
+          for (int sub = 0; sub < kSub; ++sub, ++cnt) {
+            const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
+            if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
+            uint8_t* a = As + s * kUmmaABytes;
+            if (!dead) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int m0 = (2 * dw + h) * 16 + g;  // operand rows g and g+8 of tile 2*dw+h
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {  // 32-wide sub-blocks of the stage
+                  uint4 rg, rh;
+                  if (Q4) {
+                    const uint4 q = code[h][sub];
+                    const uint32_t w0 = jj ? q.z : q.x, w1 = jj ? q.w : q.y;
+                    rg = q4_chunk(w0, w1, 0, q4_scale_dc(scl[h][0], 2 * sub + jj));
+                    rh = q4_chunk(w0, w1, 4, q4_scale_dc(scl[h][1], 2 * sub + jj));
+                  } else {  // bf16 record: W[row g][32jj + 8t ..] at jj*1024 + lane*16, row g+8 at +512
+                    rg = ldg_stream(rec[h] + jj * 1024 + lane * 16);
+                    rh = ldg_stream(rec[h] + jj * 1024 + 512 + lane * 16);
+                  }
+                  *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jj + t)) = rg;
+                  *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jj + t)) = rh;
+                }
+              }
+            }
+            fence_proxy_async_smem();  // these generic writes feed the tensor cores (async proxy)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[s]);
+          }
+        }
+        // ---- epilogue of this piece: TMEM -> fp32 partial [piece][row][ldo] ----
+        if (!waited) {
+          pdl_wait();  // the partial buffer may still be read by the previous product's fix-up
+          waited = true;
+        }
+        const int pc = (int)(c - sk_owner((long long)gidx * p.U, p.W, P));
+        if (wait_or_die(&accfull, piece & 1, dead, p.err)) {
+          tc_fence_after();
+          const int m = dw * 32 + lane;  // TMEM lane = feature of the column group
+          int si;
+          const int tile = sk_tile(p, grp, m >> 4, si);
+          const int rows = tile >= 0 ? sk_rows(p, si, mz, kUmmaRows) : 0;
+          float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mz * p.ldo +
+                       (tile >= 0 ? p.seg[si].out_col + tile * 16 + (m & 15) : 0);
+          for (int n0 = 0; n0 < kUmmaRows; n0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)n0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (n0 + i < rows) out[(size_t)(n0 + i) * p.ldo] = __uint_as_float(v[i]);
+          }
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty);
+        ++piece;
+      }
+      x += ub - ua;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kUmmaTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Output head + top-16 for many drafted rows on the tensor cores.  The prepared head (records of
+// 256 features x 64-wide K steps, the output head followed by the selector projection) is applied
+// to up to 256 rows per CTA: the rows are the MMA's M side (two 128-row accumulators in TMEM, 512
+// columns), the 256 features of a record its N side, so after a record each thread holds one
+// row's 256 logits and offers them to that row's top-16 list, kept sorted in its registers.
+//  * warp 0, one thread: TMA of the rows' [256][64] bf16 slice per K step (no multicast);
+//  * warps 4-7: permute the record's 32 KB step (the streaming head's fragment order) into the
+//    128-byte-swizzled K-major operand, then run the epilogue of each record;
+//  * warp 1: TMEM allocation and the MMA issue (2 x 4 per K step), commits.
+// CTA c works on row tile c % nrt and on records c / nrt, c / nrt + P / nrt, ...; its lists are
+// part c / nrt of the candidate lists ([P / nrt][rows][16]) that the selector merges.
+struct UHeadParams {
+  const uint8_t* W;  // prepared [lm_head; sel_proj] records
+  int V, R, H, rows, nrec, nrt;
+  float* z;           // [rows][R]
+  float* cand_val;    // [parts][rows][16]
+  int32_t* cand_id;
+  int* err;
+};
+
+constexpr int kUHeadStages = 3;
+constexpr int kUHeadStage = 2 * 32768;  // A: 256 rows x 128 B, B: 256 features x 128 B
+constexpr int kUHeadSmem = kUHeadStages * kUHeadStage + 1024;
+
+// Insert (v, id) into a sorted 16-entry list held in registers (best first; the caller has checked
+// that it beats the last entry): it replaces the last entry and bubbles up.
+DEVI void reg_list_insert(float (&lv)[16], int (&li)[16], float v, int id) {
+  lv[15] = v;
+  li[15] = id;
+#pragma unroll
+  for (int k = 15; k > 0; --k) {
+    const bool up = better(lv[k], li[k], lv[k - 1], li[k - 1]);
+    const float a = lv[k], b = lv[k - 1];
+    const int ia = li[k], ib = li[k - 1];
+    lv[k] = up ? b : a;
+    li[k] = up ? ib : ia;
+    lv[k - 1] = up ? a : b;
+    li[k - 1] = up ? ia : ib;
+  }
+}
+
+__global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_constant__ CUtensorMap tmx, UHeadParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t xfull[kUHeadStages], bfull[kUHeadStages], sempty[kUHeadStages];
+  __shared__ __align__(8) uint64_t accfull, accempty;
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.H / 64;
+  const int P = gridDim.x, c = blockIdx.x, nparts = P / p.nrt, rt = c % p.nrt, part = c / p.nrt;
+  const int row0 = rt * 256;
+  const int trows = p.rows - row0 < 256 ? p.rows - row0 : 256;
+  const int nmc = trows > 128 ? 2 : 1;  // 128-row accumulators this row tile needs
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kUHeadStages; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&bfull[s], 4);
+      mbar_init(&sempty[s], 1);
+    }
+    mbar_init(&accfull, 1);
+    mbar_init(&accempty, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- activation rows (TMA) ----
+      pdl_wait();
+      bool dead = false;
+      int cnt = 0;
+      for (int rec = part; rec < p.nrec && !dead; rec += nparts)
+        for (int st = 0; st < S && !dead; ++st, ++cnt) {
+          const int s = cnt % kUHeadStages, round = cnt / kUHeadStages;
+          if (round > 0 && !wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err)) break;
+          mbar_expect_tx(&xfull[s], 32768);
+          tma_load_2d(smem + s * kUHeadStage, &tmx, st * 64, row0, &xfull[s]);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer ----
+      bool dead = false;
+      int cnt = 0, it = 0;
+      for (int rec = part; rec < p.nrec && !dead; rec += nparts, ++it) {
+        if (it > 0 && !wait_or_die(&accempty, (it - 1) & 1, dead, p.err)) break;
+        tc_fence_after();
+        for (int st = 0; st < S && !dead; ++st, ++cnt) {
+          const int s = cnt % kUHeadStages;
+          const uint32_t par = (cnt / kUHeadStages) & 1;
+          if (!wait_or_die(&xfull[s], par, dead, p.err) || !wait_or_die(&bfull[s], par, dead, p.err)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * kUHeadStage), b0 = a0 + 32768;
+          const uint64_t bd = sw128_desc(b0);
+          for (int mc = 0; mc < nmc; ++mc) {
+            const uint64_t ad = sw128_desc(a0 + mc * 16384);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma(tmem + mc * 256, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (st == 0 && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&sempty[s]);
+        }
+        if (!dead) tc_commit(&accfull);
+      }
+    }
+  } else if (warp >= 4) {
+    // ---- weight permutation, then the per-record top-16 epilogue ----
+    const int dw = warp - 4, g = lane >> 2, t = lane & 3;
+    float lv[2][16];
+    int li[2][16];
+#pragma unroll
+    for (int mc = 0; mc < 2; ++mc)
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        lv[mc][k] = -INFINITY;
+        li[mc][k] = 0x7fffffff;
+      }
+    bool dead = false, waited = false;
+    int cnt = 0, it = 0;
+    for (int rec = part; rec < p.nrec; rec += nparts, ++it) {
+      for (int st = 0; st < S; ++st, ++cnt) {
+        const int s = cnt % kUHeadStages, round = cnt / kUHeadStages;
+        if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
+        uint8_t* b = smem + s * kUHeadStage + 32768;
+        if (!dead) {
+          const uint8_t* src = p.W + ((size_t)rec * S + st) * (size_t)kHeadSlot;
+          uint4 v[4][4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h)  // tiles 4*dw + h of the record: all loads first
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              v[h][q] = ldg_stream(src + (size_t)(4 * dw + h) * 2048 + (q >> 1) * 1024 + (q & 1) * 512 + lane * 16);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int m0 = (4 * dw + h) * 16 + g;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              *reinterpret_cast<uint4*>(b + sw128_off(m0, 4 * jj + t)) = v[h][2 * jj];
+              *reinterpret_cast<uint4*>(b + sw128_off(m0 + 8, 4 * jj + t)) = v[h][2 * jj + 1];
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bfull[s]);
+      }
+      // ---- epilogue: thread = row (TMEM lane 32*dw + lane of each accumulator) ----
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
+      if (wait_or_die(&accfull, it & 1, dead, p.err)) {
+        tc_fence_after();
+#pragma unroll
+        for (int mc = 0; mc < 2; ++mc) {
+          if (mc >= nmc) break;
+          const int rl = mc * 128 + dw * 32 + lane, row = row0 + rl;
+          for (int n0 = 0; n0 < 256; n0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)(mc * 256 + n0), r);
+            tmem_ld_wait();
+            if (rl < trows) {
+              const int f0 = rec * 256 + n0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(r[i]);
+                const int f = f0 + i;
+                if (f < p.V) {
+                  if (better(x, f, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, f);
+                } else if (f < p.V + p.R) {
+                  p.z[(size_t)row * p.R + (f - p.V)] = x;
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty);
+    }
+    // this CTA's lists -> part `part` of the candidate lists
+#pragma unroll
+    for (int mc = 0; mc < 2; ++mc) {
+      const int rl = mc * 128 + dw * 32 + lane;
+      if (rl < trows) {
+        const size_t o = ((size_t)part * p.rows + row0 + rl) * kTopK;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          p.cand_val[o + k] = lv[mc][k];
+          p.cand_id[o + k] = li[mc][k];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Split-K fix-up of the tensor-core products: the CTA of (64-row group, column group) sums the
+// pieces of its tile in piece order (deterministic) and runs the product's fused epilogue.
+// P: the tensor-core launch's grid size (p.W its stream-K plane).
+__global__ void __launch_bounds__(kGemvConsumers * 32, 1) k_umma_fixup(SGemvParams p, int P) {
+  pdl_trigger();
+  pdl_wait();
+  const int grp = blockIdx.x % p.groups, mz = (blockIdx.x / p.groups) * 64;
+  const long long gidx = (long long)(mz / kUmmaRows) * p.groups + grp;
+  const long long gstart = gidx * p.U;
+  const long long first = sk_owner(gstart, p.W, P);
+  const int npieces = (int)(sk_owner(gstart + p.U - 1, p.W, P) - first + 1);
+  int si;
+  sk_tile(p, grp, 0, si);
+  if (sk_rows(p, si, mz, 64) <= 0) return;
+  sk_fixup(p, grp, mz, 64, npieces, nullptr);
+}
+
+}  // namespace dfl

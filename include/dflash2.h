@@ -207,6 +207,66 @@ int dflash2_draft_step_static(const dflash2_config *cfg, const dflash2_weights *
 int dflash2_accept(const int32_t *draft, const int32_t *target, int32_t batch, int32_t block,
                    int32_t *accepted, int32_t *emitted, void *stream);
 
+/* Acceptance for sampled decoding by exact rejection sampling (MLX sidecar card, "Contents";
+ * Mindket listing, "For newcomers and experts": the target's distribution is preserved).  For
+ * each request, in block order: accept drafted token d_i with probability min(1, p_i(d_i) /
+ * q_i(d_i)); at the first rejection emit a token drawn from max(0, p_i - q_i) (normalised), or, when
+ * all block-1 drafted tokens are accepted, one drawn from p_{block-1}.  The decisions are exact:
+ * accept iff u_accept[b][i] * q_i(d_i) < p_i(d_i) with the product formed exactly; the residual
+ * is taken in 32-bit fixed point, floor(max(0, p - q) * 2^32) per token (fp32 subtraction), and
+ * the emitted token is the first whose running sum exceeds floor(u_sample[b] * T / 2^32), T the
+ * total; an empty residual samples p itself.  fp32 values below the normal range count as 0.
+ *   draft int32 [batch][block-1]; p_target fp32 [batch][block][vocab], row i = the target's
+ *   probabilities for block position i+1; q_draft fp32 [batch][block-1][vocab], or NULL for the
+ *   point mass on the drafted token (the selector's path is deterministic); u_accept fp32
+ *   [batch][block-1] uniforms in [0,1); u_sample uint32 [batch] uniform 32-bit integers (the
+ *   caller's random numbers: the call draws none).  accepted int32 [batch]; emitted int32
+ *   [batch][block]: the accepted tokens, the sampled token, then -1.  Device pointers;
+ *   asynchronous on `stream`. */
+int dflash2_accept_sampled(const int32_t *draft, const float *p_target, const float *q_draft, const float *u_accept,
+                           const uint32_t *u_sample, int32_t batch, int32_t block, int32_t vocab, int32_t *accepted,
+                           int32_t *emitted, void *stream);
+
+/* Greedy acceptance that also prepares the next round's draft inputs on the device, so
+ * consecutive rounds need no host work between the acceptance and the next draft (FastFlowLM
+ * card, "How it is used": the target keeps the longest agreeing prefix plus one token of its
+ * own, and drafting continues from there).  accepted and emitted as dflash2_accept; then
+ *   n_new_next[b] = accepted[b] + 1 (the accepted drafted tokens and the target's token are the
+ *     tokens whose target features the next round fuses as context rows), and
+ *   block_tokens_next[b] = {target[b][accepted[b]], mask_id, ..., mask_id} (block entries).
+ * n_new_next and block_tokens_next may be the very buffers the step just read (its n_new and
+ * block_tokens): the acceptance runs after the step on the same stream.  The caller supplies the
+ * next round's taps rows 0..accepted[b] (the target's features of those tokens).  Device
+ * pointers; mask_id >= 0; asynchronous on `stream`. */
+int dflash2_accept_chain(const int32_t *draft, const int32_t *target, int32_t batch, int32_t block, int32_t mask_id,
+                         int32_t *accepted, int32_t *emitted, int32_t *n_new_next, int32_t *block_tokens_next,
+                         void *stream);
+
+/* Per-step inputs that a speculative round updates in place (device): same meaning as
+ * dflash2_inputs; n_new and block_tokens are overwritten with the next round's values. */
+typedef struct dflash2_inputs_mut {
+  const uint16_t *taps;
+  int32_t *n_new;
+  int32_t *block_tokens;
+} dflash2_inputs_mut;
+
+/* One speculative round on device buffers, after the target has scored the previous draft:
+ * dflash2_accept_chain of prev_path (int32 [batch][block-1], the previous round's drafted path)
+ * against `target` (int32 [batch][block], the target's most likely tokens for that block's
+ * positions 1..block), which writes the next round's n_new and block tokens into `in`, then
+ * dflash2_draft_step of the next block (taps: the target's features of the accepted tokens and
+ * its own token, rows 0..accepted[b], supplied by the caller) into out_path / out_scores.  The
+ * KV cache and seq_len advance as in dflash2_draft_step.  out_path may be prev_path (the step
+ * writes it only after the acceptance has read it).  Asynchronous, no host synchronisation and
+ * no host reads of device data: a serving loop issues the target's pass and this call per round,
+ * or replays one captured CUDA graph of both (after an uncaptured step has set the kernels'
+ * attributes on the device).  0 <= mask_id < vocab.  Everything the step validates is validated
+ * before anything is queued. */
+int dflash2_spec_round(const dflash2_config *cfg, const dflash2_weights *w, dflash2_inputs_mut *in,
+                       const dflash2_kv *kv, int32_t batch, const int32_t *prev_path, const int32_t *target,
+                       int32_t mask_id, int32_t *accepted, int32_t *emitted, int32_t *out_path, float *out_scores,
+                       void *workspace, size_t ws_bytes, void *stream);
+
 /* A whole speculative draft round with HOST buffers: copies taps, n_new,
  * block_tokens and target (host, same layouts as above) into the workspace,
  * runs dflash2_draft_step and dflash2_accept, copies path, scores, accepted and

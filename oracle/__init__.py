@@ -229,6 +229,34 @@ def accept(draft, target):
     return acc, em
 
 
+def accept_chain(draft, target, mask_id: int):
+    """Acceptance plus the next round's n_new and block tokens (see orc_accept_chain)."""
+    d = _np(draft, np.int32)
+    t = _np(target, np.int32)
+    B, Bk = t.shape
+    acc = np.empty(B, np.int32)
+    em = np.empty((B, Bk), np.int32)
+    nn = np.empty(B, np.int32)
+    bt = np.empty((B, Bk), np.int32)
+    lib().orc_accept_chain(B, Bk, int(mask_id), _p(d), _p(t), _p(acc), _p(em), _p(nn), _p(bt))
+    return acc, em, nn, bt
+
+
+def accept_sampled(draft, p, u_acc, u_s, q=None):
+    """Exact rejection-sampling acceptance (see orc_accept_sampled).  draft int32 [B][D], p fp32
+    [B][Bk][V], u_acc fp32 [B][D], u_s uint32 [B], q fp32 [B][D][V] or None (point mass)."""
+    d = _np(draft, np.int32)
+    pp = np.ascontiguousarray(_np(p), np.float32)
+    B, Bk, V = pp.shape
+    qq = None if q is None else np.ascontiguousarray(_np(q), np.float32)
+    ua = np.ascontiguousarray(_np(u_acc), np.float32)
+    us = np.ascontiguousarray(_np(u_s).astype(np.uint32))
+    acc = np.empty(B, np.int32)
+    em = np.empty((B, Bk), np.int32)
+    lib().orc_accept_sampled(B, Bk, V, _p(d), _p(pp), _p(qq), _p(ua), _p(us), _p(acc), _p(em))
+    return acc, em
+
+
 def lmhead_topk(hn_bf16, lm_head, k: int):
     hn = _np(hn_bf16, np.uint16)
     rows, H = hn.shape

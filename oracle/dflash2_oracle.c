@@ -411,6 +411,98 @@ void orc_accept(int B, int Bk, const int32_t *draft, const int32_t *target, int3
   }
 }
 
+/* The next round's draft inputs from an acceptance (FastFlowLM card, "How it is used": the
+ * target keeps the longest agreeing prefix plus one token of its own, and drafting continues
+ * from there).  The accepted tokens and the target's own token are the tokens whose target
+ * features the next round fuses as context rows, so n_new_next[b] = accepted[b] + 1; the next
+ * block starts from the target's token: block_tokens_next[b][0] = target[b][accepted[b]],
+ * positions 1..Bk-1 hold the caller's mask id. */
+void orc_accept_chain(int B, int Bk, int32_t mask_id, const int32_t *draft, const int32_t *target,
+                      int32_t *accepted, int32_t *emitted, int32_t *n_new_next,
+                      int32_t *block_tokens_next) {
+  orc_accept(B, Bk, draft, target, accepted, emitted);
+  for (int b = 0; b < B; ++b) {
+    n_new_next[b] = accepted[b] + 1;
+    block_tokens_next[b * Bk] = target[b * Bk + accepted[b]];
+    for (int i = 1; i < Bk; ++i) block_tokens_next[b * Bk + i] = mask_id;
+  }
+}
+
+/* Sampled decoding: exact rejection sampling of the drafted path (MLX sidecar card, "Contents":
+ * lossless acceptance for sampled decoding; Mindket listing, "For newcomers and experts").  The
+ * pages name the rule, not its arithmetic; the reading fixed here is the standard speculative-
+ * sampling rule with the draft's own distribution q_i at block position i:
+ *   accept drafted token d_i with probability min(1, p_i(d_i) / q_i(d_i)), in order, stopping at the
+ *   first rejection; at a rejection at i emit a token drawn from max(0, p_i - q_i) (normalised); if
+ *   every drafted token is accepted emit a token drawn from p_D (the target's distribution after the
+ *   block).  The selector picks its path deterministically, so by default q_i is the point mass on
+ *   d_i (q = NULL): accept with probability p_i(d_i), resample from p_i without d_i.
+ * Decisions are exact, so every implementation takes the same ones:
+ *   accept iff u_acc[i] * q_i(d_i) < p_i(d_i), the product of the two fp32 inputs formed exactly
+ *     (in double: 24 + 24 significant bits); fp32 inputs below the normal range count as zero;
+ *   the residual r(x) = max(0, p(x) - q(x)) in fp32, then r_int(x) = floor(r(x) * 2^32) (exact),
+ *     T = sum of r_int (64-bit integer), threshold t = floor(u_s * T / 2^32) with the 32-bit uniform
+ *     integer u_s, and the emitted token is the smallest x whose running sum of r_int exceeds t
+ *     (T = 0, a residual that is empty in fp32, falls back to p itself).
+ * p: fp32 [B][Bk][V], row i = the target's probabilities for block position i+1 (row D after the
+ * drafted tokens); q: fp32 [B][D][V] or NULL; u_acc: fp32 [B][D] in [0,1); u_s: uint32 [B].
+ * accepted [B], emitted [B][Bk] (the accepted tokens, the sampled token, then -1). */
+/* fp32 values below the normal range (|v| < 2^-126) count as zero, inputs and the residual alike:
+ * the decisions then do not depend on how an implementation treats subnormal numbers. */
+static float flush32(float v) {
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  return (u & 0x7F800000u) == 0 ? 0.0f : v;
+}
+
+/* Residual mass of token x in fp32: p - q (q given), p without the drafted token (point-mass
+ * draft), or p itself (dtok < 0: the bonus position, or the fallback of an empty residual). */
+static float residual(const float *p, const float *q, int32_t dtok, int x) {
+  if (dtok < 0) return flush32(p[x]);
+  if (q) return flush32(flush32(p[x]) - flush32(q[x]));
+  return x == dtok ? flush32(flush32(p[x]) - 1.0f) : flush32(p[x]);
+}
+
+static uint64_t fixed32(float r) { return r > 0.0f ? (uint64_t)floor((double)r * 4294967296.0) : 0; }
+
+/* The smallest x whose running sum of floor(max(0, r) * 2^32) exceeds floor(us * T / 2^32). */
+static int32_t sample_residual(const float *p, const float *q, int32_t dtok, int V, uint32_t us) {
+  uint64_t T = 0;
+  for (int x = 0; x < V; ++x) T += fixed32(residual(p, q, dtok, x));
+  if (T == 0) {  /* empty residual: sample p itself */
+    dtok = -1;
+    for (int x = 0; x < V; ++x) T += fixed32(flush32(p[x]));
+    if (T == 0) return 0;
+  }
+  const uint64_t t = (uint64_t)(((unsigned __int128)us * T) >> 32);
+  uint64_t run = 0;
+  for (int x = 0; x < V; ++x) {
+    run += fixed32(residual(p, q, dtok, x));
+    if (run > t) return x;
+  }
+  return V - 1;
+}
+
+void orc_accept_sampled(int B, int Bk, int V, const int32_t *draft, const float *p, const float *q,
+                        const float *u_acc, const uint32_t *u_s, int32_t *accepted, int32_t *emitted) {
+  const int D = Bk - 1;
+  for (int b = 0; b < B; ++b) {
+    int n = 0;
+    while (n < D) {
+      const int32_t d = draft[b * D + n];
+      const float *pr = p + ((int64_t)b * Bk + n) * V;
+      const double qd = q ? (double)flush32(q[((int64_t)b * D + n) * V + d]) : 1.0;
+      if ((double)flush32(u_acc[b * D + n]) * qd < (double)flush32(pr[d])) ++n;
+      else break;
+    }
+    accepted[b] = n;
+    const float *pr = p + ((int64_t)b * Bk + n) * V;
+    const float *qr = q && n < D ? q + ((int64_t)b * D + n) * V : NULL;
+    const int32_t tok = sample_residual(pr, qr, n < D ? draft[b * D + n] : -1, V, u_s[b]);
+    for (int i = 0; i < Bk; ++i) emitted[b * Bk + i] = i < n ? draft[b * D + i] : (i == n ? tok : -1);
+  }
+}
+
 /* LM head + top-K from given bf16 rows (the shared output head, FastFlowLM card).
  * hn: [rows][H] bf16; ids, vals: [rows][K]. */
 void orc_lmhead_topk(int rows, int H, int V, int K, const uint16_t *hn, const uint16_t *lm_head,

@@ -76,6 +76,30 @@ def test_null_arguments_are_rejected(lib):
                                       None) == -1
     assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 0, *ptrs, None, ptrs[0], 0, None) == -1
     assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 1, *ptrs, None, None, 0, None) == -1
+    # the host-buffer round rejects a missing KV cache before it copies anything (weights valid-looking)
+    ws = C.create_string_buffer(512)
+    ws_al = (C.addressof(ws) + 255) // 256 * 256
+    assert lib.dflash2_spec_step_host(C.byref(cfg), C.byref(w), None, 1, *ptrs, None, ws_al, 1 << 40, None) in (-1, -6)
+    # sampled acceptance: every pointer but q (optional), a positive batch, block >= 2 and vocab >= 1
+    assert lib.dflash2_accept_sampled(None, *ptrs[1:5], 1, 8, 10, ptrs[5], ptrs[6], None) == -1
+    assert lib.dflash2_accept_sampled(*ptrs[:5], 0, 8, 10, ptrs[5], ptrs[6], None) == -1
+    assert lib.dflash2_accept_sampled(*ptrs[:5], 1, 1, 10, ptrs[5], ptrs[6], None) == -1
+    assert lib.dflash2_accept_sampled(*ptrs[:5], 1, 8, 0, ptrs[5], ptrs[6], None) == -1
+    assert lib.dflash2_accept_sampled(*ptrs[:5], 1, 8, 10, None, ptrs[6], None) == -1
+    # chained acceptance: every pointer, a positive batch, block >= 2 and mask_id >= 0 are required
+    assert lib.dflash2_accept_chain(None, ptrs[1], 1, 8, 5, *ptrs[2:6], None) == -1
+    assert lib.dflash2_accept_chain(*ptrs[:2], 0, 8, 5, *ptrs[2:6], None) == -1
+    assert lib.dflash2_accept_chain(*ptrs[:2], 1, 1, 5, *ptrs[2:6], None) == -1
+    assert lib.dflash2_accept_chain(*ptrs[:2], 1, 8, -1, *ptrs[2:6], None) == -1
+    assert lib.dflash2_accept_chain(*ptrs[:2], 1, 8, 5, ptrs[2], ptrs[3], None, ptrs[5], None) == -1
+    ins = binding.InputsMut()
+    assert lib.dflash2_spec_round(C.byref(cfg), C.byref(w), C.byref(ins), None, 1, *ptrs[:2], 5, *ptrs[2:6], ws_al,
+                                  1 << 30, None) == -1
+    ins = binding.InputsMut(ptrs[0], ptrs[1], ptrs[2])
+    assert lib.dflash2_spec_round(C.byref(cfg), C.byref(w), C.byref(ins), None, 1, *ptrs[:2], inputs.TINY.vocab,
+                                  *ptrs[2:6], ws_al, 1 << 30, None) == -1
+    assert lib.dflash2_spec_round(C.byref(cfg), C.byref(w), C.byref(ins), None, 1, *ptrs[:2], 5, *ptrs[2:6], ws_al,
+                                  1 << 30, None) == -6  # (unprepared weights: rejected before anything is queued)
 
 
 def test_unprepared_q4k_weights_are_rejected(lib):

@@ -187,3 +187,24 @@ def test_tied_candidates_are_distinct_and_in_id_order():
     parity.check_request(run2, hw_t, hw, 0)
     ids = run2["dbg"]["cand"][t_row].cpu().numpy()
     assert set(ids.tolist()) <= set(dups) | {top}, ids
+
+
+@pytest.mark.parametrize("wfmt,block,batch", [(0, 8, 12), (1, 5, 20), (0, 8, 40)])
+def test_tiny_many_rows_run_on_tensor_cores(wfmt, block, batch):
+    """More than 64 block rows: every layer product runs as a tcgen05 contraction (TMEM
+    accumulators, dequantised weight tiles, TMA-staged activations) followed by its fix-up
+    kernel; Q4_K and bf16 layers, ragged new rows (0 included), shuffled pages, and 320 rows
+    (two 256-row tiles, 640 rows for the k/v projections)."""
+    import dataclasses
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=wfmt, block=block),
+                             batch=batch, ctx_lo=0, ctx_hi=300, shuffled_pages=True)
+    w, hw_t, hw = weights_for(wl)
+    n_new = [(3 * b) % (block + 1) for b in range(batch)]
+    st = inputs.make_state(wl, "cuda", n_new=n_new)
+    sample = sorted({0, 1, batch // 2, batch - 1})
+    run = parity.run_gpu(wl, w, sample, state=st)
+    base = 3 + 6 * wl.dims.layers + 3
+    assert run["drafter"].step_kernels() == base + 6 * wl.dims.layers  # five layer products + fc, each + fix-up
+    for b in sample:
+        parity.check_request(run, hw_t, hw, b)
+    parity.check_accept(run)

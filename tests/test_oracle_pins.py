@@ -496,6 +496,126 @@ def test_accept_invariants():
     assert np.all((acc == D) == np.all(draft == target[:, :D], axis=1))
 
 
+def test_accept_chain_next_round_inputs():
+    """The next round starts from the token the target kept (emitted[n], its own argmax at the
+    first disagreement, or its bonus token after a full match) and fuses n + 1 new context rows:
+    the n accepted drafted tokens and that token."""
+    B, Bk, mask = 300, 8, 8191
+    D = Bk - 1
+    draft = rng.integers(0, 6, (B, D)).astype(np.int32)
+    target = rng.integers(0, 6, (B, Bk)).astype(np.int32)
+    m = rng.integers(0, Bk, B)
+    for b in range(B):
+        target[b, :m[b]] = draft[b, :m[b]]
+        if m[b] < D:
+            target[b, m[b]] = draft[b, m[b]] + 1
+    acc, em, nn, bt = oracle.accept_chain(draft, target, mask)
+    acc0, em0 = oracle.accept(draft, target)
+    assert np.array_equal(acc, acc0) and np.array_equal(em, em0) and np.array_equal(acc, m)
+    assert np.array_equal(nn, m + 1) and np.all((nn >= 1) & (nn <= Bk))
+    for b in range(B):
+        assert bt[b, 0] == em[b, m[b]] == target[b, m[b]]
+        assert np.all(bt[b, 1:] == mask)
+        # after a full match the next block starts from the bonus token (the target's 8th)
+        if m[b] == D:
+            assert bt[b, 0] == target[b, D]
+
+
+def _grid_uniforms(N, M):
+    """u_acc on the midpoints of N cells of [0,1), u_s on the midpoints of M cells of 2^32."""
+    ua = ((np.arange(N) + 0.5) / N).astype(np.float32)
+    us = (((np.arange(M) + 0.5) / M) * 2.0 ** 32).astype(np.uint64).astype(np.uint32)
+    return np.repeat(ua, M), np.tile(us, N)
+
+
+@pytest.mark.parametrize("with_q", [False, True])
+def test_sampled_accept_is_lossless_on_a_uniform_grid(with_q):
+    """The defining property of exact rejection sampling: over uniform u_acc and u_s (an exact
+    midpoint grid here), the first emitted token is distributed as the target's p_0, whatever the
+    draft distribution q (drafted token d drawn from q) or, by default, a fixed drafted token."""
+    V, N, M = 5, 400, 512
+    p0 = np.array([0.05, 0.4, 0.25, 0.1, 0.2], np.float32)
+    pD = np.array([0.3, 0.1, 0.1, 0.2, 0.3], np.float32)
+    q0 = np.array([0.3, 0.1, 0.4, 0.15, 0.05], np.float32)
+    ua, us = _grid_uniforms(N, M)
+    B = ua.size
+    freq = np.zeros(V)
+    for d in range(V):
+        weight = q0[d] if with_q else (1.0 if d == 2 else 0.0)
+        if weight == 0:
+            continue
+        p = np.broadcast_to(np.stack([p0, pD]), (B, 2, V)).copy()
+        q = np.broadcast_to(q0, (B, 1, V)).copy() if with_q else None
+        acc, em = oracle.accept_sampled(np.full((B, 1), d, np.int32), p, ua.reshape(B, 1), us, q=q)
+        freq += weight * np.bincount(em[:, 0], minlength=V) / B
+    assert np.allclose(freq, p0, atol=1.0 / N + 1.0 / M + 1e-6), (freq, p0)
+
+
+def test_sampled_accept_special_cases():
+    V, Bk = 50, 8
+    D = Bk - 1
+    B = 64
+    draft = rng.integers(0, V, (B, D)).astype(np.int32)
+    ua = rng.random((B, D)).astype(np.float32)
+    us = rng.integers(0, 2 ** 32, B, dtype=np.uint64).astype(np.uint32)
+    # the target is certain of every drafted token: all accepted, the bonus from p_D (one-hot 7)
+    p = np.zeros((B, Bk, V), np.float32)
+    for b in range(B):
+        p[b, np.arange(D), draft[b]] = 1.0
+    p[:, D, 7] = 1.0
+    acc, em = oracle.accept_sampled(draft, p, ua, us)
+    assert np.all(acc == D) and np.array_equal(em[:, :D], draft) and np.all(em[:, D] == 7)
+    # the target gives the first drafted token probability 0: rejected at 0 whatever u, and the
+    # resampled token is never the drafted one; u_acc = 0 accepts exactly the tokens with p > 0
+    p = rng.random((B, Bk, V)).astype(np.float32)
+    p /= p.sum(-1, keepdims=True)
+    p[np.arange(B), 0, draft[:, 0]] = 0.0
+    acc, em = oracle.accept_sampled(draft, p, ua, us)
+    assert np.all(acc == 0) and np.all(em[:, 0] != draft[:, 0]) and np.all(em[:, 1:] == -1)
+    acc0, _ = oracle.accept_sampled(draft, p, np.zeros_like(ua), us)
+    assert np.all(acc0 == 0)
+    p[np.arange(B), 0, draft[:, 0]] = 1e-30
+    acc1, _ = oracle.accept_sampled(draft, p, np.zeros_like(ua), us)
+    assert np.all(acc1 >= 1)
+
+
+def test_sampled_residual_search_matches_searchsorted():
+    """The resampled token is the inverse CDF of the fixed-point residual: numpy's searchsorted on
+    the running sums of floor(max(0, p - q) * 2^32) gives the same token, u_s = 0 and 2^32 - 1
+    included (first and last token of nonzero residual)."""
+    V, B = 1000, 200
+    p = rng.random((B, 2, V)).astype(np.float32) ** 3
+    p /= p.sum(-1, keepdims=True)
+    q = rng.random((B, 1, V)).astype(np.float32) ** 3
+    q /= q.sum(-1, keepdims=True)
+    p[:2, 0, :3] = 0.0  # leading tokens without residual mass: u_s = 0 must skip them
+    draft = rng.integers(0, V, (B, 1)).astype(np.int32)
+    ua = np.full((B, 1), 0.999999, np.float32)  # rejections (unless p(d) >= q(d))
+    us = rng.integers(0, 2 ** 32, B, dtype=np.uint64).astype(np.uint32)
+    us[:2] = [0, 2 ** 32 - 1]
+    acc, em = oracle.accept_sampled(draft, p, ua, us, q=q)
+    for b in range(B):
+        if acc[b] == 1:
+            continue
+        r = np.maximum(np.float32(0), p[b, 0] - q[b, 0])
+        fx = np.floor(r.astype(np.float64) * 2.0 ** 32).astype(np.uint64)
+        cum = np.cumsum(fx, dtype=np.uint64)
+        t = (int(us[b]) * int(cum[-1])) >> 32
+        want = int(np.searchsorted(cum, np.uint64(t), side="right"))
+        assert em[b, 0] == want, (b, em[b, 0], want)
+        if b == 0:
+            assert want == int(np.nonzero(fx)[0][0])
+        if b == 1:
+            assert want == int(np.nonzero(fx)[0][-1])
+    # a threshold exactly on a running sum: p = (1/4, 1/4, 1/2), q = (0, 0, 1) leaves the residual
+    # (1/4, 1/4, 0), in fixed point (2^30, 2^30, 0), T = 2^31; u_s = 2^31 gives t = 2^30 = the first
+    # running sum, and the token is the first whose running sum exceeds t: token 1
+    p3 = np.array([[[0.25, 0.25, 0.5], [1 / 3, 1 / 3, 1 / 3]]], np.float32)
+    acc, em = oracle.accept_sampled(np.array([[2]], np.int32), p3, np.array([[0.99]], np.float32),
+                                    np.array([2 ** 31], np.uint32), q=np.array([[[0.0, 0.0, 1.0]]], np.float32))
+    assert acc[0] == 0 and em[0, 0] == 1
+
+
 # ------------------------------------------------------------------ whole step
 
 def _tiny_step(wl=None, mutate=None, trace=True, state=None):
