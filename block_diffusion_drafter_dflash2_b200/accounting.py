@@ -13,7 +13,9 @@ def step_bytes(dims: Dims, ctx_after: List[int], n_new: List[int]) -> Dict[str, 
     ctx_after: cached tokens per request after this step's append (L_b)."""
     H, F, T, R, V = dims.hidden, dims.ffn, dims.n_taps, dims.rank, dims.vocab
     hq, hkv, hd = dims.n_q * dims.head_dim, dims.n_kv * dims.head_dim, dims.head_dim
-    per_w = Q4K_BLOCK_BYTES / Q4K_BLOCK_ELEMS if dims.wfmt == 0 else 2.0
+    # bytes per weight the step streams: Q4_K and MLX 4-bit both as 144-byte records per 256 weights;
+    # bf16 and Q8_0 (decoded to bf16 when the weights are prepared) as 2 bytes
+    per_w = Q4K_BLOCK_BYTES / Q4K_BLOCK_ELEMS if dims.wfmt in (0, 2) else 2.0
     layer_mats = (hq * H + 2 * hkv * H + H * hq + 2 * F * H + H * F) * per_w
     dyn = (2 * (H // 4) * H + 2 * H) * 2.0
     norms = (2 * H + 2 * hd) * 2.0

@@ -61,7 +61,9 @@ class InputsMut(C.Structure):
 
 EXPORTS = ("dflash2_workspace_size", "dflash2_prepared_size", "dflash2_prepare_weights", "dflash2_draft_step",
            "dflash2_draft_step_static", "dflash2_accept", "dflash2_accept_sampled", "dflash2_accept_chain", "dflash2_spec_round",
-           "dflash2_spec_step_host", "dflash2_device_error", "dflash2_step_kernels", "dflash2_strerror")
+           "dflash2_spec_step_host", "dflash2_device_error", "dflash2_step_kernels", "dflash2_strerror",
+           "dflash2_head_shard_size", "dflash2_prepare_head_shard", "dflash2_draft_step_head_shard",
+           "dflash2_select")
 
 _lib = None
 
@@ -87,6 +89,15 @@ def load(path: str = LIB_PATH):
                                               C.POINTER(KV), C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
                                               C.POINTER(Debug), C.c_void_p]
     lib.dflash2_accept.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
+    lib.dflash2_head_shard_size.restype = C.c_size_t
+    lib.dflash2_head_shard_size.argtypes = [C.POINTER(Config), C.c_int32]
+    lib.dflash2_prepare_head_shard.argtypes = [C.POINTER(Config), C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p,
+                                               C.c_size_t, C.c_void_p]
+    lib.dflash2_draft_step_head_shard.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.c_void_p, C.c_int32,
+                                                  C.c_int32, C.POINTER(Inputs), C.POINTER(KV), C.c_int32, C.c_void_p,
+                                                  C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+    lib.dflash2_select.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.c_int32, C.c_int32] + \
+        [C.c_void_p] * 7 + [C.c_size_t, C.c_void_p]
     lib.dflash2_accept_sampled.argtypes = [C.c_void_p] * 5 + [C.c_int32] * 3 + [C.c_void_p] * 3
     lib.dflash2_accept_chain.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int32] + [C.c_void_p] * 5
     lib.dflash2_spec_round.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(InputsMut), C.POINTER(KV),

@@ -25,6 +25,7 @@ struct GemvPlan {
   long long W = 1;
   size_t smem = 0;
   bool umma = false;  // tensor-core (tcgen05) product + fix-up instead of the streaming engine
+  bool mlx = false;   // 4-bit records hold MLX group-64 (scale, bias) pairs
   int rows = 0, K = 0;
 };
 
@@ -36,7 +37,7 @@ struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
   int attn_ntk;  // > 0: attention as one cluster kernel, attn_kg key groups of 8*attn_ntk keys per CTA; 0: chunks + merge
   int attn_kg;
-  bool q4;
+  bool q4, mlx;
   GemvPlan fc, dc, qkv, o, gu, dn;
   size_t off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
   int lm_nparts, lm_rows, lm_groups;
@@ -45,7 +46,7 @@ struct Plan {
   int lm_uP, lm_unrt, lm_unrec;  // its grid, row tiles of 256 and head records
   int sel_parts;                 // candidate lists per row the selector merges
   size_t off_err, off_h, off_xf, off_xb, off_yb, off_part, off_qb, off_kb, off_vb, off_ao, off_aml, off_ob,
-      off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr;
+      off_act, off_hn, off_cv, off_ci, off_z, off_g, off_ctr, off_rsg;
   size_t ctr_layer[5], ctr_per_layer, ctr_fc, ctr_head, ctr_sel, ctr_total;
   size_t off_s_taps, off_s_nnew, off_s_btok, off_s_tgt, off_s_path, off_s_scores, off_s_acc, off_s_emit;
   size_t step_bytes, total;
@@ -121,8 +122,25 @@ bool cfg_ok(const dflash2_config* c) {
          (c->n_q / c->n_kv) * c->block <= 64 && c->hidden % kUnit == 0 && c->ffn % kUnit == 0 &&
          HQ % kUnit == 0 && ((long long)c->n_taps * c->hidden) % kUnit == 0 && c->n_taps >= 1 &&
          c->vocab % 16 == 0 && c->vocab > 0 && c->rank % 16 == 0 && c->rank >= 16 && c->rank <= kMaxR &&
-         c->window >= 1 && c->window <= 4032 && c->hidden <= 16384 && (c->wfmt == 0 || c->wfmt == 1) && c->rope_theta > 0.f &&
+         c->window >= 1 && c->window <= 4032 && c->hidden <= 16384 && (c->wfmt >= 0 && c->wfmt <= 3) && c->rope_theta > 0.f &&
          c->rms_eps >= 0.f;
+}
+
+// The output head's launch shape for Vh head rows (the whole vocabulary, or a shard of it) plus the
+// selector projection.
+void plan_head(Plan& p, int Vh) {
+  const int lm_tiles = Vh / 16 + p.R / 16;
+  // the streaming head takes any number of rows in groups of 8 (one launch, a CTA per group and
+  // vocabulary part)
+  p.lm_groups = (p.lm_rows + 7) / 8;
+  p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
+  p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
+  // more than one group of 8 drafted rows: the head is a dense contraction on the tensor cores
+  p.lm_umma = p.lm_rows > 8;
+  p.lm_unrt = (p.lm_rows + 255) / 256;
+  p.lm_unrec = (lm_tiles + kHeadTiles - 1) / kHeadTiles;
+  p.lm_uP = std::max(1, p.nsm / p.lm_unrt) * p.lm_unrt;
+  p.sel_parts = p.lm_umma ? p.lm_uP / p.lm_unrt : p.lm_nparts;
 }
 
 Plan make_plan(const dflash2_config* c, int B) {
@@ -139,7 +157,8 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.V = c->vocab;
   p.R = c->rank;
   p.nsm = device_sms();
-  p.q4 = c->wfmt == 0;
+  p.q4 = c->wfmt == 0 || c->wfmt == 2;  // 4-bit records (Q4_K or MLX group-64); bf16 and Q8_0 stream bf16
+  p.mlx = c->wfmt == 2;
   p.G = c->n_q / c->n_kv;
   p.QV = p.G * p.Bk;
   p.QVP = (p.QV + 15) / 16 * 16;
@@ -174,19 +193,11 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.o = plan_gemv(p.H / 16, p.Mb, p.HQ, p.q4, p.nsm);
   p.gu = plan_gemv(2 * p.F / 16, p.Mb, p.H, p.q4, p.nsm);
   p.dn = plan_gemv(p.H / 16, p.Mb, p.F, p.q4, p.nsm);
+  for (GemvPlan* g : {&p.fc, &p.dc, &p.qkv, &p.o, &p.gu, &p.dn}) g->mlx = p.mlx;
   p.lm_rows = B * p.D;
+  plan_head(p, p.V);
   const int lm_tiles = p.V / 16 + p.R / 16;
-  // the streaming head takes any number of rows in groups of 8 (one launch, a CTA per group and
-  // vocabulary part)
-  p.lm_groups = (p.lm_rows + 7) / 8;
-  p.lm_smem = (size_t)kHeadNS * kHeadSlot + (size_t)8 * (p.H * 2 + 64) + (size_t)kGemvConsumers * 8 * kTopK * 8;
-  p.lm_nparts = (int)std::min<long long>(p.nsm, (long long)((lm_tiles + kHeadTiles - 1) / kHeadTiles) * (p.H / 64));
-  // more than one group of 8 drafted rows: the head is a dense contraction on the tensor cores
-  p.lm_umma = p.lm_rows > 8;
-  p.lm_unrt = (p.lm_rows + 255) / 256;
-  p.lm_unrec = (lm_tiles + kHeadTiles - 1) / kHeadTiles;
-  p.lm_uP = std::max(1, p.nsm / p.lm_unrt) * p.lm_unrt;
-  p.sel_parts = p.lm_umma ? p.lm_uP / p.lm_unrt : p.lm_nparts;
+
   auto part_bytes = [&](const GemvPlan& g, int rows, int ldo) { return (size_t)g.max_pieces * rows * ldo * 4; };
   size_t part = 0;
   part = std::max(part, part_bytes(p.fc, p.Mb, p.H));
@@ -228,6 +239,7 @@ Plan make_plan(const dflash2_config* c, int B) {
   p.off_hpart = take((size_t)p.lm_groups * p.lm_nparts * 2 * kGemvConsumers * 32 * 4 * 4);
   p.off_z = take((size_t)p.lm_rows * p.R * 4);
   p.off_g = take((size_t)p.Mb * (p.H / 2) * 4);
+  p.off_rsg = take((size_t)2 * p.Mb * 4);  // row scales of a folded RMSNorm (tensor-core products)
   // arrival tickets of the split-K GEMVs: one per (column group, row group) and launch
   auto nctr = [](const GemvPlan& g) { return (size_t)g.groups * g.mgroups; };
   const GemvPlan* lp[5] = {&p.dc, &p.qkv, &p.o, &p.gu, &p.dn};
@@ -326,6 +338,7 @@ struct Epi {
   const uint16_t *dyn_w = nullptr, *dyn_s0 = nullptr, *dyn_s1 = nullptr;
   uint16_t* dyn_y = nullptr;
   int Bk = 1;
+  float* rs_glob = nullptr;  // tensor-core products with rs_in: [rows] row-scale buffer
 };
 
 SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X, int ldx,
@@ -368,6 +381,8 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   prm.dyn_y = e.dyn_y;
   prm.Bk = e.Bk;
   prm.err = err;
+  prm.rs_glob = (g.umma && e.rs_in) ? e.rs_glob : nullptr;
+  prm.mlx = g.mlx ? 1 : 0;
   return prm;
 }
 
@@ -562,10 +577,11 @@ size_t dflash2_prepared_size(const dflash2_config* c) {
   const size_t H = c->hidden, F = c->ffn, HQ = (size_t)c->n_q * kHeadDim, HKV = (size_t)c->n_kv * kHeadDim;
   const size_t per_layer = HQ * H + 2 * HKV * H + H * HQ + 2 * F * H + H * F;
   const size_t mats = H * c->n_taps * H + c->layers * per_layer;
-  const size_t mat_bytes = c->wfmt == 0 ? mats / kUnit * 144 : mats * 2;
+  const size_t mat_bytes = (c->wfmt == 0 || c->wfmt == 2) ? mats / kUnit * 144 : mats * 2;
   const size_t dyn = (size_t)c->layers * 2 * (H / 4) * H * 2;
   const size_t head_groups = ((size_t)(c->vocab + c->rank) / 16 + kHeadTiles - 1) / kHeadTiles;
-  return mat_bytes + dyn + head_groups * kHeadTiles * 16 * H * 2;
+  // the head twice: the streaming kernel's records and the tensor-core operand copy
+  return mat_bytes + dyn + 2 * head_groups * kHeadTiles * 16 * H * 2;
 }
 
 int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src, void* dst, size_t dst_bytes,
@@ -585,20 +601,31 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
   uint8_t* d = (uint8_t*)dst;
   const int H = c->hidden, F = c->ffn, HQ = c->n_q * kHeadDim, HKV = c->n_kv * kHeadDim;
   // one matrix (or a set sharing one buffer) into group-interleaved records at d
-  auto place = [&](const void* w, int N, int K, bool q4, PrepPlace pl) {
-    if (q4)
+  const int fmt = c->wfmt;
+  // fmt: 0 Q4_K, 1 bf16, 2 MLX 4-bit group-64 (into the same 4-bit records), 3 Q8_0 (into bf16 records)
+  auto place_fmt = [&](const void* w, int N, int K, int fmt, PrepPlace pl) {
+    if (fmt == 0)
       k_q4k_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K, pl);
+    else if (fmt == 2)
+      k_mlx4_prepare<<<dim3(K / kUnit, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K, pl);
+    else if (fmt == 3)
+      k_q80_prepare<<<dim3(K / 64, N / 16), 32, 0, s>>>((const uint8_t*)w, d, N, K, pl);
     else
       k_bf16_prepare<<<dim3(K / 64, N / 16), 32, 0, s>>>((const uint16_t*)w, d, N, K, pl);
   };
-  auto bytes = [&](int N, int K, bool q4) { return q4 ? (size_t)N * K / kUnit * 144 : (size_t)N * K * 2; };
+  auto place = [&](const void* w, int N, int K, bool q4, PrepPlace pl) { place_fmt(w, N, K, q4 ? fmt : 1, pl); };
+  // bytes of one prepared matrix: q4 = "in the configured format" (4-bit records for Q4_K and MLX,
+  // bf16 records for bf16 and Q8_0), else bf16
+  auto bytes = [&](int N, int K, bool q4) {
+    return (q4 && (fmt == 0 || fmt == 2)) ? (size_t)N * K / kUnit * 144 : (size_t)N * K * 2;
+  };
   auto prep = [&](const void* w, int N, int K, bool q4) -> const void* {
     const void* r = d;
     place(w, N, K, q4, PrepPlace{0, 8, 0, 8});
     d += bytes(N, K, q4);
     return r;
   };
-  const bool q4 = c->wfmt == 0;
+  const bool q4 = c->wfmt != 1;  // the layer matrices in the configured format (the W_dc generators are bf16)
   out->fc = prep(src->fc, H, c->n_taps * H, q4);
   for (int l = 0; l < c->layers; ++l) {
     const dflash2_layer_weights& S = src->layer[l];
@@ -629,22 +656,44 @@ int dflash2_prepare_weights(const dflash2_config* c, const dflash2_weights* src,
   place(src->sel_proj, c->rank, H, false, PrepPlace{c->vocab / 16, kHeadTiles, 0, kHeadTiles});
   out->lm_head = (const uint16_t*)d;
   out->sel_proj = (const uint16_t*)d;  // interleaved into the head's records
+  // the tensor-core operand copy of the same head follows the records (see k_umma_head)
+  k_head_sw_prepare<<<dim3(H / 64, (unsigned)(groups * kHeadTiles / 16)), 256, 0, s>>>(
+      src->lm_head, src->sel_proj, d + groups * gbytes, c->vocab, c->rank, H);
   return fail(cudaGetLastError());
 }
 
-int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const dflash2_inputs* in,
-                       const dflash2_kv* kv, int32_t batch, int32_t* out_path, float* out_scores, void* ws,
-                       size_t ws_bytes, const dflash2_debug* dbg, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// A vocabulary shard of the output head: this rank's head rows [v0, v0 + rows) (prepared with
+// dflash2_prepare_head_shard) and where its local candidates and the selector projection go.
+struct HeadShard {
+  const uint8_t* head;  // prepared streaming records, the tensor-core operand copy following them
+  int v0, rows;
+  float* out_val;
+  int32_t* out_id;
+  float* out_z;
+};
+
+size_t head_records(const dflash2_config* c, int rows) { return ((size_t)(rows + c->rank) / 16 + kHeadTiles - 1) / kHeadTiles; }
+
+int draft_step_impl(const dflash2_config* c, const dflash2_weights* w, const dflash2_inputs* in, const dflash2_kv* kv,
+                    int32_t batch, int32_t* out_path, float* out_scores, void* ws, size_t ws_bytes,
+                    const dflash2_debug* dbg, void* stream, const HeadShard* hs) {
   if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
-  if (batch < 1 || !in || !kv || !out_path || !out_scores || !ws) return DFLASH2_ERR_ARG;
+  if (batch < 1 || !in || !kv || !ws || (!hs && (!out_path || !out_scores))) return DFLASH2_ERR_ARG;
   int rc = check_weights(c, w);
   if (rc) return rc;
   if (!in->taps || !in->n_new || !in->block_tokens) return DFLASH2_ERR_ARG;
   rc = check_kv(c, kv);
   if (rc) return rc;
   if (!aligned16(in->taps) || ((uintptr_t)ws & 255u)) return DFLASH2_ERR_ALIGN;
-  const Plan P = make_plan(c, batch);
+  Plan P = make_plan(c, batch);
   if (ws_bytes < P.step_bytes) return DFLASH2_ERR_WORKSPACE;
+  if (hs) plan_head(P, hs->rows);  // the head's launch shape for this shard (workspace sized for the whole head)
+  const uint8_t* head = hs ? hs->head : (const uint8_t*)w->lm_head;
+  const int Vh = hs ? hs->rows : P.V, id0 = hs ? hs->v0 : 0;
   cudaStream_t s = (cudaStream_t)stream;
   int* err = at<int>(ws, P.off_err);
   float* h = at<float>(ws, P.off_h);
@@ -739,6 +788,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       Epi e;
       e.mode = EPI_DYNCONV;
       e.rs_in = ssp;
+      e.rs_glob = at<float>(ws, P.off_rsg);
       e.ssp_rows = Mb;
       e.rs_H = H;
       e.eps = c->rms_eps;
@@ -822,6 +872,7 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       e.act = act;
       e.F = P.F;
       e.rs_in = ssp;
+      e.rs_glob = at<float>(ws, P.off_rsg);
       e.ssp_rows = Mb;
       e.rs_H = H;
       e.eps = c->rms_eps;
@@ -867,14 +918,15 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       CUtensorMap tm;
       CK(make_act_tmap(&tm, hn, H, H, P.lm_rows));
       UHeadParams hp{};
-      hp.W = (const uint8_t*)w->lm_head;
-      hp.V = P.V;
+      hp.Wsw = head + (size_t)P.lm_unrec * kHeadTiles * 16 * H * 2;  // the operand copy
+      hp.V = Vh;
+      hp.id0 = id0;
       hp.R = P.R;
       hp.H = H;
       hp.rows = P.lm_rows;
       hp.nrec = P.lm_unrec;
       hp.nrt = P.lm_unrt;
-      hp.z = zbuf;
+      hp.z = hs ? hs->out_z : zbuf;
       hp.cand_val = at<float>(ws, P.off_cv);
       hp.cand_id = at<int32_t>(ws, P.off_ci);
       hp.err = err;
@@ -883,13 +935,14 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
       static std::atomic<int> attr[kMaxDevices];
       CK(smem_optin(k_slmhead, kSmemLimit - kStaticSmem, attr));
       SLmParams lp{};
-      lp.W = (const uint8_t*)w->lm_head;
-      lp.V = P.V;
+      lp.W = head;
+      lp.V = Vh;
+      lp.id0 = id0;
       lp.R = P.R;
       lp.H = H;
       lp.X = hn;
       lp.rows = P.lm_rows;
-      lp.z = zbuf;
+      lp.z = hs ? hs->out_z : zbuf;
       lp.cand_val = at<float>(ws, P.off_cv);
       lp.cand_id = at<int32_t>(ws, P.off_ci);
       lp.part = at<float>(ws, P.off_hpart);
@@ -900,6 +953,12 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     }
     if (dbg && dbg->ev_lm_end) CK(cudaEventRecord((cudaEvent_t)dbg->ev_lm_end, s));
     if (dbg && dbg->z) CK(cudaMemcpyAsync(dbg->z, zbuf, (size_t)P.lm_rows * P.R * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  if (hs) {  // a shard: its local top-16 per row for the exchange; seq_len advanced here
+    CK(launch_pdl(k_merge_rows, dim3((P.lm_rows + 3) / 4), dim3(128), 0, s, (const float*)at<float>(ws, P.off_cv),
+                  (const int32_t*)at<int32_t>(ws, P.off_ci), P.sel_parts, P.lm_rows, hs->out_val, hs->out_id,
+                  kv->seq_len, in->n_new, batch));
+    return DFLASH2_OK;
   }
   // A6: candidates, selector scores, Viterbi path; seq_len advanced
   {
@@ -932,6 +991,97 @@ int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const 
     CK(smem_optin(k_sel_tau, kSelSpreadSmem, sel_attr));
     CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), kSelSpreadSmem, s, sp, tau, clg, cdg, ctr + P.ctr_sel));
   }
+  return DFLASH2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dflash2_draft_step(const dflash2_config* c, const dflash2_weights* w, const dflash2_inputs* in,
+                       const dflash2_kv* kv, int32_t batch, int32_t* out_path, float* out_scores, void* ws,
+                       size_t ws_bytes, const dflash2_debug* dbg, void* stream) {
+  return draft_step_impl(c, w, in, kv, batch, out_path, out_scores, ws, ws_bytes, dbg, stream, nullptr);
+}
+
+size_t dflash2_head_shard_size(const dflash2_config* c, int32_t rows) {
+  if (!cfg_ok(c) || rows < 16 || rows % 16) return 0;
+  return 2 * head_records(c, rows) * kHeadTiles * 16 * (size_t)c->hidden * 2;
+}
+
+int dflash2_prepare_head_shard(const dflash2_config* c, const uint16_t* lm_head_rows, int32_t rows,
+                               const uint16_t* sel_proj, void* dst, size_t dst_bytes, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (!lm_head_rows || !sel_proj || !dst || rows < 16 || rows % 16 || rows > c->vocab) return DFLASH2_ERR_ARG;
+  if (!aligned16(dst) || !aligned16(lm_head_rows) || !aligned16(sel_proj)) return DFLASH2_ERR_ALIGN;
+  if (dst_bytes < dflash2_head_shard_size(c, rows)) return DFLASH2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int H = c->hidden;
+  const size_t groups = head_records(c, rows), gbytes = (size_t)kHeadTiles * 16 * H * 2;
+  uint8_t* d = (uint8_t*)dst;
+  CK(cudaMemsetAsync(d + (groups - 1) * gbytes, 0, gbytes, s));
+  k_bf16_prepare<<<dim3(H / 64, rows / 16), 32, 0, s>>>(lm_head_rows, d, rows, H, PrepPlace{0, kHeadTiles, 0, kHeadTiles});
+  k_bf16_prepare<<<dim3(H / 64, c->rank / 16), 32, 0, s>>>(sel_proj, d, c->rank, H,
+                                                            PrepPlace{rows / 16, kHeadTiles, 0, kHeadTiles});
+  k_head_sw_prepare<<<dim3(H / 64, (unsigned)groups), 256, 0, s>>>(lm_head_rows, sel_proj, d + groups * gbytes, rows,
+                                                                   c->rank, H);
+  return fail(cudaGetLastError());
+}
+
+int dflash2_draft_step_head_shard(const dflash2_config* c, const dflash2_weights* w, const void* head_shard,
+                                  int32_t v0, int32_t rows, const dflash2_inputs* in, const dflash2_kv* kv,
+                                  int32_t batch, float* out_cand_val, int32_t* out_cand_id, float* out_z, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (!head_shard || !out_cand_val || !out_cand_id || !out_z || rows < 16 || rows % 16 || v0 < 0 ||
+      (long long)v0 + rows > c->vocab)
+    return DFLASH2_ERR_ARG;
+  if (!aligned16(head_shard) || !w) return !w ? DFLASH2_ERR_ARG : DFLASH2_ERR_ALIGN;
+  // a shard rank reads neither the whole head nor the codebooks: stand their pointers in for the
+  // weight checks (the step never reads them)
+  dflash2_weights ws_w = *w;
+  ws_w.lm_head = ws_w.sel_proj = (const uint16_t*)head_shard;
+  if (!ws_w.cb_a) ws_w.cb_a = (const uint16_t*)head_shard;
+  if (!ws_w.cb_b) ws_w.cb_b = (const uint16_t*)head_shard;
+  const HeadShard hs{(const uint8_t*)head_shard, v0, rows, out_cand_val, out_cand_id, out_z};
+  return draft_step_impl(c, &ws_w, in, kv, batch, nullptr, nullptr, ws, ws_bytes, nullptr, stream, &hs);
+}
+
+int dflash2_select(const dflash2_config* c, const dflash2_weights* w, int32_t batch, int32_t nparts,
+                   const float* cand_val, const int32_t* cand_id, const float* z, const int32_t* block_tokens,
+                   int32_t* out_path, float* out_scores, void* ws, size_t ws_bytes, void* stream) {
+  if (!cfg_ok(c)) return DFLASH2_ERR_SHAPE;
+  if (!w || !w->cb_a || !w->cb_b || !cand_val || !cand_id || !z || !block_tokens || !out_path || !out_scores || !ws ||
+      batch < 1 || nparts < 1 || nparts > 256)
+    return DFLASH2_ERR_ARG;
+  if ((uintptr_t)ws & 255u) return DFLASH2_ERR_ALIGN;
+  const Plan P = make_plan(c, batch);
+  if (ws_bytes < P.step_bytes) return DFLASH2_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  int* err = at<int>(ws, P.off_err);
+  int* ctr = at<int>(ws, P.off_ctr);
+  CK(cudaMemsetAsync(err, 0, 4, s));
+  CK(cudaMemsetAsync(ctr + P.ctr_sel, 0, (size_t)batch * 4, s));
+  SelParams sp{};
+  sp.cand_val = cand_val;
+  sp.cand_id = cand_id;
+  sp.nparts = nparts;
+  sp.rows_total = P.lm_rows;
+  sp.z = z;
+  sp.R = P.R;
+  sp.V = P.V;
+  sp.Bk = P.Bk;
+  sp.cb_a = w->cb_a;
+  sp.cb_b = w->cb_b;
+  sp.block_tokens = block_tokens;
+  sp.out_path = out_path;
+  sp.out_scores = out_scores;
+  sp.seq_len = nullptr;  // advanced by each shard's step
+  sp.err = err;
+  static std::atomic<int> sel_attr[kMaxDevices];
+  CK(smem_optin(k_sel_tau, kSelSpreadSmem, sel_attr));
+  CK(launch_pdl(k_sel_tau, dim3(P.D, batch), dim3(256), kSelSpreadSmem, s, sp, at<float>(ws, P.off_tau),
+                at<float>(ws, P.off_cfv), at<int32_t>(ws, P.off_cfi), ctr + P.ctr_sel));
   return DFLASH2_OK;
 }
 

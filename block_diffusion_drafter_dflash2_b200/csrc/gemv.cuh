@@ -67,25 +67,39 @@ DEVI float2 rope_cs(long long pos, int j, double log2_theta) {
 // Per 32-wide sub-block j: S = sum (128 + q) x by mma on the codes with the 0x4300 exponent
 // (bf16 128 + q exactly), X = sum x by an mma with all-ones weights, then
 // y += D*S - M*X with D = d*sc_j, M = dmin*m_j + 128*D.
+// The 16-byte scale record of a feature row per 256-wide K unit: Q4_K's canonical record (d, dmin,
+// 6-bit scales and mins), or for MLX 4-bit group-64 weights (mlx) four (scale, bias) bf16 pairs,
+// one per 64-wide group: word g = scale | bias << 16, weight = scale * q + bias.
 template <int NT>
 DEVI void q4_unit(const uint4 (&q)[4], const uint4 sc, float2* coef, const uint8_t* Xs, int stride, int kbyte,
-                  int ntact, float (&acc)[NT][4], int lane) {
+                  int ntact, float (&acc)[NT][4], int lane, bool mlx) {
   const int g = lane >> 2, t = lane & 3;
   // A = 1.0 in every slot: the mma then yields X_j = sum_k x_k (bf16 x, fp32 accumulate) per row
   const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
   {
-    // lane decodes (d*sc_j, dmin*m_j + 128*d*sc_j) of feature lane/2, sub-blocks 4*(lane&1) .. +3
+    // lane decodes (D_j, M_j) with weight = D_j * (128 + q) - M_j of feature lane/2, sub-blocks
+    // 4*(lane&1) .. +3: Q4_K D = d*sc_j, M = dmin*m_j + 128*D; MLX D = scale, M = 128*scale - bias
     const int f = lane >> 1, jb = (lane & 1) * 4;
-    const float d = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
-    const float dm = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
-    const uint32_t sb = (lane & 1) ? ((sc.y >> 24) | ((sc.z & 0xffffu) << 8)) : (sc.y & 0xffffffu);
-    const uint32_t mb = (lane & 1) ? (sc.w >> 8) : ((sc.z >> 16) | ((sc.w & 0xffu) << 16));
     __syncwarp();
+    if (mlx) {
+      const uint32_t w0 = (lane & 1) ? sc.z : sc.x, w1 = (lane & 1) ? sc.w : sc.y;  // groups jb/2, jb/2 + 1
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float D = d * (float)((sb >> (6 * i)) & 63u);
-      const float M = fmaf(128.f, D, dm * (float)((mb >> (6 * i)) & 63u));
-      coef[(jb + i) * 16 + f] = make_float2(D, M);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t wg = i < 2 ? w0 : w1;
+        const float D = bf2f((uint16_t)(wg & 0xffffu)), B = bf2f((uint16_t)(wg >> 16));
+        coef[(jb + i) * 16 + f] = make_float2(D, fmaf(128.f, D, -B));
+      }
+    } else {
+      const float d = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
+      const float dm = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
+      const uint32_t sb = (lane & 1) ? ((sc.y >> 24) | ((sc.z & 0xffffu) << 8)) : (sc.y & 0xffffffu);
+      const uint32_t mb = (lane & 1) ? (sc.w >> 8) : ((sc.z >> 16) | ((sc.w & 0xffu) << 16));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float D = d * (float)((sb >> (6 * i)) & 63u);
+        const float M = fmaf(128.f, D, dm * (float)((mb >> (6 * i)) & 63u));
+        coef[(jb + i) * 16 + f] = make_float2(D, M);
+      }
     }
     __syncwarp();
   }
@@ -274,6 +288,66 @@ __global__ void k_q4k_prepare(const uint8_t* __restrict__ src, uint8_t* __restri
   if (lane < 16) {
     const uint8_t* b = src + ((size_t)(T * 16 + lane) * nsb + s) * 144;
     for (int i = 0; i < 16; ++i) out[2048 + lane * 16 + i] = b[i];
+  }
+}
+
+// MLX 4-bit group-64 rows (per group of 64: 32 bytes of codes, low nibble first, then the bf16
+// scale and bias) -> the same prepared records as Q4_K: the codes in mma fragment order and, per
+// feature row, a 16-byte record of the unit's four (scale, bias) pairs.
+__global__ void k_mlx4_prepare(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K, PrepPlace pl) {
+  const int nsb = K / kUnit, ng = K / 64, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x;
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* rg = src + (size_t)(T * 16 + g) * ng * 36;
+  const uint8_t* rh = src + (size_t)(T * 16 + g + 8) * ng * 36;
+  auto q = [&](const uint8_t* row, int e) -> uint32_t {
+    const int k = s * kUnit + e;
+    const uint32_t v = row[(k >> 6) * 36 + ((k & 63) >> 1)];
+    return (k & 1) ? (v >> 4) : (v & 15u);
+  };
+  uint32_t w[8][2];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e = 32 * j + 8 * t + 4 * h;
+      w[j][h] = q(rg, e) | (q(rh, e) << 4) | (q(rg, e + 2) << 8) | (q(rh, e + 2) << 12) | (q(rg, e + 1) << 16) |
+                (q(rh, e + 1) << 20) | (q(rg, e + 3) << 24) | (q(rh, e + 3) << 28);
+    }
+  uint8_t* out = dst + prep_offset(pl, T, s, nsb, kQ4Bytes);
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    reinterpret_cast<uint4*>(out)[p * 32 + lane] = make_uint4(w[2 * p][0], w[2 * p][1], w[2 * p + 1][0], w[2 * p + 1][1]);
+  if (lane < 16) {
+    const uint8_t* row = src + (size_t)(T * 16 + lane) * ng * 36;
+    uint32_t r[4];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+      const uint8_t* gp = row + (size_t)(s * 4 + gi) * 36 + 32;
+      r[gi] = (uint32_t)gp[0] | ((uint32_t)gp[1] << 8) | ((uint32_t)gp[2] << 16) | ((uint32_t)gp[3] << 24);
+    }
+    *reinterpret_cast<uint4*>(out + 2048 + lane * 16) = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+// Q8_0 rows (blocks of 32: fp16 d, 32 signed codes) -> the prepared bf16 records: each weight d*q
+// (exact in fp32) rounded once to bf16; the step then streams them as bf16 weights.
+__global__ void k_q80_prepare(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int N, int K, PrepPlace pl) {
+  const int S = K / 64, nb = K / 32, s = blockIdx.x, T = blockIdx.y, lane = threadIdx.x, g = lane >> 2, t = lane & 3;
+  uint8_t* out = dst + prep_offset(pl, T, s, S, 2048);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint8_t* blk = src + ((size_t)(T * 16 + g + 8 * h) * nb + (size_t)s * 2 + j) * 34;
+      const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+      uint32_t r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = t * 8 + 2 * i;
+        r[i] = pack_bf2(d * (float)(int8_t)blk[2 + k], d * (float)(int8_t)blk[3 + k]);
+      }
+      *reinterpret_cast<uint4*>(out + j * 1024 + h * 512 + lane * 16) = make_uint4(r[0], r[1], r[2], r[3]);
+    }
   }
 }
 

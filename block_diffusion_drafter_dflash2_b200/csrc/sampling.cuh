@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(kSampThreads) k_accept_sampled(const int32_t* 
     int n = 0;
     while (n < D) {
       const int d = draft[(size_t)b * D + n];
+      if (d < 0 || d >= V) break;  // outside the vocabulary: probability 0, rejected (never used as an index)
       const float* pr = p + ((size_t)b * Bk + n) * V;
       const double qd = q ? (double)flush32(q[((size_t)b * D + n) * V + d]) : 1.0;
       if ((double)flush32(u_acc[(size_t)b * D + n]) * qd < (double)flush32(pr[d])) ++n;

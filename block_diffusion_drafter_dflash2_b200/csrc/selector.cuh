@@ -347,7 +347,7 @@ DEVI void selector_viterbi(const SelParams& p, int b, const float* cl, const int
     }
     jj = prev;
   }
-  if (lane == 0) p.seq_len[b] += p.n_new[b];
+  if (lane == 0 && p.seq_len) p.seq_len[b] += p.n_new[b];
 }
 
 // Final candidates of row (b, t) from the CTA lists into cl/cand (shared), ids outside [0, V)
@@ -431,6 +431,27 @@ __global__ void __launch_bounds__(256) k_sel_tau(SelParams p, float* tau_g, floa
   }
   __syncthreads();
   if (warp == 0) selector_viterbi<true>(p, b, cl_s, cd_s, tau_s);
+}
+
+// A vocabulary shard's local candidates: the final top-16 of each row from the head CTAs' lists
+// (`nparts` sorted lists [part][rows][16]) into out_v/out_id [rows][16], one warp per row; the
+// selector that would advance seq_len runs on another rank, so this kernel advances it
+// (seq_len[b] += n_new[b]).
+__global__ void __launch_bounds__(128) k_merge_rows(const float* __restrict__ cv, const int32_t* __restrict__ ci,
+                                                    int nparts, int rows, float* __restrict__ out_v,
+                                                    int32_t* __restrict__ out_id, int32_t* __restrict__ seq_len,
+                                                    const int32_t* __restrict__ n_new, int B) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __align__(16) float sv[4][512];
+  __shared__ __align__(16) int si[4][512];
+  __shared__ int surv[4];
+  const int warp = threadIdx.x >> 5, row = blockIdx.x * 4 + warp;
+  if (row < rows)
+    merge_lists_row(cv, ci, nparts, rows, row, sv[warp], si[warp], 512, &surv[warp], out_v + (size_t)row * kTopK,
+                    out_id + (size_t)row * kTopK);
+  if (blockIdx.x == 0 && seq_len)
+    for (int b = threadIdx.x; b < B; b += blockDim.x) seq_len[b] += n_new[b];
 }
 
 }  // namespace dfl

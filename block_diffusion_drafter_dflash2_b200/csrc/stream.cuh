@@ -105,6 +105,9 @@ struct SGemvParams {
   uint16_t* dyn_y;  // bf16 [rows][rs_H]
   int Bk;
   int* err;
+  // tensor-core path: the row scales of rs_in, computed once per product by its kernel, [rows]
+  float* rs_glob;
+  int mlx;  // 4-bit records carry MLX group-64 (scale, bias) pairs instead of Q4_K scale records
 };
 
 // Row scales of rows [mz, mz + rows) from quarter-column sums of squares (ssp layout
@@ -237,7 +240,8 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     // the convolution's x_{t-1} of the group's first row may be the previous row group's last
     const int pre = p.epi == EPI_DYNCONV && mz > 0 ? 1 : 0;
     if (p.rs_in) {
-      if (rs_pre && mz == 0) rsv = rs_pre;
+      if (p.rs_glob) rsv = p.rs_glob + (mz - pre);
+      else if (rs_pre && mz == 0) rsv = rs_pre;
       else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
     }
     // two outputs per thread per round: all their partial loads are in flight together
@@ -309,7 +313,8 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
   const int col0 = p.seg[si].out_col + tile0 * 16;
   const int rows = sk_rows(p, si, mz, R);
   if (p.rs_in && p.epi == EPI_STORE) {
-    if (rs_pre && mz == 0) rsv = rs_pre;
+    if (p.rs_glob) rsv = p.rs_glob + mz;
+    else if (rs_pre && mz == 0) rsv = rs_pre;
     else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
   }
   if (p.epi == EPI_QKV) {
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kSGemvThreads, 1) k_sgemv(SGemvParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) q[i] = lds_slot(sb + (i * 32 + lane) * 16);
             const uint4 sc = lds_slot(sb + 2048 + (lane >> 1) * 16);
-            q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane);
+            q4_unit<NT>(q, sc, coef, Xs, stride, (u - base) * 512, ntact, acc, lane, p.mlx != 0);
             slot_release(&empty[slot], q[0].x ^ q[1].x ^ q[2].x ^ q[3].x ^ sc.x, lane);
           } else {
             uint4 wv[4];
@@ -689,6 +694,7 @@ struct SLmParams {
   float* part;        // split records' partial accumulators [groups][parts][2][16 warps][32 lanes][4]
   int* counters;      // [groups][records] arrival tickets, zero before the launch (the last arrival re-zeroes)
   int* err;
+  int id0;            // vocabulary id of the head's first row (a shard of the vocabulary; 0 for the whole head)
 };
 
 constexpr int kHeadSlot = kHeadTiles * 2048;  // one record step: 32 KB
@@ -827,7 +833,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_slmhead(SLmParams p) {
         if (r < rows) p.z[(size_t)(row0 + r) * p.R + c0 + g + 8 * (e >> 1)] = acc[0][e];
       }
     } else {
-      offer_tile(my, acc[0], tile * 16, rows, lane);
+      offer_tile(my, acc[0], p.id0 + tile * 16, rows, lane);
     }
   }
   consumers_sync<NC>();

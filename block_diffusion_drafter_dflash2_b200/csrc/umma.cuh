@@ -32,12 +32,14 @@
 namespace dfl {
 
 constexpr int kUmmaRows = 256;                     // activation rows per tile (MMA N)
-constexpr int kUmmaStages = 4;
+constexpr int kUmmaStages = 3;                     // operand stages (64-wide K)
+constexpr int kUmmaRaw = 3;                        // raw weight-record slots (one prepared K unit each)
 constexpr int kUmmaABytes = 128 * 128;             // [128 features][64 k] bf16
 constexpr int kUmmaBBytes = kUmmaRows * 128;       // [256 rows][64 k] bf16
-constexpr int kUmmaThreads = 256;
-constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + 1024;  // + alignment slack
-constexpr int kUmmaTmemCols = 256;
+constexpr int kUmmaRawBytes = 8 * kQ4Bytes;        // one group unit (Q4_K 18 KB; bf16 units are 16 KB)
+constexpr int kUmmaThreads = 384;                  // 12 warps: roles below
+constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + kUmmaRaw * kUmmaRawBytes + 1024;
+constexpr int kUmmaTmemCols = 512;                 // two 256-column accumulators
 
 // ---- tcgen05 / TMA wrappers (one instruction each) ----
 DEVI void tmem_alloc(uint32_t* dst_smem, int cols) {
@@ -141,26 +143,52 @@ DEVI uint4 q4_chunk(uint32_t w0, uint32_t w1, int rs, float2 dc) {
   return make_uint4(q4_pair(a, dc), q4_pair(b, dc), q4_pair(c, dc), q4_pair(d, dc));
 }
 
+// Row scales 1/sqrt(mean(h^2) + eps) of rows [r0, r1) from quarter-column sums of squares
+// (layout [H/128][4][ldr]) into rs[row]; one warp.
+DEVI void rows_scale_global(const float* ssp, int ldr, int H, float eps, int r0, int r1, float* rs) {
+  const int lane = threadIdx.x & 31, nq = (H >> 7) * 4;
+  for (int r = r0; r < r1; ++r) {
+    float q = 0.f;
+    for (int i = lane; i < nq; i += 32) q += __ldcg(ssp + (size_t)i * ldr + r);
+    q = warp_sum(q);
+    if (lane == 0) rs[r] = rsqrtf(q / H + eps);
+  }
+}
+
+// Roles (12 warps): warp 0 one thread: activation TMA; warp 1: TMEM allocation, one thread issues
+// the MMAs; warp 2 one thread: raw weight records into the raw ring (bulk copies, started before
+// the dependency wait: the weights do not depend on earlier kernels); warp 3: the row scales of
+// a folded RMSNorm for the fix-up (p.rs_glob); warps 4-7: weight operand from the raw ring;
+// warps 8-11: epilogue (TMEM lane = feature), on two accumulators alternating by piece.
 template <bool Q4>
 __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t xfull[kUmmaStages], afull[kUmmaStages], sempty[kUmmaStages];
-  __shared__ __align__(8) uint64_t accfull, accempty;
+  __shared__ __align__(8) uint64_t rfull[kUmmaRaw], rempty[kUmmaRaw];
+  __shared__ __align__(8) uint64_t accfull[2], accempty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* As = smem;                              // [stages][128 x 128 B]
-  uint8_t* Bs = smem + kUmmaStages * kUmmaABytes;  // [stages][256 x 128 B]
+  uint8_t* As = smem;                                   // [stages][128 x 128 B]
+  uint8_t* Bs = As + kUmmaStages * kUmmaABytes;         // [stages][256 x 128 B]
+  uint8_t* Rs = Bs + kUmmaStages * kUmmaBBytes;         // [raw slots][group unit]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kSub = Q4 ? 4 : 1;  // 64-wide stages per prepared K unit
   constexpr int kUnitK = Q4 ? 256 : 64;
+  constexpr int kRawUnit = Ring<Q4>::kSlot;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUmmaStages; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&afull[s], 4);
       mbar_init(&sempty[s], 1);
     }
-    mbar_init(&accfull, 1);
-    mbar_init(&accempty, 4);
+    for (int r = 0; r < kUmmaRaw; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -211,8 +239,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
         int si;
         sk_tile(p, grp, 0, si);
         if (sk_rows(p, si, mz, kUmmaRows) > 0) {
-          if (piece > 0 && !wait_or_die(&accempty, (piece - 1) & 1, dead, p.err)) break;
+          const int buf = piece & 1, use = piece >> 1;
+          if (use > 0 && !wait_or_die(&accempty[buf], (use - 1) & 1, dead, p.err)) break;
           tc_fence_after();
+          const uint32_t acc = tmem + (uint32_t)(buf * kUmmaRows);
           bool first = true;
           for (int u = ua; u < ub && !dead; ++u)
             for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
@@ -224,21 +254,51 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
               const uint64_t bd = sw128_desc(smem_u32(Bs + s * kUmmaBBytes));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes inside the swizzled rows
-                tc_mma(tmem, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (first && kk == 0) ? 0u : 1u);
+                tc_mma(acc, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (first && kk == 0) ? 0u : 1u);
               first = false;
               tc_commit(&sempty[s]);  // the stage is free once these MMAs have read it
             }
-          if (!dead) tc_commit(&accfull);  // the piece's accumulator is complete
+          if (!dead) tc_commit(&accfull[buf]);  // the piece's accumulator is complete
           ++piece;
         }
         x += ub - ua;
       }
     }
-  } else if (warp >= 4) {
-    // ---- weight producers, then the piece epilogue ----
+  } else if (warp == 2) {
+    // ---- raw weight records (bulk copies; before the dependency wait) ----
+    if (lane == 0) {
+      bool dead = false;
+      int cnt = 0;
+      for (long long x = x0; x < x1 && !dead;) {
+        const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
+        const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        int si;
+        sk_tile(p, grp, 0, si);
+        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
+          const uint8_t* src = sk_group_src<Q4>(p, grp);
+          for (int u = ua; u < ub && !dead; ++u, ++cnt) {
+            const int r = cnt % kUmmaRaw, round = cnt / kUmmaRaw;
+            if (round > 0 && !wait_or_die(&rempty[r], (round - 1) & 1, dead, p.err)) break;
+            mbar_expect_tx(&rfull[r], kRawUnit);
+            bulk_g2s(Rs + r * kUmmaRawBytes, src + (size_t)u * kRawUnit, kRawUnit, &rfull[r]);
+          }
+        }
+        x += ub - ua;
+      }
+    }
+  } else if (warp == 3) {
+    // ---- row scales of a folded RMSNorm for the fix-up (rows split over the CTAs) ----
+    if (p.rs_glob) {
+      pdl_wait();  // the sums of squares come from the previous product's epilogue
+      const int r0 = (int)(c * p.rows / P), r1 = (int)((c + 1) * p.rows / P);
+      rows_scale_global(p.rs_in, p.ssp_rows, p.rs_H, p.eps, r0, r1, p.rs_glob);
+    }
+  } else if (warp < 8) {
+    // ---- weight operand: raw ring -> swizzled K-major stage ----
     const int dw = warp - 4, g = lane >> 2, t = lane & 3;
-    bool dead = false, waited = false;
-    int cnt = 0, piece = 0;
+    bool dead = false;
+    int cnt = 0, ucnt = 0;
     for (long long x = x0; x < x1;) {
       const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
       const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
@@ -246,19 +306,27 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
       int si0;
       sk_tile(p, grp, 0, si0);
       if (sk_rows(p, si0, mz, kUmmaRows) > 0) {
-        const uint8_t* src = sk_group_src<Q4>(p, grp);
-        for (int u = ua; u < ub; ++u) {
-          const uint8_t* rec[2];
-          uint4 code[2][kSub], scl[2][2];
+        for (int u = ua; u < ub; ++u, ++ucnt) {
+          const int r = ucnt % kUmmaRaw;
+          wait_or_die(&rfull[r], (ucnt / kUmmaRaw) & 1, dead, p.err);
+          const uint8_t* raw = Rs + r * kUmmaRawBytes;
+          // 4-bit records: this lane's scale records (rows g, g+8 of its two tiles), decoded once per
+          // unit (Q4_K: d, dmin and the packed 6-bit fields; MLX: the record's four bf16 pairs)
+          float dd[2][2], dm[2][2];
+          unsigned long long scp[2][2], mp[2][2];
+          uint4 mrec[2][2];
+          if (Q4 && !dead) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            rec[h] = src + (size_t)u * Ring<Q4>::kSlot + (size_t)(2 * dw + h) * Ring<Q4>::kUnitBytes;
-            if (Q4) {  // the unit's codes and the scale records of rows g, g+8 of this warp's tiles
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int q = 0; q < kSub; ++q) code[h][q] = ldg_stream(rec[h] + (q * 32 + lane) * 16);
-              scl[h][0] = __ldg(reinterpret_cast<const uint4*>(rec[h] + 2048 + g * 16));
-              scl[h][1] = __ldg(reinterpret_cast<const uint4*>(rec[h] + 2048 + (g + 8) * 16));
-            }
+              for (int e = 0; e < 2; ++e) {
+                const uint4 sc = *reinterpret_cast<const uint4*>(raw + (2 * dw + h) * kQ4Bytes + 2048 + (g + 8 * e) * 16);
+                mrec[h][e] = sc;
+                dd[h][e] = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
+                dm[h][e] = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
+                scp[h][e] = (unsigned long long)sc.y | ((unsigned long long)(sc.z & 0xffffu) << 32);
+                mp[h][e] = (unsigned long long)(sc.z >> 16) | ((unsigned long long)sc.w << 16);
+              }
           }
 #pragma unroll
           for (int sub = 0; sub < kSub; ++sub, ++cnt) {
@@ -268,18 +336,34 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
             if (!dead) {
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const int m0 = (2 * dw + h) * 16 + g;  // operand rows g and g+8 of tile 2*dw+h
+                const int tl = 2 * dw + h, m0 = tl * 16 + g;  // operand rows g and g+8 of tile tl
+                const uint8_t* rec = raw + tl * (Q4 ? kQ4Bytes : 2048);
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {  // 32-wide sub-blocks of the stage
                   uint4 rg, rh;
                   if (Q4) {
-                    const uint4 q = code[h][sub];
+                    const uint4 q = *reinterpret_cast<const uint4*>(rec + (sub * 32 + lane) * 16);
                     const uint32_t w0 = jj ? q.z : q.x, w1 = jj ? q.w : q.y;
-                    rg = q4_chunk(w0, w1, 0, q4_scale_dc(scl[h][0], 2 * sub + jj));
-                    rh = q4_chunk(w0, w1, 4, q4_scale_dc(scl[h][1], 2 * sub + jj));
+                    const int j = 2 * sub + jj;
+                    float2 dc[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                      if (p.mlx) {  // group j/2: w = scale*q + bias = (128+q)*scale + (bias - 128*scale)
+                        const uint4 r = mrec[h][e];
+                        const uint32_t wg = (j >> 1) == 0 ? r.x : (j >> 1) == 1 ? r.y : (j >> 1) == 2 ? r.z : r.w;
+                        const float D = bf2f((uint16_t)(wg & 0xffffu)), B = bf2f((uint16_t)(wg >> 16));
+                        dc[e] = make_float2(D, fmaf(-128.f, D, B));
+                      } else {
+                        const float D = dd[h][e] * (float)((scp[h][e] >> (6 * j)) & 63u);
+                        const float M = dm[h][e] * (float)((mp[h][e] >> (6 * j)) & 63u);
+                        dc[e] = make_float2(D, -fmaf(128.f, D, M));
+                      }
+                    }
+                    rg = q4_chunk(w0, w1, 0, dc[0]);
+                    rh = q4_chunk(w0, w1, 4, dc[1]);
                   } else {  // bf16 record: W[row g][32jj + 8t ..] at jj*1024 + lane*16, row g+8 at +512
-                    rg = ldg_stream(rec[h] + jj * 1024 + lane * 16);
-                    rh = ldg_stream(rec[h] + jj * 1024 + 512 + lane * 16);
+                    rg = *reinterpret_cast<const uint4*>(rec + jj * 1024 + lane * 16);
+                    rh = *reinterpret_cast<const uint4*>(rec + jj * 1024 + 512 + lane * 16);
                   }
                   *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jj + t)) = rg;
                   *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jj + t)) = rh;
@@ -290,24 +374,42 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[s]);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&rempty[r]);  // the raw unit has been read
         }
-        // ---- epilogue of this piece: TMEM -> fp32 partial [piece][row][ldo] ----
+      }
+      x += ub - ua;
+    }
+  } else {
+    // ---- epilogue: TMEM -> fp32 partial [piece][row][ldo], accumulators alternate by piece ----
+    const int ew = warp - 8;  // = warp % 4: TMEM lanes 32*ew ..
+    bool dead = false, waited = false;
+    int piece = 0;
+    for (long long x = x0; x < x1;) {
+      const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
+      const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
+      const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+      int si0;
+      sk_tile(p, grp, 0, si0);
+      if (sk_rows(p, si0, mz, kUmmaRows) > 0) {
         if (!waited) {
           pdl_wait();  // the partial buffer may still be read by the previous product's fix-up
           waited = true;
         }
+        const int buf = piece & 1, use = piece >> 1;
         const int pc = (int)(c - sk_owner((long long)gidx * p.U, p.W, P));
-        if (wait_or_die(&accfull, piece & 1, dead, p.err)) {
+        if (wait_or_die(&accfull[buf], use & 1, dead, p.err)) {
           tc_fence_after();
-          const int m = dw * 32 + lane;  // TMEM lane = feature of the column group
+          const int m = ew * 32 + lane;  // TMEM lane = feature of the column group
           int si;
           const int tile = sk_tile(p, grp, m >> 4, si);
           const int rows = tile >= 0 ? sk_rows(p, si, mz, kUmmaRows) : 0;
           float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mz * p.ldo +
                        (tile >= 0 ? p.seg[si].out_col + tile * 16 + (m & 15) : 0);
+          const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kUmmaRows);
           for (int n0 = 0; n0 < kUmmaRows; n0 += 32) {
             uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)n0, v);
+            tmem_ld32(tbase + (uint32_t)n0, v);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -316,7 +418,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           tc_fence_before();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&accempty);
+        if (lane == 0) mbar_arrive(&accempty[buf]);
         ++piece;
       }
       x += ub - ua;
@@ -331,20 +433,24 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// Output head + top-16 for many drafted rows on the tensor cores.  The prepared head (records of
-// 256 features x 64-wide K steps, the output head followed by the selector projection) is applied
-// to up to 256 rows per CTA: the rows are the MMA's M side (two 128-row accumulators in TMEM, 512
-// columns), the 256 features of a record its N side, so after a record each thread holds one
-// row's 256 logits and offers them to that row's top-16 list, kept sorted in its registers.
+// Output head + top-16 for many drafted rows on the tensor cores.  The head ([V + R] rows: the
+// output head, then the selector projection) has a second prepared copy in the tcgen05 operand
+// layout: record rec, K step st (256 features x 64 k bf16, 32 KB) at ((rec * S + st) * 32 KB),
+// feature f's 16-byte chunk c (k = 8c ..) at f * 128 + ((c ^ (f % 8)) * 16) (128-byte swizzle,
+// K-major), so one bulk copy lands it as the MMA's B operand.  The rows are the M side (two
+// 128-row accumulators in TMEM, 512 columns), the 256 features of a record the N side, so after a
+// record each thread holds one row's 256 logits and offers them to that row's top-16, kept sorted
+// in its registers.
 //  * warp 0, one thread: TMA of the rows' [256][64] bf16 slice per K step (no multicast);
-//  * warps 4-7: permute the record's 32 KB step (the streaming head's fragment order) into the
-//    128-byte-swizzled K-major operand, then run the epilogue of each record;
-//  * warp 1: TMEM allocation and the MMA issue (2 x 4 per K step), commits.
+//  * warp 2, one thread: bulk copy of the record step (weights: before the dependency wait);
+//  * warp 1: TMEM allocation and the MMA issue (2 x 4 per K step), commits;
+//  * warps 4-7: the per-record top-16 epilogue.
 // CTA c works on row tile c % nrt and on records c / nrt, c / nrt + P / nrt, ...; its lists are
 // part c / nrt of the candidate lists ([P / nrt][rows][16]) that the selector merges.
 struct UHeadParams {
-  const uint8_t* W;  // prepared [lm_head; sel_proj] records
+  const uint8_t* Wsw;  // swizzled head records
   int V, R, H, rows, nrec, nrt;
+  int id0;             // vocabulary id of the head's first row (a shard of the vocabulary; 0 for the whole head)
   float* z;           // [rows][R]
   float* cand_val;    // [parts][rows][16]
   int32_t* cand_id;
@@ -354,6 +460,20 @@ struct UHeadParams {
 constexpr int kUHeadStages = 3;
 constexpr int kUHeadStage = 2 * 32768;  // A: 256 rows x 128 B, B: 256 features x 128 B
 constexpr int kUHeadSmem = kUHeadStages * kUHeadStage + 1024;
+
+// Canonical bf16 head rows -> the swizzled operand copy (one CTA of 256 threads per record step).
+__global__ void k_head_sw_prepare(const uint16_t* __restrict__ lm_head, const uint16_t* __restrict__ sel_proj,
+                                  uint8_t* __restrict__ dst, int V, int R, int H) {
+  const int S = H / 64, st = blockIdx.x, rec = blockIdx.y, f = threadIdx.x;
+  const int row = rec * 256 + f;
+  const uint16_t* src = row < V ? lm_head + (size_t)row * H : (row < V + R ? sel_proj + (size_t)(row - V) * H : nullptr);
+  uint8_t* out = dst + ((size_t)rec * S + st) * 32768 + (size_t)f * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = src ? *reinterpret_cast<const uint4*>(src + (size_t)st * 64 + 8 * c) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(out + ((c ^ (f & 7)) << 4)) = v;
+  }
+}
 
 // Insert (v, id) into a sorted 16-entry list held in registers (best first; the caller has checked
 // that it beats the last entry): it replaces the last entry and bubbles up.
@@ -387,7 +507,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUHeadStages; ++s) {
       mbar_init(&xfull[s], 1);
-      mbar_init(&bfull[s], 4);
+      mbar_init(&bfull[s], 1);
       mbar_init(&sempty[s], 1);
     }
     mbar_init(&accfull, 1);
@@ -404,17 +524,24 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
   const uint32_t tmem = tmem_base_sh;
   pdl_trigger();
 
-  if (warp == 0) {
-    if (lane == 0) {  // ---- activation rows (TMA) ----
-      pdl_wait();
+  if (warp == 0 || warp == 2) {
+    if (lane == 0) {  // ---- warp 0: activation rows (TMA); warp 2: weight record steps (bulk) ----
+      const bool act = warp == 0;
+      if (act) pdl_wait();
       bool dead = false;
       int cnt = 0;
       for (int rec = part; rec < p.nrec && !dead; rec += nparts)
         for (int st = 0; st < S && !dead; ++st, ++cnt) {
           const int s = cnt % kUHeadStages, round = cnt / kUHeadStages;
           if (round > 0 && !wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err)) break;
-          mbar_expect_tx(&xfull[s], 32768);
-          tma_load_2d(smem + s * kUHeadStage, &tmx, st * 64, row0, &xfull[s]);
+          uint8_t* stage = smem + s * kUHeadStage;
+          if (act) {
+            mbar_expect_tx(&xfull[s], 32768);
+            tma_load_2d(stage, &tmx, st * 64, row0, &xfull[s]);
+          } else {
+            mbar_expect_tx(&bfull[s], 32768);
+            bulk_g2s(stage + 32768, p.Wsw + ((size_t)rec * S + st) * 32768, 32768, &bfull[s]);
+          }
         }
     }
   } else if (warp == 1) {
@@ -442,9 +569,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
         if (!dead) tc_commit(&accfull);
       }
     }
-  } else if (warp >= 4) {
-    // ---- weight permutation, then the per-record top-16 epilogue ----
-    const int dw = warp - 4, g = lane >> 2, t = lane & 3;
+  } else if (warp >= 4 && warp < 8) {
+    // ---- per-record top-16 epilogue: thread = row (TMEM lane 32*dw + lane of each accumulator) ----
+    const int dw = warp - 4;
     float lv[2][16];
     int li[2][16];
 #pragma unroll
@@ -454,40 +581,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
         lv[mc][k] = -INFINITY;
         li[mc][k] = 0x7fffffff;
       }
-    bool dead = false, waited = false;
-    int cnt = 0, it = 0;
+    bool dead = false;
+    int it = 0;
+    pdl_wait();  // (outputs; the dependency also orders the lists after the previous step's readers)
     for (int rec = part; rec < p.nrec; rec += nparts, ++it) {
-      for (int st = 0; st < S; ++st, ++cnt) {
-        const int s = cnt % kUHeadStages, round = cnt / kUHeadStages;
-        if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
-        uint8_t* b = smem + s * kUHeadStage + 32768;
-        if (!dead) {
-          const uint8_t* src = p.W + ((size_t)rec * S + st) * (size_t)kHeadSlot;
-          uint4 v[4][4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h)  // tiles 4*dw + h of the record: all loads first
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              v[h][q] = ldg_stream(src + (size_t)(4 * dw + h) * 2048 + (q >> 1) * 1024 + (q & 1) * 512 + lane * 16);
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int m0 = (4 * dw + h) * 16 + g;
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              *reinterpret_cast<uint4*>(b + sw128_off(m0, 4 * jj + t)) = v[h][2 * jj];
-              *reinterpret_cast<uint4*>(b + sw128_off(m0 + 8, 4 * jj + t)) = v[h][2 * jj + 1];
-            }
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bfull[s]);
-      }
-      // ---- epilogue: thread = row (TMEM lane 32*dw + lane of each accumulator) ----
-      if (!waited) {
-        pdl_wait();
-        waited = true;
-      }
       if (wait_or_die(&accfull, it & 1, dead, p.err)) {
         tc_fence_after();
 #pragma unroll
@@ -500,14 +597,23 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
             tmem_ld_wait();
             if (rl < trows) {
               const int f0 = rec * 256 + n0;
+              if (f0 + 32 <= p.V) {
+                const int g0 = f0 + p.id0;  // vocabulary id of feature f0
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(r[i]);
-                const int f = f0 + i;
-                if (f < p.V) {
-                  if (better(x, f, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, f);
-                } else if (f < p.V + p.R) {
-                  p.z[(size_t)row * p.R + (f - p.V)] = x;
+                for (int i = 0; i < 32; ++i) {
+                  const float x = __uint_as_float(r[i]);
+                  if (better(x, g0 + i, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, g0 + i);
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const float x = __uint_as_float(r[i]);
+                  const int f = f0 + i;
+                  if (f < p.V) {
+                    if (better(x, f + p.id0, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, f + p.id0);
+                  } else if (f < p.V + p.R) {
+                    p.z[(size_t)row * p.R + (f - p.V)] = x;
+                  }
                 }
               }
             }

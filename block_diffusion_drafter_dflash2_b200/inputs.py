@@ -53,7 +53,7 @@ class Dims:
     page_size: int = 16
     rope_theta: float = 1.0e6
     rms_eps: float = 1.0e-6
-    wfmt: int = 0  # layer + fc matrices: 0 = Q4_K, 1 = bf16
+    wfmt: int = 0  # layer + fc matrices: 0 = Q4_K, 1 = bf16, 2 = MLX 4-bit group-64, 3 = Q8_0
 
     @property
     def drafted(self) -> int:
@@ -102,6 +102,9 @@ WORKLOADS: Dict[str, Workload] = {
     # profiling case: full layer shapes, one layer, a 65536-token vocabulary (about 1.7 GB on the device)
     "prof_small": Workload("prof_small", dataclasses.replace(FULL, layers=1, vocab=65536), 1, 4096, 4096, False, False,
                            False, "first_mismatch", 1006, "profiling case: 1 full-shape layer, vocab 65536"),
+    # the same for 64 requests (the tensor-core products and head), about 2.5 GB on the device
+    "prof_b64": Workload("prof_b64", dataclasses.replace(FULL, layers=1, vocab=65536), 64, 512, 4096, False, False,
+                         False, "first_mismatch", 1007, "profiling case: 1 full-shape layer, vocab 65536, 64 requests"),
 }
 
 
@@ -168,17 +171,66 @@ def quantize_q4k(w: torch.Tensor) -> torch.Tensor:
     return out.reshape(n, nb * Q4K_BLOCK_BYTES)
 
 
+def quantize_mlx4(w: torch.Tensor) -> torch.Tensor:
+    """fp32 [N, K] -> uint8 [N, K/64*36]: MLX-style 4-bit groups of 64 (the MLX sidecar card ships
+    4-bit group-64 weights).  Per group: 32 bytes of codes (element e at byte e/2, low nibble
+    first), then the bf16 scale and bias; weight = scale * q + bias.  Scale (max - min)/15 and bias
+    = min, both rounded to bf16 first; codes by round-half-even of (w - bias)/scale, clamped."""
+    assert w.dim() == 2 and w.shape[1] % 64 == 0
+    n, k = w.shape
+    x = w.float().reshape(n, k // 64, 64)
+    mn, mx = x.amin(-1), x.amax(-1)
+    sc = ((mx - mn) / 15.0).to(torch.bfloat16)
+    bi = mn.to(torch.bfloat16)
+    scf, bif = sc.float().unsqueeze(-1), bi.float().unsqueeze(-1)
+    q = torch.where(scf > 0, torch.round((x - bif) / torch.where(scf > 0, scf, torch.ones_like(scf))),
+                    torch.zeros_like(x)).clamp(0, 15).to(torch.int32)
+    out = torch.empty((n, k // 64, 36), dtype=torch.uint8, device=w.device)
+    out[..., :32] = (q[..., 0::2] | (q[..., 1::2] << 4)).to(torch.uint8)
+    sb = sc.view(torch.int16).to(torch.int32) & 0xFFFF
+    bb = bi.view(torch.int16).to(torch.int32) & 0xFFFF
+    out[..., 32] = (sb & 0xFF).to(torch.uint8)
+    out[..., 33] = (sb >> 8).to(torch.uint8)
+    out[..., 34] = (bb & 0xFF).to(torch.uint8)
+    out[..., 35] = (bb >> 8).to(torch.uint8)
+    return out.reshape(n, k // 64 * 36)
+
+
+def quantize_q8_0(w: torch.Tensor) -> torch.Tensor:
+    """fp32 [N, K] -> uint8 [N, K/32*34]: Q8_0 blocks of 32 (the GGUF listing ships Q8_0 files):
+    fp16 d = max|w|/127, then 32 signed codes round-half-even(w/d) clamped to [-127, 127]."""
+    assert w.dim() == 2 and w.shape[1] % 32 == 0
+    n, k = w.shape
+    x = w.float().reshape(n, k // 32, 32)
+    d16 = (x.abs().amax(-1) / 127.0).to(torch.float16)
+    d = d16.float().unsqueeze(-1)
+    q = torch.where(d > 0, torch.round(x / torch.where(d > 0, d, torch.ones_like(d))),
+                    torch.zeros_like(x)).clamp(-127, 127).to(torch.int32)
+    out = torch.empty((n, k // 32, 34), dtype=torch.uint8, device=w.device)
+    db = d16.view(torch.int16).to(torch.int32) & 0xFFFF
+    out[..., 0] = (db & 0xFF).to(torch.uint8)
+    out[..., 1] = (db >> 8).to(torch.uint8)
+    out[..., 2:] = (q & 0xFF).to(torch.uint8)
+    return out.reshape(n, k // 32 * 34)
+
+
+# bytes per row per 256 weights of each storage format of fc and the layer matrices
+FORMAT_BYTES_PER_256 = {0: Q4K_BLOCK_BYTES, 1: 512, 2: 4 * 36, 3: 8 * 34}
+
+
 def _linear(out_f, in_f, dims: Dims, seed, name, device, quantized: bool):
-    """A linear layer [out_f, in_f] with N(0, 0.02) weights, as Q4_K bytes or bf16."""
-    if not quantized:
+    """A linear layer [out_f, in_f] with N(0, 0.02) weights, stored in the format dims.wfmt
+    (0 = Q4_K, 1 = bf16, 2 = MLX 4-bit group-64, 3 = Q8_0)."""
+    if not quantized or dims.wfmt == 1:
         return _normal((out_f, in_f), 0.02, 0.0, seed, name, device)
+    enc = {0: quantize_q4k, 2: quantize_mlx4, 3: quantize_q8_0}[dims.wfmt]
     g = _gen(seed, name, device)
-    out = torch.empty((out_f, in_f // Q4K_BLOCK_ELEMS * Q4K_BLOCK_BYTES), dtype=torch.uint8, device=device)
+    out = torch.empty((out_f, in_f // 256 * FORMAT_BYTES_PER_256[dims.wfmt]), dtype=torch.uint8, device=device)
     step = 2048
     for r0 in range(0, out_f, step):
         r1 = min(out_f, r0 + step)
         w = torch.randn((r1 - r0, in_f), generator=g, device=device, dtype=torch.float32) * 0.02
-        out[r0:r1] = quantize_q4k(w)
+        out[r0:r1] = enc(w)
     return out
 
 
@@ -186,7 +238,7 @@ def make_weights(dims: Dims, seed: int, device="cpu") -> dict:
     """All drafter weights for ``dims``; every tensor has its own seeded stream."""
     H, F, T, R, V = dims.hidden, dims.ffn, dims.n_taps, dims.rank, dims.vocab
     hq, hkv, hd = dims.n_q * dims.head_dim, dims.n_kv * dims.head_dim, dims.head_dim
-    qz = dims.wfmt == 0
+    qz = dims.wfmt != 1
     norm = lambda n, name: _normal((n,), 0.01, 1.0, seed, name, device)
     w = {
         "fc": _linear(H, T * H, dims, seed, "fc", device, qz),

@@ -59,7 +59,13 @@ extern "C" {
  * n_q % n_kv == 0, (n_q / n_kv) * block <= 64, hidden, ffn, n_q*head_dim and
  * n_taps*hidden multiples of 256, vocab and rank multiples of 16, rank <= 256.
  * rope_theta: RoPE base (1e6); rms_eps: RMSNorm epsilon (1e-6).
- * wfmt: storage of fc and the layer matrices, 0 = Q4_K, 1 = bf16. */
+ * wfmt: storage of fc and the layer matrices: 0 = Q4_K; 1 = bf16; 2 = MLX-style 4-bit group-64
+ * (MLX sidecar card, "Contents"): per row, per group of 64 inputs, 32 bytes of 4-bit codes (low
+ * nibble first) then the group's bf16 scale and bias, weight = scale*q + bias (36 bytes per 64
+ * weights); 3 = Q8_0 (Mindket listing, "Good to know"): per block of 32 inputs an fp16 d then 32
+ * signed 8-bit codes, weight = d*q (34 bytes per 32).  The W_dc generators are bf16 in every
+ * format.  Q4_K and MLX weights are decoded inside the products; Q8_0 is decoded when the weights
+ * are prepared (each weight rounded once to bf16) and then streamed as bf16. */
 typedef struct dflash2_config {
   int32_t layers, hidden, ffn, n_q, n_kv, head_dim, window, vocab, n_taps, block, topk, rank,
       page_size;
@@ -146,7 +152,8 @@ typedef struct dflash2_debug {
 size_t dflash2_workspace_size(const dflash2_config *cfg, int32_t batch);
 
 /* Bytes of the prepared weight copy: every streamed matrix (fc, the layer matrices, the
- * dynamic-convolution generators, the output head with the selector projection). */
+ * dynamic-convolution generators, the output head with the selector projection; the head twice:
+ * in the streaming records and in the tensor cores' operand layout used for many drafted rows). */
 size_t dflash2_prepared_size(const dflash2_config *cfg);
 
 /* Repack the streamed matrices of `src` (canonical layouts, device) into `dst`
@@ -157,7 +164,8 @@ size_t dflash2_prepared_size(const dflash2_config *cfg);
  * records of 16 tiles per 64-wide step (32 KB), padded to whole records.  Values are not
  * changed: the prepared copy holds the same bits, reordered.  Fills `out` (host struct)
  * with `src`'s pointers except the streamed matrices, which point into dst (wu aliases
- * wg; lm_head and sel_proj both point at the combined head); out->prepared = 1.  The embedding
+ * wg; lm_head and sel_proj both point at the combined head, whose tensor-core operand copy follows
+ * it: records of 256 features x 64-wide K steps, 32 KB each, 128-byte swizzled); out->prepared = 1.  The embedding
  * table, norms, static taps and codebooks stay where they are.  Asynchronous on `stream`. */
 int dflash2_prepare_weights(const dflash2_config *cfg, const dflash2_weights *src, void *dst,
                             size_t dst_bytes, dflash2_weights *out, void *stream);
@@ -207,6 +215,38 @@ int dflash2_draft_step_static(const dflash2_config *cfg, const dflash2_weights *
 int dflash2_accept(const int32_t *draft, const int32_t *target, int32_t batch, int32_t block,
                    int32_t *accepted, int32_t *emitted, void *stream);
 
+/* The output head sharded by vocabulary across GPUs (one process per GPU), for the latency of a
+ * single request: the head is 69 % of a step's bytes and, like the NPU's separate 8-row head
+ * (FastFlowLM card, "How it is used"), can run apart from the layers.  Every rank holds the
+ * layers; rank r holds head rows [v0, v0 + rows) (and the selector projection).  Each rank runs
+ * dflash2_draft_step_head_shard: the layers, its shard of the head, and its local top-16 per drafted
+ * row (global vocabulary ids, logit descending, smaller id first) into out_cand_val /
+ * out_cand_id [batch*(block-1)][16], the selector projection into out_z
+ * [batch*(block-1)][rank]; it appends the context rows and advances seq_len like
+ * dflash2_draft_step.  The caller exchanges the candidates (an all-gather of [G][rows][16] values
+ * and ids: bytes, not megabytes) and one rank runs dflash2_select on the G gathered lists with the
+ * codebooks, which produces the path and scores exactly as the unsharded step would from the same
+ * candidates.  The codebooks are not sharded: only the 2 x 16 x 7 gathered rows are read per step,
+ * so they cost no bandwidth.
+ *  - dflash2_head_shard_size / dflash2_prepare_head_shard: bytes and preparation of a shard from
+ *    its canonical bf16 rows lm_head_rows [rows][hidden] and sel_proj [rank][hidden] (rows a
+ *    multiple of 16); the prepared shard is what head_shard points to.
+ *  - dflash2_draft_step_head_shard: w's lm_head and sel_proj are not used, its codebooks may be
+ *    NULL; workspace as dflash2_draft_step; 0 <= v0, v0 + rows <= vocab.
+ *  - dflash2_select: nparts (1..256) lists cand_val/cand_id [nparts][batch*(block-1)][16], z from
+ *    any shard, block_tokens [batch][block]; writes out_path / out_scores; does not touch seq_len.
+ * Device pointers; asynchronous on `stream`. */
+size_t dflash2_head_shard_size(const dflash2_config *cfg, int32_t rows);
+int dflash2_prepare_head_shard(const dflash2_config *cfg, const uint16_t *lm_head_rows, int32_t rows,
+                               const uint16_t *sel_proj, void *dst, size_t dst_bytes, void *stream);
+int dflash2_draft_step_head_shard(const dflash2_config *cfg, const dflash2_weights *w, const void *head_shard,
+                                  int32_t v0, int32_t rows, const dflash2_inputs *in, const dflash2_kv *kv,
+                                  int32_t batch, float *out_cand_val, int32_t *out_cand_id, float *out_z,
+                                  void *workspace, size_t ws_bytes, void *stream);
+int dflash2_select(const dflash2_config *cfg, const dflash2_weights *w, int32_t batch, int32_t nparts,
+                   const float *cand_val, const int32_t *cand_id, const float *z, const int32_t *block_tokens,
+                   int32_t *out_path, float *out_scores, void *workspace, size_t ws_bytes, void *stream);
+
 /* Acceptance for sampled decoding by exact rejection sampling (MLX sidecar card, "Contents";
  * Mindket listing, "For newcomers and experts": the target's distribution is preserved).  For
  * each request, in block order: accept drafted token d_i with probability min(1, p_i(d_i) /
@@ -220,7 +260,8 @@ int dflash2_accept(const int32_t *draft, const int32_t *target, int32_t batch, i
  *   probabilities for block position i+1; q_draft fp32 [batch][block-1][vocab], or NULL for the
  *   point mass on the drafted token (the selector's path is deterministic); u_accept fp32
  *   [batch][block-1] uniforms in [0,1); u_sample uint32 [batch] uniform 32-bit integers (the
- *   caller's random numbers: the call draws none).  accepted int32 [batch]; emitted int32
+ *   caller's random numbers: the call draws none).  A drafted id outside [0, vocab) is rejected
+ *   (probability 0) and never used as an index.  accepted int32 [batch]; emitted int32
  *   [batch][block]: the accepted tokens, the sampled token, then -1.  Device pointers;
  *   asynchronous on `stream`. */
 int dflash2_accept_sampled(const int32_t *draft, const float *p_target, const float *q_draft, const float *u_accept,

@@ -134,6 +134,22 @@ def q4k_dequant(blocks) -> np.ndarray:
     return out
 
 
+def mlx4_dequant(groups) -> np.ndarray:
+    b = _np(groups, np.uint8).reshape(-1)
+    assert b.size % 36 == 0
+    out = np.empty(b.size // 36 * 64, np.float64)
+    lib().orc_mlx4_dequant(_p(b), C.c_int64(b.size // 36), _p(out))
+    return out
+
+
+def q8_0_dequant(blocks) -> np.ndarray:
+    b = _np(blocks, np.uint8).reshape(-1)
+    assert b.size % 34 == 0
+    out = np.empty(b.size // 34 * 32, np.float64)
+    lib().orc_q8_0_dequant(_p(b), C.c_int64(b.size // 34), _p(out))
+    return out
+
+
 def matmul(fmt: int, W, N: int, K: int, X: np.ndarray) -> np.ndarray:
     w = _np(W)
     x = np.ascontiguousarray(X, np.float64).reshape(-1, K)

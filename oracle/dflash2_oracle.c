@@ -50,7 +50,7 @@
 
 typedef struct {
   int32_t layers, hidden, ffn, n_q, n_kv, head_dim, window, vocab, n_taps, block, topk, rank,
-      page_size, wfmt; /* wfmt: 0 = Q4_K, 1 = bf16 for fc and the layer matrices */
+      page_size, wfmt; /* fc and layer matrices: 0 = Q4_K, 1 = bf16, 2 = MLX 4-bit g64, 3 = Q8_0 */
   double rope_theta, rms_eps;
 } orc_dims;
 
@@ -140,10 +140,41 @@ void orc_q4k_dequant(const uint8_t *blocks, int64_t nblocks, double *out) {
   for (int64_t i = 0; i < nblocks; ++i) q4k_block(blocks + 144 * i, out + 256 * i);
 }
 
-/* Row n of a [N, K] matrix stored as Q4_K (fmt 0) or bf16 (fmt 1). */
+/* MLX-style 4-bit group-64 (MLX sidecar card, "Contents": 4-bit weights in groups of 64): each
+ * group of 64 consecutive weights of a row is stored as 32 bytes of 4-bit codes (element e at byte
+ * e/2, low nibble first; the uint32-packed order of MLX read little-endian) followed by its scale
+ * and bias in bf16 (36 bytes per group); weight e = scale * q_e + bias. */
+void orc_mlx4_dequant(const uint8_t *groups, int64_t ngroups, double *out) {
+  for (int64_t g = 0; g < ngroups; ++g) {
+    const uint8_t *b = groups + 36 * g;
+    const double sc = orc_bf16((uint16_t)(b[32] | (b[33] << 8)));
+    const double bi = orc_bf16((uint16_t)(b[34] | (b[35] << 8)));
+    for (int e = 0; e < 64; ++e) {
+      const int q = (e & 1) ? (b[e / 2] >> 4) : (b[e / 2] & 15);
+      out[64 * g + e] = sc * q + bi;
+    }
+  }
+}
+
+/* Q8_0 (Mindket listing, "Good to know": Q8_0 files): blocks of 32 weights, an fp16 scale d then
+ * 32 signed 8-bit codes (34 bytes); weight e = d * q_e. */
+void orc_q8_0_dequant(const uint8_t *blocks, int64_t nblocks, double *out) {
+  for (int64_t i = 0; i < nblocks; ++i) {
+    const uint8_t *b = blocks + 34 * i;
+    const double d = orc_fp16((uint16_t)(b[0] | (b[1] << 8)));
+    for (int e = 0; e < 32; ++e) out[32 * i + e] = d * (double)(int8_t)b[2 + e];
+  }
+}
+
+/* Row n of a [N, K] matrix stored as Q4_K (fmt 0), bf16 (fmt 1), MLX 4-bit group-64 (fmt 2) or
+ * Q8_0 (fmt 3). */
 static void weight_row(int fmt, const void *W, int K, int64_t n, double *row) {
   if (fmt == 0) {
     orc_q4k_dequant((const uint8_t *)W + (int64_t)n * (K / 256) * 144, K / 256, row);
+  } else if (fmt == 2) {
+    orc_mlx4_dequant((const uint8_t *)W + (int64_t)n * (K / 64) * 36, K / 64, row);
+  } else if (fmt == 3) {
+    orc_q8_0_dequant((const uint8_t *)W + (int64_t)n * (K / 32) * 34, K / 32, row);
   } else {
     const uint16_t *r = (const uint16_t *)W + (int64_t)n * K;
     for (int k = 0; k < K; ++k) row[k] = orc_bf16(r[k]);
@@ -446,7 +477,8 @@ void orc_accept_chain(int B, int Bk, int32_t mask_id, const int32_t *draft, cons
  *     (T = 0, a residual that is empty in fp32, falls back to p itself).
  * p: fp32 [B][Bk][V], row i = the target's probabilities for block position i+1 (row D after the
  * drafted tokens); q: fp32 [B][D][V] or NULL; u_acc: fp32 [B][D] in [0,1); u_s: uint32 [B].
- * accepted [B], emitted [B][Bk] (the accepted tokens, the sampled token, then -1). */
+ * accepted [B], emitted [B][Bk] (the accepted tokens, the sampled token, then -1).  A drafted id
+ * outside [0, V) has probability 0 under the target: it is rejected (no table is indexed by it). */
 /* fp32 values below the normal range (|v| < 2^-126) count as zero, inputs and the residual alike:
  * the decisions then do not depend on how an implementation treats subnormal numbers. */
 static float flush32(float v) {
@@ -490,6 +522,7 @@ void orc_accept_sampled(int B, int Bk, int V, const int32_t *draft, const float 
     int n = 0;
     while (n < D) {
       const int32_t d = draft[b * D + n];
+      if (d < 0 || d >= V) break; /* a token outside the vocabulary has target probability 0 */
       const float *pr = p + ((int64_t)b * Bk + n) * V;
       const double qd = q ? (double)flush32(q[((int64_t)b * D + n) * V + d]) : 1.0;
       if ((double)flush32(u_acc[b * D + n]) * qd < (double)flush32(pr[d])) ++n;

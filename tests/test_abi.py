@@ -41,18 +41,19 @@ def test_strerror_and_sizes(lib):
     mats = H * d.n_taps * H + d.layers * (HQ * H + 2 * HKV * H + H * HQ + 3 * F * H)
     dyn = d.layers * 2 * (H // 4) * H * 2
     head = -(-(d.vocab + d.rank) // 256) * 256 * H * 2  # output head + selector projection, whole 16-tile records
-    # prepared copy: the Q4_K matrices keep their size, bf16 matrices and the output head theirs
-    assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144 + dyn + head
+    # prepared copy: the Q4_K matrices keep their size, bf16 matrices theirs, and the output head is
+    # held twice (the streaming kernel's records and the tensor-core operand layout)
+    assert lib.dflash2_prepared_size(C.byref(cfg)) == mats // 256 * 144 + dyn + 2 * head
     full = binding.config(inputs.FULL)
-    # full drafter: 973.2 MB of Q4_K matrices + 131.1 MB dynamic-convolution generators + 2545.5 MB head
-    assert abs(lib.dflash2_prepared_size(C.byref(full)) / 1e6 - (973.2 + 131.1 + 2545.5)) < 1.0
+    # full drafter: 973.2 MB of Q4_K matrices + 131.1 MB dynamic-convolution generators + 2 x 2545.5 MB head
+    assert abs(lib.dflash2_prepared_size(C.byref(full)) / 1e6 - (973.2 + 131.1 + 2 * 2545.5)) < 1.0
     bf = binding.config(inputs.FULL_BF16_B5)
     assert lib.dflash2_prepared_size(C.byref(bf)) > lib.dflash2_prepared_size(C.byref(full))
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 64), ("page_size", 32), ("topk", 8), ("block", 1),
                                          ("block", 17), ("hidden", 500), ("n_kv", 3), ("rank", 512),
-                                         ("vocab", 8200), ("layers", 9), ("wfmt", 2)])
+                                         ("vocab", 8200), ("layers", 9), ("wfmt", 4)])
 def test_unsupported_config_is_rejected(lib, field, value):
     cfg = binding.config(inputs.TINY)
     setattr(cfg, field, value)

@@ -208,3 +208,19 @@ def test_tiny_many_rows_run_on_tensor_cores(wfmt, block, batch):
     for b in sample:
         parity.check_request(run, hw_t, hw, b)
     parity.check_accept(run)
+
+
+@pytest.mark.parametrize("wfmt,batch", [(2, 1), (2, 12), (3, 1), (3, 12)])
+def test_tiny_alternate_codecs(wfmt, batch):
+    """MLX-style 4-bit group-64 layers (decoded inside the products, streaming engine at one request,
+    tensor cores at 96 rows) and Q8_0 layers (decoded once into bf16 records when the weights are
+    prepared) against the oracle, which decodes both formats exactly."""
+    import dataclasses
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=wfmt),
+                             batch=batch, ctx_lo=3, ctx_hi=150, shuffled_pages=batch > 1)
+    w, hw_t, hw = weights_for(wl)
+    sample = sorted({0, batch - 1})
+    run = parity.run_gpu(wl, w, sample)
+    for b in sample:
+        parity.check_request(run, hw_t, hw, b)
+    parity.check_accept(run)

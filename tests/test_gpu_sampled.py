@@ -43,15 +43,19 @@ def test_sampled_acceptance_matches_oracle(V, B, with_q):
     draft, p, q, ua, us = _case(B, Bk, V, 7 + V + B, with_q)
     dims = inputs.Dims(layers=1, hidden=256, ffn=256, n_q=1, n_kv=1, head_dim=128, window=16, vocab=V, n_taps=1,
                        block=Bk, topk=16, rank=16)
+    draft[0, 3] = V + 5  # an id outside the vocabulary: rejected, never used as an index
+    draft[-1, 1] = -2
     lib = binding.load()
-    t = lambda a, dt: torch.as_tensor(a).to("cuda", dt)
+    t = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a)).to("cuda", dt)
     acc = torch.full((B,), -5, dtype=torch.int32, device="cuda")
     em = torch.full((B, Bk), -5, dtype=torch.int32, device="cuda")
+    # every device buffer stays referenced until the call has completed
+    d_draft, d_p, d_ua = t(draft, torch.int32), t(p, torch.float32), t(ua, torch.float32)
+    d_us = t(us.view(np.int32), torch.int32)
     d_q = t(q, torch.float32) if q is not None else None
-    rc = lib.dflash2_accept_sampled(t(draft, torch.int32).data_ptr(), t(p, torch.float32).data_ptr(),
-                                    d_q.data_ptr() if d_q is not None else None, t(ua, torch.float32).data_ptr(),
-                                    t(us.view(np.int32), torch.int32).data_ptr(), B, Bk, V, acc.data_ptr(),
-                                    em.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    rc = lib.dflash2_accept_sampled(d_draft.data_ptr(), d_p.data_ptr(), d_q.data_ptr() if d_q is not None else None,
+                                    d_ua.data_ptr(), d_us.data_ptr(), B, Bk, V, acc.data_ptr(), em.data_ptr(),
+                                    torch.cuda.current_stream().cuda_stream)
     assert rc == 0
     torch.cuda.synchronize()
     o_acc, o_em = oracle.accept_sampled(draft, p, ua, us, q=q)

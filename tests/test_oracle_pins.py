@@ -89,6 +89,48 @@ def test_q4k_all_zero_block_is_exact():
     assert np.array_equal(oracle.q4k_dequant(inputs.quantize_q4k(z)), np.zeros(4 * 512))
 
 
+def test_mlx4_hand_group_and_round_trip():
+    """MLX 4-bit group-64: a hand-packed group decodes to scale * q + bias exactly (scale 0.5,
+    bias -3, q = e mod 16), nibble order low first; the synthetic quantiser's round trip on
+    N(0, 0.02) rows has the relative L2 error of 4-bit codes over a group's range (about 0.1)."""
+    q = [e % 16 for e in range(64)]
+    b = bytearray(36)
+    for e in range(0, 64, 2):
+        b[e // 2] = q[e] | (q[e + 1] << 4)
+    b[32:34] = bf16_bits([0.5]).tobytes()
+    b[34:36] = bf16_bits([-3.0]).tobytes()
+    got = oracle.mlx4_dequant(np.frombuffer(bytes(b), np.uint8))
+    assert np.array_equal(got, 0.5 * np.array(q) - 3.0)
+    w = torch.randn(64, 512, generator=torch.Generator().manual_seed(5)) * 0.02
+    enc = inputs.quantize_mlx4(w)
+    dec = oracle.mlx4_dequant(enc.numpy()).reshape(64, 512)
+    rel = np.linalg.norm(dec - w.double().numpy()) / np.linalg.norm(w.double().numpy())
+    assert 0.05 < rel < 0.15, rel
+
+
+def test_q8_0_hand_block_and_round_trip():
+    """Q8_0: a hand-packed block decodes to d * q exactly (d = 0.25, q = -127, -3, 0, 5, 127, ...);
+    the round trip on N(0, 0.02) rows has the error of 8-bit codes (well under 1 %)."""
+    qv = np.array([-127, -3, 0, 5, 127] + list(range(-13, 14)), np.int8)
+    b = np.frombuffer(np.float16(0.25).tobytes() + qv.tobytes(), np.uint8)
+    got = oracle.q8_0_dequant(b)
+    assert np.array_equal(got, 0.25 * qv.astype(np.float64))
+    w = torch.randn(64, 512, generator=torch.Generator().manual_seed(6)) * 0.02
+    dec = oracle.q8_0_dequant(inputs.quantize_q8_0(w).numpy()).reshape(64, 512)
+    rel = np.linalg.norm(dec - w.double().numpy()) / np.linalg.norm(w.double().numpy())
+    assert 0.001 < rel < 0.01, rel
+
+
+@pytest.mark.parametrize("fmt", [2, 3])
+def test_matmul_of_alternate_codecs_matches_decoded_numpy(fmt):
+    N, K = 48, 512
+    w = torch.randn(N, K, generator=torch.Generator().manual_seed(7 + fmt)) * 0.02
+    enc = (inputs.quantize_mlx4 if fmt == 2 else inputs.quantize_q8_0)(w)
+    dec = (oracle.mlx4_dequant if fmt == 2 else oracle.q8_0_dequant)(enc.numpy()).reshape(N, K)
+    x = rng.standard_normal((5, K))
+    assert np.allclose(oracle.matmul(fmt, enc, N, K, x), x @ dec.T, rtol=1e-12, atol=1e-12)
+
+
 def test_q4k_round_trip_matches_card_error():
     """FastFlowLM card: about 0.07 relative L2 per Q4_K matrix (N(0, 0.02) weights here)."""
     w = torch.randn((256, 4096), generator=torch.Generator().manual_seed(7)) * 0.02
@@ -461,11 +503,13 @@ def test_selector_chain_codebooks_force_consecutive_ids():
     for b in range(1, V):
         Bc[b, b - 1] = 1.0
     x0 = 20
+    g = np.random.default_rng(77)  # own stream: independent of the order the other tests run in
     cand = np.zeros((D, K), np.int32)
     for t in range(D):
-        others = [i for i in rng.permutation(V) if i != x0 + 1 + t][:K - 1]
+        # the alternative first token x0 + 30 below must have no chain successor among the candidates
+        others = [i for i in g.permutation(V) if i != x0 + 1 + t and i != x0 + 31][:K - 1]
         cand[t] = others[:K - 1 - (t % 5)] + [x0 + 1 + t] + others[K - 1 - (t % 5):K - 1]
-    cl = -np.sort(-rng.standard_normal((D, K)), axis=1)
+    cl = -np.sort(-g.standard_normal((D, K)), axis=1)
     z = np.full((D, R), 50.0)
     path, sc = oracle.selector(cand, cl, z, x0, bf16_bits(A), bf16_bits(Bc))
     assert np.array_equal(path, x0 + 1 + np.arange(D))
