@@ -282,6 +282,9 @@ def main():
         barrier(ws)
     ms = t0.elapsed_time(t1) / K
     ms_max = all_max(ms, ws)
+    # accepted drafted tokens per request in the last timed step (synthetic targets: the first
+    # mismatch sits at a seeded position, so this is the workload's own distribution)
+    acc_hist = [int(v) for v in torch.bincount(acc.long().cpu(), minlength=Bk)[:Bk]]
     lm_ms = sum(a.elapsed_time(b) for a, b in ev) / K
     assert dr.device_error() == 0, "device error during the timed steps"
 
@@ -348,6 +351,7 @@ def main():
         "data": "synthetic (seeded N(0,0.02) weights quantised to Q4_K, bf16 LM head/codebooks, N(0,1) taps and KV)",
         "config": bench_config(wl, ws),
         "request_steps_per_s": value * B,
+        "accepted_hist": {"counts_by_accepted_0_to_7": acc_hist, "kind": "synthetic targets (seeded first mismatch)"},
         "step_hbm": {"algorithmic_bytes": byt["total"], "achieved_gbs": byt["total"] / (ms_max * 1e-3) / 1e9,
                      "frac_of_8tbs": byt["total"] / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                      "frac_of_measured": byt["total"] / (ms_max * 1e-3) / 1e9 / hbm, "peak_kind": peak_kind},

@@ -228,6 +228,31 @@ DEVI void sum_pieces4(const SGemvParams& p, int npieces, const int (&row)[4], co
   }
 }
 
+// Split-K sums of N outputs (row[k], col[k]; ok[k] false: 0), each in piece order (the same
+// additions as sum_pieces); all loads of a round of 4 pieces for all N outputs go out together.
+template <int N>
+DEVI void sum_pieces_n(const SGemvParams& p, int npieces, const int (&row)[N], const int (&col)[N],
+                       const bool (&ok)[N], float (&v)[N]) {
+  const float* b[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    b[k] = p.part + (size_t)row[k] * p.ldo + col[k];
+    v[k] = 0.f;
+  }
+  for (int s0 = 0; s0 < npieces; s0 += 4) {
+    float x[N][4];
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        x[k][j] = ok[k] && s0 + j < npieces ? __ldcg(b[k] + (size_t)(s0 + j) * p.piece_stride) : 0.f;
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[k] += x[k][j];
+  }
+}
+
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 // rs_pre: row scales of rows [0, rows) computed at the kernel's start (single row group), or null.
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, const float* rs_pre = nullptr) {
@@ -244,17 +269,18 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
       else if (rs_pre && mz == 0) rsv = rs_pre;
       else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
     }
-    // two outputs per thread per round: all their partial loads are in flight together
-    for (int i0 = tid; i0 < rows * 64; i0 += 2 * nthr) {
-      float gv[2], uv[2];
-      float4 hc[2], hp[2];
-      uint2 wv[2], e0[2], e1[2];
+    // four outputs per thread per round: all their partial loads are in flight together
+    constexpr int NO = 4;
+    for (int i0 = tid; i0 < rows * 64; i0 += NO * nthr) {
+      float gv[NO], uv[NO];
+      float4 hc[NO], hp[NO];
+      uint2 wv[NO], e0[NO], e1[NO];
       {
-        int rw[4], cl[4];
-        bool okk[4];
-        float sv[4];
+        int rw[2 * NO], cl[2 * NO];
+        bool okk[2 * NO];
+        float sv[2 * NO];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < NO; ++k) {
           const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
           okk[2 * k] = okk[2 * k + 1] = i < rows * 64;
           rw[2 * k] = rw[2 * k + 1] = mz + r;
@@ -272,15 +298,15 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
             e1[k] = *reinterpret_cast<const uint2*>(p.dyn_s1 + 4 * f);
           }
         }
-        sum_pieces4(p, npieces, rw, cl, okk, sv);
+        sum_pieces_n<2 * NO>(p, npieces, rw, cl, okk, sv);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < NO; ++k) {
           gv[k] = sv[2 * k];
           uv[k] = sv[2 * k + 1];
         }
       }
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < NO; ++k) {
         const int i = i0 + k * nthr, r = i >> 6, f = f0 + (i & 63);
         if (i >= rows * 64) continue;
         const float sc = p.rs_in ? rsv[pre + r] : 1.f;
@@ -330,15 +356,16 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     }
     return;
   }
-  // four outputs per thread per round: all their partial loads (and the residual reads) are in
+  // eight outputs per thread per round: all their partial loads (and the residual reads) are in
   // flight together before any store
-  for (int i0 = tid; i0 < rows * 128; i0 += 4 * nthr) {
-    float v[4], old[4], hwf[4];
+  constexpr int NR = 8;
+  for (int i0 = tid; i0 < rows * 128; i0 += NR * nthr) {
+    float v[NR], old[NR], hwf[NR];
     {
-      int rw[4], cl[4];
-      bool okk[4];
+      int rw[NR], cl[NR];
+      bool okk[NR];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < NR; ++k) {
         const int i = i0 + k * nthr;
         rw[k] = mz + (i >> 7);
         cl[k] = col0 + (i & 127);
@@ -347,10 +374,10 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
         old[k] = okk[k] && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)rw[k] * p.ldy + cl[k]) : 0.f;
         hwf[k] = okk[k] && p.epi == EPI_RESID && p.hw ? bf2f(p.hw_w[cl[k]]) : 0.f;
       }
-      sum_pieces4(p, npieces, rw, cl, okk, v);
+      sum_pieces_n<NR>(p, npieces, rw, cl, okk, v);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < NR; ++k) {
       const int i = i0 + k * nthr, r = i >> 7, c = col0 + (i & 127);
       if (i >= rows * 128) break;  // warp-uniform: rows * 128 is a multiple of 32
       float* y = p.y + (size_t)(mz + r) * p.ldy + c;

@@ -37,7 +37,8 @@ constexpr int kUmmaRaw = 3;                        // raw weight-record slots (o
 constexpr int kUmmaABytes = 128 * 128;             // [128 features][64 k] bf16
 constexpr int kUmmaBBytes = kUmmaRows * 128;       // [256 rows][64 k] bf16
 constexpr int kUmmaRawBytes = 8 * kQ4Bytes;        // one group unit (Q4_K 18 KB; bf16 units are 16 KB)
-constexpr int kUmmaThreads = 384;                  // 12 warps: roles below
+constexpr int kUmmaDq = 8;                         // weight-operand warps (one tile of the group each)
+constexpr int kUmmaThreads = (4 + kUmmaDq + 4) * 32; // roles below
 constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + kUmmaRaw * kUmmaRawBytes + 1024;
 constexpr int kUmmaTmemCols = 512;                 // two 256-column accumulators
 
@@ -155,11 +156,13 @@ DEVI void rows_scale_global(const float* ssp, int ldr, int H, float eps, int r0,
   }
 }
 
-// Roles (12 warps): warp 0 one thread: activation TMA; warp 1: TMEM allocation, one thread issues
+// Roles (16 warps): warp 0 one thread: activation TMA; warp 1: TMEM allocation, one thread issues
 // the MMAs; warp 2 one thread: raw weight records into the raw ring (bulk copies, started before
 // the dependency wait: the weights do not depend on earlier kernels); warp 3: the row scales of
-// a folded RMSNorm for the fix-up (p.rs_glob); warps 4-7: weight operand from the raw ring;
-// warps 8-11: epilogue (TMEM lane = feature), on two accumulators alternating by piece.
+// a folded RMSNorm for the fix-up (p.rs_glob); warps 4-11: the weight operand from the raw ring,
+// one 16-feature tile each (two warps per SM sub-partition, so one's latencies hide behind the
+// other's work: with one per sub-partition the dequantisation bounded the kernel); warps 12-15:
+// epilogue (TMEM lane = feature), on two accumulators alternating by piece.
 template <bool Q4>
 __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -178,12 +181,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUmmaStages; ++s) {
       mbar_init(&xfull[s], 1);
-      mbar_init(&afull[s], 4);
+      mbar_init(&afull[s], kUmmaDq);
       mbar_init(&sempty[s], 1);
     }
     for (int r = 0; r < kUmmaRaw; ++r) {
       mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], 4);
+      mbar_init(&rempty[r], kUmmaDq);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
@@ -294,9 +297,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
       const int r0 = (int)(c * p.rows / P), r1 = (int)((c + 1) * p.rows / P);
       rows_scale_global(p.rs_in, p.ssp_rows, p.rs_H, p.eps, r0, r1, p.rs_glob);
     }
-  } else if (warp < 8) {
-    // ---- weight operand: raw ring -> swizzled K-major stage ----
-    const int dw = warp - 4, g = lane >> 2, t = lane & 3;
+  } else if (warp < 4 + kUmmaDq) {
+    // ---- weight operand: raw ring -> swizzled K-major stage (warp = one tile of the group) ----
+    const int tl = warp - 4, g = lane >> 2, t = lane & 3;
     bool dead = false;
     int cnt = 0, ucnt = 0;
     for (long long x = x0; x < x1;) {
@@ -310,23 +313,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           const int r = ucnt % kUmmaRaw;
           wait_or_die(&rfull[r], (ucnt / kUmmaRaw) & 1, dead, p.err);
           const uint8_t* raw = Rs + r * kUmmaRawBytes;
-          // 4-bit records: this lane's scale records (rows g, g+8 of its two tiles), decoded once per
+          // 4-bit records: this lane's scale records (rows g, g+8 of its tile), decoded once per
           // unit (Q4_K: d, dmin and the packed 6-bit fields; MLX: the record's four bf16 pairs)
-          float dd[2][2], dm[2][2];
-          unsigned long long scp[2][2], mp[2][2];
-          uint4 mrec[2][2];
+          float dd[2], dm[2];
+          unsigned long long scp[2], mp[2];
+          uint4 mrec[2];
           if (Q4 && !dead) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const uint4 sc = *reinterpret_cast<const uint4*>(raw + (2 * dw + h) * kQ4Bytes + 2048 + (g + 8 * e) * 16);
-                mrec[h][e] = sc;
-                dd[h][e] = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
-                dm[h][e] = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
-                scp[h][e] = (unsigned long long)sc.y | ((unsigned long long)(sc.z & 0xffffu) << 32);
-                mp[h][e] = (unsigned long long)(sc.z >> 16) | ((unsigned long long)sc.w << 16);
-              }
+            for (int e = 0; e < 2; ++e) {
+              const uint4 sc = *reinterpret_cast<const uint4*>(raw + tl * kQ4Bytes + 2048 + (g + 8 * e) * 16);
+              mrec[e] = sc;
+              dd[e] = __half2float(__ushort_as_half((unsigned short)(sc.x & 0xffffu)));
+              dm[e] = __half2float(__ushort_as_half((unsigned short)(sc.x >> 16)));
+              scp[e] = (unsigned long long)sc.y | ((unsigned long long)(sc.z & 0xffffu) << 32);
+              mp[e] = (unsigned long long)(sc.z >> 16) | ((unsigned long long)sc.w << 16);
+            }
           }
 #pragma unroll
           for (int sub = 0; sub < kSub; ++sub, ++cnt) {
@@ -334,40 +335,37 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
             if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
             uint8_t* a = As + s * kUmmaABytes;
             if (!dead) {
+              const int m0 = tl * 16 + g;  // operand rows g and g+8 of tile tl
+              const uint8_t* rec = raw + tl * (Q4 ? kQ4Bytes : 2048);
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int tl = 2 * dw + h, m0 = tl * 16 + g;  // operand rows g and g+8 of tile tl
-                const uint8_t* rec = raw + tl * (Q4 ? kQ4Bytes : 2048);
+              for (int jj = 0; jj < 2; ++jj) {  // 32-wide sub-blocks of the stage
+                uint4 rg, rh;
+                if (Q4) {
+                  const uint4 q = *reinterpret_cast<const uint4*>(rec + (sub * 32 + lane) * 16);
+                  const uint32_t w0 = jj ? q.z : q.x, w1 = jj ? q.w : q.y;
+                  const int j = 2 * sub + jj;
+                  float2 dc[2];
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {  // 32-wide sub-blocks of the stage
-                  uint4 rg, rh;
-                  if (Q4) {
-                    const uint4 q = *reinterpret_cast<const uint4*>(rec + (sub * 32 + lane) * 16);
-                    const uint32_t w0 = jj ? q.z : q.x, w1 = jj ? q.w : q.y;
-                    const int j = 2 * sub + jj;
-                    float2 dc[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                      if (p.mlx) {  // group j/2: w = scale*q + bias = (128+q)*scale + (bias - 128*scale)
-                        const uint4 r = mrec[h][e];
-                        const uint32_t wg = (j >> 1) == 0 ? r.x : (j >> 1) == 1 ? r.y : (j >> 1) == 2 ? r.z : r.w;
-                        const float D = bf2f((uint16_t)(wg & 0xffffu)), B = bf2f((uint16_t)(wg >> 16));
-                        dc[e] = make_float2(D, fmaf(-128.f, D, B));
-                      } else {
-                        const float D = dd[h][e] * (float)((scp[h][e] >> (6 * j)) & 63u);
-                        const float M = dm[h][e] * (float)((mp[h][e] >> (6 * j)) & 63u);
-                        dc[e] = make_float2(D, -fmaf(128.f, D, M));
-                      }
+                  for (int e = 0; e < 2; ++e) {
+                    if (p.mlx) {  // group j/2: w = scale*q + bias = (128+q)*scale + (bias - 128*scale)
+                      const uint4 r = mrec[e];
+                      const uint32_t wg = (j >> 1) == 0 ? r.x : (j >> 1) == 1 ? r.y : (j >> 1) == 2 ? r.z : r.w;
+                      const float D = bf2f((uint16_t)(wg & 0xffffu)), B = bf2f((uint16_t)(wg >> 16));
+                      dc[e] = make_float2(D, fmaf(-128.f, D, B));
+                    } else {
+                      const float D = dd[e] * (float)((scp[e] >> (6 * j)) & 63u);
+                      const float M = dm[e] * (float)((mp[e] >> (6 * j)) & 63u);
+                      dc[e] = make_float2(D, -fmaf(128.f, D, M));
                     }
-                    rg = q4_chunk(w0, w1, 0, dc[0]);
-                    rh = q4_chunk(w0, w1, 4, dc[1]);
-                  } else {  // bf16 record: W[row g][32jj + 8t ..] at jj*1024 + lane*16, row g+8 at +512
-                    rg = *reinterpret_cast<const uint4*>(rec + jj * 1024 + lane * 16);
-                    rh = *reinterpret_cast<const uint4*>(rec + jj * 1024 + 512 + lane * 16);
                   }
-                  *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jj + t)) = rg;
-                  *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jj + t)) = rh;
+                  rg = q4_chunk(w0, w1, 0, dc[0]);
+                  rh = q4_chunk(w0, w1, 4, dc[1]);
+                } else {  // bf16 record: W[row g][32jj + 8t ..] at jj*1024 + lane*16, row g+8 at +512
+                  rg = *reinterpret_cast<const uint4*>(rec + jj * 1024 + lane * 16);
+                  rh = *reinterpret_cast<const uint4*>(rec + jj * 1024 + 512 + lane * 16);
                 }
+                *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jj + t)) = rg;
+                *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jj + t)) = rh;
               }
             }
             fence_proxy_async_smem();  // these generic writes feed the tensor cores (async proxy)
@@ -382,7 +380,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
     }
   } else {
     // ---- epilogue: TMEM -> fp32 partial [piece][row][ldo], accumulators alternate by piece ----
-    const int ew = warp - 8;  // = warp % 4: TMEM lanes 32*ew ..
+    const int ew = warp - (4 + kUmmaDq);  // = warp % 4: TMEM lanes 32*ew ..
     bool dead = false, waited = false;
     int piece = 0;
     for (long long x = x0; x < x1;) {
@@ -596,24 +594,28 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
             tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)(mc * 256 + n0), r);
             tmem_ld_wait();
             if (rl < trows) {
-              const int f0 = rec * 256 + n0;
-              if (f0 + 32 <= p.V) {
-                const int g0 = f0 + p.id0;  // vocabulary id of feature f0
+              const int f0 = rec * 256 + n0, g0 = f0 + p.id0;  // g0: vocabulary id of feature f0
+              const int nv = min(32, max(0, p.V - f0));          // head features of this chunk
+              // the features that beat the row's 16th entry (compact: one compare each), then one
+              // insertion site for the few that do (the list's 16th only rises as entries go in)
+              const float th = lv[mc][15];
+              const int thi = li[mc][15];
+              unsigned m = 0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) m |= (i < nv && better(__uint_as_float(r[i]), g0 + i, th, thi)) ? 1u << i : 0u;
+              while (m) {
+                const int i = __ffs(m) - 1;
+                m &= m - 1;
+                float x = __uint_as_float(r[0]);
+#pragma unroll
+                for (int k = 1; k < 32; ++k) x = k == i ? __uint_as_float(r[k]) : x;
+                if (better(x, g0 + i, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, g0 + i);
+              }
+              if (f0 + 32 > p.V) {  // selector projection features of this chunk
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                  const float x = __uint_as_float(r[i]);
-                  if (better(x, g0 + i, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, g0 + i);
-                }
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  const float x = __uint_as_float(r[i]);
                   const int f = f0 + i;
-                  if (f < p.V) {
-                    if (better(x, f + p.id0, lv[mc][15], li[mc][15])) reg_list_insert(lv[mc], li[mc], x, f + p.id0);
-                  } else if (f < p.V + p.R) {
-                    p.z[(size_t)row * p.R + (f - p.V)] = x;
-                  }
+                  if (f >= p.V && f < p.V + p.R) p.z[(size_t)row * p.R + (f - p.V)] = __uint_as_float(r[i]);
                 }
               }
             }
