@@ -1,0 +1,319 @@
+// Sliding-window GQA attention for many requests (FastFlowLM card, "Draft" row: 32 query / 8
+// key-value heads of 128, sliding window 2048): one CTA per (request, kv head) streams the
+// window's cache pages through a ring of TMA stages.
+//
+// With many requests the cluster kernel (attention.cuh) runs thousands of short CTAs, one per SM at
+// a time, each paying the whole load-compute-merge latency.  Here a CTA owns a (request, kv head)
+// for the whole window, two CTAs share an SM, and the loads run ahead of the math:
+//  * warp 4, one thread: for each 64-key chunk (4 pages of 16 tokens), the 4 KiB K and V rows of
+//    this kv head in each page by 2-D TMA (cp.async.bulk.tensor, no multicast) as two 64-dim boxes
+//    with 128-byte swizzle into one of two 32 KB stages; unmapped pages are skipped and flagged;
+//  * warps 0-3: warp (qt, kh) takes query tile qt (16 of the kv head's G x Bk query vectors) and
+//    key half kh (32 keys) of every chunk: S = Q K^T and P V on mma.sync m16n8k16 with an online
+//    softmax (running max, sum and output in registers); then the block's own keys (all visible);
+//    the two key halves of a query tile merge in shared memory at the end.
+// Visibility as everywhere: block row t at position p = Lb + t sees cache keys
+// max(0, p - W + 1) <= j < Lb and every block key.  Softmax in fp32, scale 1/sqrt(128).
+#pragma once
+#include <cuda.h>
+
+#include "attention.cuh"
+#include "umma.cuh"
+
+namespace dfl {
+
+constexpr int kAttnStreamMinBatch = 8;  // requests from which the streaming kernel is used
+constexpr int kAsStages = 2;
+constexpr int kAsKeys = 64;                  // cache keys per stage (4 pages)
+constexpr int kAsHalf = kAsKeys * 128;       // one 64-dim half of a stage's K or V: 8 KB (128-byte rows)
+constexpr int kAsStage = 4 * kAsHalf;        // K lo | K hi | V lo | V hi
+constexpr int kAsBlk = 4 * 16 * 128;         // the block keys (<= 16) in the same layout: 8 KB
+constexpr int kAsQ = 32 * 256;               // 32 query vectors x 128 bf16
+constexpr int kAsThreads = 5 * 32;
+constexpr int kAsSmem = kAsStages * kAsStage + kAsBlk + kAsQ + 1024;
+
+// byte offset of dims [8c, 8c + 8) of key row r in a 128-byte-swizzled half block
+DEVI uint32_t as_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// S for NT * 8 keys (NT n-tiles of 8) of one 16-query tile; kbase: the K half-blocks (dims 0..63 at
+// +0, 64..127 at +half), keys key0 .. key0 + 8 NT - 1 of them.
+template <int NT>
+DEVI void as_scores(const uint32_t (&qa)[8][4], const uint8_t* kbase, int half, int key0, float (&s)[4][4], int lane) {
+#pragma unroll
+  for (int n = 0; n < 4; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int hf = ks >> 2, c = (ks & 3) * 2 + ((lane >> 3) & 1);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int r = key0 + n * 8 + (lane & 7);
+      uint32_t b0, b1;
+      ldmatrix_x2(b0, b1, kbase + hf * half + as_off(r, c));
+      mma16816(s[n], qa[ks], b0, b1);
+    }
+  }
+}
+
+// P V for the same keys (KK steps of 16): o[16 dim tiles][4] += P (s, already exponentiated) x V.
+template <int KK>
+DEVI void as_pv(const float (&s)[4][4], const uint8_t* vbase, int half, int key0, float (&o)[16][4], int lane) {
+#pragma unroll
+  for (int kk = 0; kk < KK; ++kk) {
+    uint32_t a[4];
+    a[0] = pack_bf2(s[2 * kk][0], s[2 * kk][1]);
+    a[1] = pack_bf2(s[2 * kk][2], s[2 * kk][3]);
+    a[2] = pack_bf2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+    a[3] = pack_bf2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+    const int r = key0 + kk * 16 + (lane & 15);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      uint32_t b0, b1;
+      ldmatrix_x2_trans(b0, b1, vbase + (n >> 3) * half + as_off(r, n & 7));
+      mma16816(o[n], a, b0, b1);
+    }
+  }
+}
+
+// Online softmax update of one warp's two rows (h = 0, 1: query vectors g, g + 8 of its tile) with
+// this chunk's masked scores (already scaled to log2 units, -inf where not visible); only the first
+// NT n-tiles hold keys.
+template <int NT>
+DEVI void as_softmax(float (&s)[4][4], float (&m)[2], float (&l)[2], float (&o)[16][4]) {
+  float mx[2] = {m[0], m[1]};
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+  }
+  float corr[2], add[2] = {0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) corr[h] = mx[h] == -INFINITY ? 1.f : exp2f(m[h] - mx[h]);
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mm = mx[e >> 1];
+      const float pv = mm == -INFINITY ? 0.f : exp2f(s[n][e] - mm);
+      s[n][e] = pv;
+      add[e >> 1] += pv;
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    add[h] += __shfl_xor_sync(0xffffffffu, add[h], 1);
+    add[h] += __shfl_xor_sync(0xffffffffu, add[h], 2);
+    l[h] = l[h] * corr[h] + add[h];
+    m[h] = mx[h];
+  }
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    o[n][0] *= corr[0];
+    o[n][1] *= corr[0];
+    o[n][2] *= corr[1];
+    o[n][3] *= corr[1];
+  }
+}
+
+// tmk / tmv: the layer's K and V caches as [pages * nkv * 16 rows][128] bf16 tensors (boxes of 16
+// rows x 64 dims, 128-byte swizzle).  Grid (nkv, B).  Requires G * Bk <= 32 (two query tiles).
+__global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_constant__ CUtensorMap tmk,
+                                                              const __grid_constant__ CUtensorMap tmv, AttnParams p,
+                                                              uint16_t* __restrict__ ob) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kAsStages], empty[kAsStages];
+  __shared__ int pvalid[kAsStages][4];
+  __shared__ float mrg_m[2][16], mrg_l[2][16];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* stages = smem;
+  uint8_t* blk = smem + kAsStages * kAsStage;  // block keys: K lo | K hi | V lo | V hi, 16 rows each
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(blk + kAsBlk);  // [32][128] bf16
+  const int kvh = blockIdx.x, b = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.nq / p.nkv, nqv = G * p.Bk;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAsStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    fence_mbar_init();
+  }
+  // Keys of pages that are never loaded (past the window's end, or unmapped) get P = 0, and their V
+  // rows must be finite for 0 x V to vanish: the stages start zeroed, and later hold only loaded rows.
+  for (int i = threadIdx.x; i < kAsStages * kAsStage / 16; i += kAsThreads)
+    reinterpret_cast<uint4*>(stages)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the queries, the block's keys and this step's context rows come from the QKV kernel
+  const long long S0 = p.seq_len[b], Lb = S0 + p.n_new[b];
+  long long s0 = Lb - p.W + 1;
+  if (s0 < 0) s0 = 0;
+  const long long cs = (s0 / kPage) * kPage;
+  const int nc = (int)((Lb - cs + kAsKeys - 1) / kAsKeys);
+
+  if (warp == 4) {
+    // ---- producer: the window's pages, chunk by chunk ----
+    if (lane == 0) {
+      bool dead = false;
+      int issued = 0;
+      for (int c = 0; c < nc && !dead; ++c) {
+        const int s = c % kAsStages, round = c / kAsStages;
+        if (round > 0 && !wait_or_die(&empty[s], (round - 1) & 1, dead, p.err)) break;
+        int pg[4];
+        uint32_t bytes = 0;
+        for (int pi = 0; pi < 4; ++pi) {
+          const long long j0 = cs + (long long)c * kAsKeys + pi * kPage;  // first token of the page
+          int g = -2;  // -2: past the cached tokens (nothing to load), -1: unmapped
+          if (j0 < Lb) {
+            const long long lp = j0 / kPage;
+            g = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+            if (g >= p.num_pages) g = -1;
+            if (g < 0) {
+              g = -1;
+              set_err(p.err, DFLASH2_DEV_PAGE);
+            } else {
+              bytes += 4 * 2048;
+            }
+          }
+          pg[pi] = g;
+          pvalid[s][pi] = g >= 0 ? 1 : 0;
+        }
+        uint8_t* st = stages + s * kAsStage;
+        if (bytes) {
+          mbar_expect_tx(&full[s], bytes);
+          for (int pi = 0; pi < 4; ++pi)
+            if (pg[pi] >= 0) {
+              const int row = (pg[pi] * p.nkv + kvh) * kPage;
+              tma_load_2d(st + 0 * kAsHalf + pi * 2048, &tmk, 0, row, &full[s]);
+              tma_load_2d(st + 1 * kAsHalf + pi * 2048, &tmk, 64, row, &full[s]);
+              tma_load_2d(st + 2 * kAsHalf + pi * 2048, &tmv, 0, row, &full[s]);
+              tma_load_2d(st + 3 * kAsHalf + pi * 2048, &tmv, 64, row, &full[s]);
+            }
+        } else {
+          mbar_arrive(&full[s]);  // (releases the page flags)
+        }
+        issued = c + 1;
+      }
+      // the CTA must not retire with copies into its shared memory still in flight (the math warps
+      // may have stopped early on a timeout): wait, bounded, for the last stages issued
+      for (int c = issued > kAsStages ? issued - kAsStages : 0; c < issued; ++c) {
+        bool d2 = false;
+        wait_or_die(&full[c % kAsStages], (c / kAsStages) & 1, d2, p.err);
+      }
+    }
+    return;
+  }
+
+  // ---- math warps: stage Q and the block keys (cp.async), then stream the chunks ----
+  for (int i = threadIdx.x; i < 32 * 16; i += 128) {  // Q: 32 vectors x 16 chunks of 16 B
+    const int qv = i >> 4, ch = i & 15;
+    const bool ok = qv < nqv;
+    const uint16_t* src = p.qb;
+    if (ok) src += ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim + ch * 8;
+    cp_async16(reinterpret_cast<uint8_t*>(Qs) + qv * 256 + ch * 16, src, ok);
+  }
+  for (int i = threadIdx.x; i < 2 * 16 * 16; i += 128) {  // block keys: {K, V} x 16 rows x 16 chunks
+    const int kv = i >> 8, r = (i >> 4) & 15, ch = i & 15;
+    const bool ok = r < p.Bk;
+    const uint16_t* src = kv ? p.vb : p.kb;
+    if (ok) src += ((size_t)(b * p.Bk + r) * p.nkv + kvh) * kHeadDim + ch * 8;
+    cp_async16(blk + (2 * kv + (ch >> 3)) * (16 * 128) + as_off(r, ch & 7), src, ok);
+  }
+  cp_async_wait_all();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int qt = warp & 1, kh = warp >> 1, g = lane >> 2, t4 = lane & 3;
+  uint32_t qa[8][4];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+    ldmatrix_x4(qa[ks], reinterpret_cast<const uint8_t*>(Qs) + (qt * 16 + (lane & 15)) * 256 + (ks * 16 + (lane >> 4) * 8) * 2);
+  int trow[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int qv = qt * 16 + g + 8 * h;
+    trow[h] = qv < nqv ? qv / G : -1;  // -1: padding vector, sees nothing
+  }
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  bool dead = false;
+  for (int c = 0; c < nc; ++c) {
+    const int s = c % kAsStages;
+    if (!wait_or_die(&full[s], (c / kAsStages) & 1, dead, p.err)) break;
+    const uint8_t* st = stages + s * kAsStage;
+    float sc[4][4];
+    as_scores<4>(qa, st, kAsHalf, kh * 32, sc, lane);
+    // mask: cache key j = cs + 64c + kk visible to block row t iff its page is mapped, j < Lb and
+    // j >= Lb + t - W + 1
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kk = kh * 32 + n * 8 + 2 * t4 + (e & 1);
+        const long long j = cs + (long long)c * kAsKeys + kk;
+        const int t = trow[e >> 1];
+        const bool vis = t >= 0 && pvalid[s][kk >> 4] && j < Lb && j >= Lb + t - p.W + 1;
+        sc[n][e] = vis ? sc[n][e] * p.scale_log2 : -INFINITY;
+      }
+    as_softmax<4>(sc, m, l, o);
+    as_pv<2>(sc, st + 2 * kAsHalf, kAsHalf, kh * 32, o, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
+  }
+  // the block's own keys (rows 0 .. Bk-1 of the block area, zero-filled to 16), all visible: both
+  // key halves score the 16 rows, half kh keeps rows 8kh .. 8kh + 7
+  if (!dead) {
+    float sc[4][4];
+    as_scores<2>(qa, blk, 16 * 128, 0, sc, lane);
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kk = n * 8 + 2 * t4 + (e & 1);
+        const bool vis = trow[e >> 1] >= 0 && kk < p.Bk && n == kh;
+        sc[n][e] = vis ? sc[n][e] * p.scale_log2 : -INFINITY;
+      }
+    as_softmax<2>(sc, m, l, o);
+    as_pv<1>(sc, blk + 2 * (16 * 128), 16 * 128, 0, o, lane);
+  }
+  // ---- merge the two key halves of each query tile; kh = 0 writes the output ----
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // every warp is done with the stages and blk
+  float* red = reinterpret_cast<float*>(stages);  // [qt][16 rows][128] of the kh = 1 warps
+  if (kh == 1) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = g + 8 * h;
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2*>(red + ((size_t)qt * 16 + row) * 128 + n * 8 + 2 * t4) =
+            make_float2(o[n][2 * h], o[n][2 * h + 1]);
+      if (t4 == 0) {
+        mrg_m[qt][row] = m[h];
+        mrg_l[qt][row] = l[h];
+      }
+    }
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (kh == 0) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = g + 8 * h, qv = qt * 16 + row;
+      const float m1 = mrg_m[qt][row], l1 = mrg_l[qt][row];
+      const float M = fmaxf(m[h], m1);
+      const float w0 = M == -INFINITY ? 0.f : exp2f(m[h] - M), w1 = M == -INFINITY ? 0.f : exp2f(m1 - M);
+      const float L = w0 * l[h] + w1 * l1, inv = L > 0.f ? 1.f / L : 0.f;
+      if (qv < nqv) {
+        uint16_t* dst = ob + ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          const float2 v1 = *reinterpret_cast<const float2*>(red + ((size_t)qt * 16 + row) * 128 + n * 8 + 2 * t4);
+          const float x = (w0 * o[n][2 * h] + w1 * v1.x) * inv, y = (w0 * o[n][2 * h + 1] + w1 * v1.y) * inv;
+          *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * t4) = pack_bf2(x, y);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace dfl

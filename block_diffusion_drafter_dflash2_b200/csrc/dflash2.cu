@@ -8,6 +8,7 @@
 #include <atomic>
 
 #include "attention.cuh"
+#include "attn_stream.cuh"
 #include "common.cuh"
 #include "gemv.cuh"
 #include "rowops.cuh"
@@ -37,6 +38,7 @@ struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
   int attn_ntk;  // > 0: attention as one cluster kernel, attn_kg key groups of 8*attn_ntk keys per CTA; 0: chunks + merge
   int attn_kg;
+  bool attn_stream;  // one streaming CTA per (request, kv head) with TMA-staged pages (many requests)
   bool q4, mlx;
   GemvPlan fc, dc, qkv, o, gu, dn;
   size_t off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
@@ -92,11 +94,12 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   g.P = (int)std::min<long long>(nsm, g.W);
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
   const int ring = ns * slot;
-  const int per_unit = g.R * unitK * 2;
+  // per unit: the activation chunk (bf16) and, for 4-bit records, its 8 sub-block sums per row (fp32)
+  const int per_unit = g.R * unitK * 2 + (q4 ? g.R * 8 * 4 : 0);
   const int extra = kGemvConsumers * 1024 + kConsumers * 32 * g.NT * 4 * 4;  // per-warp scale tables, set reduction
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra + (q4 ? (size_t)g.kc_units * g.R * 32 : 0);
   return g;
 }
 
@@ -187,6 +190,9 @@ Plan make_plan(const dflash2_config* c, int B) {
           }
     }
   }
+  // With 8 or more requests the (request, kv head) pairs fill the SMs two deep, and a CTA that keeps
+  // its window's pages streaming beats clusters that each pay the whole load-compute-merge latency.
+  p.attn_stream = B >= kAttnStreamMinBatch && p.QV <= 32;
   p.fc = plan_gemv(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
   p.dc = plan_gemv((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
   p.qkv = plan_gemv((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
@@ -468,6 +474,31 @@ cudaError_t launch_attn_t(const Plan& P, const AttnParams& ap, cudaStream_t s) {
   const cudaError_t e = smem_optin(k_attn_chunk<MT>, (int)smem, attr);
   if (e != cudaSuccess) return e;
   return launch_pdl(k_attn_chunk<MT>, dim3(P.NC + 1, ap.nkv, P.B), dim3(kAttnThreads), smem, s, ap);
+}
+
+// Tensor map of one layer's K or V cache viewed as [pages * nkv * 16 rows][128] bf16: boxes of
+// 16 rows (one page of one kv head) x 64 dims, 128-byte swizzle.
+cudaError_t make_kv_tmap(CUtensorMap* tm, const uint16_t* cache, int num_pages, int nkv) {
+  const EncodeTiledFn f = encode_tiled();
+  if (!f) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)num_pages * nkv * kPage};
+  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kPage};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = f(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(cache), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_stream(const Plan& P, const AttnParams& ap, uint16_t* ob, cudaStream_t s) {
+  static std::atomic<int> attr[kMaxDevices];
+  cudaError_t e = smem_optin(k_attn_stream, kAsSmem, attr);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tk, tv;
+  if ((e = make_kv_tmap(&tk, ap.kc, ap.num_pages, ap.nkv)) != cudaSuccess) return e;
+  if ((e = make_kv_tmap(&tv, ap.vc, ap.num_pages, ap.nkv)) != cudaSuccess) return e;
+  return launch_pdl(k_attn_stream, dim3(ap.nkv, P.B), dim3(kAsThreads), (size_t)kAsSmem, s, tk, tv, ap, ob);
 }
 
 template <int MT, int NTK, int KG>
@@ -837,7 +868,9 @@ int draft_step_impl(const dflash2_config* c, const dflash2_weights* w, const dfl
     {
       ap.kc = kv->k[l];
       ap.vc = kv->v[l];
-      if (P.attn_ntk > 0) {
+      if (P.attn_stream) {
+        CK(launch_attn_stream(P, ap, ob, s));
+      } else if (P.attn_ntk > 0) {
         if (P.MT == 1) CK(launch_attn_cluster_mt<1>(P, ap, ob, s));
         else CK(launch_attn_cluster_mt<2>(P, ap, ob, s));
       } else {
@@ -1231,7 +1264,7 @@ int32_t dflash2_step_kernels(const dflash2_config* c, int32_t batch) {
   int extra = 0;
   for (int i = 0; i < 5; ++i) extra += gp[i]->umma ? c->layers : 0;
   extra += P.fc.umma ? 1 : 0;
-  return 3 + (P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + 1 + 1 + extra;
+  return 3 + (P.attn_stream || P.attn_ntk > 0 ? 6 : 7) * c->layers + 1 + 1 + 1 + extra;
 }
 
 int dflash2_device_error(const void* ws, int32_t* out_bits, void* stream) {

@@ -56,6 +56,29 @@ def test_unmapped_append_page_sets_page_bit(tiny):
     assert _step(wl, dr, st) & binding.DEV_PAGE
 
 
+def test_unmapped_page_in_window_sets_page_bit_many_requests():
+    """Same check in the streaming attention kernel (eight requests)."""
+    import dataclasses
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], batch=8)
+    w = inputs.make_weights(wl.dims, wl.wseed, "cuda")
+    dr = binding.Drafter(wl.dims, w, 8)
+    D = wl.dims.block - 1
+
+    def step(st):
+        path = torch.zeros((8, D), dtype=torch.int32, device="cuda")
+        scores = torch.zeros((8, D), dtype=torch.float32, device="cuda")
+        dr.draft_step({"taps": st["taps"], "n_new": st["n_new"], "block_tokens": st["block_tokens"]}, st, path,
+                      scores)
+        torch.cuda.synchronize()
+        return dr.device_error()
+
+    assert step(inputs.make_state(wl, "cuda")) == 0
+    st = inputs.make_state(wl, "cuda")
+    L = int(st["seq_len"][5])
+    st["page_table"][5, (L - 5) // 16] = -1
+    assert step(st) & binding.DEV_PAGE
+
+
 def test_misaligned_taps_are_rejected(tiny):
     wl, dr = tiny
     st = inputs.make_state(wl, "cuda")

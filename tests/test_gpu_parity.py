@@ -83,6 +83,32 @@ def test_tiny_batch_of_requests_is_independent():
     parity.check_accept(run)
 
 
+def test_tiny_many_requests_stream_the_window():
+    """Ten requests (the streaming attention kernel's range): context lengths at page and window
+    boundaries, an empty cache, ragged appends and shuffled physical pages in one call."""
+    import dataclasses
+    ctx = [0, 1, 15, 16, 57, 63, 64, 65, 200, 130]
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], batch=10, shuffled_pages=True)
+    w, hw_t, hw = weights_for(wl)
+    st = inputs.make_state(wl, "cuda", seq_len=ctx, n_new=[8, 1, 0, 5, 8, 3, 8, 0, 2, 8])
+    run = parity.run_gpu(wl, w, range(10), state=st)
+    for b in range(10):
+        parity.check_request(run, hw_t, hw, b)
+    parity.check_accept(run)
+
+
+def test_tiny_many_requests_window_pages_only_block5():
+    """Eight bf16-layer requests of block 5 (ragged 20-vector query tiles) whose pages before the
+    window are unbacked."""
+    import dataclasses
+    wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=1, block=5),
+                             batch=8, ctx_lo=1, ctx_hi=500, window_pages_only=True, shuffled_pages=True)
+    w, hw_t, hw = weights_for(wl)
+    run = parity.run_gpu(wl, w, range(8))
+    for b in range(8):
+        parity.check_request(run, hw_t, hw, b)
+
+
 def test_tiny_bf16_layers_block5():
     import dataclasses
     wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=1, block=5),
