@@ -94,12 +94,11 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   g.P = (int)std::min<long long>(nsm, g.W);
   g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
   const int ring = ns * slot;
-  // per unit: the activation chunk (bf16) and, for 4-bit records, its 8 sub-block sums per row (fp32)
-  const int per_unit = g.R * unitK * 2 + (q4 ? g.R * 8 * 4 : 0);
+  const int per_unit = g.R * unitK * 2;
   const int extra = kGemvConsumers * 1024 + kConsumers * 32 * g.NT * 4 * 4;  // per-warp scale tables, set reduction
   const int budget = kSmemLimit - kStaticSmem - ring - extra - 64 * g.R;
   g.kc_units = std::max(1, std::min(g.U, budget / per_unit));
-  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra + (q4 ? (size_t)g.kc_units * g.R * 32 : 0);
+  g.smem = (size_t)ring + (size_t)g.R * (g.kc_units * unitK * 2 + 64) + extra;
   return g;
 }
 
@@ -442,7 +441,14 @@ cudaError_t launch_umma_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_
   e = launch_pdl(k_umma<Q4>, dim3(g.P), dim3(kUmmaThreads), (size_t)kUmmaSmem, s, tm, prm);
   if (e != cudaSuccess) return e;
   const int fix_blocks = prm.groups * ((prm.rows + 63) / 64);
-  return launch_pdl(k_umma_fixup, dim3(fix_blocks), dim3(kGemvConsumers * 32), 0, s, prm, g.P);
+  const dim3 fg(fix_blocks), fb(kGemvConsumers * 32);
+  switch (prm.epi) {
+    case EPI_RESID: return launch_pdl(k_umma_fixup<EPI_RESID, 2>, fg, fb, 0, s, prm, g.P);
+    case EPI_SWIGLU: return launch_pdl(k_umma_fixup<EPI_SWIGLU, 2>, fg, fb, 0, s, prm, g.P);
+    case EPI_STORE: return launch_pdl(k_umma_fixup<EPI_STORE, 2>, fg, fb, 0, s, prm, g.P);
+    case EPI_QKV: return launch_pdl(k_umma_fixup<EPI_QKV, 1>, fg, fb, 0, s, prm, g.P);
+    default: return launch_pdl(k_umma_fixup<EPI_DYNCONV, 1>, fg, fb, 0, s, prm, g.P);
+  }
 }
 
 cudaError_t launch_gemv(const GemvPlan& g, bool q4, const GemvSeg* segs, int nseg, bool paired, const uint16_t* X,

@@ -253,9 +253,46 @@ DEVI void sum_pieces_n(const SGemvParams& p, int npieces, const int (&row)[N], c
   }
 }
 
+// Split-K sums of N groups of 4 consecutive outputs (row[k], col[k] .. col[k] + 3, col[k] a
+// multiple of 4; ok[k] false: 0), each output in piece order (the same additions as sum_pieces),
+// with 16-byte loads: all loads of a round of 2 pieces for all N groups go out together.
+template <int N>
+DEVI void sum_pieces_q(const SGemvParams& p, int npieces, const int (&row)[N], const int (&col)[N],
+                       const bool (&ok)[N], float4 (&v)[N]) {
+  const float* b[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    b[k] = p.part + (size_t)row[k] * p.ldo + col[k];
+    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int s0 = 0; s0 < npieces; s0 += 2) {
+    float4 x[N][2];
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        x[k][j] = ok[k] && s0 + j < npieces
+                      ? __ldcg(reinterpret_cast<const float4*>(b[k] + (size_t)(s0 + j) * p.piece_stride))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        v[k].x += x[k][j].x;
+        v[k].y += x[k][j].y;
+        v[k].z += x[k][j].z;
+        v[k].w += x[k][j].w;
+      }
+  }
+}
+
+DEVI uint2 pack_bf4(float a, float b, float c, float d) { return make_uint2(pack_bf2(a, b), pack_bf2(c, d)); }
+
 // Epilogue of one column group over rows [mz, mz + R) (consumer threads only).
 // rs_pre: row scales of rows [0, rows) computed at the kernel's start (single row group), or null.
+template <int E = -1>
 DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, const float* rs_pre = nullptr) {
+  const int epi = E >= 0 ? E : p.epi;  // a compile-time epilogue lets a kernel drop the other branches
   const int tid = threadIdx.x, nthr = kGemvConsumers * 32, warp = tid >> 5, lane = tid & 31;
   __shared__ float s_rs[72];
   const float* rsv = s_rs;
@@ -263,13 +300,51 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     const int f0 = grp * 64;
     const int rows = sk_rows(p, 0, mz, R);
     // the convolution's x_{t-1} of the group's first row may be the previous row group's last
-    const int pre = p.epi == EPI_DYNCONV && mz > 0 ? 1 : 0;
+    const int pre = epi == EPI_DYNCONV && mz > 0 ? 1 : 0;
     if (p.rs_in) {
       if (p.rs_glob) rsv = p.rs_glob + (mz - pre);
       else if (rs_pre && mz == 0) rsv = rs_pre;
       else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz - pre, rows + pre, s_rs);
     }
-    // four outputs per thread per round: all their partial loads are in flight together
+    if (epi != EPI_DYNCONV) {
+      // two groups of 4 features (gate and up partials each) per thread per round, 16-byte loads
+      constexpr int NQ = 2;
+      for (int i0 = tid; i0 < rows * 16; i0 += NQ * nthr) {
+        float4 sv[2 * NQ];
+        {
+          int rw[2 * NQ], cl[2 * NQ];
+          bool okk[2 * NQ];
+#pragma unroll
+          for (int k = 0; k < NQ; ++k) {
+            const int i = i0 + k * nthr, r = i >> 4, f = f0 + (i & 15) * 4;
+            okk[2 * k] = okk[2 * k + 1] = i < rows * 16;
+            rw[2 * k] = rw[2 * k + 1] = mz + r;
+            cl[2 * k] = p.seg[0].out_col + f;
+            cl[2 * k + 1] = p.seg[1].out_col + f;
+          }
+          sum_pieces_q<2 * NQ>(p, npieces, rw, cl, okk, sv);
+        }
+#pragma unroll
+        for (int k = 0; k < NQ; ++k) {
+          const int i = i0 + k * nthr, r = i >> 4, f = f0 + (i & 15) * 4;
+          if (i >= rows * 16) continue;
+          const float sc = p.rs_in ? rsv[r] : 1.f;
+          const float4 g = make_float4(sv[2 * k].x * sc, sv[2 * k].y * sc, sv[2 * k].z * sc, sv[2 * k].w * sc);
+          const float4 u =
+              make_float4(sv[2 * k + 1].x * sc, sv[2 * k + 1].y * sc, sv[2 * k + 1].z * sc, sv[2 * k + 1].w * sc);
+          if (epi == EPI_SWIGLU) {
+            *reinterpret_cast<uint2*>(p.act + (size_t)(mz + r) * p.F + f) =
+                pack_bf4(g.x / (1.f + __expf(-g.x)) * u.x, g.y / (1.f + __expf(-g.y)) * u.y,
+                         g.z / (1.f + __expf(-g.z)) * u.z, g.w / (1.f + __expf(-g.w)) * u.w);
+          } else {  // EPI_STORE
+            *reinterpret_cast<float4*>(p.y + (size_t)(mz + r) * p.ldy + p.seg[0].out_col + f) = g;
+            *reinterpret_cast<float4*>(p.y + (size_t)(mz + r) * p.ldy + p.seg[1].out_col + f) = u;
+          }
+        }
+      }
+      return;
+    }
+    // the convolution: four outputs per thread per round, all their partial loads in flight together
     constexpr int NO = 4;
     for (int i0 = tid; i0 < rows * 64; i0 += NO * nthr) {
       float gv[NO], uv[NO];
@@ -289,7 +364,7 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
           // the convolution's operands go out with the partial loads
           hc[k] = hp[k] = make_float4(0.f, 0.f, 0.f, 0.f);
           wv[k] = e0[k] = e1[k] = make_uint2(0, 0);
-          if (okk[2 * k] && p.epi == EPI_DYNCONV) {
+          if (okk[2 * k] && epi == EPI_DYNCONV) {
             const int row = mz + r, H = p.rs_H;
             hc[k] = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)row * H + 4 * f));
             if (row % p.Bk > 0) hp[k] = __ldcg(reinterpret_cast<const float4*>(p.dyn_h + (size_t)(row - 1) * H + 4 * f));
@@ -311,9 +386,9 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
         if (i >= rows * 64) continue;
         const float sc = p.rs_in ? rsv[pre + r] : 1.f;
         const float g = gv[k] * sc, u = uv[k] * sc;
-        if (p.epi == EPI_SWIGLU) {
+        if (epi == EPI_SWIGLU) {
           p.act[(size_t)(mz + r) * p.F + f] = f2bf(g / (1.f + __expf(-g)) * u);
-        } else if (p.epi == EPI_STORE) {
+        } else if (epi == EPI_STORE) {
           p.y[(size_t)(mz + r) * p.ldy + p.seg[0].out_col + f] = g;
           p.y[(size_t)(mz + r) * p.ldy + p.seg[1].out_col + f] = u;
         } else {  // EPI_DYNCONV: channels 4f .. 4f + 3 of block row mz + r, gates (g, u) of that row
@@ -338,12 +413,12 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
   if (tile0 < 0) return;
   const int col0 = p.seg[si].out_col + tile0 * 16;
   const int rows = sk_rows(p, si, mz, R);
-  if (p.rs_in && p.epi == EPI_STORE) {
+  if (p.rs_in && epi == EPI_STORE) {
     if (p.rs_glob) rsv = p.rs_glob + mz;
     else if (rs_pre && mz == 0) rsv = rs_pre;
     else rows_scale(p.rs_in, p.ssp_rows, p.rs_H, p.eps, mz, rows, s_rs);
   }
-  if (p.epi == EPI_QKV) {
+  if (epi == EPI_QKV) {
     const int head = tile0 / 8;
     for (int r = warp; r < rows; r += kGemvConsumers) {
       float x[4];
@@ -356,41 +431,52 @@ DEVI void sk_fixup(const SGemvParams& p, int grp, int mz, int R, int npieces, co
     }
     return;
   }
-  // eight outputs per thread per round: all their partial loads (and the residual reads) are in
-  // flight together before any store
-  constexpr int NR = 8;
-  for (int i0 = tid; i0 < rows * 128; i0 += NR * nthr) {
-    float v[NR], old[NR], hwf[NR];
+  // four groups of 4 consecutive columns per thread per round: all their partial loads (and the
+  // residual reads) are in flight together before any store; a warp covers one row's 128 columns
+  constexpr int NR = 4;
+  for (int i0 = tid; i0 < rows * 32; i0 += NR * nthr) {
+    float4 v[NR], old[NR];
+    uint2 hwv[NR];
     {
       int rw[NR], cl[NR];
       bool okk[NR];
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
         const int i = i0 + k * nthr;
-        rw[k] = mz + (i >> 7);
-        cl[k] = col0 + (i & 127);
-        okk[k] = i < rows * 128;
+        rw[k] = mz + (i >> 5);
+        cl[k] = col0 + (i & 31) * 4;
+        okk[k] = i < rows * 32;
         // L2 read: another CTA may have written the residual row
-        old[k] = okk[k] && p.epi == EPI_RESID ? __ldcg(p.y + (size_t)rw[k] * p.ldy + cl[k]) : 0.f;
-        hwf[k] = okk[k] && p.epi == EPI_RESID && p.hw ? bf2f(p.hw_w[cl[k]]) : 0.f;
+        old[k] = okk[k] && epi == EPI_RESID
+                     ? __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)rw[k] * p.ldy + cl[k]))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        hwv[k] = okk[k] && epi == EPI_RESID && p.hw ? *reinterpret_cast<const uint2*>(p.hw_w + cl[k])
+                                                     : make_uint2(0u, 0u);
       }
-      sum_pieces_n<NR>(p, npieces, rw, cl, okk, v);
+      sum_pieces_q<NR>(p, npieces, rw, cl, okk, v);
     }
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
-      const int i = i0 + k * nthr, r = i >> 7, c = col0 + (i & 127);
-      if (i >= rows * 128) break;  // warp-uniform: rows * 128 is a multiple of 32
+      const int i = i0 + k * nthr, r = i >> 5, c = col0 + (i & 31) * 4;
+      if (i >= rows * 32) break;  // warp-uniform: rows * 32 is a multiple of 32
       float* y = p.y + (size_t)(mz + r) * p.ldy + c;
-      if (p.epi == EPI_RESID) {
-        const float nv = old[k] + v[k];
-        *y = nv;
-        if (p.hw) p.hw[(size_t)(mz + r) * p.hw_ld + c] = f2bf(nv * hwf[k]);
-        if (p.ssp) {  // sum of squares of this warp's 32 columns of the new row, for the next RMSNorm
-          const float q = warp_sum(nv * nv);
-          if (lane == 0) p.ssp[((size_t)(col0 >> 7) * 4 + ((i >> 5) & 3)) * p.ssp_rows + mz + r] = q;
+      if (epi == EPI_RESID) {
+        const float4 nv = make_float4(old[k].x + v[k].x, old[k].y + v[k].y, old[k].z + v[k].z, old[k].w + v[k].w);
+        *reinterpret_cast<float4*>(y) = nv;
+        if (p.hw)
+          *reinterpret_cast<uint2*>(p.hw + (size_t)(mz + r) * p.hw_ld + c) =
+              pack_bf4(nv.x * bf2f(hwv[k].x & 0xffff), nv.y * bf2f(hwv[k].x >> 16), nv.z * bf2f(hwv[k].y & 0xffff),
+                       nv.w * bf2f(hwv[k].y >> 16));
+        if (p.ssp) {  // sum of squares of each 32-column quarter of the new row (8 lanes), for the next RMSNorm
+          float q = nv.x * nv.x + nv.y * nv.y + nv.z * nv.z + nv.w * nv.w;
+          q += __shfl_xor_sync(0xffffffffu, q, 1);
+          q += __shfl_xor_sync(0xffffffffu, q, 2);
+          q += __shfl_xor_sync(0xffffffffu, q, 4);
+          if ((lane & 7) == 0) p.ssp[((size_t)(col0 >> 7) * 4 + (lane >> 3)) * p.ssp_rows + mz + r] = q;
         }
       } else {
-        *y = p.rs_in ? v[k] * rsv[r] : v[k];
+        const float sc = p.rs_in ? rsv[r] : 1.f;
+        *reinterpret_cast<float4*>(y) = make_float4(v[k].x * sc, v[k].y * sc, v[k].z * sc, v[k].w * sc);
       }
     }
   }

@@ -650,8 +650,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_cons
 
 // Split-K fix-up of the tensor-core products: the CTA of (64-row group, column group) sums the
 // pieces of its tile in piece order (deterministic) and runs the product's fused epilogue.
-// P: the tensor-core launch's grid size (p.W its stream-K plane).
-__global__ void __launch_bounds__(kGemvConsumers * 32, 1) k_umma_fixup(SGemvParams p, int P) {
+// P: the tensor-core launch's grid size (p.W its stream-K plane).  E: the epilogue, fixed at compile
+// time so that the light ones (residual, SwiGLU, store) fit two CTAs per SM.
+template <int E, int MINB>
+__global__ void __launch_bounds__(kGemvConsumers * 32, MINB) k_umma_fixup(SGemvParams p, int P) {
   pdl_trigger();
   pdl_wait();
   const int grp = blockIdx.x % p.groups, mz = (blockIdx.x / p.groups) * 64;
@@ -662,7 +664,7 @@ __global__ void __launch_bounds__(kGemvConsumers * 32, 1) k_umma_fixup(SGemvPara
   int si;
   sk_tile(p, grp, 0, si);
   if (sk_rows(p, si, mz, 64) <= 0) return;
-  sk_fixup(p, grp, mz, 64, npieces, nullptr);
+  sk_fixup<E>(p, grp, mz, 64, npieces, nullptr);
 }
 
 }  // namespace dfl
