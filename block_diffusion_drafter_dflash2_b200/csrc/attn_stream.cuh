@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
                                                               uint16_t* __restrict__ ob) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[kAsStages], empty[kAsStages];
-  __shared__ int pvalid[kAsStages][4];
+  __shared__ int pvalid[kAsStages];  // bit i: page i of the stage's chunk is mapped
   __shared__ float mrg_m[2][16], mrg_l[2][16];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = smem;
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
       for (int c = 0; c < nc && !dead; ++c) {
         const int s = c % kAsStages, round = c / kAsStages;
         if (round > 0 && !wait_or_die(&empty[s], (round - 1) & 1, dead, p.err)) break;
-        int pg[4];
+        int pg[4], pv = 0;
         uint32_t bytes = 0;
         for (int pi = 0; pi < 4; ++pi) {
           const long long j0 = cs + (long long)c * kAsKeys + pi * kPage;  // first token of the page
@@ -178,8 +178,9 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
             }
           }
           pg[pi] = g;
-          pvalid[s][pi] = g >= 0 ? 1 : 0;
+          pv |= (g >= 0 ? 1 : 0) << pi;
         }
+        pvalid[s] = pv;
         uint8_t* st = stages + s * kAsStage;
         if (bytes) {
           mbar_expect_tx(&full[s], bytes);
@@ -228,11 +229,15 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks)
     ldmatrix_x4(qa[ks], reinterpret_cast<const uint8_t*>(Qs) + (qt * 16 + (lane & 15)) * 256 + (ks * 16 + (lane >> 4) * 8) * 2);
+  // window start of each of the thread's two rows relative to the first cached key of the walk:
+  // block row t sees cache keys j >= Lb + t - W + 1 (padding vectors see no key)
   int trow[2];
+  long long lo0[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int qv = qt * 16 + g + 8 * h;
-    trow[h] = qv < nqv ? qv / G : -1;  // -1: padding vector, sees nothing
+    trow[h] = qv < nqv ? qv / G : -1;
+    lo0[h] = trow[h] >= 0 ? Lb + trow[h] - p.W + 1 - cs : (long long)INT_MAX;
   }
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, o[16][4];
 #pragma unroll
@@ -244,18 +249,29 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
     const uint8_t* st = stages + s * kAsStage;
     float sc[4][4];
     as_scores<4>(qa, st, kAsHalf, kh * 32, sc, lane);
-    // mask: cache key j = cs + 64c + kk visible to block row t iff its page is mapped, j < Lb and
-    // j >= Lb + t - W + 1
+    // mask: key kk of the chunk (cache key j = cs + 64c + kk) is visible to the row iff its page is
+    // mapped, j < Lb and j >= Lb + t - W + 1; chunk-relative bounds in int, clamped to [0, 65]
+    const long long c64 = (long long)c * kAsKeys;
+    const int hi = (int)min(max(Lb - cs - c64, 0ll), 65ll);
+    int lo[2];
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int h = 0; h < 2; ++h) lo[h] = (int)min(max(lo0[h] - c64, 0ll), 65ll);
+    const int pv = pvalid[s];
+    if (__all_sync(0xffffffffu, lo[0] == 0 && lo[1] == 0 && hi >= kAsKeys && pv == 0xF)) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kk = kh * 32 + n * 8 + 2 * t4 + (e & 1);
-        const long long j = cs + (long long)c * kAsKeys + kk;
-        const int t = trow[e >> 1];
-        const bool vis = t >= 0 && pvalid[s][kk >> 4] && j < Lb && j >= Lb + t - p.W + 1;
-        sc[n][e] = vis ? sc[n][e] * p.scale_log2 : -INFINITY;
-      }
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[n][e] *= p.scale_log2;
+    } else {
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kk = kh * 32 + n * 8 + 2 * t4 + (e & 1);
+          const bool vis = kk >= lo[e >> 1] && kk < hi && ((pv >> (kk >> 4)) & 1);
+          sc[n][e] = vis ? sc[n][e] * p.scale_log2 : -INFINITY;
+        }
+    }
     as_softmax<4>(sc, m, l, o);
     as_pv<2>(sc, st + 2 * kAsHalf, kAsHalf, kh * 32, o, lane);
     __syncwarp();
