@@ -3,15 +3,17 @@
 // window's cache pages through a ring of TMA stages.
 //
 // With many requests the cluster kernel (attention.cuh) runs thousands of short CTAs, one per SM at
-// a time, each paying the whole load-compute-merge latency.  Here a CTA owns a (request, kv head)
-// for the whole window, two CTAs share an SM, and the loads run ahead of the math:
+// a time, each paying the whole load-compute-merge latency.  Here a cluster of S CTAs (S = 1 when
+// the (request, kv head) pairs alone fill the SMs two deep) owns a pair for the whole window, CTA
+// r of it taking chunks r, r + S, ...; two CTAs share an SM, and the loads run ahead of the math:
 //  * warp 4, one thread: for each 64-key chunk (4 pages of 16 tokens), the 4 KiB K and V rows of
 //    this kv head in each page by 2-D TMA (cp.async.bulk.tensor, no multicast) as two 64-dim boxes
 //    with 128-byte swizzle into one of two 32 KB stages; unmapped pages are skipped and flagged;
 //  * warps 0-3: warp (qt, kh) takes query tile qt (16 of the kv head's G x Bk query vectors) and
 //    key half kh (32 keys) of every chunk: S = Q K^T and P V on mma.sync m16n8k16 with an online
 //    softmax (running max, sum and output in registers); then the block's own keys (all visible);
-//    the two key halves of a query tile merge in shared memory at the end.
+//    the two key halves of a query tile merge in shared memory, then the S CTAs' (max, sum,
+//    output) merge over distributed shared memory, CTA r finishing 32/S of the query vectors.
 // Visibility as everywhere: block row t at position p = Lb + t sees cache keys
 // max(0, p - W + 1) <= j < Lb and every block key.  Softmax in fp32, scale 1/sqrt(128).
 #pragma once
@@ -118,7 +120,8 @@ DEVI void as_softmax(float (&s)[4][4], float (&m)[2], float (&l)[2], float (&o)[
 }
 
 // tmk / tmv: the layer's K and V caches as [pages * nkv * 16 rows][128] bf16 tensors (boxes of 16
-// rows x 64 dims, 128-byte swizzle).  Grid (nkv, B).  Requires G * Bk <= 32 (two query tiles).
+// rows x 64 dims, 128-byte swizzle).  Grid (S, nkv, B), clusters of (S, 1, 1), S in 1..8.
+// Requires G * Bk <= 32 (two query tiles).
 __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_constant__ CUtensorMap tmk,
                                                               const __grid_constant__ CUtensorMap tmv, AttnParams p,
                                                               uint16_t* __restrict__ ob) {
@@ -126,11 +129,13 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
   __shared__ __align__(8) uint64_t full[kAsStages], empty[kAsStages];
   __shared__ int pvalid[kAsStages];  // bit i: page i of the stage's chunk is mapped
   __shared__ float mrg_m[2][16], mrg_l[2][16];
+  __shared__ float fin_m[32], fin_l[32];  // this CTA's running max and sum per query vector
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = smem;
   uint8_t* blk = smem + kAsStages * kAsStage;  // block keys: K lo | K hi | V lo | V hi, 16 rows each
   uint16_t* Qs = reinterpret_cast<uint16_t*>(blk + kAsBlk);  // [32][128] bf16
-  const int kvh = blockIdx.x, b = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = gridDim.x, rank = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.nq / p.nkv, nqv = G * p.Bk;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAsStages; ++s) {
@@ -152,14 +157,15 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
   if (s0 < 0) s0 = 0;
   const long long cs = (s0 / kPage) * kPage;
   const int nc = (int)((Lb - cs + kAsKeys - 1) / kAsKeys);
+  const int nloc = nc > rank ? (nc - rank + S - 1) / S : 0;  // this CTA's chunks: rank + i S
 
   if (warp == 4) {
-    // ---- producer: the window's pages, chunk by chunk ----
+    // ---- producer: this CTA's share of the window's pages, chunk by chunk ----
     if (lane == 0) {
       bool dead = false;
       int issued = 0;
-      for (int c = 0; c < nc && !dead; ++c) {
-        const int s = c % kAsStages, round = c / kAsStages;
+      for (int i = 0; i < nloc && !dead; ++i) {
+        const int c = rank + i * S, s = i % kAsStages, round = i / kAsStages;
         if (round > 0 && !wait_or_die(&empty[s], (round - 1) & 1, dead, p.err)) break;
         int pg[4], pv = 0;
         uint32_t bytes = 0;
@@ -195,17 +201,17 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
         } else {
           mbar_arrive(&full[s]);  // (releases the page flags)
         }
-        issued = c + 1;
+        issued = i + 1;
       }
       // the CTA must not retire with copies into its shared memory still in flight (the math warps
       // may have stopped early on a timeout): wait, bounded, for the last stages issued
-      for (int c = issued > kAsStages ? issued - kAsStages : 0; c < issued; ++c) {
+      for (int i = issued > kAsStages ? issued - kAsStages : 0; i < issued; ++i) {
         bool d2 = false;
-        wait_or_die(&full[c % kAsStages], (c / kAsStages) & 1, d2, p.err);
+        wait_or_die(&full[i % kAsStages], (i / kAsStages) & 1, d2, p.err);
       }
     }
-    return;
-  }
+    __syncwarp();
+  } else {
 
   // ---- math warps: stage Q and the block keys (cp.async), then stream the chunks ----
   for (int i = threadIdx.x; i < 32 * 16; i += 128) {  // Q: 32 vectors x 16 chunks of 16 B
@@ -243,9 +249,9 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
 #pragma unroll
   for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   bool dead = false;
-  for (int c = 0; c < nc; ++c) {
-    const int s = c % kAsStages;
-    if (!wait_or_die(&full[s], (c / kAsStages) & 1, dead, p.err)) break;
+  for (int i = 0; i < nloc; ++i) {
+    const int c = rank + i * S, s = i % kAsStages;
+    if (!wait_or_die(&full[s], (i / kAsStages) & 1, dead, p.err)) break;
     const uint8_t* st = stages + s * kAsStage;
     float sc[4][4];
     as_scores<4>(qa, st, kAsHalf, kh * 32, sc, lane);
@@ -277,9 +283,9 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);  // this warp's reads of the stage are done
   }
-  // the block's own keys (rows 0 .. Bk-1 of the block area, zero-filled to 16), all visible: both
-  // key halves score the 16 rows, half kh keeps rows 8kh .. 8kh + 7
-  if (!dead) {
+  // the block's own keys (rows 0 .. Bk-1 of the block area, zero-filled to 16), all visible, in CTA
+  // 0 of the cluster: both key halves score the 16 rows, half kh keeps rows 8kh .. 8kh + 7
+  if (!dead && rank == 0) {
     float sc[4][4];
     as_scores<2>(qa, blk, 16 * 128, 0, sc, lane);
 #pragma unroll
@@ -293,9 +299,10 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
     as_softmax<2>(sc, m, l, o);
     as_pv<1>(sc, blk + 2 * (16 * 128), 16 * 128, 0, o, lane);
   }
-  // ---- merge the two key halves of each query tile; kh = 0 writes the output ----
+  // ---- merge the two key halves of each query tile into this CTA's (max, sum, output) ----
   asm volatile("bar.sync 1, 128;" ::: "memory");  // every warp is done with the stages and blk
-  float* red = reinterpret_cast<float*>(stages);  // [qt][16 rows][128] of the kh = 1 warps
+  float* red = reinterpret_cast<float*>(stages);                  // [qt][16 rows][128], key half 1
+  float* fin = reinterpret_cast<float*>(stages) + 2 * 16 * 128;  // [32 vectors][128], unnormalised
   if (kh == 1) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -318,18 +325,44 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
       const float m1 = mrg_m[qt][row], l1 = mrg_l[qt][row];
       const float M = fmaxf(m[h], m1);
       const float w0 = M == -INFINITY ? 0.f : exp2f(m[h] - M), w1 = M == -INFINITY ? 0.f : exp2f(m1 - M);
-      const float L = w0 * l[h] + w1 * l1, inv = L > 0.f ? 1.f / L : 0.f;
-      if (qv < nqv) {
-        uint16_t* dst = ob + ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          const float2 v1 = *reinterpret_cast<const float2*>(red + ((size_t)qt * 16 + row) * 128 + n * 8 + 2 * t4);
-          const float x = (w0 * o[n][2 * h] + w1 * v1.x) * inv, y = (w0 * o[n][2 * h + 1] + w1 * v1.y) * inv;
-          *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * t4) = pack_bf2(x, y);
-        }
+      for (int n = 0; n < 16; ++n) {
+        const float2 v1 = *reinterpret_cast<const float2*>(red + ((size_t)qt * 16 + row) * 128 + n * 8 + 2 * t4);
+        *reinterpret_cast<float2*>(fin + (size_t)qv * 128 + n * 8 + 2 * t4) =
+            make_float2(w0 * o[n][2 * h] + w1 * v1.x, w0 * o[n][2 * h + 1] + w1 * v1.y);
+      }
+      if (t4 == 0) {
+        fin_m[qv] = M;
+        fin_l[qv] = w0 * l[h] + w1 * l1;
       }
     }
   }
+  }  // math warps
+  // ---- the cluster's CTAs merge: CTA `rank` finishes query vectors [rank * 32 / S, ...) ----
+  cluster_sync_all();  // every CTA's (max, sum, output) is in its shared memory
+  {
+    float* fin = reinterpret_cast<float*>(stages) + 2 * 16 * 128;
+    const int v0 = rank * 32 / S, v1 = (rank + 1) * 32 / S;
+    for (int i = threadIdx.x; i < (v1 - v0) * 64; i += kAsThreads) {
+      const int qv = v0 + i / 64, d = (i % 64) * 2;
+      if (qv >= nqv) continue;
+      float M = -INFINITY;
+      for (int r = 0; r < S; ++r) M = fmaxf(M, ld_cluster_f32(cluster_map(&fin_m[qv], r)));
+      float L = 0.f, x = 0.f, y = 0.f;
+      for (int r = 0; r < S; ++r) {
+        const float mr = ld_cluster_f32(cluster_map(&fin_m[qv], r));
+        const float wr = mr == -INFINITY ? 0.f : exp2f(mr - M);
+        const float2 orr = ld_cluster_f32x2(cluster_map(fin + (size_t)qv * 128 + d, r));
+        L += wr * ld_cluster_f32(cluster_map(&fin_l[qv], r));
+        x += wr * orr.x;
+        y += wr * orr.y;
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      uint16_t* dst = ob + ((size_t)(b * p.Bk + qv / G) * p.nq + kvh * G + qv % G) * kHeadDim;
+      *reinterpret_cast<uint32_t*>(dst + d) = pack_bf2(x * inv, y * inv);
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
 }
 
 }  // namespace dfl

@@ -38,7 +38,8 @@ struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
   int attn_ntk;  // > 0: attention as one cluster kernel, attn_kg key groups of 8*attn_ntk keys per CTA; 0: chunks + merge
   int attn_kg;
-  bool attn_stream;  // one streaming CTA per (request, kv head) with TMA-staged pages (many requests)
+  bool attn_stream;  // streaming CTAs per (request, kv head) with TMA-staged pages (many requests)
+  int attn_split;    // its cluster size: CTAs sharing one (request, kv head)'s window
   bool q4, mlx;
   GemvPlan fc, dc, qkv, o, gu, dn;
   size_t off_cfv, off_cfi, off_ssp, off_tau, off_hpart, off_rope, off_rpage;
@@ -192,6 +193,10 @@ Plan make_plan(const dflash2_config* c, int B) {
   // With 8 or more requests the (request, kv head) pairs fill the SMs two deep, and a CTA that keeps
   // its window's pages streaming beats clusters that each pay the whole load-compute-merge latency.
   p.attn_stream = B >= kAttnStreamMinBatch && p.QV <= 32;
+  // CTAs per (request, kv head) for the streaming kernel: the fewest (a power of two, at most 8)
+  // that give about two CTAs per SM
+  p.attn_split = 1;
+  while (p.attn_split < 8 && (long long)B * c->n_kv * p.attn_split * 5 < 4LL * 2 * p.nsm) p.attn_split *= 2;
   p.fc = plan_gemv(p.H / 16, p.Mb, p.T * p.H, p.q4, p.nsm);
   p.dc = plan_gemv((p.H / 2) / 16, p.Mb, p.H, false, p.nsm);
   p.qkv = plan_gemv((p.HQ + 2 * p.HKV) / 16, 2 * p.Mb, p.H, p.q4, p.nsm);
@@ -504,7 +509,21 @@ cudaError_t launch_attn_stream(const Plan& P, const AttnParams& ap, uint16_t* ob
   CUtensorMap tk, tv;
   if ((e = make_kv_tmap(&tk, ap.kc, ap.num_pages, ap.nkv)) != cudaSuccess) return e;
   if ((e = make_kv_tmap(&tv, ap.vc, ap.num_pages, ap.nkv)) != cudaSuccess) return e;
-  return launch_pdl(k_attn_stream, dim3(ap.nkv, P.B), dim3(kAsThreads), (size_t)kAsSmem, s, tk, tv, ap, ob);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.attn_split, ap.nkv, P.B);
+  cfg.blockDim = dim3(kAsThreads);
+  cfg.dynamicSmemBytes = kAsSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = P.attn_split;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_attn_stream, tk, tv, ap, ob);
 }
 
 template <int MT, int NTK, int KG>
