@@ -988,7 +988,7 @@ int draft_step_impl(const dflash2_config* c, const dflash2_weights* w, const dfl
       hp.cand_val = at<float>(ws, P.off_cv);
       hp.cand_id = at<int32_t>(ws, P.off_ci);
       hp.err = err;
-      CK(launch_pdl(k_umma_head, dim3(P.lm_uP), dim3(kUmmaThreads), (size_t)kUHeadSmem, s, tm, hp));
+      CK(launch_pdl(k_umma_head, dim3(P.lm_uP), dim3(kUHeadThreads), (size_t)kUHeadSmem, s, tm, hp));
     } else {
       static std::atomic<int> attr[kMaxDevices];
       CK(smem_optin(k_slmhead, kSmemLimit - kStaticSmem, attr));

@@ -37,8 +37,9 @@ constexpr int kUmmaRaw = 3;                        // raw weight-record slots (o
 constexpr int kUmmaABytes = 128 * 128;             // [128 features][64 k] bf16
 constexpr int kUmmaBBytes = kUmmaRows * 128;       // [256 rows][64 k] bf16
 constexpr int kUmmaRawBytes = 8 * kQ4Bytes;        // one group unit (Q4_K 18 KB; bf16 units are 16 KB)
-constexpr int kUmmaDq = 8;                         // weight-operand warps (one tile of the group each)
+constexpr int kUmmaDq = 16;                        // weight-operand warps (a tile's 32-wide half each)
 constexpr int kUmmaThreads = (4 + kUmmaDq + 4) * 32; // roles below
+constexpr int kUHeadThreads = 16 * 32;               // the output head's roles
 constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + kUmmaRaw * kUmmaRawBytes + 1024;
 constexpr int kUmmaTmemCols = 512;                 // two 256-column accumulators
 
@@ -156,13 +157,14 @@ DEVI void rows_scale_global(const float* ssp, int ldr, int H, float eps, int r0,
   }
 }
 
-// Roles (16 warps): warp 0 one thread: activation TMA; warp 1: TMEM allocation, one thread issues
+// Roles (24 warps): warp 0 one thread: activation TMA; warp 1: TMEM allocation, one thread issues
 // the MMAs; warp 2 one thread: raw weight records into the raw ring (bulk copies, started before
 // the dependency wait: the weights do not depend on earlier kernels); warp 3: the row scales of
-// a folded RMSNorm for the fix-up (p.rs_glob); warps 4-11: the weight operand from the raw ring,
-// one 16-feature tile each (two warps per SM sub-partition, so one's latencies hide behind the
-// other's work: with one per sub-partition the dequantisation bounded the kernel); warps 12-15:
-// epilogue (TMEM lane = feature), on two accumulators alternating by piece.
+// a folded RMSNorm for the fix-up (p.rs_glob); warps 4-19: the weight operand from the raw ring,
+// one 32-wide half of one 16-feature tile each (four warps per SM sub-partition, so their
+// latencies hide behind one another's work: the dequantisation's dependent chains bounded the
+// kernel with one or two per sub-partition); warps 20-23: epilogue (TMEM lane = feature), on two
+// accumulators alternating by piece.
 template <bool Q4>
 __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -299,7 +301,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
     }
   } else if (warp < 4 + kUmmaDq) {
     // ---- weight operand: raw ring -> swizzled K-major stage (warp = one tile of the group) ----
-    const int tl = warp - 4, g = lane >> 2, t = lane & 3;
+    // warp = one 32-wide half jh of every 64-wide stage of tile tl
+    const int tl = (warp - 4) % 8, jh = (warp - 4) / 8, g = lane >> 2, t = lane & 3;
     bool dead = false;
     int cnt = 0, ucnt = 0;
     for (long long x = x0; x < x1;) {
@@ -332,14 +335,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
 #pragma unroll
           for (int sub = 0; sub < kSub; ++sub, ++cnt) {
             const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
-            if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
             uint8_t* a = As + s * kUmmaABytes;
+            // features g and g + 8 of tile tl go to operand rows 16 tl + a8(g) and + 8: a8 puts the
+            // two features of each 8-lane store phase 4 rows apart, so that the phase's 16-byte
+            // chunks land in distinct swizzled bank groups (the epilogue maps TMEM lanes back)
+            const int m0 = tl * 16 + ((g >> 1) | ((g & 1) << 2));
+            // the operand values are formed from the raw unit first, so that only the stores wait
+            // for the tensor cores to free the stage
+            uint4 rg = make_uint4(0u, 0u, 0u, 0u), rh = rg;
             if (!dead) {
-              const int m0 = tl * 16 + g;  // operand rows g and g+8 of tile tl
               const uint8_t* rec = raw + tl * (Q4 ? kQ4Bytes : 2048);
-#pragma unroll
-              for (int jj = 0; jj < 2; ++jj) {  // 32-wide sub-blocks of the stage
-                uint4 rg, rh;
+              {
+                const int jj = jh;  // this warp's 32-wide sub-block of the stage
                 if (Q4) {
                   const uint4 q = *reinterpret_cast<const uint4*>(rec + (sub * 32 + lane) * 16);
                   const uint32_t w0 = jj ? q.z : q.x, w1 = jj ? q.w : q.y;
@@ -364,9 +371,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
                   rg = *reinterpret_cast<const uint4*>(rec + jj * 1024 + lane * 16);
                   rh = *reinterpret_cast<const uint4*>(rec + jj * 1024 + 512 + lane * 16);
                 }
-                *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jj + t)) = rg;
-                *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jj + t)) = rh;
               }
+            }
+            if (round > 0) wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err);
+            if (!dead) {
+              *reinterpret_cast<uint4*>(a + sw128_off(m0, 4 * jh + t)) = rg;
+              *reinterpret_cast<uint4*>(a + sw128_off(m0 + 8, 4 * jh + t)) = rh;
             }
             fence_proxy_async_smem();  // these generic writes feed the tensor cores (async proxy)
             __syncwarp();
@@ -398,12 +408,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
         const int pc = (int)(c - sk_owner((long long)gidx * p.U, p.W, P));
         if (wait_or_die(&accfull[buf], use & 1, dead, p.err)) {
           tc_fence_after();
-          const int m = ew * 32 + lane;  // TMEM lane = feature of the column group
+          const int m = ew * 32 + lane;  // TMEM lane = operand row: feature 16 (m / 16) + fo
+          const int fo = (m & 8) | ((m & 3) << 1) | ((m >> 2) & 1);
           int si;
           const int tile = sk_tile(p, grp, m >> 4, si);
           const int rows = tile >= 0 ? sk_rows(p, si, mz, kUmmaRows) : 0;
           float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mz * p.ldo +
-                       (tile >= 0 ? p.seg[si].out_col + tile * 16 + (m & 15) : 0);
+                       (tile >= 0 ? p.seg[si].out_col + tile * 16 + fo : 0);
           const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kUmmaRows);
           for (int n0 = 0; n0 < kUmmaRows; n0 += 32) {
             uint32_t v[32];
@@ -490,7 +501,7 @@ DEVI void reg_list_insert(float (&lv)[16], int (&li)[16], float v, int id) {
   }
 }
 
-__global__ void __launch_bounds__(kUmmaThreads, 1) k_umma_head(const __grid_constant__ CUtensorMap tmx, UHeadParams p) {
+__global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_constant__ CUtensorMap tmx, UHeadParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t xfull[kUHeadStages], bfull[kUHeadStages], sempty[kUHeadStages];
   __shared__ __align__(8) uint64_t accfull, accempty;
