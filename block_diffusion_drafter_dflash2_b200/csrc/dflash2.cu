@@ -26,13 +26,17 @@ struct GemvPlan {
   long long W = 1;
   size_t smem = 0;
   bool umma = false;  // tensor-core (tcgen05) product + fix-up instead of the streaming engine
+  int un = 0;         // its activation rows per tile (MMA N): all rows up to 256, rounded up to 16
   bool mlx = false;   // 4-bit records hold MLX group-64 (scale, bias) pairs
   int rows = 0, K = 0;
 };
 
-// Above this many activation rows a product runs on the tcgen05 tensor cores (k_umma): the
-// streaming engine would need several 64-row groups, each re-reading the weights.
-constexpr int kUmmaMinRows = 65;
+// From this many activation rows on a product runs on the tcgen05 tensor cores (k_umma, the
+// tile's N = the rows rounded up to 16): the streaming engine's warps re-read every activation
+// fragment from shared memory for each weight fragment, which at 32 rows and more costs more than
+// the tensor-core path's dequantisation (measured: full shape at 4, 5 and 8 requests 2.29 -> 2.04,
+// 2.97 -> 2.11 and 3.67 -> 2.14 ms per step; at 24 rows the streaming engine is still ahead).
+constexpr int kUmmaMinRows = 32;
 
 struct Plan {
   int B, Bk, D, Mb, H, F, HQ, HKV, T, V, R, nsm, G, QV, QVP, MT, NC;
@@ -73,6 +77,7 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
   if (rows >= kUmmaMinRows) {
     g.umma = true;
     g.R = kUmmaRows;
+    g.un = rows >= kUmmaRows ? kUmmaRows : (rows + 15) / 16 * 16;
     g.NT = 8;
     g.mgroups = (rows + kUmmaRows - 1) / kUmmaRows;
     g.groups = (tiles + kConsumers - 1) / kConsumers;
@@ -393,6 +398,7 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   prm.err = err;
   prm.rs_glob = (g.umma && e.rs_in) ? e.rs_glob : nullptr;
   prm.mlx = g.mlx ? 1 : 0;
+  prm.un = g.un;
   return prm;
 }
 
@@ -418,14 +424,15 @@ EncodeTiledFn encode_tiled() {
   return f;
 }
 
-// Tensor map of a bf16 activation matrix [rows][ldx] (K valid columns): boxes of 64 columns x 256
-// rows, 128-byte swizzle (the tcgen05 K-major operand layout); rows past the end read as zero.
-cudaError_t make_act_tmap(CUtensorMap* tm, const uint16_t* X, int K, int ldx, int rows) {
+// Tensor map of a bf16 activation matrix [rows][ldx] (K valid columns): boxes of 64 columns x
+// box_rows rows, 128-byte swizzle (the tcgen05 K-major operand layout); rows past the end read as
+// zero.
+cudaError_t make_act_tmap(CUtensorMap* tm, const uint16_t* X, int K, int ldx, int rows, int box_rows = kUmmaRows) {
   const EncodeTiledFn f = encode_tiled();
   if (!f) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kUmmaRows};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = f(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -441,7 +448,7 @@ cudaError_t launch_umma_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_
   cudaError_t e = smem_optin(k_umma<Q4>, kUmmaSmem, attr);
   if (e != cudaSuccess) return e;
   CUtensorMap tm;
-  e = make_act_tmap(&tm, prm.X, g.K, prm.ldx, prm.rows);
+  e = make_act_tmap(&tm, prm.X, g.K, prm.ldx, prm.rows, g.un);
   if (e != cudaSuccess) return e;
   e = launch_pdl(k_umma<Q4>, dim3(g.P), dim3(kUmmaThreads), (size_t)kUmmaSmem, s, tm, prm);
   if (e != cudaSuccess) return e;

@@ -108,6 +108,7 @@ struct SGemvParams {
   // tensor-core path: the row scales of rs_in, computed once per product by its kernel, [rows]
   float* rs_glob;
   int mlx;  // 4-bit records carry MLX group-64 (scale, bias) pairs instead of Q4_K scale records
+  int un;   // tensor-core path: activation rows per tile (the MMA's N and the TMA box height)
 };
 
 // Row scales of rows [mz, mz + rows) from quarter-column sums of squares (ssp layout

@@ -98,9 +98,12 @@ DEVI uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
          ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
-// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N = 256, M = 128.
-constexpr uint32_t kUmmaIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kUmmaRows >> 3) << 17) |
-                                ((uint32_t)(128 >> 4) << 24);
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M = 128, N = n (a multiple
+// of 16 up to 256).
+DEVI constexpr uint32_t umma_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+constexpr uint32_t kUmmaIdesc = umma_idesc(kUmmaRows);
 
 // Byte offset of the 16-byte chunk c (k = 8c .. 8c+7) of row m in a 128-byte-swizzled stage.
 DEVI uint32_t sw128_off(int m, int c) { return (uint32_t)(m * 128 + ((c ^ (m & 7)) << 4)); }
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
             for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
               const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
               if (round > 0 && !wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err)) break;
-              mbar_expect_tx(&xfull[s], kUmmaBBytes);
+              mbar_expect_tx(&xfull[s], (uint32_t)p.un * 128u);  // the box: un rows of 64 k
               tma_load_2d(Bs + s * kUmmaBBytes, &tmx, u * kUnitK + sub * 64, mz, &xfull[s]);
             }
         }
@@ -248,6 +251,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           if (use > 0 && !wait_or_die(&accempty[buf], (use - 1) & 1, dead, p.err)) break;
           tc_fence_after();
           const uint32_t acc = tmem + (uint32_t)(buf * kUmmaRows);
+          const uint32_t idesc = umma_idesc(p.un);  // N = the tile's rows
           bool first = true;
           for (int u = ua; u < ub && !dead; ++u)
             for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
@@ -259,7 +263,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
               const uint64_t bd = sw128_desc(smem_u32(Bs + s * kUmmaBBytes));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes inside the swizzled rows
-                tc_mma(acc, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (first && kk == 0) ? 0u : 1u);
+                tc_mma(acc, ad + 2 * kk, bd + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
               first = false;
               tc_commit(&sempty[s]);  // the stage is free once these MMAs have read it
             }
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mz * p.ldo +
                        (tile >= 0 ? p.seg[si].out_col + tile * 16 + fo : 0);
           const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kUmmaRows);
-          for (int n0 = 0; n0 < kUmmaRows; n0 += 32) {
+          for (int n0 = 0; n0 < rows && n0 < p.un; n0 += 32) {
             uint32_t v[32];
             tmem_ld32(tbase + (uint32_t)n0, v);
             tmem_ld_wait();
