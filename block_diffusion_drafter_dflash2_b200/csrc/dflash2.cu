@@ -452,14 +452,18 @@ cudaError_t launch_umma_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_
   if (e != cudaSuccess) return e;
   e = launch_pdl(k_umma<Q4>, dim3(g.P), dim3(kUmmaThreads), (size_t)kUmmaSmem, s, tm, prm);
   if (e != cudaSuccess) return e;
-  const int fix_blocks = prm.groups * ((prm.rows + 63) / 64);
+  // rows per fix-up CTA: 64, halved (down to 16) while the grid would leave SMs idle (the fix-ups
+  // of products with few column groups are latency-bound)
+  int fr = 64;
+  while (fr > 16 && (long long)prm.groups * ((prm.rows + fr - 1) / fr) < g.P) fr /= 2;
+  const int fix_blocks = prm.groups * ((prm.rows + fr - 1) / fr);
   const dim3 fg(fix_blocks), fb(kGemvConsumers * 32);
   switch (prm.epi) {
-    case EPI_RESID: return launch_pdl(k_umma_fixup<EPI_RESID, 2>, fg, fb, 0, s, prm, g.P);
-    case EPI_SWIGLU: return launch_pdl(k_umma_fixup<EPI_SWIGLU, 2>, fg, fb, 0, s, prm, g.P);
-    case EPI_STORE: return launch_pdl(k_umma_fixup<EPI_STORE, 2>, fg, fb, 0, s, prm, g.P);
-    case EPI_QKV: return launch_pdl(k_umma_fixup<EPI_QKV, 1>, fg, fb, 0, s, prm, g.P);
-    default: return launch_pdl(k_umma_fixup<EPI_DYNCONV, 1>, fg, fb, 0, s, prm, g.P);
+    case EPI_RESID: return launch_pdl(k_umma_fixup<EPI_RESID, 2>, fg, fb, 0, s, prm, g.P, fr);
+    case EPI_SWIGLU: return launch_pdl(k_umma_fixup<EPI_SWIGLU, 2>, fg, fb, 0, s, prm, g.P, fr);
+    case EPI_STORE: return launch_pdl(k_umma_fixup<EPI_STORE, 2>, fg, fb, 0, s, prm, g.P, fr);
+    case EPI_QKV: return launch_pdl(k_umma_fixup<EPI_QKV, 1>, fg, fb, 0, s, prm, g.P, fr);
+    default: return launch_pdl(k_umma_fixup<EPI_DYNCONV, 1>, fg, fb, 0, s, prm, g.P, fr);
   }
 }
 

@@ -663,23 +663,24 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
   }
 }
 
-// Split-K fix-up of the tensor-core products: the CTA of (64-row group, column group) sums the
+// Split-K fix-up of the tensor-core products: the CTA of (fr-row group, column group) sums the
 // pieces of its tile in piece order (deterministic) and runs the product's fused epilogue.
 // P: the tensor-core launch's grid size (p.W its stream-K plane).  E: the epilogue, fixed at compile
 // time so that the light ones (residual, SwiGLU, store) fit two CTAs per SM.
 template <int E, int MINB>
-__global__ void __launch_bounds__(kGemvConsumers * 32, MINB) k_umma_fixup(SGemvParams p, int P) {
+// fr: rows per CTA (16, 32 or 64; fewer rows give few-row products more CTAs in flight).
+__global__ void __launch_bounds__(kGemvConsumers * 32, MINB) k_umma_fixup(SGemvParams p, int P, int fr) {
   pdl_trigger();
   pdl_wait();
-  const int grp = blockIdx.x % p.groups, mz = (blockIdx.x / p.groups) * 64;
+  const int grp = blockIdx.x % p.groups, mz = (blockIdx.x / p.groups) * fr;
   const long long gidx = (long long)(mz / kUmmaRows) * p.groups + grp;
   const long long gstart = gidx * p.U;
   const long long first = sk_owner(gstart, p.W, P);
   const int npieces = (int)(sk_owner(gstart + p.U - 1, p.W, P) - first + 1);
   int si;
   sk_tile(p, grp, 0, si);
-  if (sk_rows(p, si, mz, 64) <= 0) return;
-  sk_fixup<E>(p, grp, mz, 64, npieces, nullptr);
+  if (sk_rows(p, si, mz, fr) <= 0) return;
+  sk_fixup<E>(p, grp, mz, fr, npieces, nullptr);
 }
 
 }  // namespace dfl
