@@ -47,11 +47,12 @@ DEVI void as_scores(const uint32_t (&qa)[8][4], const uint8_t* kbase, int half, 
   for (int ks = 0; ks < 8; ++ks) {
     const int hf = ks >> 2, c = (ks & 3) * 2 + ((lane >> 3) & 1);
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int r = key0 + n * 8 + (lane & 7);
-      uint32_t b0, b1;
-      ldmatrix_x2(b0, b1, kbase + hf * half + as_off(r, c));
-      mma16816(s[n], qa[ks], b0, b1);
+    for (int n = 0; n < NT; n += 2) {  // two n-tiles per ldmatrix: lanes 16-31 address tile n + 1
+      const int r = key0 + (n + (lane >> 4)) * 8 + (lane & 7);
+      uint32_t b[4];
+      ldmatrix_x4(b, kbase + hf * half + as_off(r, c));
+      mma16816(s[n], qa[ks], b[0], b[1]);
+      mma16816(s[n + 1], qa[ks], b[2], b[3]);
     }
   }
 }
@@ -68,10 +69,12 @@ DEVI void as_pv(const float (&s)[4][4], const uint8_t* vbase, int half, int key0
     a[3] = pack_bf2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
     const int r = key0 + kk * 16 + (lane & 15);
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      uint32_t b0, b1;
-      ldmatrix_x2_trans(b0, b1, vbase + (n >> 3) * half + as_off(r, n & 7));
-      mma16816(o[n], a, b0, b1);
+    for (int n = 0; n < 16; n += 2) {  // two dim tiles per ldmatrix: lanes 16-31 address tile n + 1
+      const int nn = n + (lane >> 4);
+      uint32_t b[4];
+      ldmatrix_x4_trans(b, vbase + (nn >> 3) * half + as_off(r, nn & 7));
+      mma16816(o[n], a, b[0], b[1]);
+      mma16816(o[n + 1], a, b[2], b[3]);
     }
   }
 }
@@ -110,12 +113,14 @@ DEVI void as_softmax(float (&s)[4][4], float (&m)[2], float (&l)[2], float (&o)[
     l[h] = l[h] * corr[h] + add[h];
     m[h] = mx[h];
   }
+  if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {  // (most chunks keep the max)
 #pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    o[n][0] *= corr[0];
-    o[n][1] *= corr[0];
-    o[n][2] *= corr[1];
-    o[n][3] *= corr[1];
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= corr[0];
+      o[n][1] *= corr[0];
+      o[n][2] *= corr[1];
+      o[n][3] *= corr[1];
+    }
   }
 }
 

@@ -84,6 +84,11 @@ DEVI void ldmatrix_x2(uint32_t& r0, uint32_t& r1, const void* p) {
                : "=r"(r0), "=r"(r1)
                : "r"(smem_u32(p)));
 }
+DEVI void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
 DEVI void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                : "=r"(r0), "=r"(r1)
