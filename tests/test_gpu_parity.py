@@ -215,12 +215,13 @@ def test_tied_candidates_are_distinct_and_in_id_order():
     assert set(ids.tolist()) <= set(dups) | {top}, ids
 
 
-@pytest.mark.parametrize("wfmt,block,batch", [(0, 8, 12), (1, 5, 20), (0, 8, 40)])
+@pytest.mark.parametrize("wfmt,block,batch", [(0, 8, 4), (0, 8, 6), (0, 8, 12), (1, 5, 20), (0, 8, 40)])
 def test_tiny_many_rows_run_on_tensor_cores(wfmt, block, batch):
-    """More than 64 block rows: every layer product runs as a tcgen05 contraction (TMEM
-    accumulators, dequantised weight tiles, TMA-staged activations) followed by its fix-up
-    kernel; Q4_K and bf16 layers, ragged new rows (0 included), shuffled pages, and 320 rows
-    (two 256-row tiles, 640 rows for the k/v projections)."""
+    """32 or more block rows: every layer product runs as a tcgen05 contraction (TMEM
+    accumulators, dequantised weight tiles, TMA-staged activations; the tile's N is the rows
+    rounded up to 16: 32, 48, 96, 112) followed by its fix-up kernel; Q4_K and bf16 layers, ragged
+    new rows (0 included), shuffled pages, and 320 rows (two 256-row tiles, 640 rows for the k/v
+    projections)."""
     import dataclasses
     wl = dataclasses.replace(inputs.WORKLOADS["tiny"], dims=dataclasses.replace(inputs.TINY, wfmt=wfmt, block=block),
                              batch=batch, ctx_lo=0, ctx_hi=300, shuffled_pages=True)
