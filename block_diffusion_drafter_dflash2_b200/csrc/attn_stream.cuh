@@ -33,6 +33,7 @@ constexpr int kAsBlk = 4 * 16 * 128;         // the block keys (<= 16) in the sa
 constexpr int kAsQ = 32 * 256;               // 32 query vectors x 128 bf16
 constexpr int kAsThreads = 5 * 32;
 constexpr int kAsSmem = kAsStages * kAsStage + kAsBlk + kAsQ + 1024;
+constexpr int kAsMaxPages = 256;  // page-table entries a CTA reads ahead (64 chunks: windows to 4032)
 
 // byte offset of dims [8c, 8c + 8) of key row r in a 128-byte-swizzled half block
 DEVI uint32_t as_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[kAsStages], empty[kAsStages];
   __shared__ int pvalid[kAsStages];  // bit i: page i of the stage's chunk is mapped
+  __shared__ int s_pg[kAsMaxPages];  // physical page of (local chunk i, page pi) at 4 i + pi
   __shared__ float mrg_m[2][16], mrg_l[2][16];
   __shared__ float fin_m[32], fin_l[32];  // this CTA's running max and sum per query vector
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -166,28 +168,34 @@ __global__ void __launch_bounds__(kAsThreads, 2) k_attn_stream(const __grid_cons
 
   if (warp == 4) {
     // ---- producer: this CTA's share of the window's pages, chunk by chunk ----
+    // page (local chunk i, page pi): -2 past the cached tokens (nothing to load), -1 unmapped
+    auto page_of = [&](int i, int pi) -> int {
+      const long long j0 = cs + (long long)(rank + i * S) * kAsKeys + pi * kPage;  // first token
+      if (j0 >= Lb) return -2;
+      const long long lp = j0 / kPage;
+      int g = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+      if (g >= p.num_pages || g < 0) {
+        g = -1;
+        set_err(p.err, DFLASH2_DEV_PAGE);
+      }
+      return g;
+    };
+    // the whole warp reads the page-table entries ahead, all loads in flight together (one by
+    // one they put a global-memory round trip per page on the chunk's critical path)
+    const int npre = nloc * 4 < kAsMaxPages ? nloc * 4 : kAsMaxPages;
+    for (int k = lane; k < npre; k += 32) s_pg[k] = page_of(k >> 2, k & 3);
+    __syncwarp();
     if (lane == 0) {
       bool dead = false;
       int issued = 0;
       for (int i = 0; i < nloc && !dead; ++i) {
-        const int c = rank + i * S, s = i % kAsStages, round = i / kAsStages;
+        const int s = i % kAsStages, round = i / kAsStages;
         if (round > 0 && !wait_or_die(&empty[s], (round - 1) & 1, dead, p.err)) break;
         int pg[4], pv = 0;
         uint32_t bytes = 0;
         for (int pi = 0; pi < 4; ++pi) {
-          const long long j0 = cs + (long long)c * kAsKeys + pi * kPage;  // first token of the page
-          int g = -2;  // -2: past the cached tokens (nothing to load), -1: unmapped
-          if (j0 < Lb) {
-            const long long lp = j0 / kPage;
-            g = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
-            if (g >= p.num_pages) g = -1;
-            if (g < 0) {
-              g = -1;
-              set_err(p.err, DFLASH2_DEV_PAGE);
-            } else {
-              bytes += 4 * 2048;
-            }
-          }
+          const int g = 4 * i + pi < npre ? s_pg[4 * i + pi] : page_of(i, pi);
+          if (g >= 0) bytes += 4 * 2048;
           pg[pi] = g;
           pv |= (g >= 0 ? 1 : 0) << pi;
         }
