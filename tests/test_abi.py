@@ -114,6 +114,23 @@ def test_unprepared_q4k_weights_are_rejected(lib):
     assert rc == -6
 
 
+@pytest.mark.parametrize("dims_name,batch,umma_products", [
+    ("tiny", 3, 1),   # 24 block rows stream; only q/k/v (48 rows: block + context) on the tensor cores
+    ("tiny", 4, 6),   # 32 rows: every layer product and fc on the tensor cores
+    ("full", 1, 0),   # 8 rows (16 for q/k/v): all streamed
+    ("full", 2, 5),   # q/k/v of 5 layers at 32 rows
+    ("full", 4, 26),  # 5 layers x 5 products + fc
+    ("full", 64, 26),
+])
+def test_tensor_core_products_from_32_rows(lib, dims_name, batch, umma_products):
+    """A product runs on the tensor cores (two launches: product and fix-up) from 32 activation rows
+    on; the plan is visible on the host through the per-step launch count."""
+    dims = inputs.TINY if dims_name == "tiny" else inputs.FULL
+    cfg = binding.config(dims)
+    base = 3 + 6 * dims.layers + 1 + 1 + 1
+    assert lib.dflash2_step_kernels(C.byref(cfg), batch) == base + umma_products
+
+
 def test_step_kernel_count_without_a_device(lib):
     cfg = binding.config(inputs.TINY)
     # embed, fc, fc norm | 7 per layer | final norm, LM head, selector tau + Viterbi
