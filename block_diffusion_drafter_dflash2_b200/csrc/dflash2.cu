@@ -27,6 +27,7 @@ struct GemvPlan {
   size_t smem = 0;
   bool umma = false;  // tensor-core (tcgen05) product + fix-up instead of the streaming engine
   int un = 0;         // its activation rows per tile (MMA N): all rows up to 256, rounded up to 16
+  bool upair = false; // its tiles are two 256-row halves (more than 256 rows)
   bool mlx = false;   // 4-bit records hold MLX group-64 (scale, bias) pairs
   int rows = 0, K = 0;
 };
@@ -79,14 +80,18 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
     g.R = kUmmaRows;
     g.un = rows >= kUmmaRows ? kUmmaRows : (rows + 15) / 16 * 16;
     g.NT = 8;
-    g.mgroups = (rows + kUmmaRows - 1) / kUmmaRows;
+    // 4-bit weights and more than 256 rows: tiles of two 256-row halves, each weight stage
+    // dequantised once for both (bf16 weights keep double-buffered accumulators and three stages:
+    // measured faster without the pairing)
+    g.upair = q4 && rows > kUmmaRows;
+    g.mgroups = (rows + (g.upair ? 2 : 1) * kUmmaRows - 1) / ((g.upair ? 2 : 1) * kUmmaRows);
     g.groups = (tiles + kConsumers - 1) / kConsumers;
     g.U = K / (q4 ? Ring<true>::kUnitK : Ring<false>::kUnitK);
     g.W = (long long)g.groups * g.mgroups * g.U;
     g.P = (int)std::min<long long>(nsm, g.W);
     g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
     g.kc_units = g.U;
-    g.smem = kUmmaSmem;
+    g.smem = g.upair ? kUmmaPairSmem : kUmmaSmem;
     return g;
   }
   g.R = rows <= 8 ? 8 : rows <= 16 ? 16 : rows <= 32 ? 32 : 64;
@@ -399,6 +404,7 @@ SGemvParams sgemv_params(const GemvPlan& g, const GemvSeg* segs, int nseg, bool 
   prm.rs_glob = (g.umma && e.rs_in) ? e.rs_glob : nullptr;
   prm.mlx = g.mlx ? 1 : 0;
   prm.un = g.un;
+  prm.upair = g.upair ? 1 : 0;
   return prm;
 }
 
@@ -442,15 +448,21 @@ cudaError_t make_act_tmap(CUtensorMap* tm, const uint16_t* X, int K, int ldx, in
 
 // Tensor-core product (stream-K pieces into the partial buffer) and its fix-up kernel (piece sums
 // in order + the product's epilogue), both with programmatic dependent launch.
+template <bool Q4, bool PAIR>
+cudaError_t launch_umma_k(const GemvPlan& g, const SGemvParams& prm, const CUtensorMap& tm, cudaStream_t s) {
+  static std::atomic<int> attr[kMaxDevices];
+  const int smem = PAIR ? kUmmaPairSmem : kUmmaSmem;
+  const cudaError_t e = smem_optin(k_umma<Q4, PAIR>, smem, attr);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_umma<Q4, PAIR>, dim3(g.P), dim3(kUmmaThreads), (size_t)smem, s, tm, prm);
+}
+
 template <bool Q4>
 cudaError_t launch_umma_t(const GemvPlan& g, const SGemvParams& prm, cudaStream_t s) {
-  static std::atomic<int> attr[kMaxDevices];
-  cudaError_t e = smem_optin(k_umma<Q4>, kUmmaSmem, attr);
-  if (e != cudaSuccess) return e;
   CUtensorMap tm;
-  e = make_act_tmap(&tm, prm.X, g.K, prm.ldx, prm.rows, g.un);
+  cudaError_t e = make_act_tmap(&tm, prm.X, g.K, prm.ldx, prm.rows, g.un);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(k_umma<Q4>, dim3(g.P), dim3(kUmmaThreads), (size_t)kUmmaSmem, s, tm, prm);
+  e = g.upair ? launch_umma_k<Q4, true>(g, prm, tm, s) : launch_umma_k<Q4, false>(g, prm, tm, s);
   if (e != cudaSuccess) return e;
   // rows per fix-up CTA: 64, halved (down to 16) while the grid would leave SMs idle (the fix-ups
   // of products with few column groups are latency-bound)

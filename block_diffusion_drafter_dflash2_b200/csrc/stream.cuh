@@ -109,6 +109,7 @@ struct SGemvParams {
   float* rs_glob;
   int mlx;  // 4-bit records carry MLX group-64 (scale, bias) pairs instead of Q4_K scale records
   int un;   // tensor-core path: activation rows per tile (the MMA's N and the TMA box height)
+  int upair;  // and 1 when a tile is two 256-row halves sharing each weight stage
 };
 
 // Row scales of rows [mz, mz + rows) from quarter-column sums of squares (ssp layout

@@ -41,6 +41,7 @@ constexpr int kUmmaDq = 16;                        // weight-operand warps (a ti
 constexpr int kUmmaThreads = (4 + kUmmaDq + 4) * 32; // roles below
 constexpr int kUHeadThreads = 16 * 32;               // the output head's roles
 constexpr int kUmmaSmem = kUmmaStages * (kUmmaABytes + kUmmaBBytes) + kUmmaRaw * kUmmaRawBytes + 1024;
+constexpr int kUmmaPairSmem = 2 * (kUmmaABytes + 2 * kUmmaBBytes) + kUmmaRaw * kUmmaRawBytes + 1024;
 constexpr int kUmmaTmemCols = 512;                 // two 256-column accumulators
 
 // ---- tcgen05 / TMA wrappers (one instruction each) ----
@@ -168,23 +169,28 @@ DEVI void rows_scale_global(const float* ssp, int ldr, int H, float eps, int r0,
 // latencies hide behind one another's work: the dequantisation's dependent chains bounded the
 // kernel with one or two per sub-partition); warps 20-23: epilogue (TMEM lane = feature), on two
 // accumulators alternating by piece.
-template <bool Q4>
+template <bool Q4, bool PAIR>
 __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
+  // PAIR: a tile is two 256-row halves sharing each weight stage (the operand is dequantised once
+  // for both), accumulated in all 512 TMEM columns; two stages of 80 KB instead of three of 48 KB
+  constexpr int NS = PAIR ? 2 : kUmmaStages;
+  constexpr int BST = PAIR ? 2 * kUmmaBBytes : kUmmaBBytes;
+  constexpr int MROWS = PAIR ? 2 * kUmmaRows : kUmmaRows;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t xfull[kUmmaStages], afull[kUmmaStages], sempty[kUmmaStages];
+  __shared__ __align__(8) uint64_t xfull[NS], afull[NS], sempty[NS];
   __shared__ __align__(8) uint64_t rfull[kUmmaRaw], rempty[kUmmaRaw];
   __shared__ __align__(8) uint64_t accfull[2], accempty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* As = smem;                                   // [stages][128 x 128 B]
-  uint8_t* Bs = As + kUmmaStages * kUmmaABytes;         // [stages][256 x 128 B]
-  uint8_t* Rs = Bs + kUmmaStages * kUmmaBBytes;         // [raw slots][group unit]
+  uint8_t* As = smem;                    // [NS][128 x 128 B]
+  uint8_t* Bs = As + NS * kUmmaABytes;   // [NS][1 or 2 halves][256 x 128 B]
+  uint8_t* Rs = Bs + NS * BST;           // [raw slots][group unit]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kSub = Q4 ? 4 : 1;  // 64-wide stages per prepared K unit
   constexpr int kUnitK = Q4 ? 256 : 64;
   constexpr int kRawUnit = Ring<Q4>::kSlot;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kUmmaStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&afull[s], kUmmaDq);
       mbar_init(&sempty[s], 1);
@@ -220,16 +226,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
       for (long long x = x0; x < x1 && !dead;) {
         const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
         const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
-        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * MROWS;
         int si;
         sk_tile(p, grp, 0, si);
-        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
+        if (sk_rows(p, si, mz, MROWS) > 0) {
+          const bool h2 = PAIR && sk_rows(p, si, mz + kUmmaRows, kUmmaRows) > 0;  // second half rows
           for (int u = ua; u < ub && !dead; ++u)
             for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
-              const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
+              const int s = cnt % NS, round = cnt / NS;
               if (round > 0 && !wait_or_die(&sempty[s], (round - 1) & 1, dead, p.err)) break;
-              mbar_expect_tx(&xfull[s], (uint32_t)p.un * 128u);  // the box: un rows of 64 k
-              tma_load_2d(Bs + s * kUmmaBBytes, &tmx, u * kUnitK + sub * 64, mz, &xfull[s]);
+              mbar_expect_tx(&xfull[s], (uint32_t)p.un * 128u * (h2 ? 2u : 1u));  // boxes: un rows of 64 k
+              tma_load_2d(Bs + s * BST, &tmx, u * kUnitK + sub * 64, mz, &xfull[s]);
+              if (h2) tma_load_2d(Bs + s * BST + kUmmaBBytes, &tmx, u * kUnitK + sub * 64, mz + kUmmaRows, &xfull[s]);
             }
         }
         x += ub - ua;
@@ -243,11 +251,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
       for (long long x = x0; x < x1 && !dead;) {
         const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
         const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
-        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * MROWS;
         int si;
         sk_tile(p, grp, 0, si);
-        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
-          const int buf = piece & 1, use = piece >> 1;
+        if (sk_rows(p, si, mz, MROWS) > 0) {
+          const bool h2 = PAIR && sk_rows(p, si, mz + kUmmaRows, kUmmaRows) > 0;
+          // a pair tile fills all 512 columns, so its pieces take turns with the epilogue
+          const int buf = PAIR ? 0 : piece & 1, use = PAIR ? piece : piece >> 1;
           if (use > 0 && !wait_or_die(&accempty[buf], (use - 1) & 1, dead, p.err)) break;
           tc_fence_after();
           const uint32_t acc = tmem + (uint32_t)(buf * kUmmaRows);
@@ -255,15 +265,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           bool first = true;
           for (int u = ua; u < ub && !dead; ++u)
             for (int sub = 0; sub < kSub && !dead; ++sub, ++cnt) {
-              const int s = cnt % kUmmaStages;
-              const uint32_t par = (cnt / kUmmaStages) & 1;
+              const int s = cnt % NS;
+              const uint32_t par = (cnt / NS) & 1;
               if (!wait_or_die(&xfull[s], par, dead, p.err) || !wait_or_die(&afull[s], par, dead, p.err)) break;
               tc_fence_after();
               const uint64_t ad = sw128_desc(smem_u32(As + s * kUmmaABytes));
-              const uint64_t bd = sw128_desc(smem_u32(Bs + s * kUmmaBBytes));
+              const uint64_t bd = sw128_desc(smem_u32(Bs + s * BST));
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes inside the swizzled rows
+              for (int kk = 0; kk < 4; ++kk) {  // 16-wide K slices: +32 bytes inside the swizzled rows
                 tc_mma(acc, ad + 2 * kk, bd + 2 * kk, idesc, (first && kk == 0) ? 0u : 1u);
+                if (h2)  // the second half: the same weights, rows 256 on, accumulator columns 256 on
+                  tc_mma(acc + (uint32_t)kUmmaRows, ad + 2 * kk, bd + (uint64_t)(kUmmaBBytes >> 4) + 2 * kk, idesc,
+                         (first && kk == 0) ? 0u : 1u);
+              }
               first = false;
               tc_commit(&sempty[s]);  // the stage is free once these MMAs have read it
             }
@@ -281,10 +295,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
       for (long long x = x0; x < x1 && !dead;) {
         const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
         const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
-        const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+        const int grp = gidx % p.groups, mz = (gidx / p.groups) * MROWS;
         int si;
         sk_tile(p, grp, 0, si);
-        if (sk_rows(p, si, mz, kUmmaRows) > 0) {
+        if (sk_rows(p, si, mz, MROWS) > 0) {
           const uint8_t* src = sk_group_src<Q4>(p, grp);
           for (int u = ua; u < ub && !dead; ++u, ++cnt) {
             const int r = cnt % kUmmaRaw, round = cnt / kUmmaRaw;
@@ -312,10 +326,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
     for (long long x = x0; x < x1;) {
       const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
       const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
-      const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+      const int grp = gidx % p.groups, mz = (gidx / p.groups) * MROWS;
       int si0;
       sk_tile(p, grp, 0, si0);
-      if (sk_rows(p, si0, mz, kUmmaRows) > 0) {
+      if (sk_rows(p, si0, mz, MROWS) > 0) {
         for (int u = ua; u < ub; ++u, ++ucnt) {
           const int r = ucnt % kUmmaRaw;
           wait_or_die(&rfull[r], (ucnt / kUmmaRaw) & 1, dead, p.err);
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           }
 #pragma unroll
           for (int sub = 0; sub < kSub; ++sub, ++cnt) {
-            const int s = cnt % kUmmaStages, round = cnt / kUmmaStages;
+            const int s = cnt % NS, round = cnt / NS;
             uint8_t* a = As + s * kUmmaABytes;
             // features g and g + 8 of tile tl go to operand rows 16 tl + a8(g) and + 8: a8 puts the
             // two features of each 8-lane store phase 4 rows apart, so that the phase's 16-byte
@@ -400,15 +414,15 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
     for (long long x = x0; x < x1;) {
       const int gidx = (int)(x / p.U), ua = (int)(x % p.U);
       const int ub = (int)((x1 - x) < (long long)(p.U - ua) ? ua + (x1 - x) : p.U);
-      const int grp = gidx % p.groups, mz = (gidx / p.groups) * kUmmaRows;
+      const int grp = gidx % p.groups, mz = (gidx / p.groups) * MROWS;
       int si0;
       sk_tile(p, grp, 0, si0);
-      if (sk_rows(p, si0, mz, kUmmaRows) > 0) {
+      if (sk_rows(p, si0, mz, MROWS) > 0) {
         if (!waited) {
           pdl_wait();  // the partial buffer may still be read by the previous product's fix-up
           waited = true;
         }
-        const int buf = piece & 1, use = piece >> 1;
+        const int buf = PAIR ? 0 : piece & 1, use = PAIR ? piece : piece >> 1;
         const int pc = (int)(c - sk_owner((long long)gidx * p.U, p.W, P));
         if (wait_or_die(&accfull[buf], use & 1, dead, p.err)) {
           tc_fence_after();
@@ -416,17 +430,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant_
           const int fo = (m & 8) | ((m & 3) << 1) | ((m >> 2) & 1);
           int si;
           const int tile = sk_tile(p, grp, m >> 4, si);
-          const int rows = tile >= 0 ? sk_rows(p, si, mz, kUmmaRows) : 0;
-          float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mz * p.ldo +
-                       (tile >= 0 ? p.seg[si].out_col + tile * 16 + fo : 0);
-          const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kUmmaRows);
-          for (int n0 = 0; n0 < rows && n0 < p.un; n0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(tbase + (uint32_t)n0, v);
-            tmem_ld_wait();
+#pragma unroll 1
+          for (int h = 0; h < (PAIR ? 2 : 1); ++h) {  // the tile's halves: rows mz + 256 h ..
+            const int mh = mz + h * kUmmaRows;
+            const int rows = tile >= 0 ? sk_rows(p, si, mh, kUmmaRows) : 0;
+            float* out = p.part + (size_t)pc * p.piece_stride + (size_t)mh * p.ldo +
+                         (tile >= 0 ? p.seg[si].out_col + tile * 16 + fo : 0);
+            const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)((buf + h) * kUmmaRows);
+            for (int n0 = 0; n0 < rows && n0 < p.un; n0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(tbase + (uint32_t)n0, v);
+              tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < rows) out[(size_t)(n0 + i) * p.ldo] = __uint_as_float(v[i]);
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < rows) out[(size_t)(n0 + i) * p.ldo] = __uint_as_float(v[i]);
+            }
           }
           tc_fence_before();
         }
@@ -673,7 +691,7 @@ __global__ void __launch_bounds__(kGemvConsumers * 32, MINB) k_umma_fixup(SGemvP
   pdl_trigger();
   pdl_wait();
   const int grp = blockIdx.x % p.groups, mz = (blockIdx.x / p.groups) * fr;
-  const long long gidx = (long long)(mz / kUmmaRows) * p.groups + grp;
+  const long long gidx = (long long)(mz / (p.upair ? 2 * kUmmaRows : kUmmaRows)) * p.groups + grp;
   const long long gstart = gidx * p.U;
   const long long first = sk_owner(gstart, p.W, P);
   const int npieces = (int)(sk_owner(gstart + p.U - 1, p.W, P) - first + 1);
