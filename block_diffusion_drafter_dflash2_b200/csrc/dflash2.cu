@@ -80,13 +80,14 @@ GemvPlan plan_gemv(int tiles, int rows, int K, bool q4, int nsm) {
     g.R = kUmmaRows;
     g.un = rows >= kUmmaRows ? kUmmaRows : (rows + 15) / 16 * 16;
     g.NT = 8;
-    // 4-bit weights and more than 256 rows: tiles of two 256-row halves, each weight stage
-    // dequantised once for both (bf16 weights keep double-buffered accumulators and three stages:
-    // measured faster without the pairing)
-    g.upair = q4 && rows > kUmmaRows;
-    g.mgroups = (rows + (g.upair ? 2 : 1) * kUmmaRows - 1) / ((g.upair ? 2 : 1) * kUmmaRows);
     g.groups = (tiles + kConsumers - 1) / kConsumers;
     g.U = K / (q4 ? Ring<true>::kUnitK : Ring<false>::kUnitK);
+    // 4-bit weights and more than 256 rows: tiles of two 256-row halves, each weight stage
+    // dequantised once for both, as long as every CTA still gets 8 or more K units (measured: bf16
+    // weights, and products as small as W_o, run faster with double-buffered 256-row tiles)
+    const int mg1 = (rows + kUmmaRows - 1) / kUmmaRows, mg2 = (rows + 2 * kUmmaRows - 1) / (2 * kUmmaRows);
+    g.upair = q4 && rows > kUmmaRows && (long long)g.groups * mg2 * g.U >= 8LL * nsm;
+    g.mgroups = g.upair ? mg2 : mg1;
     g.W = (long long)g.groups * g.mgroups * g.U;
     g.P = (int)std::min<long long>(nsm, g.W);
     g.max_pieces = (int)((long long)(g.U - 1) * g.P / g.W) + 2;
