@@ -167,8 +167,8 @@ DEVI void rows_scale_global(const float* ssp, int ldr, int H, float eps, int r0,
 // a folded RMSNorm for the fix-up (p.rs_glob); warps 4-19: the weight operand from the raw ring,
 // one 32-wide half of one 16-feature tile each (four warps per SM sub-partition, so their
 // latencies hide behind one another's work: the dequantisation's dependent chains bounded the
-// kernel with one or two per sub-partition); warps 20-23: epilogue (TMEM lane = feature), on two
-// accumulators alternating by piece.
+// kernel with one or two per sub-partition); warps 20-23: epilogue (TMEM lane = operand row), on
+// two accumulators alternating by piece, or (PAIR) on the two halves of each piece in turn.
 template <bool Q4, bool PAIR>
 __global__ void __launch_bounds__(kUmmaThreads, 1) k_umma(const __grid_constant__ CUtensorMap tmx, SGemvParams p) {
   // PAIR: a tile is two 256-row halves sharing each weight stage (the operand is dequantised once
