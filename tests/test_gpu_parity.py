@@ -186,6 +186,21 @@ def test_full_size_configs(name, sample):
     parity.check_accept(run)
 
 
+@pytest.mark.slow
+def test_full_size_320_rows_run_as_paired_tiles():
+    """40 requests (320 block rows, 640 for k/v): the 4-bit layer products run as tensor-core tiles
+    of two 256-row halves whose second half is partly filled (rows 256-319; for k/v 512-639 with
+    an empty second half)."""
+    import dataclasses
+    wl = dataclasses.replace(inputs.WORKLOADS["full_b64"], batch=40)
+    w, hw_t, hw = weights_for(wl)
+    sample = [0, 33, 39]
+    run = parity.run_gpu(wl, w, sample)
+    for b in sample:
+        parity.check_request(run, hw_t, hw, b)
+    parity.check_accept(run)
+
+
 def test_tied_candidates_are_distinct_and_in_id_order():
     """Exact logit ties in the output head: the head row of one drafted position's best token is
     copied onto 23 other ids (in its own 16-row tile, in other tiles of its 256-id record, and in
