@@ -526,7 +526,7 @@ DEVI void reg_list_insert(float (&lv)[16], int (&li)[16], float v, int id) {
 __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_constant__ CUtensorMap tmx, UHeadParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t xfull[kUHeadStages], bfull[kUHeadStages], sempty[kUHeadStages];
-  __shared__ __align__(8) uint64_t accfull, accempty;
+  __shared__ __align__(8) uint64_t accfull[2], accempty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -535,14 +535,20 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
   const int row0 = rt * 256;
   const int trows = p.rows - row0 < 256 ? p.rows - row0 : 256;
   const int nmc = trows > 128 ? 2 : 1;  // 128-row accumulators this row tile needs
+  // with one accumulator (at most 128 rows) the records alternate between TMEM columns 0 and 256,
+  // so that the next record's MMAs run while the epilogue drains this one
+  auto acc_buf = [&](int it) { return nmc == 1 ? (it & 1) : 0; };
+  auto acc_use = [&](int it) { return nmc == 1 ? (it >> 1) : it; };
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUHeadStages; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&bfull[s], 1);
       mbar_init(&sempty[s], 1);
     }
-    mbar_init(&accfull, 1);
-    mbar_init(&accempty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -580,7 +586,8 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
       bool dead = false;
       int cnt = 0, it = 0;
       for (int rec = part; rec < p.nrec && !dead; rec += nparts, ++it) {
-        if (it > 0 && !wait_or_die(&accempty, (it - 1) & 1, dead, p.err)) break;
+        const int buf = acc_buf(it), use = acc_use(it);
+        if (use > 0 && !wait_or_die(&accempty[buf], (use - 1) & 1, dead, p.err)) break;
         tc_fence_after();
         for (int st = 0; st < S && !dead; ++st, ++cnt) {
           const int s = cnt % kUHeadStages;
@@ -593,11 +600,11 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
             const uint64_t ad = sw128_desc(a0 + mc * 16384);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc_mma(tmem + mc * 256, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (st == 0 && kk == 0) ? 0u : 1u);
+              tc_mma(tmem + (buf + mc) * 256, ad + 2 * kk, bd + 2 * kk, kUmmaIdesc, (st == 0 && kk == 0) ? 0u : 1u);
           }
           tc_commit(&sempty[s]);
         }
-        if (!dead) tc_commit(&accfull);
+        if (!dead) tc_commit(&accfull[buf]);
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -616,7 +623,8 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
     int it = 0;
     pdl_wait();  // (outputs; the dependency also orders the lists after the previous step's readers)
     for (int rec = part; rec < p.nrec; rec += nparts, ++it) {
-      if (wait_or_die(&accfull, it & 1, dead, p.err)) {
+      const int buf = acc_buf(it), use = acc_use(it);
+      if (wait_or_die(&accfull[buf], use & 1, dead, p.err)) {
         tc_fence_after();
 #pragma unroll
         for (int mc = 0; mc < 2; ++mc) {
@@ -624,7 +632,7 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
           const int rl = mc * 128 + dw * 32 + lane, row = row0 + rl;
           for (int n0 = 0; n0 < 256; n0 += 32) {
             uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)(mc * 256 + n0), r);
+            tmem_ld32(tmem + ((uint32_t)(dw * 32) << 16) + (uint32_t)((buf + mc) * 256 + n0), r);
             tmem_ld_wait();
             if (rl < trows) {
               const int f0 = rec * 256 + n0, g0 = f0 + p.id0;  // g0: vocabulary id of feature f0
@@ -657,7 +665,7 @@ __global__ void __launch_bounds__(kUHeadThreads, 1) k_umma_head(const __grid_con
         tc_fence_before();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty);
+      if (lane == 0) mbar_arrive(&accempty[buf]);
     }
     // this CTA's lists -> part `part` of the candidate lists
 #pragma unroll
